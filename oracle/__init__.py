@@ -1,0 +1,160 @@
+"""fp64 CPU oracle for sink-softmax GQA attention -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` /
+``--impl reference`` legs of ``bench.py`` may import this package.  The CUDA
+product path (``gqa_softmax_attention_attn_b200``) never imports it, and the
+two share no code.
+
+The arithmetic lives in ``attn_sink_oracle.c`` (plain C, fp64, OpenMP); this
+module only compiles it with gcc and marshals numpy float64 arrays.  The
+definition it follows is stated in the C file's header ("GPT-OSS on day 0",
+sections "Attention: GQA with Attention Sinks" and "Sink Attention").
+
+Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
+against library routines (PyTorch CPU fp64 SDPA and autograd), closed forms,
+invariants, brute force and finite differences.  The pages print no worked
+example, so no stored golden values from the pages exist.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "attn_sink_oracle.c")
+_BUILD_DIR = os.path.join(_HERE, "_build")
+_LIB_PATH = os.path.join(_BUILD_DIR, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the C oracle into oracle/_build/liboracle.so (generic x86-64 flags)."""
+    os.makedirs(_BUILD_DIR, exist_ok=True)
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-shared", "-fPIC", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load(path: str | None = None):
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(path or build())
+        P = ctypes.c_void_p
+        I = ctypes.c_int
+        Dd = ctypes.c_double
+        lib.oracle_fwd.argtypes = [P] * 6 + [I] * 7 + [Dd]
+        lib.oracle_fwd_rows.argtypes = [P] * 7 + [I] + [P, P] + [I] * 7 + [Dd]
+        lib.oracle_decode.argtypes = [P] * 7 + [I] * 6 + [Dd]
+        lib.oracle_bwd.argtypes = [P] * 9 + [I] * 7 + [Dd]
+        lib.oracle_row_stats.argtypes = [P] * 7 + [I] * 7 + [Dd]
+        lib.oracle_num_threads.restype = I
+        _lib = lib
+    return _lib
+
+
+class use_library:
+    """Context manager that points this module at another build of the C
+    oracle (used only by the mutation test, which compiles planted mistakes)."""
+
+    def __init__(self, path: str):
+        self.path = path
+
+    def __enter__(self):
+        global _lib
+        self.saved = _lib
+        _lib = None
+        _load(self.path)
+        return self
+
+    def __exit__(self, *exc):
+        global _lib
+        _lib = self.saved
+        return False
+
+
+def _f64(a) -> np.ndarray:
+    if hasattr(a, "detach"):
+        a = a.detach().to("cpu").double().numpy()
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+def fwd(q, k, v, sinks, window: int, scale: float):
+    """q [B,Lq,Hq,D], k/v [B,Lk,Hkv,D], sinks [Hq] -> (out [B,Lq,Hq,D], lse [B,Hq,Lq])."""
+    q, k, v, sinks = _f64(q), _f64(k), _f64(v), _f64(sinks)
+    B, Lq, Hq, D = q.shape
+    Lk, Hkv = k.shape[1], k.shape[2]
+    assert Hq % Hkv == 0 and sinks.shape == (Hq,)
+    out = np.empty_like(q)
+    lse = np.empty((B, Hq, Lq))
+    _load().oracle_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(sinks), _ptr(out), _ptr(lse),
+                       B, Lq, Lk, Hq, Hkv, D, int(window), float(scale))
+    return out, lse
+
+
+def fwd_rows(q, k, v, sinks, rows_b, rows_h, rows_i, window: int, scale: float):
+    """Forward for sampled rows only: returns (out_rows [n,D], lse_rows [n])."""
+    q, k, v, sinks = _f64(q), _f64(k), _f64(v), _f64(sinks)
+    B, Lq, Hq, D = q.shape
+    Lk, Hkv = k.shape[1], k.shape[2]
+    rb = np.ascontiguousarray(rows_b, dtype=np.int32)
+    rh = np.ascontiguousarray(rows_h, dtype=np.int32)
+    ri = np.ascontiguousarray(rows_i, dtype=np.int32)
+    n = len(rb)
+    out = np.empty((n, D))
+    lse = np.empty((n,))
+    _load().oracle_fwd_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(sinks), _ptr(rb), _ptr(rh), _ptr(ri), n,
+                            _ptr(out), _ptr(lse), B, Lq, Lk, Hq, Hkv, D, int(window), float(scale))
+    return out, lse
+
+
+def decode(q, k_cache, v_cache, seqlens, sinks, window: int, scale: float):
+    """q [B,Hq,D], caches [B,Lmax,Hkv,D], seqlens [B] -> (out [B,Hq,D], lse [B,Hq])."""
+    q, kc, vc, sinks = _f64(q), _f64(k_cache), _f64(v_cache), _f64(sinks)
+    sl = np.ascontiguousarray(np.asarray(seqlens.cpu() if hasattr(seqlens, "cpu") else seqlens), dtype=np.int32)
+    B, Hq, D = q.shape
+    Lmax, Hkv = kc.shape[1], kc.shape[2]
+    assert sl.min() >= 1 and sl.max() <= Lmax
+    out = np.empty_like(q)
+    lse = np.empty((B, Hq))
+    _load().oracle_decode(_ptr(q), _ptr(kc), _ptr(vc), _ptr(sl), _ptr(sinks), _ptr(out), _ptr(lse),
+                          B, Lmax, Hq, Hkv, D, int(window), float(scale))
+    return out, lse
+
+
+def bwd(q, k, v, sinks, dout, window: int, scale: float):
+    """Returns (dq, dk, dv, dsinks) in fp64, recomputing the forward internally."""
+    q, k, v, sinks, dout = _f64(q), _f64(k), _f64(v), _f64(sinks), _f64(dout)
+    B, Lq, Hq, D = q.shape
+    Lk, Hkv = k.shape[1], k.shape[2]
+    dq = np.empty_like(q)
+    dk = np.empty_like(k)
+    dv = np.empty_like(v)
+    ds = np.empty((Hq,))
+    _load().oracle_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(sinks), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
+                       _ptr(ds), B, Lq, Lk, Hq, Hkv, D, int(window), float(scale))
+    return dq, dk, dv, ds
+
+
+def row_stats(q, k, v, sinks, dout, window: int, scale: float):
+    """Per-row D_i = <dO_i, O_i> and P_sink_i = exp(sink - LSE_i), each [B,Hq,Lq]."""
+    q, k, v, sinks, dout = _f64(q), _f64(k), _f64(v), _f64(sinks), _f64(dout)
+    B, Lq, Hq, D = q.shape
+    Lk, Hkv = k.shape[1], k.shape[2]
+    Dr = np.empty((B, Hq, Lq))
+    Ps = np.empty((B, Hq, Lq))
+    _load().oracle_row_stats(_ptr(q), _ptr(k), _ptr(v), _ptr(sinks), _ptr(dout), _ptr(Dr), _ptr(Ps),
+                             B, Lq, Lk, Hq, Hkv, D, int(window), float(scale))
+    return Dr, Ps

@@ -1,0 +1,312 @@
+"""Pins for the fp64 oracle, against things other than itself (CPU only).
+
+The pages print no worked example, so the oracle is pinned by:
+  * library routines: PyTorch CPU fp64 scaled_dot_product_attention (SDPA) and
+    autograd through it -- sink = -inf must reduce to ordinary causal GQA
+    attention ("GPT-OSS on day 0", section "Attention: GQA with Attention
+    Sinks": the sink only adds a logit), and sink attention must equal SDPA
+    over keys augmented with one zero-value key whose logit is the sink
+    (section "Sink Attention": the sink is a bias term entering the softmax
+    but carrying no value row);
+  * closed forms: window = 1, window = 2, a dominant sink;
+  * invariants: row mass + sink mass = 1, a common shift of all logits,
+    window >= Lk equals dense bit for bit;
+  * brute force on tiny inputs written as a separate pure-Python path;
+  * central finite differences for the backward.
+Masks in these tests are built with torch.tril(diagonal=...) (a library
+routine), independently of the oracle's index arithmetic.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+from gqa_softmax_attention_attn_b200.inputs import decode_inputs, prefill_inputs
+
+TOL = 1e-11
+
+
+def _mask_bool(Lq, Lk, window):
+    """Visible[i, j] with bottom-right causal alignment, via torch.tril."""
+    ones = torch.ones(Lq, Lk, dtype=torch.bool)
+    vis = torch.tril(ones, diagonal=Lk - Lq)
+    if window > 0:
+        vis = vis & ~torch.tril(ones, diagonal=Lk - Lq - window)
+    return vis
+
+
+def _sdpa_aug(q, k, v, sinks, scale, window, grad=False):
+    """Sink attention as SDPA over keys augmented with a zero key whose additive
+    mask entry is the sink logit; an extra value channel that is 1 only on the
+    sink key returns the sink's probability P_sink, hence LSE = sink - ln P_sink.
+    q [B,Lq,Hq,D], k/v [B,Lk,Hkv,D] (fp64)."""
+    B, Lq, Hq, D = q.shape
+    Lk, Hkv = k.shape[1], k.shape[2]
+    qt = q.permute(0, 2, 1, 3)
+    kt = k.permute(0, 2, 1, 3)
+    vt = v.permute(0, 2, 1, 3)
+    zk = torch.zeros(B, Hkv, 1, D, dtype=q.dtype)
+    k_aug = torch.cat([kt, zk], dim=2)
+    v_aug = torch.cat([vt, zk], dim=2)
+    chan = torch.zeros(B, Hkv, Lk + 1, 1, dtype=q.dtype)
+    chan[:, :, Lk, 0] = 1.0
+    v_aug = torch.cat([v_aug, chan], dim=3)
+    vis = _mask_bool(Lq, Lk, window)
+    base = torch.zeros(Lq, Lk, dtype=q.dtype).masked_fill(~vis, float("-inf"))
+    mask = torch.cat([base.expand(Hq, Lq, Lk),
+                      sinks.view(Hq, 1, 1).expand(Hq, Lq, 1)], dim=2).unsqueeze(0)
+    o = F.scaled_dot_product_attention(qt, k_aug, v_aug, attn_mask=mask, scale=scale, enable_gqa=True)
+    o = o.permute(0, 2, 1, 3)
+    out = o[..., :D]
+    psink = o[..., D]  # [B, Lq, Hq]
+    lse = sinks.view(1, 1, Hq) - torch.log(psink)
+    return out, lse.permute(0, 2, 1)
+
+
+def _inp(B, Lq, Lk, Hq, Hkv, D, seed, sink_std=1.0, with_dout=False, sink_fill=None):
+    t = prefill_inputs(B, Lq, Lk, Hq, Hkv, D, dtype=torch.float64, qkv_std=1.0, sink_std=sink_std,
+                       dout_std=1.0, seed=seed, with_dout=with_dout, sink_fill=sink_fill)
+    t["sinks"] = t["sinks"].double()
+    return t
+
+
+@pytest.mark.parametrize("Lq,Lk", [(33, 33), (20, 47), (1, 9)])
+def test_sink_neg_inf_is_plain_causal_gqa_sdpa(Lq, Lk):
+    t = _inp(2, Lq, Lk, 8, 2, 16, seed=1, sink_fill=float("-inf"))
+    scale = 0.3
+    out, lse = oracle.fwd(t["q"], t["k"], t["v"], t["sinks"], 0, scale)
+    vis = _mask_bool(Lq, Lk, 0)
+    ref = F.scaled_dot_product_attention(t["q"].permute(0, 2, 1, 3), t["k"].permute(0, 2, 1, 3),
+                                         t["v"].permute(0, 2, 1, 3), attn_mask=vis, scale=scale,
+                                         enable_gqa=True).permute(0, 2, 1, 3)
+    assert np.abs(out - ref.numpy()).max() < TOL
+    if Lq == Lk:
+        ref2 = F.scaled_dot_product_attention(t["q"].permute(0, 2, 1, 3), t["k"].permute(0, 2, 1, 3),
+                                              t["v"].permute(0, 2, 1, 3), is_causal=True, scale=scale,
+                                              enable_gqa=True).permute(0, 2, 1, 3)
+        assert np.abs(out - ref2.numpy()).max() < TOL
+
+
+@pytest.mark.parametrize("window", [0, 1, 5, 16])
+@pytest.mark.parametrize("Lq,Lk,Hq,Hkv", [(40, 40, 8, 2), (17, 30, 4, 4), (25, 25, 6, 1)])
+def test_matches_augmented_sdpa(window, Lq, Lk, Hq, Hkv):
+    t = _inp(2, Lq, Lk, Hq, Hkv, 8, seed=2 + window)
+    scale = 1.0 / math.sqrt(8)
+    out, lse = oracle.fwd(t["q"], t["k"], t["v"], t["sinks"], window, scale)
+    ref_o, ref_lse = _sdpa_aug(t["q"], t["k"], t["v"], t["sinks"], scale, window)
+    assert np.abs(out - ref_o.numpy()).max() < TOL
+    assert np.abs(lse - ref_lse.numpy()).max() < 1e-10
+
+
+def test_window_ge_lk_is_dense_bitwise():
+    t = _inp(1, 50, 50, 4, 2, 16, seed=3)
+    o0, l0 = oracle.fwd(t["q"], t["k"], t["v"], t["sinks"], 0, 0.25)
+    for w in (50, 51, 1000):
+        o1, l1 = oracle.fwd(t["q"], t["k"], t["v"], t["sinks"], w, 0.25)
+        assert np.array_equal(o0, o1) and np.array_equal(l0, l1)
+
+
+def test_window_one_closed_form():
+    """window = 1: each row sees only its own key, so O_i = v_i * sigmoid(z_ii - sink)."""
+    t = _inp(1, 30, 30, 4, 2, 8, seed=4)
+    scale = 0.4
+    out, lse = oracle.fwd(t["q"], t["k"], t["v"], t["sinks"], 1, scale)
+    q, k, v, s = t["q"].numpy(), t["k"].numpy(), t["v"].numpy(), t["sinks"].numpy()
+    for h in range(4):
+        g = h // 2
+        z = scale * np.einsum("id,id->i", q[0, :, h], k[0, :, g])
+        sig = 1.0 / (1.0 + np.exp(-(z - s[h])))
+        assert np.abs(out[0, :, h] - v[0, :, g] * sig[:, None]).max() < 1e-12
+        assert np.abs(lse[0, h] - np.logaddexp(z, s[h])).max() < 1e-12
+
+
+def test_window_two_closed_form():
+    t = _inp(1, 12, 12, 2, 1, 4, seed=5)
+    scale = 0.7
+    out, lse = oracle.fwd(t["q"], t["k"], t["v"], t["sinks"], 2, scale)
+    q, k, v, s = t["q"].numpy(), t["k"].numpy(), t["v"].numpy(), t["sinks"].numpy()
+    for h in range(2):
+        for i in range(12):
+            zs = [scale * q[0, i, h] @ k[0, j, 0] for j in range(max(0, i - 1), i + 1)]
+            vs = [v[0, j, 0] for j in range(max(0, i - 1), i + 1)]
+            den = math.exp(s[h]) + sum(math.exp(z) for z in zs)
+            o = sum(math.exp(z) * vv for z, vv in zip(zs, vs)) / den
+            assert np.abs(out[0, i, h] - o).max() < 1e-12
+            assert abs(lse[0, h, i] - math.log(den)) < 1e-12
+
+
+def test_dominant_sink_drives_output_to_zero():
+    t = _inp(1, 40, 40, 4, 2, 16, seed=6, sink_fill=50.0)
+    scale = 0.25
+    out, lse = oracle.fwd(t["q"], t["k"], t["v"], t["sinks"], 0, scale)
+    z = scale * torch.einsum("bihd,bjhd->bhij", t["q"], t["k"].repeat_interleave(2, dim=2))
+    bound = math.exp(float(z.max()) - 50.0) * float(t["v"].abs().max()) * 40
+    assert np.abs(out).max() <= bound
+    assert np.abs(out).max() < 1e-12
+    assert np.abs(lse - 50.0).max() < 1e-12
+
+
+@pytest.mark.parametrize("window", [0, 7])
+def test_row_mass_plus_sink_mass_is_one(window):
+    t = _inp(2, 31, 31, 8, 2, 16, seed=7)
+    scale = 0.25
+    _, lse = oracle.fwd(t["q"], t["k"], t["v"], t["sinks"], window, scale)
+    z = scale * torch.einsum("bihd,bjhd->bhij", t["q"], t["k"].repeat_interleave(4, dim=2))
+    vis = _mask_bool(31, 31, window)
+    lse_t = torch.from_numpy(lse)
+    mass = (torch.exp(z - lse_t[..., None]) * vis).sum(-1) + torch.exp(t["sinks"].view(1, 8, 1) - lse_t)
+    assert (mass - 1.0).abs().max() < 1e-12
+
+
+def test_common_logit_shift_invariance():
+    """Appending a coordinate c/scale to every q and 1 to every k adds c to all
+    z_ij; adding c to the sink too must leave O unchanged and shift LSE by c."""
+    t = _inp(1, 20, 20, 4, 2, 8, seed=8)
+    scale, c = 0.5, 3.7
+    o0, l0 = oracle.fwd(t["q"], t["k"], t["v"], t["sinks"], 0, scale)
+    q1 = torch.cat([t["q"], torch.full((1, 20, 4, 1), c / scale, dtype=torch.float64)], -1)
+    k1 = torch.cat([t["k"], torch.ones(1, 20, 2, 1, dtype=torch.float64)], -1)
+    v1 = torch.cat([t["v"], torch.zeros(1, 20, 2, 1, dtype=torch.float64)], -1)
+    o1, l1 = oracle.fwd(q1, k1, v1, t["sinks"] + c, 0, scale)
+    assert np.abs(o1[..., :8] - o0).max() < 1e-12
+    assert np.abs(l1 - (l0 + c)).max() < 1e-12
+
+
+def _brute(q, k, v, sinks, scale, window):
+    """Separate pure-Python path: full score matrix with -inf masks, sink column appended, explicit softmax."""
+    B, Lq, Hq, D = q.shape
+    Lk, Hkv = k.shape[1], k.shape[2]
+    out = np.zeros((B, Lq, Hq, D))
+    lse = np.zeros((B, Hq, Lq))
+    for b in range(B):
+        for h in range(Hq):
+            g = h // (Hq // Hkv)
+            for i in range(Lq):
+                row = []
+                for j in range(Lk):
+                    p = i + Lk - Lq
+                    ok = (j <= p) and (window <= 0 or p - j < window)
+                    row.append(scale * float(np.dot(q[b, i, h], k[b, j, g])) if ok else -math.inf)
+                row.append(float(sinks[h]))
+                mx = max(row)
+                ex = [math.exp(x - mx) if x != -math.inf else 0.0 for x in row]
+                s = sum(ex)
+                for j in range(Lk):
+                    out[b, i, h] += ex[j] / s * v[b, j, g]
+                lse[b, h, i] = mx + math.log(s)
+    return out, lse
+
+
+@pytest.mark.parametrize("window", [0, 1, 3])
+@pytest.mark.parametrize("Lq,Lk", [(8, 8), (5, 8), (8, 5)])
+def test_brute_force_tiny(window, Lq, Lk):
+    t = _inp(2, Lq, Lk, 4, 2, 4, seed=9 + Lq + Lk)
+    q, k, v, s = (t[x].numpy() for x in ("q", "k", "v", "sinks"))
+    bo, bl = _brute(q, k, v, s, 0.6, window)
+    out, lse = oracle.fwd(t["q"], t["k"], t["v"], t["sinks"], window, 0.6)
+    assert np.abs(out - bo).max() < 1e-12
+    assert np.abs(lse - bl).max() < 1e-12
+
+
+def test_rows_without_visible_keys():
+    """Lq > Lk: the first Lq - Lk rows see no key; O = 0 and LSE = sink, or
+    LSE = -inf when the sink is -inf (no NaN anywhere)."""
+    t = _inp(1, 10, 4, 2, 1, 4, seed=10)
+    out, lse = oracle.fwd(t["q"], t["k"], t["v"], t["sinks"], 0, 0.5)
+    assert np.all(out[0, :6] == 0.0)
+    assert np.allclose(lse[0, :, :6], t["sinks"].numpy()[:, None], atol=0, rtol=0)
+    t2 = _inp(1, 10, 4, 2, 1, 4, seed=10, sink_fill=float("-inf"), with_dout=True)
+    out2, lse2 = oracle.fwd(t2["q"], t2["k"], t2["v"], t2["sinks"], 0, 0.5)
+    assert np.all(out2[0, :6] == 0.0) and np.all(np.isneginf(lse2[0, :, :6]))
+    assert not np.isnan(out2).any()
+    dq, dk, dv, ds = oracle.bwd(t2["q"], t2["k"], t2["v"], t2["sinks"], t2["dout"], 0, 0.5)
+    for a in (dq, dk, dv, ds):
+        assert not np.isnan(a).any()
+    assert np.all(dq[0, :6] == 0.0) and np.all(ds == 0.0)
+
+
+def test_fwd_rows_matches_full():
+    t = _inp(2, 40, 40, 8, 2, 16, seed=11)
+    out, lse = oracle.fwd(t["q"], t["k"], t["v"], t["sinks"], 9, 0.3)
+    rb = np.array([0, 1, 1, 0]); rh = np.array([0, 7, 3, 5]); ri = np.array([0, 39, 17, 8])
+    o, l = oracle.fwd_rows(t["q"], t["k"], t["v"], t["sinks"], rb, rh, ri, 9, 0.3)
+    for n in range(4):
+        assert np.array_equal(o[n], out[rb[n], ri[n], rh[n]])
+        assert l[n] == lse[rb[n], rh[n], ri[n]]
+
+
+@pytest.mark.parametrize("window", [0, 6])
+def test_decode_is_last_prefill_row_and_sdpa(window):
+    d = decode_inputs(3, 40, 8, 2, 16, 1, 40, dtype=torch.float64, qkv_std=1.0, seed=12)
+    d["sinks"] = d["sinks"].double()
+    lens = d["seqlens"].tolist()
+    scale = 0.25
+    out, lse = oracle.decode(d["q"], d["k_cache"], d["v_cache"], d["seqlens"], d["sinks"], window, scale)
+    for b, L in enumerate(lens):
+        qb = d["q"][b].view(1, 1, 8, 16)
+        kb = d["k_cache"][b:b + 1, :L]
+        vb = d["v_cache"][b:b + 1, :L]
+        ro, rl = oracle.fwd(qb, kb, vb, d["sinks"], window, scale)
+        assert np.abs(out[b] - ro[0, 0]).max() < 1e-13
+        assert np.abs(lse[b] - rl[0, :, 0]).max() < 1e-13
+        so, sl = _sdpa_aug(qb, kb, vb, d["sinks"], scale, window)
+        assert np.abs(out[b] - so[0, 0].numpy()).max() < TOL
+        assert np.abs(lse[b] - sl[0, :, 0].numpy()).max() < 1e-10
+
+
+@pytest.mark.parametrize("window", [0, 5])
+@pytest.mark.parametrize("Lq,Lk", [(24, 24), (13, 21)])
+def test_backward_matches_autograd_of_augmented_sdpa(window, Lq, Lk):
+    t = _inp(2, Lq, Lk, 8, 2, 8, seed=13, with_dout=True)
+    scale = 0.35
+    dq, dk, dv, ds = oracle.bwd(t["q"], t["k"], t["v"], t["sinks"], t["dout"], window, scale)
+    q = t["q"].clone().requires_grad_(True)
+    k = t["k"].clone().requires_grad_(True)
+    v = t["v"].clone().requires_grad_(True)
+    s = t["sinks"].clone().requires_grad_(True)
+    o, _ = _sdpa_aug(q, k, v, s, scale, window)
+    (o * t["dout"]).sum().backward()
+    assert np.abs(dq - q.grad.numpy()).max() < 1e-10
+    assert np.abs(dk - k.grad.numpy()).max() < 1e-10
+    assert np.abs(dv - v.grad.numpy()).max() < 1e-10
+    assert np.abs(ds - s.grad.numpy()).max() < 1e-10
+
+
+def test_backward_finite_differences():
+    """Central differences of L = sum(dO * O(x)) through the oracle forward, h = 1e-6."""
+    t = _inp(1, 32, 32, 4, 2, 8, seed=14, with_dout=True)
+    scale, window, h = 0.3, 9, 1e-6
+    dq, dk, dv, ds = oracle.bwd(t["q"], t["k"], t["v"], t["sinks"], t["dout"], window, scale)
+    dO = t["dout"].numpy()
+
+    def loss(q, k, v, s):
+        o, _ = oracle.fwd(q, k, v, s, window, scale)
+        return float((o * dO).sum())
+
+    base = {x: t[x].numpy().copy() for x in ("q", "k", "v", "sinks")}
+    rng = np.random.default_rng(0)
+
+    def fd(name, idx):
+        a = {x: base[x].copy() for x in base}
+        a[name][idx] += h
+        lp = loss(a["q"], a["k"], a["v"], a["sinks"])
+        a[name][idx] -= 2 * h
+        lm = loss(a["q"], a["k"], a["v"], a["sinks"])
+        return (lp - lm) / (2 * h)
+
+    for hh in range(4):
+        assert abs(fd("sinks", (hh,)) - ds[hh]) <= 1e-7 * max(1.0, abs(ds[hh]))
+    for name, grad in (("q", dq), ("k", dk), ("v", dv)):
+        for _ in range(6):
+            idx = tuple(int(rng.integers(0, n)) for n in base[name].shape)
+            assert abs(fd(name, idx) - grad[idx]) <= 1e-7 * max(1.0, abs(grad[idx]))
+
+
+def test_row_stats_reduce_to_dsink():
+    t = _inp(2, 20, 20, 4, 2, 8, seed=15, with_dout=True)
+    _, _, _, ds = oracle.bwd(t["q"], t["k"], t["v"], t["sinks"], t["dout"], 6, 0.4)
+    Dr, Ps = oracle.row_stats(t["q"], t["k"], t["v"], t["sinks"], t["dout"], 6, 0.4)
+    assert np.abs(-(Ps * Dr).sum(axis=(0, 2)) - ds).max() < 1e-12

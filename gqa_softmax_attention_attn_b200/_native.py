@@ -1,0 +1,166 @@
+"""ctypes binding of libattn_sink.so -- argument marshalling only.
+
+Every function here has the name of the C entry point it calls
+(include/attn_sink.h) and does nothing but check tensor shapes/devices,
+take data pointers and raise on a non-zero status.  All arithmetic runs in the
+library's CUDA kernels; there is no CPU or library fallback.  If the shared
+library is missing the first call raises ``AttnSinkLibraryMissing``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "lib", "libattn_sink.so")
+
+DTYPE_F32 = 0
+DTYPE_BF16 = 1
+
+_lock = threading.Lock()
+_lib = None
+
+
+class AttnSinkLibraryMissing(RuntimeError):
+    pass
+
+
+class AttnSinkError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: status {status} ({strerror(status)})")
+
+
+def load():
+    """Loads the in-tree libattn_sink.so (built by gqa_softmax_attention_attn_b200.build)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(LIB_PATH):
+            raise AttnSinkLibraryMissing(
+                f"{LIB_PATH} not found: build it with `python -m gqa_softmax_attention_attn_b200.build` "
+                "(there is no fallback implementation)")
+        lib = ctypes.CDLL(LIB_PATH)
+        P, I, F, Z, LL = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.c_longlong
+        lib.attn_sink_fwd.argtypes = [P] * 6 + [I] * 7 + [F, I, P]
+        lib.attn_sink_fwd.restype = I
+        lib.attn_sink_decode.argtypes = [P] * 7 + [I] * 6 + [F, I, P, Z, I, P]
+        lib.attn_sink_decode.restype = I
+        lib.attn_sink_decode_workspace_size.argtypes = [I] * 6
+        lib.attn_sink_decode_workspace_size.restype = Z
+        lib.attn_sink_bwd.argtypes = [P] * 11 + [I] * 7 + [F, P, Z, I, P]
+        lib.attn_sink_bwd.restype = I
+        lib.attn_sink_bwd_workspace_size.argtypes = [I] * 7
+        lib.attn_sink_bwd_workspace_size.restype = Z
+        lib.attn_sink_get_device_status.argtypes = [P]
+        lib.attn_sink_get_device_status.restype = I
+        lib.attn_sink_set_wait_timeout_ns.argtypes = [LL]
+        lib.attn_sink_set_wait_timeout_ns.restype = LL
+        lib.attn_sink_strerror.argtypes = [I]
+        lib.attn_sink_strerror.restype = ctypes.c_char_p
+        lib.attn_sink_version.argtypes = []
+        lib.attn_sink_version.restype = I
+        _lib = lib
+        return lib
+
+
+def strerror(status: int) -> str:
+    return load().attn_sink_strerror(int(status)).decode()
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return DTYPE_F32
+    if t.dtype == torch.bfloat16:
+        return DTYPE_BF16
+    raise TypeError(f"unsupported dtype {t.dtype} (float32 or bfloat16)")
+
+
+def _dev(t: torch.Tensor, name: str, dtype=None) -> int:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _check(rc: int, where: str):
+    if rc != 0:
+        raise AttnSinkError(rc, where)
+
+
+def attn_sink_fwd(q, k, v, sinks, out, lse, window: int, scale: float, stream=None):
+    """q [B,Lq,Hq,D], k/v [B,Lk,Hkv,D], sinks [Hq] fp32 -> writes out [B,Lq,Hq,D], lse [B,Hq,Lq] fp32."""
+    B, Lq, Hq, D = q.shape
+    Lk, Hkv = k.shape[1], k.shape[2]
+    dt = q.dtype
+    rc = load().attn_sink_fwd(_dev(q, "q"), _dev(k, "k", dt), _dev(v, "v", dt), _dev(sinks, "sinks", torch.float32),
+                              _dev(out, "out", dt), _dev(lse, "lse", torch.float32), B, Lq, Lk, Hq, Hkv, D,
+                              int(window), float(scale), _dtype_code(q), _stream(stream))
+    _check(rc, "attn_sink_fwd")
+
+
+def attn_sink_decode_workspace_size(B: int, Hq: int, D: int, Lmax: int, window: int, num_splits: int) -> int:
+    return int(load().attn_sink_decode_workspace_size(B, Hq, D, Lmax, int(window), int(num_splits)))
+
+
+def attn_sink_decode(q, k_cache, v_cache, seqlens, sinks, out, lse, window: int, scale: float,
+                     num_splits: int = 0, workspace=None, stream=None):
+    """q [B,Hq,D], caches [B,Lmax,Hkv,D], seqlens [B] int32 -> writes out [B,Hq,D], lse [B,Hq]."""
+    B, Hq, D = q.shape
+    Lmax, Hkv = k_cache.shape[1], k_cache.shape[2]
+    dt = q.dtype
+    ws_ptr, ws_bytes = 0, 0
+    if workspace is not None:
+        ws_ptr = _dev(workspace, "workspace")
+        ws_bytes = workspace.numel() * workspace.element_size()
+    rc = load().attn_sink_decode(_dev(q, "q"), _dev(k_cache, "k_cache", dt), _dev(v_cache, "v_cache", dt),
+                                 _dev(seqlens, "seqlens", torch.int32), _dev(sinks, "sinks", torch.float32),
+                                 _dev(out, "out", dt), _dev(lse, "lse", torch.float32), B, Lmax, Hq, Hkv, D,
+                                 int(window), float(scale), int(num_splits), ws_ptr, ws_bytes, _dtype_code(q),
+                                 _stream(stream))
+    _check(rc, "attn_sink_decode")
+
+
+def attn_sink_bwd_workspace_size(B: int, Lq: int, Lk: int, Hq: int, Hkv: int, D: int, dtype: int) -> int:
+    return int(load().attn_sink_bwd_workspace_size(B, Lq, Lk, Hq, Hkv, D, dtype))
+
+
+def attn_sink_bwd(q, k, v, sinks, out, dout, lse, dq, dk, dv, dsinks, window: int, scale: float,
+                  workspace, stream=None):
+    B, Lq, Hq, D = q.shape
+    Lk, Hkv = k.shape[1], k.shape[2]
+    dt = q.dtype
+    rc = load().attn_sink_bwd(_dev(q, "q"), _dev(k, "k", dt), _dev(v, "v", dt), _dev(sinks, "sinks", torch.float32),
+                              _dev(out, "out", dt), _dev(dout, "dout", dt), _dev(lse, "lse", torch.float32),
+                              _dev(dq, "dq", dt), _dev(dk, "dk", dt), _dev(dv, "dv", dt),
+                              _dev(dsinks, "dsinks", torch.float32), B, Lq, Lk, Hq, Hkv, D, int(window),
+                              float(scale), _dev(workspace, "workspace"),
+                              workspace.numel() * workspace.element_size(), _dtype_code(q), _stream(stream))
+    _check(rc, "attn_sink_bwd")
+
+
+def attn_sink_get_device_status(stream=None) -> int:
+    return int(load().attn_sink_get_device_status(_stream(stream)))
+
+
+def attn_sink_set_wait_timeout_ns(ns: int) -> int:
+    return int(load().attn_sink_set_wait_timeout_ns(int(ns)))
+
+
+def attn_sink_version() -> int:
+    return int(load().attn_sink_version())

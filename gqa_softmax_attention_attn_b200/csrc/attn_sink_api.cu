@@ -1,0 +1,336 @@
+// attn_sink_api.cu -- the C ABI declared in include/attn_sink.h: argument
+// checks, the one-time per-device set-up, and kernel dispatch.  The library
+// allocates no device or host memory on any call path.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/attn_sink.h"
+#include "kernels.h"
+
+namespace attn_sink {
+
+__device__ unsigned g_device_status = 0;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr long long kDefaultTimeoutNs = 2000000000LL;
+
+std::atomic<long long> g_timeout_ns{kDefaultTimeoutNs};
+
+struct DeviceState {
+    std::once_flag once;
+    int status = ATTN_SINK_ERR_CUDA;  // result of the set-up
+    unsigned *status_ptr = nullptr;
+};
+DeviceState g_dev[kMaxDevices];
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                   CUtensorMapFloatOOBfill);
+std::once_flag g_encode_once;
+EncodeTiledFn g_encode = nullptr;
+
+int current_device(int *dev)
+{
+    int n = 0;
+    if (cudaGetDeviceCount(&n) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        return ATTN_SINK_ERR_NO_DEVICE;
+    }
+    if (cudaGetDevice(dev) != cudaSuccess || *dev < 0 || *dev >= kMaxDevices) {
+        cudaGetLastError();
+        return ATTN_SINK_ERR_CUDA;
+    }
+    return ATTN_SINK_OK;
+}
+
+// One-time per-device set-up, run with that device current: the device must
+// be an sm_100 part (the clean counterpart of a backend that only runs on one
+// architecture), and the status word's device address is looked up.
+int ensure_device()
+{
+    int dev = 0;
+    int rc = current_device(&dev);
+    if (rc != ATTN_SINK_OK) return rc;
+    DeviceState &d = g_dev[dev];
+    std::call_once(d.once, [&d, dev]() {
+        cudaDeviceProp prop;
+        if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) {
+            cudaGetLastError();
+            d.status = ATTN_SINK_ERR_CUDA;
+            return;
+        }
+        if (prop.major != 10 || prop.minor != 0) {
+            d.status = ATTN_SINK_ERR_ARCH;
+            return;
+        }
+        void *ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_device_status) != cudaSuccess) {
+            cudaGetLastError();
+            d.status = ATTN_SINK_ERR_CUDA;
+            return;
+        }
+        d.status_ptr = static_cast<unsigned *>(ptr);
+        d.status = ATTN_SINK_OK;
+    });
+    return d.status;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_common(int B, int Lq, int Lk, int Hq, int Hkv, int D, int dtype)
+{
+    if (B <= 0 || Lq <= 0 || Lk <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0) return ATTN_SINK_ERR_INVALID_ARG;
+    if (Hq % Hkv != 0) return ATTN_SINK_ERR_INVALID_ARG;
+    if (D != 64) return ATTN_SINK_ERR_UNSUPPORTED;
+    if (dtype != ATTN_SINK_DTYPE_F32 && dtype != ATTN_SINK_DTYPE_BF16) return ATTN_SINK_ERR_UNSUPPORTED;
+    if (B > 65535 || Hq > 65535) return ATTN_SINK_ERR_UNSUPPORTED;
+    return ATTN_SINK_OK;
+}
+
+int launch_status(cudaError_t e)
+{
+    if (e == cudaSuccess) return ATTN_SINK_OK;
+    cudaGetLastError();
+    return ATTN_SINK_ERR_CUDA;
+}
+
+int auto_splits(int Lmax, int window)
+{
+    const int lvis = window > 0 ? (window < Lmax ? window : Lmax) : Lmax;
+    int s = (lvis + 2047) / 2048;
+    if (s < 1) s = 1;
+    if (s > 32) s = 32;
+    return s;
+}
+
+DecodeShape decode_shape(int B, int Lmax, int Hq, int Hkv, int D, int window, float scale, int num_splits)
+{
+    DecodeShape s;
+    s.B = B;
+    s.Lmax = Lmax;
+    s.Hq = Hq;
+    s.Hkv = Hkv;
+    s.D = D;
+    s.window = window;
+    s.scale = scale;
+    const int lvis = window > 0 ? (window < Lmax ? window : Lmax) : Lmax;
+    s.splits = num_splits > 0 ? num_splits : auto_splits(Lmax, window);
+    int chunk = (lvis + s.splits - 1) / s.splits;
+    chunk = (chunk + 63) / 64 * 64;
+    s.chunk = chunk;
+    // splits that can actually be used by the longest visible range
+    s.splits = (lvis + chunk - 1) / chunk;
+    return s;
+}
+
+size_t decode_ws_bytes(const DecodeShape &s)
+{
+    if (s.splits <= 1) return 0;
+    return (size_t)s.B * s.Hq * s.splits * (s.D + 2) * sizeof(float);
+}
+
+}  // namespace
+
+unsigned *device_status_ptr()
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    return g_dev[dev].status_ptr;
+}
+
+long long wait_timeout_ns() { return g_timeout_ns.load(); }
+
+bool encode_tensor_map_4d(void *map, void *gaddr, int elem_bytes, const uint64_t dims[4],
+                          const uint64_t strides_bytes[3], const uint32_t box[4], bool swizzle128)
+{
+    std::call_once(g_encode_once, []() {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+        else
+            cudaGetLastError();
+    });
+    if (!g_encode || elem_bytes != 2) return false;
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    const CUresult r = g_encode(static_cast<CUtensorMap *>(map), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, gaddr,
+                                reinterpret_cast<const cuuint64_t *>(dims),
+                                reinterpret_cast<const cuuint64_t *>(strides_bytes),
+                                reinterpret_cast<const cuuint32_t *>(box), estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+}  // namespace attn_sink
+
+using namespace attn_sink;
+
+extern "C" {
+
+int attn_sink_version(void) { return 100; }
+
+const char *attn_sink_strerror(int status)
+{
+    switch (status) {
+    case ATTN_SINK_OK: return "ok";
+    case ATTN_SINK_ERR_INVALID_ARG: return "invalid argument";
+    case ATTN_SINK_ERR_UNSUPPORTED: return "unsupported configuration (head dim must be 64; dtype f32 or bf16)";
+    case ATTN_SINK_ERR_MISALIGNED: return "tensor pointer not 16-byte aligned";
+    case ATTN_SINK_ERR_ARCH: return "device is not sm_100 (B200); this library only runs on sm_100a";
+    case ATTN_SINK_ERR_WORKSPACE: return "workspace missing or too small";
+    case ATTN_SINK_ERR_CUDA: return "CUDA call or kernel launch failed";
+    case ATTN_SINK_ERR_TIMEOUT: return "a bounded device-side wait expired";
+    case ATTN_SINK_ERR_NO_DEVICE: return "no CUDA device visible";
+    default: return "unknown status";
+    }
+}
+
+long long attn_sink_set_wait_timeout_ns(long long ns)
+{
+    return g_timeout_ns.exchange(ns > 0 ? ns : kDefaultTimeoutNs);
+}
+
+int attn_sink_fwd(const void *q, const void *k, const void *v, const float *sinks, void *out, float *lse, int B,
+                  int Lq, int Lk, int Hq, int Hkv, int D, int window, float scale, int dtype, void *stream)
+{
+    if (!q || !k || !v || !sinks || !out || !lse) return ATTN_SINK_ERR_INVALID_ARG;
+    int rc = check_common(B, Lq, Lk, Hq, Hkv, D, dtype);
+    if (rc != ATTN_SINK_OK) return rc;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse) ||
+        !aligned16(sinks))
+        return ATTN_SINK_ERR_MISALIGNED;
+    rc = ensure_device();
+    if (rc != ATTN_SINK_OK) return rc;
+    AttnShape s{B, Lq, Lk, Hq, Hkv, D, window, scale};
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (dtype == ATTN_SINK_DTYPE_F32)
+        return launch_status(launch_fwd_simt<float>(static_cast<const float *>(q), static_cast<const float *>(k),
+                                                    static_cast<const float *>(v), sinks,
+                                                    static_cast<float *>(out), lse, s, st));
+    if (!fwd_tc_supported(s)) return ATTN_SINK_ERR_UNSUPPORTED;
+    return launch_status(launch_fwd_tc(q, k, v, sinks, out, lse, s, st));
+}
+
+size_t attn_sink_decode_workspace_size(int B, int Hq, int D, int Lmax, int window, int num_splits)
+{
+    if (B <= 0 || Hq <= 0 || D <= 0 || Lmax <= 0 || num_splits < 0 || num_splits > 32) return 0;
+    return decode_ws_bytes(decode_shape(B, Lmax, Hq, 1, D, window, 1.f, num_splits));
+}
+
+int attn_sink_decode(const void *q, const void *k_cache, const void *v_cache, const int *seqlens,
+                     const float *sinks, void *out, float *lse, int B, int Lmax, int Hq, int Hkv, int D,
+                     int window, float scale, int num_splits, void *workspace, size_t ws_bytes, int dtype,
+                     void *stream)
+{
+    if (!q || !k_cache || !v_cache || !seqlens || !sinks || !out || !lse) return ATTN_SINK_ERR_INVALID_ARG;
+    if (num_splits < 0 || num_splits > 32) return ATTN_SINK_ERR_INVALID_ARG;
+    int rc = check_common(B, 1, Lmax, Hq, Hkv, D, dtype);
+    if (rc != ATTN_SINK_OK) return rc;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) || !aligned16(lse) ||
+        !aligned16(sinks) || !aligned16(seqlens))
+        return ATTN_SINK_ERR_MISALIGNED;
+    const DecodeShape s = decode_shape(B, Lmax, Hq, Hkv, D, window, scale, num_splits);
+    const size_t need = decode_ws_bytes(s);
+    if (need > 0 && (!workspace || ws_bytes < need)) return ATTN_SINK_ERR_WORKSPACE;
+    if (need > 0 && !aligned16(workspace)) return ATTN_SINK_ERR_MISALIGNED;
+    rc = ensure_device();
+    if (rc != ATTN_SINK_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    float *ws_o = static_cast<float *>(workspace);
+    float *ws_ml = need > 0 ? ws_o + (size_t)s.B * s.Hq * s.splits * s.D : nullptr;
+    cudaError_t e;
+    if (dtype == ATTN_SINK_DTYPE_F32) {
+        e = launch_decode_simt<float>(static_cast<const float *>(q), static_cast<const float *>(k_cache),
+                                      static_cast<const float *>(v_cache), seqlens, sinks,
+                                      static_cast<float *>(out), lse, s, ws_o, ws_ml, st);
+        if (e == cudaSuccess && s.splits > 1)
+            e = launch_decode_combine<float>(seqlens, sinks, static_cast<float *>(out), lse, s, ws_o, ws_ml, st);
+    } else {
+        if (decode_bf16_supported(s))
+            e = launch_decode_bf16(q, k_cache, v_cache, seqlens, sinks, out, lse, s, ws_o, ws_ml, st);
+        else
+            e = launch_decode_simt<__nv_bfloat16>(static_cast<const __nv_bfloat16 *>(q),
+                                                  static_cast<const __nv_bfloat16 *>(k_cache),
+                                                  static_cast<const __nv_bfloat16 *>(v_cache), seqlens, sinks,
+                                                  static_cast<__nv_bfloat16 *>(out), lse, s, ws_o, ws_ml, st);
+        if (e == cudaSuccess && s.splits > 1)
+            e = launch_decode_combine<__nv_bfloat16>(seqlens, sinks, static_cast<__nv_bfloat16 *>(out), lse, s,
+                                                     ws_o, ws_ml, st);
+    }
+    return launch_status(e);
+}
+
+size_t attn_sink_bwd_workspace_size(int B, int Lq, int Lk, int Hq, int Hkv, int D, int dtype)
+{
+    if (check_common(B, Lq, Lk, Hq, Hkv, D, dtype) != ATTN_SINK_OK) return 0;
+    AttnShape s{B, Lq, Lk, Hq, Hkv, D, 0, 1.f};
+    return bwd_simt_workspace_bytes(s);
+}
+
+int attn_sink_bwd(const void *q, const void *k, const void *v, const float *sinks, const void *out,
+                  const void *dout, const float *lse, void *dq, void *dk, void *dv, float *dsinks, int B, int Lq,
+                  int Lk, int Hq, int Hkv, int D, int window, float scale, void *workspace, size_t ws_bytes,
+                  int dtype, void *stream)
+{
+    if (!q || !k || !v || !sinks || !out || !dout || !lse || !dq || !dk || !dv || !dsinks)
+        return ATTN_SINK_ERR_INVALID_ARG;
+    int rc = check_common(B, Lq, Lk, Hq, Hkv, D, dtype);
+    if (rc != ATTN_SINK_OK) return rc;
+    const void *ptrs[] = {q, k, v, sinks, out, dout, lse, dq, dk, dv, dsinks};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return ATTN_SINK_ERR_MISALIGNED;
+    AttnShape s{B, Lq, Lk, Hq, Hkv, D, window, scale};
+    const size_t need = bwd_simt_workspace_bytes(s);
+    if (!workspace || ws_bytes < need) return ATTN_SINK_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return ATTN_SINK_ERR_MISALIGNED;
+    rc = ensure_device();
+    if (rc != ATTN_SINK_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (dtype == ATTN_SINK_DTYPE_F32)
+        return launch_status(launch_bwd_simt<float>(
+            static_cast<const float *>(q), static_cast<const float *>(k), static_cast<const float *>(v), sinks,
+            static_cast<const float *>(out), static_cast<const float *>(dout), lse, static_cast<float *>(dq),
+            static_cast<float *>(dk), static_cast<float *>(dv), dsinks, s, workspace, st));
+    using bf = __nv_bfloat16;
+    return launch_status(launch_bwd_simt<bf>(
+        static_cast<const bf *>(q), static_cast<const bf *>(k), static_cast<const bf *>(v), sinks,
+        static_cast<const bf *>(out), static_cast<const bf *>(dout), lse, static_cast<bf *>(dq),
+        static_cast<bf *>(dk), static_cast<bf *>(dv), dsinks, s, workspace, st));
+}
+
+int attn_sink_get_device_status(void *stream)
+{
+    int dev = 0;
+    int rc = current_device(&dev);
+    if (rc != ATTN_SINK_OK) return rc;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_SINK_ERR_CUDA;
+    }
+    unsigned v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(v)) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_SINK_ERR_CUDA;
+    }
+    if (v != 0) {
+        const unsigned zero = 0;
+        if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(zero)) != cudaSuccess) {
+            cudaGetLastError();
+            return ATTN_SINK_ERR_CUDA;
+        }
+    }
+    return (v & STATUS_TIMEOUT) ? ATTN_SINK_ERR_TIMEOUT : ATTN_SINK_OK;
+}
+
+}  // extern "C"

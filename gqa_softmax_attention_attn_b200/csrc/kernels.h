@@ -1,0 +1,63 @@
+// kernels.h -- internal launch interface between the C ABI (attn_sink_api.cu)
+// and the kernel translation units.  Not part of the public ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace attn_sink {
+
+// Device status word bits (read back by attn_sink_get_device_status).
+enum : unsigned { STATUS_TIMEOUT = 1u };
+
+struct AttnShape {
+    int B, Lq, Lk, Hq, Hkv, D, window;
+    float scale;
+};
+
+struct DecodeShape {
+    int B, Lmax, Hq, Hkv, D, window;
+    float scale;
+    int splits;  // maximum number of chunks per sequence
+    int chunk;   // keys per chunk (multiple of 64)
+};
+
+// Per-device status word (bit STATUS_TIMEOUT set by an expired bounded wait).
+unsigned *device_status_ptr();
+long long wait_timeout_ns();
+
+// Exact CUDA-core path (T = float or __nv_bfloat16).
+template <typename T>
+cudaError_t launch_fwd_simt(const T *q, const T *k, const T *v, const float *sinks, T *out, float *lse,
+                            const AttnShape &s, cudaStream_t st);
+template <typename T>
+cudaError_t launch_bwd_simt(const T *q, const T *k, const T *v, const float *sinks, const T *out,
+                            const T *dout, const float *lse, T *dq, T *dk, T *dv, float *dsinks,
+                            const AttnShape &s, void *ws, cudaStream_t st);
+size_t bwd_simt_workspace_bytes(const AttnShape &s);
+
+template <typename T>
+cudaError_t launch_decode_simt(const T *q, const T *kc, const T *vc, const int *seqlens, const float *sinks,
+                               T *out, float *lse, const DecodeShape &s, float *ws_o, float *ws_ml,
+                               cudaStream_t st);
+template <typename T>
+cudaError_t launch_decode_combine(const int *seqlens, const float *sinks, T *out, float *lse,
+                                  const DecodeShape &s, const float *ws_o, const float *ws_ml, cudaStream_t st);
+
+// Tensor-core (tcgen05 / TMEM / TMA) bf16 prefill forward.
+cudaError_t launch_fwd_tc(const void *q, const void *k, const void *v, const float *sinks, void *out,
+                          float *lse, const AttnShape &s, cudaStream_t st);
+bool fwd_tc_supported(const AttnShape &s);
+
+// bf16 split-KV decode: TMA-staged K/V, tensor-core (mma.sync) group scores.
+cudaError_t launch_decode_bf16(const void *q, const void *kc, const void *vc, const int *seqlens,
+                               const float *sinks, void *out, float *lse, const DecodeShape &s, float *ws_o,
+                               float *ws_ml, cudaStream_t st);
+bool decode_bf16_supported(const DecodeShape &s);
+
+// Driver entry point for cuTensorMapEncodeTiled (resolved once through the runtime).
+bool encode_tensor_map_4d(void *map, void *gaddr, int elem_bytes, const uint64_t dims[4],
+                          const uint64_t strides_bytes[3], const uint32_t box[4], bool swizzle128);
+
+}  // namespace attn_sink

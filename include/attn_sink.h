@@ -1,0 +1,176 @@
+/*
+ * attn_sink.h -- C ABI of libattn_sink.so: grouped-query attention whose
+ * softmax carries a learned per-head sink logit, on NVIDIA B200 (sm_100a).
+ *
+ * The operation ("GPT-OSS on day 0", Perplexity, sections "Attention: GQA
+ * with Attention Sinks" and "Sink Attention"): every query head h owns a
+ * sink logit sink_h that joins the softmax denominator but carries no value
+ * row.  For query row i and the keys j it may see,
+ *
+ *     s_ij  = scale * <q_i, k_j>
+ *     M_i   = max(sink_h, max_j s_ij)
+ *     Z_i   = exp(sink_h - M_i) + sum_j exp(s_ij - M_i)
+ *     out_i = sum_j exp(s_ij - M_i) v_j / Z_i
+ *     lse_i = M_i + ln Z_i                        (the sink term included)
+ *
+ * The sink is a raw logit: it is not multiplied by `scale`.  Query head h
+ * reads KV head h / (Hq / Hkv) (grouped-query attention, "GPT-OSS 20B
+ * Egitimi: Unsloth, A100 ve Hopper Uyumlulugu", section 1).  Layers are
+ * either dense causal (window <= 0) or causal and banded to the last
+ * `window` keys (window = 128 in gpt-oss: "GPT-OSS-120B 4-bit ...",
+ * section 3).  Query row i of Lq sits at absolute position
+ * p_i = i + (Lk - Lq); key j is visible iff j <= p_i and, when window > 0,
+ * j > p_i - window.  A row with no visible key gets out = 0 and
+ * lse = sink_h (lse = -inf, out = 0 when sink_h = -inf as well).
+ *
+ * Conventions shared by every call below.
+ *   Pointers      device memory owned by the caller, except where a
+ *                 parameter says "host".  The library never allocates,
+ *                 frees or retains any of them.  Every tensor pointer must be
+ *                 16-byte aligned.
+ *   dtype         element type of q/k/v/out/dout/dq/dk/dv/caches:
+ *                 ATTN_SINK_DTYPE_F32 (exact fp32 CUDA-core path) or
+ *                 ATTN_SINK_DTYPE_BF16 (tensor-core path, fp32 accumulation).
+ *                 sinks, dsinks and lse are always fp32.
+ *   D             head dimension; only 64 is supported.
+ *   stream        a cudaStream_t (NULL = legacy default stream).  Calls are
+ *                 asynchronous: they enqueue kernels on `stream` and return.
+ *   Return value  ATTN_SINK_OK (0) or a negative attn_sink_status.  On a
+ *                 non-zero return nothing has been enqueued, except for
+ *                 ATTN_SINK_ERR_CUDA, which reports a failed launch.
+ *   Timeouts      every device-side wait is bounded; a wait that expires sets
+ *                 a per-device status word, and the kernel winds down without
+ *                 trapping.  attn_sink_get_device_status() reports it.
+ *   Threads       the library keeps no state between calls apart from a
+ *                 one-time per-device set-up (kernel attributes, the device
+ *                 check), so calls from several host threads are safe.
+ */
+#ifndef ATTN_SINK_H
+#define ATTN_SINK_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define ATTN_SINK_API __attribute__((visibility("default")))
+#else
+#define ATTN_SINK_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum attn_sink_status {
+    ATTN_SINK_OK = 0,
+    ATTN_SINK_ERR_INVALID_ARG = -1,   /* null pointer, non-positive size, Hq % Hkv != 0, ... */
+    ATTN_SINK_ERR_UNSUPPORTED = -2,   /* D != 64, unknown dtype, group size not supported */
+    ATTN_SINK_ERR_MISALIGNED = -3,    /* a tensor pointer is not 16-byte aligned */
+    ATTN_SINK_ERR_ARCH = -4,          /* the current device is not sm_100 (B200) */
+    ATTN_SINK_ERR_WORKSPACE = -5,     /* workspace missing or smaller than required */
+    ATTN_SINK_ERR_CUDA = -6,          /* a CUDA runtime/driver call or launch failed */
+    ATTN_SINK_ERR_TIMEOUT = -7,       /* a bounded device-side wait expired */
+    ATTN_SINK_ERR_NO_DEVICE = -8      /* no CUDA device is visible */
+} attn_sink_status;
+
+enum { ATTN_SINK_DTYPE_F32 = 0, ATTN_SINK_DTYPE_BF16 = 1 };
+
+/*
+ * Prefill forward ("GPT-OSS on day 0", section "Sink Attention": the sink
+ * seeds the running maximum of the online softmax).
+ *   q     [B, Lq, Hq, D]   k, v [B, Lk, Hkv, D]   (dtype)
+ *   sinks [Hq] fp32
+ *   out   [B, Lq, Hq, D]   (dtype, written)
+ *   lse   [B, Hq, Lq] fp32 (written; natural log, sink included)
+ *   window <= 0: dense causal; window > 0: causal band of `window` keys.
+ *   scale: multiplies <q, k> (usually 1/sqrt(D)).
+ * Lq > Lk is allowed (leading rows then see no key).  B*Lq*Hq*D and
+ * B*Lk*Hkv*D must stay below 2^31 elements per tensor for dtype F32.
+ */
+ATTN_SINK_API int attn_sink_fwd(const void *q, const void *k, const void *v, const float *sinks,
+                  void *out, float *lse, int B, int Lq, int Lk, int Hq, int Hkv, int D,
+                  int window, float scale, int dtype, void *stream);
+
+/*
+ * Split-KV decode over a contiguous per-sequence KV cache with ragged
+ * lengths ("GPT-OSS on day 0", section "Sink Attention": attention is split
+ * along the KV length as well as across heads, and the sink must be counted
+ * once, not once per split).
+ *   q        [B, Hq, D]            one query per sequence (dtype)
+ *   k_cache, v_cache [B, Lmax, Hkv, D]  (dtype)
+ *   seqlens  [B] int32, device     cached length of each sequence, in
+ *                                  [1, Lmax]; the query sits at position
+ *                                  seqlens[b] - 1 (its own key is already
+ *                                  in the cache).  Values outside [1, Lmax]
+ *                                  are clamped on the device.
+ *   sinks    [Hq] fp32
+ *   out      [B, Hq, D] (dtype)    lse [B, Hq] fp32
+ *   num_splits  0 = choose automatically, else 1..32: the visible range of
+ *               the longest possible sequence is cut into num_splits chunks
+ *               of equal length (a multiple of 64 keys); sequence b uses as
+ *               many chunks as its own range needs.
+ *   workspace   device scratch of at least
+ *               attn_sink_decode_workspace_size(B, Hq, D, Lmax, window, num_splits)
+ *               bytes (may be NULL when that size is 0).  Its contents on
+ *               entry do not matter.
+ */
+ATTN_SINK_API int attn_sink_decode(const void *q, const void *k_cache, const void *v_cache,
+                     const int *seqlens, const float *sinks, void *out, float *lse,
+                     int B, int Lmax, int Hq, int Hkv, int D, int window, float scale,
+                     int num_splits, void *workspace, size_t ws_bytes, int dtype,
+                     void *stream);
+
+/* Bytes of decode workspace for these sizes (0 when a single split suffices). */
+ATTN_SINK_API size_t attn_sink_decode_workspace_size(int B, int Hq, int D, int Lmax, int window, int num_splits);
+
+/*
+ * Backward of attn_sink_fwd, derived from the definition above (the pages
+ * give no gradient).  With P_ij = exp(s_ij - lse_i), P_sink_i =
+ * exp(sink_h - lse_i) and D_i = <dout_i, out_i>:
+ *   dS_ij  = P_ij (<dout_i, v_j> - D_i)
+ *   dq_i   = scale * sum_j dS_ij k_j
+ *   dk_j   = scale * sum over (query heads of j's group, rows i) dS_ij q_i
+ *   dv_j   = sum over (query heads of j's group, rows i) P_ij dout_i
+ *   dsinks_h = - sum over (b, i) P_sink_i D_i
+ * Inputs: q, k, v, sinks as for attn_sink_fwd; out and lse as written by
+ * attn_sink_fwd for the same arguments; dout [B, Lq, Hq, D] (dtype).
+ * Outputs (overwritten, not accumulated): dq [B, Lq, Hq, D],
+ * dk, dv [B, Lk, Hkv, D] (dtype); dsinks [Hq] fp32, summed over the batch.
+ * The result is deterministic run to run.
+ *   workspace  device scratch of at least
+ *              attn_sink_bwd_workspace_size(B, Lq, Lk, Hq, Hkv, D, dtype)
+ *              bytes; contents on entry do not matter.
+ */
+ATTN_SINK_API int attn_sink_bwd(const void *q, const void *k, const void *v, const float *sinks,
+                  const void *out, const void *dout, const float *lse,
+                  void *dq, void *dk, void *dv, float *dsinks,
+                  int B, int Lq, int Lk, int Hq, int Hkv, int D, int window, float scale,
+                  void *workspace, size_t ws_bytes, int dtype, void *stream);
+
+ATTN_SINK_API size_t attn_sink_bwd_workspace_size(int B, int Lq, int Lk, int Hq, int Hkv, int D, int dtype);
+
+/*
+ * Synchronises `stream`, then reads and clears the current device's status
+ * word.  Returns ATTN_SINK_OK, ATTN_SINK_ERR_TIMEOUT if a bounded device
+ * wait expired since the last call, or ATTN_SINK_ERR_CUDA if the
+ * synchronisation itself failed.
+ */
+ATTN_SINK_API int attn_sink_get_device_status(void *stream);
+
+/*
+ * Upper bound, in nanoseconds, on any single device-side wait in kernels
+ * launched after this call (default 2e9, i.e. 2 s; values <= 0 restore the
+ * default).  Process-wide.  Returns the previous value.
+ */
+ATTN_SINK_API long long attn_sink_set_wait_timeout_ns(long long ns);
+
+/* Static description of a status code. */
+ATTN_SINK_API const char *attn_sink_strerror(int status);
+
+/* Library version as 10000*major + 100*minor + patch. */
+ATTN_SINK_API int attn_sink_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_SINK_H */

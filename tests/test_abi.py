@@ -1,0 +1,101 @@
+"""The C-ABI library loads, exports every symbol its header declares, and
+rejects bad arguments on the host before touching any device (CPU only)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import gqa_softmax_attention_attn_b200 as attn
+from gqa_softmax_attention_attn_b200 import _native
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "attn_sink.h")
+
+OK, INVALID, UNSUPPORTED, MISALIGNED, ARCH, WORKSPACE, CUDA, TIMEOUT, NODEV = 0, -1, -2, -3, -4, -5, -6, -7, -8
+
+
+def declared_symbols():
+    txt = open(HEADER).read()
+    return sorted(set(re.findall(r"ATTN_SINK_API\s+[\w\s\*]+?\b(attn_sink_\w+)\s*\(", txt)))
+
+
+def test_header_declares_the_three_calls():
+    syms = declared_symbols()
+    for s in ("attn_sink_fwd", "attn_sink_decode", "attn_sink_bwd"):
+        assert s in syms
+
+
+def test_library_exports_every_declared_symbol():
+    lib = attn.load()
+    for s in declared_symbols():
+        assert hasattr(lib, s), s
+    out = os.popen(f"nm -D --defined-only {_native.LIB_PATH}").read()
+    exported = set(re.findall(r" T (\w+)", out))
+    assert set(declared_symbols()) <= exported
+    # nothing else leaks out of the library
+    assert all(e.startswith("attn_sink_") for e in exported), exported
+
+
+def test_strerror_and_version():
+    assert attn.attn_sink_version() >= 100
+    for code in (OK, INVALID, UNSUPPORTED, MISALIGNED, ARCH, WORKSPACE, CUDA, TIMEOUT, NODEV):
+        assert len(attn.strerror(code)) > 0
+    assert attn.strerror(-99) == "unknown status"
+
+
+def _fake(n=8):
+    # distinct, 256-byte aligned, non-null addresses; never dereferenced by the host checks
+    return [0x7f0000000000 + 0x1000 * i for i in range(n)]
+
+
+def test_fwd_host_checks():
+    lib = attn.load()
+    q, k, v, s, o, l = _fake(6)
+    assert lib.attn_sink_fwd(None, k, v, s, o, l, 1, 16, 16, 8, 2, 64, 0, 0.125, 1, None) == INVALID
+    assert lib.attn_sink_fwd(q, k, v, s, o, l, 0, 16, 16, 8, 2, 64, 0, 0.125, 1, None) == INVALID
+    assert lib.attn_sink_fwd(q, k, v, s, o, l, 1, 16, 16, 8, 3, 64, 0, 0.125, 1, None) == INVALID
+    assert lib.attn_sink_fwd(q, k, v, s, o, l, 1, 16, 16, 8, 2, 128, 0, 0.125, 1, None) == UNSUPPORTED
+    assert lib.attn_sink_fwd(q, k, v, s, o, l, 1, 16, 16, 8, 2, 64, 0, 0.125, 7, None) == UNSUPPORTED
+    assert lib.attn_sink_fwd(q + 2, k, v, s, o, l, 1, 16, 16, 8, 2, 64, 0, 0.125, 1, None) == MISALIGNED
+
+
+def test_decode_host_checks():
+    lib = attn.load()
+    q, kc, vc, sl, s, o, l, ws = _fake(8)
+    args = [q, kc, vc, sl, s, o, l, 4, 4096, 8, 2, 64, 0, 0.125]
+    assert lib.attn_sink_decode(*args, 33, ws, 1 << 20, 1, None) == INVALID
+    need = attn.attn_sink_decode_workspace_size(4, 8, 64, 4096, 0, 8)
+    assert need == 4 * 8 * 8 * (64 + 2) * 4
+    assert lib.attn_sink_decode(*args, 8, None, 0, 1, None) == WORKSPACE
+    assert lib.attn_sink_decode(*args, 8, ws, need - 4, 1, None) == WORKSPACE
+    # one split needs no workspace
+    assert attn.attn_sink_decode_workspace_size(4, 8, 64, 4096, 128, 0) == 0
+
+
+def test_bwd_host_checks():
+    lib = attn.load()
+    p = _fake(12)
+    need = attn.attn_sink_bwd_workspace_size(2, 32, 32, 8, 2, 64, 1)
+    assert need > 0
+    base = p[:11] + [2, 32, 32, 8, 2, 64, 0, 0.125]
+    assert lib.attn_sink_bwd(*base, None, 0, 1, None) == WORKSPACE
+    assert lib.attn_sink_bwd(*base, p[11], need - 1, 1, None) == WORKSPACE
+    bad = [None] + p[1:11] + [2, 32, 32, 8, 2, 64, 0, 0.125]
+    assert lib.attn_sink_bwd(*bad, p[11], need, 1, None) == INVALID
+
+
+def test_no_device_is_reported_cleanly():
+    import torch
+
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    lib = attn.load()
+    q, k, v, s, o, l = _fake(6)
+    assert lib.attn_sink_fwd(q, k, v, s, o, l, 1, 16, 16, 8, 2, 64, 0, 0.125, 1, None) == NODEV
+    assert lib.attn_sink_get_device_status(None) == NODEV
+
+
+def test_wait_timeout_setting_round_trips():
+    old = attn.attn_sink_set_wait_timeout_ns(123456789)
+    assert attn.attn_sink_set_wait_timeout_ns(old) == 123456789

@@ -1,0 +1,75 @@
+"""GPU parity of attn_sink_bwd (through the C ABI) against the fp64 oracle."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from _harness import assert_close_bf16, assert_close_fp32, errors
+from gqa_softmax_attention_attn_b200 import attn_sink_bwd, attn_sink_bwd_workspace_size, attn_sink_fwd
+from gqa_softmax_attention_attn_b200.inputs import SEEDS, TINY_FP32, TRAIN, WINDOW, prefill_inputs, workload_inputs
+
+pytestmark = pytest.mark.gpu
+
+# dsink: a sum of B*Lq row terms; its bound scales with the largest entry.
+DSINK_REL = 5e-3
+
+
+def run_bwd(t, window, scale):
+    dev = "cuda"
+    q, k, v = t["q"].to(dev), t["k"].to(dev), t["v"].to(dev)
+    s, do = t["sinks"].to(dev), t["dout"].to(dev)
+    B, Lq, Hq, D = q.shape
+    Lk, Hkv = k.shape[1], k.shape[2]
+    out = torch.empty_like(q)
+    lse = torch.empty(B, Hq, Lq, device=dev, dtype=torch.float32)
+    attn_sink_fwd(q, k, v, s, out, lse, window, scale)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ds = torch.empty(Hq, device=dev, dtype=torch.float32)
+    code = 0 if q.dtype == torch.float32 else 1
+    ws = torch.empty(attn_sink_bwd_workspace_size(B, Lq, Lk, Hq, Hkv, D, code), dtype=torch.uint8, device=dev)
+    attn_sink_bwd(q, k, v, s, out, do, lse, dq, dk, dv, ds, window, scale, ws)
+    torch.cuda.synchronize()
+    return dq, dk, dv, ds
+
+
+@pytest.mark.parametrize("window", [0, WINDOW])
+def test_tiny_fp32_bwd_exact(window):
+    w = TINY_FP32
+    t = workload_inputs(w, SEEDS["tiny"], with_dout=True)
+    scale = 1.0 / math.sqrt(w.D)
+    dq, dk, dv, ds = run_bwd(t, window, scale)
+    rq, rk, rv, rs = oracle.bwd(t["q"], t["k"], t["v"], t["sinks"], t["dout"], window, scale)
+    assert_close_fp32(dq, rq, "dq")
+    assert_close_fp32(dk, rk, "dk")
+    assert_close_fp32(dv, rv, "dv")
+    assert_close_fp32(ds, rs, "dsink")
+
+
+def _check_bf16(t, window, scale, what):
+    dq, dk, dv, ds = run_bwd(t, window, scale)
+    rq, rk, rv, rs = oracle.bwd(t["q"], t["k"], t["v"], t["sinks"], t["dout"], window, scale)
+    assert_close_bf16(dq, rq, f"{what} dq")
+    assert_close_bf16(dk, rk, f"{what} dk")
+    assert_close_bf16(dv, rv, f"{what} dv")
+    ma, _ = errors(ds, rs)
+    assert ma <= DSINK_REL * np.abs(rs).max() + 1e-5, f"{what} dsink max_abs={ma:.3e}"
+
+
+@pytest.mark.parametrize("window", [0, 1, 128])
+@pytest.mark.parametrize("shape", [(1, 200, 200, 16, 2), (2, 129, 129, 8, 1), (1, 70, 150, 8, 4), (1, 96, 64, 8, 2)])
+def test_bf16_bwd_small(shape, window):
+    B, Lq, Lk, Hq, Hkv = shape
+    t = prefill_inputs(B, Lq, Lk, Hq, Hkv, 64, torch.bfloat16, 0.5, 1.0, 0.1, seed=31 + window, with_dout=True)
+    _check_bf16(t, window, 0.125, f"{shape} w={window}")
+
+
+@pytest.mark.parametrize("window", [0, WINDOW])
+def test_bf16_bwd_one_train_group(window):
+    """One (b, kv-group) slice of the training shape at full length L = 8192
+    (all 8 query heads of the group): the backward is separable per slice."""
+    w = TRAIN
+    t = prefill_inputs(1, 2048, 2048, 8, 1, 64, torch.bfloat16, w.qkv_std, w.sink_std, w.dout_std,
+                       seed=SEEDS["train"], with_dout=True)
+    _check_bf16(t, window, 1.0 / math.sqrt(64), f"train-slice w={window}")

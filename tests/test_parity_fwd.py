@@ -1,0 +1,139 @@
+"""GPU parity of attn_sink_fwd (through the C ABI) against the fp64 oracle."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from _harness import assert_close_bf16, assert_close_fp32, assert_lse, errors
+from gqa_softmax_attention_attn_b200 import attn_sink_fwd
+from gqa_softmax_attention_attn_b200.inputs import (LONG_BANDED, LONG_DENSE, PREFILL_20B, SEEDS, TINY_FP32, TRAIN,
+                                                    WINDOW, prefill_inputs, sample_rows, workload_inputs)
+
+pytestmark = pytest.mark.gpu
+
+
+def run_fwd(t, window, scale):
+    dev = "cuda"
+    q, k, v = t["q"].to(dev), t["k"].to(dev), t["v"].to(dev)
+    s = t["sinks"].to(dev)
+    B, Lq, Hq, D = q.shape
+    out = torch.empty_like(q)
+    lse = torch.empty(B, Hq, Lq, device=dev, dtype=torch.float32)
+    attn_sink_fwd(q, k, v, s, out, lse, window, scale)
+    torch.cuda.synchronize()
+    return out, lse
+
+
+@pytest.mark.parametrize("window", [0, WINDOW])
+def test_tiny_fp32_exact(window):
+    w = TINY_FP32
+    t = workload_inputs(w, SEEDS["tiny"])
+    scale = 1.0 / math.sqrt(w.D)
+    out, lse = run_fwd(t, window, scale)
+    ro, rl = oracle.fwd(t["q"], t["k"], t["v"], t["sinks"], window, scale)
+    assert_close_fp32(out, ro, "out")
+    assert_close_fp32(lse, rl, "lse")
+
+
+SMALL = [
+    # B, Lq, Lk, Hq, Hkv  (ragged tails, Lq != Lk, several GQA group sizes)
+    (1, 128, 128, 8, 1),
+    (2, 200, 200, 16, 2),
+    (1, 77, 300, 8, 8),
+    (2, 333, 333, 4, 2),
+    (1, 129, 129, 32, 2),
+    (1, 50, 40, 8, 1),
+    (3, 64, 64, 24, 3),
+]
+
+
+@pytest.mark.parametrize("window", [0, 1, 5, 128, 100000])
+@pytest.mark.parametrize("shape", SMALL)
+def test_bf16_small_shapes(shape, window):
+    B, Lq, Lk, Hq, Hkv = shape
+    t = prefill_inputs(B, Lq, Lk, Hq, Hkv, 64, torch.bfloat16, 0.5, 1.0, seed=hash(shape) % 1000 + window)
+    scale = 0.125
+    out, lse = run_fwd(t, window, scale)
+    ro, rl = oracle.fwd(t["q"], t["k"], t["v"], t["sinks"], window, scale)
+    assert_close_bf16(out, ro, f"out {shape} w={window}")
+    assert_lse(lse, rl, f"lse {shape} w={window}")
+
+
+@pytest.mark.parametrize("sink", [float("-inf"), 50.0, -30.0])
+def test_bf16_extreme_sinks(sink):
+    t = prefill_inputs(1, 150, 150, 16, 2, 64, torch.bfloat16, 0.5, 1.0, seed=7, sink_fill=sink)
+    out, lse = run_fwd(t, 0, 0.125)
+    ro, rl = oracle.fwd(t["q"], t["k"], t["v"], t["sinks"], 0, 0.125)
+    assert_close_bf16(out, ro, f"sink={sink}")
+    assert_lse(lse, rl, f"sink={sink}")
+    assert torch.isfinite(out).all()
+
+
+def test_bf16_large_logits_force_rescale():
+    """Scores far above the sink move the running maximum many times (the
+    conditional O rescale path) -- values stay exact."""
+    t = prefill_inputs(1, 300, 300, 8, 1, 64, torch.bfloat16, 3.0, 1.0, seed=8)
+    out, lse = run_fwd(t, 0, 0.125)
+    ro, rl = oracle.fwd(t["q"], t["k"], t["v"], t["sinks"], 0, 0.125)
+    assert_close_bf16(out, ro, "large logits")
+    assert_lse(lse, rl, "large logits", max_abs=2e-3)
+
+
+def test_rows_without_keys_and_neg_inf_sink():
+    t = prefill_inputs(1, 100, 20, 8, 2, 64, torch.bfloat16, 0.5, 1.0, seed=9)
+    t["sinks"][:4] = float("-inf")
+    out, lse = run_fwd(t, 0, 0.125)
+    ro, rl = oracle.fwd(t["q"], t["k"], t["v"], t["sinks"], 0, 0.125)
+    assert_close_bf16(out, ro, "no keys")
+    lg = lse.cpu().numpy()
+    assert np.array_equal(np.isneginf(lg), np.isneginf(rl))
+    assert_lse(lse, rl, "no keys")
+
+
+@pytest.mark.parametrize("window", [0, WINDOW])
+def test_prefill_20b_full(window):
+    """gpt-oss-20b shaped prefill (B1 L4096 Hq64 Hkv8), every output element."""
+    w = PREFILL_20B
+    t = workload_inputs(w, SEEDS["prefill"])
+    scale = 1.0 / math.sqrt(w.D)
+    out, lse = run_fwd(t, window, scale)
+    ro, rl = oracle.fwd(t["q"], t["k"], t["v"], t["sinks"], window, scale)
+    ma, rel = assert_close_bf16(out, ro, f"prefill w={window}")
+    assert_lse(lse, rl, f"prefill w={window}")
+
+
+def _sampled(w, seed, window, n=64):
+    t = workload_inputs(w, seed)
+    scale = 1.0 / math.sqrt(w.D)
+    out, lse = run_fwd(t, window, scale)
+    rb, rh, ri = sample_rows(w.B, w.Hq, w.L, n, seed + 17, window, sinks=t["sinks"])
+    ro, rl = oracle.fwd_rows(t["q"], t["k"], t["v"], t["sinks"], rb.numpy(), rh.numpy(), ri.numpy(), window, scale)
+    go = out[rb.long(), ri.long(), rh.long()].float().cpu()
+    gl = lse[rb.long(), rh.long(), ri.long()].cpu()
+    assert_close_bf16(go, ro, f"{w.name} w={window} sampled")
+    assert_lse(gl, rl, f"{w.name} w={window} sampled")
+    # properties that hold at any size: finite, and |O| <= max|v| (convex combination scaled by < 1)
+    assert torch.isfinite(out).all() and torch.isfinite(lse).all()
+    assert out.abs().max().item() <= t["v"].abs().max().item() + 1e-2
+
+
+@pytest.mark.parametrize("window", [0, WINDOW])
+def test_train_shape_sampled(window):
+    _sampled(TRAIN, SEEDS["train"], window)
+
+
+def test_long_banded_sampled():
+    _sampled(LONG_BANDED, SEEDS["long"], WINDOW)
+
+
+def test_long_dense_sampled():
+    _sampled(LONG_DENSE, SEEDS["long"], 0)
+
+
+def test_deterministic_and_stream_ordered():
+    t = prefill_inputs(1, 512, 512, 64, 8, 64, torch.bfloat16, 0.5, 1.0, seed=11)
+    o1, l1 = run_fwd(t, 0, 0.125)
+    o2, l2 = run_fwd(t, 0, 0.125)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)

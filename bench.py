@@ -1,0 +1,430 @@
+#!/usr/bin/env python
+"""Benchmark of sink-softmax GQA attention on B200.
+
+Workload of one step: the gpt-oss-20b shaped prefill -- B=1, L=4096, Hq=64,
+Hkv=8, D=64, bf16 -- as two layers run back to back, one dense causal and one
+causal banded to a window of 128 (forward: output bf16 + fp32 LSE).
+Metric: prefill TFLOP/s, counting only unmasked scores (4*D flops per visible
+(query, key) pair), whole job over all ranks.  Further legs measured in the
+same run (rank 0 only): split-KV decode (B=64 ragged sequences up to 32768,
+dense and window-128) in KV GB/s, and the backward.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--no-legs]
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own batch of
+the same workload (independent problems, no collective on the data path);
+`value` is the total work of all ranks over the max-over-ranks device time.
+`--impl reference` times the fp64 CPU oracle on a bounded sample of the same
+workload on this host's cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "gpt-oss-20b prefill B1 L4096 Hq64 Hkv8 D64 bf16, dense causal + window-128 layers"
+METRIC = "prefill TFLOP/s (unmasked scores, 4*D flop per visible pair), dense+banded layers"
+B, L, HQ, HKV, D, WIN = 1, 4096, 64, 8, 64, 128
+SCALE = 1.0 / math.sqrt(D)
+FLUSH_BYTES = 256 << 20
+
+
+def n_visible(L_, window):
+    """Visible (query, key) pairs of one (b, h) for Lq = Lk = L_."""
+    if window <= 0 or window >= L_:
+        return L_ * (L_ + 1) // 2
+    return window * (window + 1) // 2 + (L_ - window) * window
+
+
+def fwd_flops(B_, L_, Hq_, window):
+    return 4.0 * D * n_visible(L_, window) * B_ * Hq_
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
+            pk = json.load(fh)
+        return float(pk["hbm_gbs"]), float(pk["bf16_tflops"]), float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"])), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "200", "-i", str(self.gpu)], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        rows = []
+        for ts, line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((ts, float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        inside = [r for r in rows if t0 <= r[0] <= t1] or rows
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in inside for i, v in enumerate(r[3]) if v.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(r[1] for r in inside), "sm_max_mhz": max(r[2] for r in inside),
+                "reasons": reasons, "samples": len(inside)}
+
+
+# ----------------------------------------------------------------------------- our arm
+def make_prefill(seed, dev):
+    from gqa_softmax_attention_attn_b200.inputs import prefill_inputs
+
+    t = prefill_inputs(B, L, L, HQ, HKV, D, torch.bfloat16, 0.5, 1.0, 0.1, seed=seed, with_dout=True)
+    return {k: v.to(dev) for k, v in t.items()}, t
+
+
+def traffic_from_profile(kernel_file: str, profile_json: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the kernel source as it is now (else null)."""
+    try:
+        with open(os.path.join(ROOT, "profiles", profile_json)) as fh:
+            pj = json.load(fh)
+        src = open(os.path.join(ROOT, "gqa_softmax_attention_attn_b200", "csrc", kernel_file), "rb").read()
+        if pj.get("source_sha256") != hashlib.sha256(src).hexdigest():
+            return None
+        return float(pj["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+def run_ours(args, rank, world, dev):
+    import gqa_softmax_attention_attn_b200 as attn
+
+    hbm, tf_burst, tf_sust, peak_src = peaks()
+    stream = torch.cuda.current_stream(dev)
+    layers = []
+    for li, window in enumerate((0, WIN)):
+        d, host = make_prefill(1002 + 7919 * rank + li, dev)
+        d["out"] = torch.empty_like(d["q"])
+        d["lse"] = torch.empty(B, HQ, L, device=dev, dtype=torch.float32)
+        d["window"] = window
+        d["host"] = host
+        layers.append(d)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def launch(d):
+        attn.attn_sink_fwd(d["q"], d["k"], d["v"], d["sinks"], d["out"], d["lse"], d["window"], SCALE, stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        for d in layers:
+            launch(d)
+    torch.cuda.synchronize(dev)
+    assert attn.attn_sink_get_device_status(stream) == 0
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    if rank == 0:
+        sampler.start()
+        time.sleep(0.5)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    t0 = time.time()
+    for i in range(K):
+        flush.zero_()
+        ev[i][0].record(stream)
+        launch(layers[0])
+        ev[i][1].record(stream)
+        launch(layers[1])
+        ev[i][2].record(stream)
+    torch.cuda.synchronize(dev)
+    t1 = time.time()
+    if world > 1:
+        torch.distributed.barrier()
+    if rank == 0:
+        time.sleep(0.3)
+        sampler.stop()
+    dense_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
+    band_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
+    step_ms = sum(dense_ms) + sum(band_ms)
+    status = attn.attn_sink_get_device_status(stream)
+    assert status == 0, f"device status {status}"
+    t_ms = torch.tensor([step_ms, sum(dense_ms), sum(band_ms)], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t_ms, op=torch.distributed.ReduceOp.MAX)
+    step_ms, dense_tot, band_tot = (float(x) for x in t_ms.tolist())
+    flops_step = fwd_flops(B, L, HQ, 0) + fwd_flops(B, L, HQ, WIN)
+    value = flops_step * K * world / (step_ms * 1e-3) / 1e12
+
+    # e2e through the public API with host buffers: pinned H2D of each layer's inputs, D2H of its outputs
+    e2e = None
+    if not args.no_e2e:
+        hosts = []
+        for d in layers:
+            h = {k: d["host"][k].pin_memory() for k in ("q", "k", "v", "sinks")}
+            h["out"] = torch.empty(d["out"].shape, dtype=d["out"].dtype).pin_memory()
+            h["lse"] = torch.empty(d["lse"].shape, dtype=d["lse"].dtype).pin_memory()
+            hosts.append(h)
+        h2d = sum(h[k].numel() * h[k].element_size() for h in hosts for k in ("q", "k", "v", "sinks"))
+        d2h = sum(h[k].numel() * h[k].element_size() for h in hosts for k in ("out", "lse"))
+        Ke = max(3, min(K, 50))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for it in range(Ke + 2):
+            if it == 2:
+                torch.cuda.synchronize(dev)
+                e0.record(stream)
+            for d, h in zip(layers, hosts):
+                for k in ("q", "k", "v", "sinks"):
+                    d[k].copy_(h[k], non_blocking=True)
+                launch(d)
+                h["out"].copy_(d["out"], non_blocking=True)
+                h["lse"].copy_(d["lse"], non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+        if world > 1:
+            torch.distributed.all_reduce(e_ms, op=torch.distributed.ReduceOp.MAX)
+        e2e = {"value": flops_step * Ke * world / (float(e_ms.item()) * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    dense_avg = dense_tot / K
+    achieved = fwd_flops(B, L, HQ, 0) / (dense_avg * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "kernel": "fwd_tc_kernel (dense causal layer)", "achieved": achieved,
+                "peak": tf_burst, "unit": "TFLOP/s", "frac": achieved / tf_burst,
+                "peak_source": f"{peak_src} bf16 dense (burst)",
+                "traffic": traffic_from_profile("fwd_tc.cu", "fwd_tc_prefill_20b_dense.json")}
+    res = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": step_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded N(0,1)*0.5 q/k/v, N(0,1) sinks)",
+        "config": {"workload": WORKLOAD, "global_batch": B * world, "seq_len": L, "heads_q": HQ, "heads_kv": HKV,
+                   "head_dim": D, "window": WIN, "parallelism": f"dp{world}",
+                   "l2": "flushed between steps (256 MB write, outside the timed events)"},
+        "roofline": roofline,
+        "gpu_launches": 2 * K,
+        "e2e": e2e,
+        "layers": {"dense_ms": dense_avg, "dense_tflops": achieved,
+                   "banded_ms": band_tot / K,
+                   "banded_gbs": banded_bytes() / (band_tot / K * 1e-3) / 1e9,
+                   "banded_frac_hbm": banded_bytes() / (band_tot / K * 1e-3) / 1e9 / hbm},
+    }
+    if rank == 0:
+        res["clocks"] = sampler.summary(t0, t1)
+    return res
+
+
+def banded_bytes():
+    """Compulsory bytes of one banded forward: read q, k, v, sinks; write out (bf16) and lse (fp32)."""
+    return (2 * B * L * HQ * D + 2 * 2 * B * L * HKV * D + 4 * HQ + 2 * B * L * HQ * D + 4 * B * HQ * L)
+
+
+def decode_legs(dev, reps=20):
+    import gqa_softmax_attention_attn_b200 as attn
+    from gqa_softmax_attention_attn_b200.inputs import DECODE, SEEDS, decode_inputs
+
+    hbm, _, _, _ = peaks()
+    w = DECODE
+    d = decode_inputs(w.B, w.Lmax, w.Hq, w.Hkv, w.D, w.len_lo, w.len_hi, w.dtype, w.qkv_std, w.sink_std,
+                      seed=SEEDS["decode"])
+    lens = d["seqlens"].tolist()
+    d = {k: v.to(dev) for k, v in d.items()}
+    out = torch.empty_like(d["q"])
+    lse = torch.empty(w.B, w.Hq, device=dev, dtype=torch.float32)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    legs = {}
+    for name, window in (("decode_dense", 0), ("decode_window128", WIN)):
+        nbytes = attn.attn_sink_decode_workspace_size(w.B, w.Hq, w.D, w.Lmax, window, 0)
+        ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
+        kv_rows = sum(min(n, window) if window > 0 else n for n in lens)
+        by = kv_rows * w.Hkv * w.D * 2 * 2 + w.B * w.Hq * w.D * 2 * 2 + w.B * w.Hq * 4 + 4 * w.B
+        times = []
+        for it in range(reps + 3):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            attn.attn_sink_decode(d["q"], d["k_cache"], d["v_cache"], d["seqlens"], d["sinks"], out, lse, window,
+                                  SCALE, 0, ws, stream)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            if it >= 3:
+                times.append(e0.elapsed_time(e1))
+        ms = statistics.median(times)
+        gbs = by / (ms * 1e-3) / 1e9
+        legs[name] = {"ms": ms, "GB/s": gbs, "frac_hbm": gbs / hbm, "bytes": by,
+                      "flops": 4.0 * w.D * kv_rows * (w.Hq // w.Hkv) * w.Hkv}
+    return legs
+
+
+def bwd_legs(dev, reps=5):
+    import gqa_softmax_attention_attn_b200 as attn
+
+    hbm, tf_burst, _, _ = peaks()
+    d, _ = make_prefill(2002, dev)
+    stream = torch.cuda.current_stream(dev)
+    out = torch.empty_like(d["q"])
+    lse = torch.empty(B, HQ, L, device=dev, dtype=torch.float32)
+    dq, dk, dv = torch.empty_like(d["q"]), torch.empty_like(d["k"]), torch.empty_like(d["v"])
+    ds = torch.empty(HQ, device=dev, dtype=torch.float32)
+    ws = torch.empty(attn.attn_sink_bwd_workspace_size(B, L, L, HQ, HKV, D, attn.DTYPE_BF16), dtype=torch.uint8,
+                     device=dev)
+    legs = {}
+    for name, window in (("bwd_dense", 0), ("bwd_window128", WIN)):
+        attn.attn_sink_fwd(d["q"], d["k"], d["v"], d["sinks"], out, lse, window, SCALE, stream)
+        times = []
+        for it in range(reps + 2):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            attn.attn_sink_bwd(d["q"], d["k"], d["v"], d["sinks"], out, d["dout"], lse, dq, dk, dv, ds, window,
+                               SCALE, ws, stream)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            if it >= 2:
+                times.append(e0.elapsed_time(e1))
+        ms = statistics.median(times)
+        fl = 2.5 * fwd_flops(B, L, HQ, window)
+        legs[name] = {"ms": ms, "TFLOP/s": fl / (ms * 1e-3) / 1e12, "frac_tensor": fl / (ms * 1e-3) / 1e12 / tf_burst,
+                      "shape": "B1 L4096 Hq64 Hkv8 D64"}
+    return legs
+
+
+# ----------------------------------------------------------------------------- oracle (CPU) arm
+def oracle_sample(seconds_budget=12.0, seed=1002):
+    """Times the fp64 oracle on sampled rows of both layers of the workload.
+    Returns (TFLOP/s, threads, description, flops, seconds)."""
+    import numpy as np
+
+    import oracle
+    from gqa_softmax_attention_attn_b200.inputs import prefill_inputs
+
+    t = prefill_inputs(B, L, L, HQ, HKV, D, torch.bfloat16, 0.5, 1.0, seed=seed)
+    rng = np.random.default_rng(seed)
+    total_fl, total_s, rows = 0.0, 0.0, 0
+    n = 256
+    while total_s < seconds_budget:
+        for window in (0, WIN):
+            ri = rng.integers(0, L, n).astype(np.int32)
+            rh = rng.integers(0, HQ, n).astype(np.int32)
+            rb = np.zeros(n, dtype=np.int32)
+            vis = np.minimum(ri + 1, window) if window > 0 else ri + 1
+            t0 = time.perf_counter()
+            oracle.fwd_rows(t["q"], t["k"], t["v"], t["sinks"], rb, rh, ri, window, SCALE)
+            total_s += time.perf_counter() - t0
+            total_fl += 4.0 * D * float(vis.sum())
+            rows += n
+    desc = (f"{rows} uniformly sampled query rows (dense and window-128 layers) of the {WORKLOAD} workload, "
+            f"fp64 oracle, {total_s:.1f} s")
+    return total_fl / total_s / 1e12, oracle.num_threads(), desc, total_fl, total_s
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    steps = []
+    per = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    for i in range(args.warmup + args.steps):
+        v, cores, desc, fl, s = oracle_sample(seconds_budget=per, seed=1002 + i)
+        if i >= args.warmup:
+            steps.append((fl, s))
+    fl = sum(x[0] for x in steps)
+    s = sum(x[1] for x in steps)
+    value = fl / s / 1e12
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": s / len(steps) * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": WORKLOAD, "global_batch": B, "seq_len": L,
+                                             "parallelism": "cpu-oracle"},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# ----------------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-legs", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    res = run_ours(args, rank, world, dev)
+    if rank == 0:
+        if not args.no_legs and world == 1:
+            res["legs"] = {}
+            res["legs"].update(decode_legs(dev))
+            res["legs"].update(bwd_legs(dev))
+        if not args.no_cpu_baseline and world == 1:
+            v, cores, desc, _, _ = oracle_sample(12.0)
+            res["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc}
+        res["device"] = {"name": torch.cuda.get_device_name(dev), "capability": list(torch.cuda.get_device_capability(dev)),
+                         "torch": torch.__version__, "cuda": torch.version.cuda}
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -77,7 +77,9 @@ def test_bf16_large_logits_force_rescale():
     t = prefill_inputs(1, 300, 300, 8, 1, 64, torch.bfloat16, 3.0, 1.0, seed=8)
     out, lse = run_fwd(t, 0, 0.125)
     ro, rl = oracle.fwd(t["q"], t["k"], t["v"], t["sinks"], 0, 0.125)
-    assert_close_bf16(out, ro, "large logits")
+    # Inputs with std 3 give |O| up to ~12, where rounding O itself to bf16
+    # (2^-9 relative) already exceeds 2e-2: the bound scales with max|O| here.
+    assert_close_bf16(out, ro, "large logits", max_abs=2e-2 * max(1.0, float(np.abs(ro).max()) / 4))
     assert_lse(lse, rl, "large logits", max_abs=2e-3)
 
 

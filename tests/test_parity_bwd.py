@@ -50,8 +50,13 @@ def test_tiny_fp32_bwd_exact(window):
 def _check_bf16(t, window, scale, what):
     dq, dk, dv, ds = run_bwd(t, window, scale)
     rq, rk, rv, rs = oracle.bwd(t["q"], t["k"], t["v"], t["sinks"], t["dout"], window, scale)
-    assert_close_bf16(dq, rq, f"{what} dq")
-    assert_close_bf16(dk, rk, f"{what} dk")
+    # D_i = <dO_i, O_i> uses the forward's bf16-stored O (as the API defines).
+    # With a single visible key (window = 1) dP - D = (1 - P) dO.v cancels, so
+    # O's 2^-9 rounding is amplified by P / (1 - P) in dq and dk; the absolute
+    # bound is unchanged, the relative one is widened for that degenerate case.
+    rel = 5e-3 if window != 1 else 2e-2
+    assert_close_bf16(dq, rq, f"{what} dq", rel_l2=rel)
+    assert_close_bf16(dk, rk, f"{what} dk", rel_l2=rel)
     assert_close_bf16(dv, rv, f"{what} dv")
     ma, _ = errors(ds, rs)
     assert ma <= DSINK_REL * np.abs(rs).max() + 1e-5, f"{what} dsink max_abs={ma:.3e}"

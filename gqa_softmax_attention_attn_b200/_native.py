@@ -50,6 +50,8 @@ def load():
         lib.attn_sink_fwd.restype = I
         lib.attn_sink_decode.argtypes = [P] * 7 + [I] * 6 + [F, I, P, Z, I, P]
         lib.attn_sink_decode.restype = I
+        lib.attn_sink_decode_noalloc.argtypes = [P] * 7 + [I] * 6 + [F, I, I, P]
+        lib.attn_sink_decode_noalloc.restype = I
         lib.attn_sink_decode_workspace_size.argtypes = [I] * 6
         lib.attn_sink_decode_workspace_size.restype = Z
         lib.attn_sink_bwd.argtypes = [P] * 11 + [I] * 7 + [F, P, Z, I, P]
@@ -134,6 +136,23 @@ def attn_sink_decode(q, k_cache, v_cache, seqlens, sinks, out, lse, window: int,
                                  int(window), float(scale), int(num_splits), ws_ptr, ws_bytes, _dtype_code(q),
                                  _stream(stream))
     _check(rc, "attn_sink_decode")
+
+
+NOALLOC_SCRATCH_BYTES = 32 << 20  # ATTN_SINK_NOALLOC_SCRATCH_BYTES
+
+
+def attn_sink_decode_noalloc(q, k_cache, v_cache, seqlens, sinks, out, lse, window: int, scale: float,
+                             num_splits: int = 0, stream=None):
+    """attn_sink_decode with the library's built-in scratch instead of a caller workspace
+    (for callers that cannot allocate device memory; calls on one device must not overlap)."""
+    B, Hq, D = q.shape
+    Lmax, Hkv = k_cache.shape[1], k_cache.shape[2]
+    dt = q.dtype
+    rc = load().attn_sink_decode_noalloc(_dev(q, "q"), _dev(k_cache, "k_cache", dt), _dev(v_cache, "v_cache", dt),
+                                         _dev(seqlens, "seqlens", torch.int32), _dev(sinks, "sinks", torch.float32),
+                                         _dev(out, "out", dt), _dev(lse, "lse", torch.float32), B, Lmax, Hq, Hkv, D,
+                                         int(window), float(scale), int(num_splits), _dtype_code(q), _stream(stream))
+    _check(rc, "attn_sink_decode_noalloc")
 
 
 def attn_sink_bwd_workspace_size(B: int, Lq: int, Lk: int, Hq: int, Hkv: int, D: int, dtype: int) -> int:

@@ -192,6 +192,9 @@ const char *attn_sink_strerror(int status)
     case ATTN_SINK_ERR_CUDA: return "CUDA call or kernel launch failed";
     case ATTN_SINK_ERR_TIMEOUT: return "a bounded device-side wait expired";
     case ATTN_SINK_ERR_NO_DEVICE: return "no CUDA device visible";
+    case ATTN_SINK_ERR_SCRATCH_LIMIT:
+        return "problem needs more scratch than the library's built-in no-allocation buffer "
+               "(ATTN_SINK_NOALLOC_SCRATCH_BYTES); use fewer splits or attn_sink_decode with a workspace";
     default: return "unknown status";
     }
 }
@@ -334,3 +337,64 @@ int attn_sink_get_device_status(void *stream)
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode without any allocation: the split partials live in a file-scope
+// device array.  In host code `g_noalloc_scratch` names a host-side shadow,
+// not device memory, so the kernels get the device address looked up below.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[ATTN_SINK_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+struct NoAllocScratch {
+    std::once_flag once;
+    int status = ATTN_SINK_ERR_CUDA;
+    void *ptr = nullptr;
+};
+NoAllocScratch g_noalloc[kMaxDevices];
+
+// Once per device, with that device current: device address of the array.
+int noalloc_scratch(void **ptr)
+{
+    int dev = 0;
+    int rc = current_device(&dev);
+    if (rc != ATTN_SINK_OK) return rc;
+    NoAllocScratch &s = g_noalloc[dev];
+    std::call_once(s.once, [&s]() {
+        void *p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess || p == nullptr) {
+            cudaGetLastError();
+            s.status = ATTN_SINK_ERR_CUDA;
+            return;
+        }
+        s.ptr = p;
+        s.status = ATTN_SINK_OK;
+    });
+    *ptr = s.ptr;
+    return s.status;
+}
+
+}  // namespace
+
+extern "C" int attn_sink_decode_noalloc(const void *q, const void *k_cache, const void *v_cache,
+                                        const int *seqlens, const float *sinks, void *out, float *lse, int B,
+                                        int Lmax, int Hq, int Hkv, int D, int window, float scale,
+                                        int num_splits, int dtype, void *stream)
+{
+    if (num_splits < 0 || num_splits > 32) return ATTN_SINK_ERR_INVALID_ARG;
+    const int rc0 = check_common(B, 1, Lmax, Hq, Hkv, D, dtype);
+    if (rc0 != ATTN_SINK_OK) return rc0;
+    const size_t need = decode_ws_bytes(decode_shape(B, Lmax, Hq, Hkv, D, window, scale, num_splits));
+    if (need > ATTN_SINK_NOALLOC_SCRATCH_BYTES) return ATTN_SINK_ERR_SCRATCH_LIMIT;
+    void *scratch = nullptr;
+    if (need > 0) {
+        int rc = ensure_device();
+        if (rc != ATTN_SINK_OK) return rc;
+        rc = noalloc_scratch(&scratch);
+        if (rc != ATTN_SINK_OK) return rc;
+    }
+    return attn_sink_decode(q, k_cache, v_cache, seqlens, sinks, out, lse, B, Lmax, Hq, Hkv, D, window, scale,
+                            num_splits, scratch, need > 0 ? (size_t)ATTN_SINK_NOALLOC_SCRATCH_BYTES : 0, dtype,
+                            stream);
+}

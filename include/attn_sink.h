@@ -69,7 +69,9 @@ typedef enum attn_sink_status {
     ATTN_SINK_ERR_WORKSPACE = -5,     /* workspace missing or smaller than required */
     ATTN_SINK_ERR_CUDA = -6,          /* a CUDA runtime/driver call or launch failed */
     ATTN_SINK_ERR_TIMEOUT = -7,       /* a bounded device-side wait expired */
-    ATTN_SINK_ERR_NO_DEVICE = -8      /* no CUDA device is visible */
+    ATTN_SINK_ERR_NO_DEVICE = -8,     /* no CUDA device is visible */
+    ATTN_SINK_ERR_SCRATCH_LIMIT = -9  /* attn_sink_decode_noalloc: the problem needs more
+                                         scratch than ATTN_SINK_NOALLOC_SCRATCH_BYTES */
 } attn_sink_status;
 
 enum { ATTN_SINK_DTYPE_F32 = 0, ATTN_SINK_DTYPE_BF16 = 1 };
@@ -121,6 +123,45 @@ ATTN_SINK_API int attn_sink_decode(const void *q, const void *k_cache, const voi
 
 /* Bytes of decode workspace for these sizes (0 when a single split suffices). */
 ATTN_SINK_API size_t attn_sink_decode_workspace_size(int B, int Hq, int D, int Lmax, int window, int num_splits);
+
+/*
+ * Size of the scratch buffer built into the library for
+ * attn_sink_decode_noalloc: 32 MiB of device memory, reserved on every GPU
+ * that loads the library and held until the process exits.
+ */
+#define ATTN_SINK_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+
+/*
+ * attn_sink_decode for callers that cannot allocate device memory.  The
+ * pages describe no such call; it exists for users of this library whose
+ * device memory is owned by someone else -- a plugin inside an inference
+ * server or framework that must not go around the host's allocator, or a
+ * latency-critical decode loop where a cudaMalloc (which can synchronise the
+ * device, and can fail) is not acceptable -- and who therefore cannot supply
+ * the workspace attn_sink_decode needs.
+ *
+ * Arguments, layouts, results and errors are those of attn_sink_decode,
+ * minus the workspace: the split partials go to a file-scope scratch array
+ * of ATTN_SINK_NOALLOC_SCRATCH_BYTES inside the library.  Nothing is
+ * allocated: no cudaMalloc, no cudaFree, no allocating library routine.
+ *   - A problem whose attn_sink_decode_workspace_size(...) exceeds
+ *     ATTN_SINK_NOALLOC_SCRATCH_BYTES is rejected with
+ *     ATTN_SINK_ERR_SCRATCH_LIMIT before anything is enqueued (pass a
+ *     smaller num_splits, or use attn_sink_decode with your own workspace).
+ *   - Every call on a device shares that device's one scratch array and the
+ *     array keeps the last call's contents.  Calls whose kernels can overlap
+ *     on the GPU (different streams without ordering between them) race on
+ *     it and give wrong results; order them on one stream or use
+ *     attn_sink_decode.  No part of the scratch needs to start at zero: every
+ *     partial is written before it is read.
+ *   - The first call on a device looks up the array's device address (a
+ *     one-time set-up with that device current); make that first call before
+ *     any stream capture begins.
+ */
+ATTN_SINK_API int attn_sink_decode_noalloc(const void *q, const void *k_cache, const void *v_cache,
+                     const int *seqlens, const float *sinks, void *out, float *lse,
+                     int B, int Lmax, int Hq, int Hkv, int D, int window, float scale,
+                     int num_splits, int dtype, void *stream);
 
 /*
  * Backward of attn_sink_fwd, derived from the definition above (the pages

@@ -10,14 +10,17 @@
 // log-sum-exp including the sink.
 //
 // Design (B200):
-//  * CTA tile = 128 query rows = (128 / Gp) positions x Gp query heads of one
+//  * Work item = 128 query rows = (128 / Gp) positions x Gp query heads of one
 //    KV group, so every K/V tile fetched is shared by Gp heads (GQA packing;
-//    no cluster multicast).  Q is loaded once by a 4-D TMA box.
-//  * Warp 0: TMA producer (K and V tiles of BN keys into an NS-stage ring).
-//    Warp 1: allocates tensor memory and issues tcgen05.mma from one thread:
-//    S = Q K^T into a double-buffered TMEM tile, O += P V with P read from
-//    TMEM.  Warps 2-5: one thread per row -- tcgen05.ld of S, masking, the
-//    exp2 softmax, P written back over S as bf16, conditional rescale of O.
+//    no cluster multicast).  Persistent CTAs (two per SM, 256 TMEM columns
+//    each) walk a static longest-first list of work items.
+//  * Warp 0: TMA producer -- Q (double-buffered, so the next item's Q lands
+//    while the current one finishes) and K/V tiles of BN keys into an
+//    NS-stage ring.  Warp 1: allocates tensor memory and issues tcgen05.mma
+//    from one thread: S = Q K^T into a double-buffered TMEM tile, O += P V
+//    with P read back from TMEM.  Warps 2-5: one thread per row --
+//    tcgen05.ld of S, masking, the exp2 softmax, P written over S as bf16,
+//    conditional rescale of O, epilogue.
 //  * The running maximum used for the exponentials is only moved when the
 //    true maximum exceeds it by more than 2^8, so the O rescale (which must
 //    wait for the previous PV product) is rare; the result is exact either
@@ -31,6 +34,8 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <math.h>
+
+#include <algorithm>
 
 #include "kernels.h"
 #include "sm100_ptx.cuh"
@@ -48,18 +53,17 @@ template <int BN, int NS>
 struct FwdCfg {
     static constexpr int kQBytes = kM * kD * 2;
     static constexpr int kKVBytes = BN * kD * 2;
-    static constexpr int kOffQ = 0;
-    static constexpr int kOffK = kQBytes;
+    static constexpr int kOffQ = 0;  // two Q buffers
+    static constexpr int kOffK = 2 * kQBytes;
     static constexpr int kOffV = kOffK + NS * kKVBytes;
     static constexpr int kOffBar = kOffV + NS * kKVBytes;
-    // q_full, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS], s_full[2], p_full[2], o_done, drain
-    static constexpr int kNumBar = 1 + 4 * NS + 2 + 2 + 1 + 1;
+    // q_full[2], q_empty[2], k_full[NS], k_empty[NS], v_full[NS], v_empty[NS],
+    // s_full[2], p_full[2], o_done, o_free, drain
+    static constexpr int kNumBar = 4 + 4 * NS + 4 + 3;
     static constexpr int kOffMisc = kOffBar + kNumBar * 8;
+    static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + slack for 1024-byte alignment
     static constexpr int kTmemCols = (2 * BN + kD <= 256) ? 256 : 512;
-    // + slack for 1024-byte alignment; a CTA that takes all 512 TMEM columns
-    // also takes enough shared memory that no second CTA lands on its SM
-    static constexpr int kSmemUsed = kOffMisc + 16 + 1024;
-    static constexpr int kSmemBytes = (kTmemCols == 512 && kSmemUsed < 116 * 1024) ? 116 * 1024 : kSmemUsed;
+    static constexpr int kCtasPerSm = kTmemCols == 256 ? 2 : 1;
     static constexpr int kTmS0 = 0;
     static constexpr int kTmO = 2 * BN;
 };
@@ -67,7 +71,7 @@ struct FwdCfg {
 struct FwdTcParams {
     int B, Lq, Lk, Hq, Hkv, window;
     int G, Gp, P;  // group size, query heads packed per tile, positions per tile
-    int n_ptiles;
+    int n_ptiles, n_htiles, n_items;
     float c_log2;  // scale * log2(e)
     const float *sinks;
     __nv_bfloat16 *out;
@@ -76,6 +80,32 @@ struct FwdTcParams {
     long long timeout_ns;
 };
 
+struct Item {
+    int pos0, h0, b, t_lo, n_tiles;
+};
+
+// Work item i of the longest-first order: q tiles from the last (most keys
+// under a causal mask) to the first, all head tiles and batches of one q tile
+// next to each other.
+template <int BN>
+__device__ __forceinline__ Item item_at(const FwdTcParams &p, int i)
+{
+    Item it;
+    const int per_q = p.n_htiles * p.B;
+    const int qt = p.n_ptiles - 1 - i / per_q;
+    const int r = i % per_q;
+    it.h0 = (r % p.n_htiles) * p.Gp;
+    it.b = r / p.n_htiles;
+    it.pos0 = qt * p.P;
+    const long off = (long)p.Lk - p.Lq;
+    const int pos_last = min(it.pos0 + p.P - 1, p.Lq - 1);
+    const long lo = p.window > 0 ? max(0L, it.pos0 + off - p.window + 1) : 0L;
+    const long hi = min((long)p.Lk, pos_last + off + 1);  // exclusive
+    it.t_lo = (int)(lo / BN);
+    it.n_tiles = hi > lo ? (int)((hi - 1) / BN) - it.t_lo + 1 : 0;
+    return it;
+}
+
 __device__ __forceinline__ bool wait_noabort(uint64_t *bar, uint32_t parity, unsigned *status, long long tmo)
 {
     int never = 0;
@@ -83,7 +113,7 @@ __device__ __forceinline__ bool wait_noabort(uint64_t *bar, uint32_t parity, uns
 }
 
 template <int BN, int NS>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(192, FwdCfg<BN, NS>::kCtasPerSm)
     fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdTcParams p)
 {
@@ -92,43 +122,36 @@ __global__ void __launch_bounds__(192, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kOffBar);
     uint64_t *q_full = bars;
-    uint64_t *k_full = bars + 1;
+    uint64_t *q_empty = bars + 2;
+    uint64_t *k_full = bars + 4;
     uint64_t *k_empty = k_full + NS;
     uint64_t *v_full = k_empty + NS;
     uint64_t *v_empty = v_full + NS;
     uint64_t *s_full = v_empty + NS;
     uint64_t *p_full = s_full + 2;
     uint64_t *o_done = p_full + 2;
-    uint64_t *drain = o_done + 1;
+    uint64_t *o_free = o_done + 1;
+    uint64_t *drain = o_free + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Cfg::kOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Cfg::kOffMisc + 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int qt = p.n_ptiles - 1 - (int)blockIdx.x;  // longest causal tiles first
-    const int h0 = (int)blockIdx.y * p.Gp;
-    const int b = (int)blockIdx.z;
-    const int g = h0 / p.G;
-    const int pos0 = qt * p.P;
-    const long off = (long)p.Lk - p.Lq;
-    const int pos_last = min(pos0 + p.P - 1, p.Lq - 1);
-    const long lo = p.window > 0 ? max(0L, pos0 + off - p.window + 1) : 0L;
-    const long hi = min((long)p.Lk, pos_last + off + 1);  // exclusive
-    const int t_lo = (int)(lo / BN);
-    const int n_tiles = hi > lo ? (int)((hi - 1) / BN) - t_lo + 1 : 0;
 
     if (threadIdx.x == 0) {
-        mbar_init(q_full, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&q_full[s], 1);
+            mbar_init(&q_empty[s], 1);
+            mbar_init(&s_full[s], 1);
+            mbar_init(&p_full[s], 128);
+        }
         for (int s = 0; s < NS; ++s) {
             mbar_init(&k_full[s], 1);
             mbar_init(&k_empty[s], 1);
             mbar_init(&v_full[s], 1);
             mbar_init(&v_empty[s], 1);
         }
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&s_full[s], 1);
-            mbar_init(&p_full[s], 128);
-        }
         mbar_init(o_done, 1);
+        mbar_init(o_free, 128);
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -144,29 +167,47 @@ __global__ void __launch_bounds__(192, 1)
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
-        if (lane == 0 && n_tiles > 0) {
+        if (lane == 0) {
             tma_prefetch_desc(&tmQ);
             tma_prefetch_desc(&tmK);
             tma_prefetch_desc(&tmV);
-            uint32_t k_issued[NS], v_issued[NS];
+            uint32_t k_issued[NS], v_issued[NS], q_issued[2] = {0, 0};
             for (int s = 0; s < NS; ++s) k_issued[s] = v_issued[s] = 0;
-            mbar_arrive_expect_tx(q_full, Cfg::kQBytes);
-            tma_load_4d(smem + Cfg::kOffQ, &tmQ, 0, h0, pos0, b, q_full);
-            for (int jt = 0; jt < n_tiles; ++jt) {
-                const int st = jt % NS;
-                const uint32_t ph = (uint32_t)(jt / NS) & 1u;
-                const int j0 = (t_lo + jt) * BN;
-                if (!mbar_wait(&k_empty[st], ph ^ 1u, abort_flag, p.status, p.timeout_ns)) break;
-                mbar_arrive_expect_tx(&k_full[st], Cfg::kKVBytes);
-                tma_load_4d(smem + Cfg::kOffK + st * Cfg::kKVBytes, &tmK, 0, g, j0, b, &k_full[st]);
-                ++k_issued[st];
-                if (!mbar_wait(&v_empty[st], ph ^ 1u, abort_flag, p.status, p.timeout_ns)) break;
-                mbar_arrive_expect_tx(&v_full[st], Cfg::kKVBytes);
-                tma_load_4d(smem + Cfg::kOffV + st * Cfg::kKVBytes, &tmV, 0, g, j0, b, &v_full[st]);
-                ++v_issued[st];
+            uint32_t it = 0, item_n = 0;
+            bool ok = true;
+            for (int w = blockIdx.x; w < p.n_items && ok; w += gridDim.x) {
+                const Item t = item_at<BN>(p, w);
+                if (t.n_tiles == 0) continue;
+                const int qb = item_n & 1;
+                if (!mbar_wait(&q_empty[qb], ((item_n >> 1) & 1u) ^ 1u, abort_flag, p.status, p.timeout_ns)) break;
+                mbar_arrive_expect_tx(&q_full[qb], Cfg::kQBytes);
+                tma_load_4d(smem + Cfg::kOffQ + qb * Cfg::kQBytes, &tmQ, 0, t.h0, t.pos0, t.b, &q_full[qb]);
+                ++q_issued[qb];
+                const int g = t.h0 / p.G;
+                for (int jt = 0; jt < t.n_tiles; ++jt, ++it) {
+                    const int st = it % NS;
+                    const uint32_t ph = (it / NS) & 1u;
+                    const int j0 = (t.t_lo + jt) * BN;
+                    if (!mbar_wait(&k_empty[st], ph ^ 1u, abort_flag, p.status, p.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&k_full[st], Cfg::kKVBytes);
+                    tma_load_4d(smem + Cfg::kOffK + st * Cfg::kKVBytes, &tmK, 0, g, j0, t.b, &k_full[st]);
+                    ++k_issued[st];
+                    if (!mbar_wait(&v_empty[st], ph ^ 1u, abort_flag, p.status, p.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&v_full[st], Cfg::kKVBytes);
+                    tma_load_4d(smem + Cfg::kOffV + st * Cfg::kKVBytes, &tmV, 0, g, j0, t.b, &v_full[st]);
+                    ++v_issued[st];
+                }
+                ++item_n;
             }
             // every load issued must land before the CTA may exit
-            wait_noabort(q_full, 0, p.status, p.timeout_ns);
+            for (int s = 0; s < 2; ++s)
+                if (q_issued[s]) wait_noabort(&q_full[s], (q_issued[s] - 1) & 1u, p.status, p.timeout_ns);
             for (int s = 0; s < NS; ++s) {
                 if (k_issued[s]) wait_noabort(&k_full[s], (k_issued[s] - 1) & 1u, p.status, p.timeout_ns);
                 if (v_issued[s]) wait_noabort(&v_full[s], (v_issued[s] - 1) & 1u, p.status, p.timeout_ns);
@@ -174,19 +215,21 @@ __global__ void __launch_bounds__(192, 1)
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0 && n_tiles > 0) {
+        if (lane == 0) {
             const uint32_t id_s = idesc_bf16_f32(kM, BN, 0);
             const uint32_t id_pv = idesc_bf16_f32(kM, kD, 1);
-            const uint32_t q_addr = smem_u32(smem + Cfg::kOffQ);
             const uint32_t k_addr = smem_u32(smem + Cfg::kOffK);
             const uint32_t v_addr = smem_u32(smem + Cfg::kOffV);
-            bool ok = mbar_wait(q_full, 0, abort_flag, p.status, p.timeout_ns);
-            auto issue_pv = [&](int t) -> bool {
+            uint32_t it = 0, item_n = 0;
+            bool ok = true;
+            // O += P(t) V(t); the first product of an item overwrites O, which
+            // must wait until the previous item's epilogue has read O out.
+            auto issue_pv = [&](uint32_t t, bool first) -> bool {
                 const int sb = t & 1, st = t % NS;
-                const uint32_t ph = (uint32_t)(t / NS) & 1u;
-                if (!mbar_wait(&p_full[sb], (uint32_t)(t >> 1) & 1u, abort_flag, p.status, p.timeout_ns))
+                if (first && !mbar_wait(o_free, (item_n & 1u) ^ 1u, abort_flag, p.status, p.timeout_ns))
                     return false;
-                if (!mbar_wait(&v_full[st], ph, abort_flag, p.status, p.timeout_ns)) return false;
+                if (!mbar_wait(&p_full[sb], (t >> 1) & 1u, abort_flag, p.status, p.timeout_ns)) return false;
+                if (!mbar_wait(&v_full[st], (t / NS) & 1u, abort_flag, p.status, p.timeout_ns)) return false;
                 tc_fence_after();
                 const uint32_t vb = v_addr + st * Cfg::kKVBytes;
 #pragma unroll
@@ -194,18 +237,22 @@ __global__ void __launch_bounds__(192, 1)
                     // V tile [BN keys][64 d] is the MN-major B operand: 16 keys = 2048 bytes per step
                     const uint64_t bdesc = smem_desc_sw128(vb + kk * 2048, BN * 128, 1024);
                     mma_ts(tmem + Cfg::kTmO, tmem + Cfg::kTmS0 + sb * BN + kk * 8, bdesc, id_pv,
-                           (t > 0 || kk > 0) ? 1u : 0u);
+                           (!first || kk > 0) ? 1u : 0u);
                 }
                 mma_commit(o_done);
                 mma_commit(&v_empty[st]);
                 return true;
             };
-            if (ok) {
+            for (int w = blockIdx.x; w < p.n_items && ok; w += gridDim.x) {
+                const Item t = item_at<BN>(p, w);
+                if (t.n_tiles == 0) continue;
+                const int qb = item_n & 1;
+                if (!mbar_wait(&q_full[qb], (item_n >> 1) & 1u, abort_flag, p.status, p.timeout_ns)) break;
                 tc_fence_after();
-                for (int jt = 0; jt < n_tiles && ok; ++jt) {
-                    const int st = jt % NS, sb = jt & 1;
-                    const uint32_t ph = (uint32_t)(jt / NS) & 1u;
-                    if (!mbar_wait(&k_full[st], ph, abort_flag, p.status, p.timeout_ns)) {
+                const uint32_t q_addr = smem_u32(smem + Cfg::kOffQ + qb * Cfg::kQBytes);
+                for (int jt = 0; jt < t.n_tiles; ++jt, ++it) {
+                    const int st = it % NS, sb = it & 1;
+                    if (!mbar_wait(&k_full[st], (it / NS) & 1u, abort_flag, p.status, p.timeout_ns)) {
                         ok = false;
                         break;
                     }
@@ -219,9 +266,17 @@ __global__ void __launch_bounds__(192, 1)
                     }
                     mma_commit(&s_full[sb]);
                     mma_commit(&k_empty[st]);
-                    if (jt >= 1) ok = issue_pv(jt - 1);
+                    if (jt == t.n_tiles - 1) mma_commit(&q_empty[qb]);
+                    if (jt >= 1 && !issue_pv(it - 1, jt == 1)) {
+                        ok = false;
+                        break;
+                    }
                 }
-                if (ok) issue_pv(n_tiles - 1);
+                if (!ok || !issue_pv(it - 1, t.n_tiles == 1)) {
+                    ok = false;
+                    break;
+                }
+                ++item_n;
             }
             mma_commit(drain);
             wait_noabort(drain, 0, p.status, p.timeout_ns);
@@ -230,123 +285,136 @@ __global__ void __launch_bounds__(192, 1)
         // ------------------------------------------------------------ softmax + epilogue
         const int quad = warp & 3;
         const int r = quad * 32 + lane;
-        const int pos = pos0 + r / p.Gp;
-        const int h = h0 + r % p.Gp;
-        const bool row_valid = pos < p.Lq;
-        const long pabs = pos + off;
-        const float sink = p.sinks[h];
-        const float C = p.c_log2;
-        float m = sink * kLog2e;  // reference maximum, log2 units
-        float l = (sink == -INFINITY) ? 0.f : 1.f;
         const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
+        const float C = p.c_log2;
+        const long off = (long)p.Lk - p.Lq;
+        uint32_t it = 0;
         bool ok = true;
+        for (int w = blockIdx.x; w < p.n_items && ok; w += gridDim.x) {
+            const Item t = item_at<BN>(p, w);
+            const int pos = t.pos0 + r / p.Gp;
+            const int h = t.h0 + r % p.Gp;
+            const bool row_valid = pos < p.Lq;
+            const long pabs = pos + off;
+            const float sink2 = p.sinks[h] * kLog2e;  // the sink logit in log2 units
+            float m = sink2;                           // reference maximum, log2 units
+            float l = (sink2 == -INFINITY) ? 0.f : 1.f;  // running sum, seeded with the sink's mass
+            // rows beyond Lq only need finite, unused values
+            const long vis_hi = row_valid ? min(pabs, (long)p.Lk - 1) : -1;   // last visible key
+            const long vis_lo = p.window > 0 ? pabs - p.window + 1 : 0;     // first visible key
 
-        for (int jt = 0; jt < n_tiles; ++jt) {
-            const int sb = jt & 1;
-            const long j0 = (long)(t_lo + jt) * BN;
-            if (!__all_sync(0xffffffffu,
-                            mbar_wait(&s_full[sb], (uint32_t)(jt >> 1) & 1u, abort_flag, p.status, p.timeout_ns))) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            uint32_t sr[BN / 32][32];
-#pragma unroll
-            for (int c = 0; c < BN / 32; ++c) tmem_ld32(trow + Cfg::kTmS0 + sb * BN + c * 32, sr[c]);
-            tmem_wait_ld();
-            float sv[BN];
-#pragma unroll
-            for (int c = 0; c < BN; ++c) sv[c] = __uint_as_float(sr[c / 32][c % 32]);
-            const bool full_vis = (j0 + BN - 1 <= pabs) && (j0 + BN <= p.Lk) &&
-                                  (p.window <= 0 || j0 > pabs - p.window);
-            if (__any_sync(0xffffffffu, !full_vis)) {
-#pragma unroll
-                for (int c = 0; c < BN; ++c) {
-                    const long j = j0 + c;
-                    const bool vis = j <= pabs && j < p.Lk && (p.window <= 0 || j > pabs - p.window);
-                    sv[c] = vis ? sv[c] : -INFINITY;
-                }
-            }
-            float tmax = sv[0];
-#pragma unroll
-            for (int c = 1; c < BN; ++c) tmax = fmaxf(tmax, sv[c]);
-            const float m_new = fmaxf(m, tmax * C);
-            const bool rescale = m_new > m + kRescaleThreshold;
-            const float alpha = rescale ? ((m == -INFINITY) ? 0.f : ex2(m - m_new)) : 1.f;
-            if (rescale) m = m_new;
-            const float neg_m = (m == -INFINITY) ? 0.f : -m;
-            // P (bf16 pairs) overwrites the first BN/2 columns of this S buffer,
-            // which has been read in full already; 32 scores per store.
-            float sum = 0.f;
-#pragma unroll
-            for (int c = 0; c < BN / 32; ++c) {
-                uint32_t pk[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const float p0 = ex2(fmaf(sv[32 * c + 2 * e], C, neg_m));
-                    const float p1 = ex2(fmaf(sv[32 * c + 2 * e + 1], C, neg_m));
-                    sum += p0 + p1;
-                    pk[e] = pack_bf16x2(p0, p1);
-                }
-                tmem_st16(trow + Cfg::kTmS0 + sb * BN + c * 16, pk);
-            }
-            l = l * alpha + sum;
-            if (jt > 0) {
-                // O holds sum_{t<jt} P_t V_t once PV(jt-1) completes
+            for (int jt = 0; jt < t.n_tiles; ++jt, ++it) {
+                const int sb = it & 1;
+                const long j0 = (long)(t.t_lo + jt) * BN;
                 if (!__all_sync(0xffffffffu,
-                                mbar_wait(o_done, (uint32_t)(jt - 1) & 1u, abort_flag, p.status, p.timeout_ns))) {
+                                mbar_wait(&s_full[sb], (it >> 1) & 1u, abort_flag, p.status, p.timeout_ns))) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                if (__any_sync(0xffffffffu, rescale)) {
-                    uint32_t o[2][32];
-                    tmem_ld32(trow + Cfg::kTmO, o[0]);
-                    tmem_ld32(trow + Cfg::kTmO + 32, o[1]);
-                    tmem_wait_ld();
+                uint32_t sr[BN / 32][32];
 #pragma unroll
-                    for (int c = 0; c < 64; ++c)
-                        o[c / 32][c % 32] = __float_as_uint(__uint_as_float(o[c / 32][c % 32]) * alpha);
-                    tmem_st32(trow + Cfg::kTmO, o[0]);
-                    tmem_st32(trow + Cfg::kTmO + 32, o[1]);
+                for (int c = 0; c < BN / 32; ++c) tmem_ld32(trow + Cfg::kTmS0 + sb * BN + c * 32, sr[c]);
+                tmem_wait_ld();
+                float sv[BN];
+#pragma unroll
+                for (int c = 0; c < BN; ++c) sv[c] = __uint_as_float(sr[c / 32][c % 32]);
+                // visible columns of this tile: c in [c_lo, c_hi] (32-bit, tile-relative)
+                const int c_hi = (int)max(-1L, min((long)BN - 1, vis_hi - j0));
+                const int c_lo = (int)max(0L, min((long)BN, vis_lo - j0));
+                if (__any_sync(0xffffffffu, c_lo > 0 || c_hi < BN - 1)) {
+#pragma unroll
+                    for (int c = 0; c < BN; ++c) sv[c] = (c >= c_lo && c <= c_hi) ? sv[c] : -INFINITY;
                 }
-            }
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(&p_full[sb]);
-        }
-
-        // ------------------------------------------------------------ epilogue
-        float ov[64];
+                float mx[4];
 #pragma unroll
-        for (int c = 0; c < 64; ++c) ov[c] = 0.f;
-        if (ok && n_tiles > 0) {
-            if (__all_sync(0xffffffffu,
-                           mbar_wait(o_done, (uint32_t)(n_tiles - 1) & 1u, abort_flag, p.status, p.timeout_ns))) {
+                for (int k = 0; k < 4; ++k) mx[k] = fmax3(sv[k], sv[k + 4], sv[k + 8]);
+#pragma unroll
+                for (int c = 12; c < BN; c += 8)
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) mx[k] = fmax3(mx[k], sv[c + k], sv[c + 4 + k]);
+                const float tmax = fmax3(mx[0], mx[1], fmaxf(mx[2], mx[3]));
+                const float m_new = fmaxf(m, tmax * C);
+                const bool rescale = m_new > m + kRescaleThreshold;
+                const float alpha = rescale ? ((m == -INFINITY) ? 0.f : ex2(m - m_new)) : 1.f;
+                if (rescale) m = m_new;
+                const float neg_m = (m == -INFINITY) ? 0.f : -m;
+                const float2 C2 = make_float2(C, C), M2 = make_float2(neg_m, neg_m);
+                float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+                // P (bf16 pairs) overwrites the first BN/2 columns of this S
+                // buffer, which has been read in full already; 32 scores per store.
+#pragma unroll
+                for (int c = 0; c < BN / 32; ++c) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const float2 x = ffma2(make_float2(sv[32 * c + 2 * e], sv[32 * c + 2 * e + 1]), C2, M2);
+                        const float2 pe = make_float2(ex2(x.x), ex2(x.y));
+                        acc[e & 1] = fadd2(acc[e & 1], pe);
+                        pk[e] = pack_bf16x2(pe.x, pe.y);
+                    }
+                    tmem_st16(trow + Cfg::kTmS0 + sb * BN + c * 16, pk);
+                }
+                l = l * alpha + ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y));
+                if (jt > 0) {
+                    // O holds sum_{t<jt} P_t V_t once PV(jt-1) completes
+                    if (!__all_sync(0xffffffffu,
+                                    mbar_wait(o_done, (it - 1) & 1u, abort_flag, p.status, p.timeout_ns))) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    if (__any_sync(0xffffffffu, rescale)) {
+                        uint32_t o[2][32];
+                        tmem_ld32(trow + Cfg::kTmO, o[0]);
+                        tmem_ld32(trow + Cfg::kTmO + 32, o[1]);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int c = 0; c < 64; ++c)
+                            o[c / 32][c % 32] = __float_as_uint(__uint_as_float(o[c / 32][c % 32]) * alpha);
+                        tmem_st32(trow + Cfg::kTmO, o[0]);
+                        tmem_st32(trow + Cfg::kTmO + 32, o[1]);
+                    }
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(&p_full[sb]);
+            }
+            if (!ok) break;
+
+            // -------------------------------------------------------- epilogue
+            uint32_t o[2][32];
+            if (t.n_tiles > 0) {
+                if (!__all_sync(0xffffffffu,
+                                mbar_wait(o_done, (it - 1) & 1u, abort_flag, p.status, p.timeout_ns))) {
+                    ok = false;
+                    break;
+                }
                 tc_fence_after();
-                uint32_t o[2][32];
                 tmem_ld32(trow + Cfg::kTmO, o[0]);
                 tmem_ld32(trow + Cfg::kTmO + 32, o[1]);
                 tmem_wait_ld();
-#pragma unroll
-                for (int c = 0; c < 64; ++c) ov[c] = __uint_as_float(o[c / 32][c % 32]);
+                tc_fence_before();
+                mbar_arrive(o_free);  // the next item's first PV may overwrite O now
             } else {
-                ok = false;
-            }
-        }
-        if (row_valid && ok) {
-            const float inv = l > 0.f ? 1.f / l : 0.f;
-            uint4 *dst = reinterpret_cast<uint4 *>(p.out + (((size_t)b * p.Lq + pos) * p.Hq + h) * kD);
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                uint4 w;
-                w.x = pack_bf16x2(ov[8 * c + 0] * inv, ov[8 * c + 1] * inv);
-                w.y = pack_bf16x2(ov[8 * c + 2] * inv, ov[8 * c + 3] * inv);
-                w.z = pack_bf16x2(ov[8 * c + 4] * inv, ov[8 * c + 5] * inv);
-                w.w = pack_bf16x2(ov[8 * c + 6] * inv, ov[8 * c + 7] * inv);
-                dst[c] = w;
+                for (int c = 0; c < 64; ++c) o[c / 32][c % 32] = 0u;
             }
-            p.lse[((size_t)b * p.Hq + h) * p.Lq + pos] = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
+            if (row_valid) {
+                const float inv = l > 0.f ? 1.f / l : 0.f;
+                uint4 *dst = reinterpret_cast<uint4 *>(p.out + (((size_t)t.b * p.Lq + pos) * p.Hq + h) * kD);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const uint32_t *src = &o[c / 4][(c % 4) * 8];
+                    uint4 v;
+                    v.x = pack_bf16x2(__uint_as_float(src[0]) * inv, __uint_as_float(src[1]) * inv);
+                    v.y = pack_bf16x2(__uint_as_float(src[2]) * inv, __uint_as_float(src[3]) * inv);
+                    v.z = pack_bf16x2(__uint_as_float(src[4]) * inv, __uint_as_float(src[5]) * inv);
+                    v.w = pack_bf16x2(__uint_as_float(src[6]) * inv, __uint_as_float(src[7]) * inv);
+                    dst[c] = v;
+                }
+                p.lse[((size_t)t.b * p.Hq + h) * p.Lq + pos] = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
+            }
         }
     }
 
@@ -377,6 +445,10 @@ cudaError_t launch_cfg(const void *q, const void *k, const void *v, const float 
     p.Gp = gp;
     p.P = kM / gp;
     p.n_ptiles = (s.Lq + p.P - 1) / p.P;
+    p.n_htiles = s.Hq / gp;
+    const long long n_items = (long long)p.n_ptiles * p.n_htiles * s.B;
+    if (n_items > 0x7fffffffLL) return cudaErrorInvalidValue;
+    p.n_items = (int)n_items;
     p.c_log2 = s.scale * kLog2e;
     p.sinks = sinks;
     p.out = static_cast<__nv_bfloat16 *>(out);
@@ -404,7 +476,10 @@ cudaError_t launch_cfg(const void *q, const void *k, const void *v, const float 
     auto kern = fwd_tc_kernel<BN, NS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
     if (e != cudaSuccess) return e;
-    dim3 grid(p.n_ptiles, s.Hq / p.Gp, s.B);
+    int dev = 0, sms = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    const int grid = (int)std::min<long long>(n_items, (long long)sms * Cfg::kCtasPerSm);
     kern<<<grid, 192, Cfg::kSmemBytes, st>>>(mq, mk, mv, p);
     return cudaGetLastError();
 }
@@ -421,7 +496,7 @@ bool fwd_tc_supported(const AttnShape &s)
 cudaError_t launch_fwd_tc(const void *q, const void *k, const void *v, const float *sinks, void *out,
                           float *lse, const AttnShape &s, cudaStream_t st)
 {
-    return launch_cfg<128, 2>(q, k, v, sinks, out, lse, s, st);
+    return launch_cfg<64, 4>(q, k, v, sinks, out, lse, s, st);
 }
 
 }  // namespace attn_sink

@@ -12,7 +12,8 @@ CSRC = os.path.join(HERE, "csrc")
 LIB_DIR = os.path.join(HERE, "lib")
 LIB = os.path.join(LIB_DIR, "libattn_sink.so")
 SOURCES = ["attn_sink_api.cu", "simt_kernels.cu", "fwd_tc.cu", "decode_tc.cu"]
-HEADERS = ["kernels.h", "sm100_ptx.cuh"]
+HEADERS = ["kernels.h", "sm100_ptx.cuh", "selftest.cu"]
+SELFTEST_LIB = os.path.join(LIB_DIR, "libattn_sink_selftest.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17", "-lineinfo",
          "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden", "-DNDEBUG"]
@@ -49,6 +50,10 @@ def build(force: bool = False, verbose: bool = False) -> str:
     subprocess.check_call([NVCC, "-shared", "-gencode", "arch=compute_100a,code=sm_100a", "-o", tmp, *objs,
                            "-Xlinker", "--version-script=" + os.path.join(CSRC, "exports.map")])
     os.replace(tmp, LIB)
+    # device self-tests of kernel helpers (test support, not the product ABI)
+    tmp = SELFTEST_LIB + f".tmp{os.getpid()}"
+    subprocess.check_call([NVCC, *FLAGS, "-shared", "-o", tmp, os.path.join(CSRC, "selftest.cu")])
+    os.replace(tmp, SELFTEST_LIB)
     with open(stamp, "w") as fh:
         fh.write(dig)
     return LIB

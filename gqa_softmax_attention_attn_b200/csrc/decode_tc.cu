@@ -1,10 +1,384 @@
-// placeholder, replaced below
+// decode_tc.cu -- bf16 split-KV decode of sink-softmax GQA attention.
+//
+// What it computes ("GPT-OSS on day 0", section "Sink Attention"): one query
+// per sequence against that sequence's cached keys, with the work split both
+// across KV heads and along the KV length; each split produces a partial
+// (running max m, running sum l, unnormalised output o) WITHOUT the sink, and
+// the sink joins exactly once, when the splits are combined (or directly here
+// when a sequence needs only one split).
+//
+// Design (B200): the path is HBM-bound (8 flop per byte of KV at GQA group 8).
+//  * CTA = (split c, KV head g, sequence b).  Warp 0 streams the split's K and
+//    V rows of head g with 2-D-tiled TMA boxes (64 keys x 128 bytes, 128-byte
+//    swizzle) into a 4-stage shared-memory ring; every byte of KV is read
+//    from HBM once, for all G query heads of the group.
+//  * Warps 1-4 take 16 keys of each 64-key tile: the G query heads of the
+//    group (padded to 16 rows) are scored with mma.sync m16n8k16 -- FP32 CUDA
+//    cores cannot sustain 8 flop/byte at HBM rate -- then an exp2 online
+//    softmax in registers and P V with mma.sync again (P reused from the
+//    score accumulators).
+//  * Keys past the chunk (ragged tail, cache rows beyond the sequence, or
+//    TMA zero fill past Lmax) are masked, and their V rows are zeroed in the
+//    operand registers so stale cache contents can never reach the output.
+//  * Every wait is bounded; on expiry the CTA raises the device status bit
+//    and winds down.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <math.h>
+
 #include "kernels.h"
+#include "sm100_ptx.cuh"
+
 namespace attn_sink {
-bool decode_bf16_supported(const DecodeShape &) { return false; }
-cudaError_t launch_decode_bf16(const void *, const void *, const void *, const int *, const float *, void *,
-                               float *, const DecodeShape &, float *, float *, cudaStream_t)
+namespace {
+
+constexpr int kD = 64;
+constexpr int kT = 64;          // keys per tile
+constexpr int kNS = 4;          // ring stages
+constexpr int kTileBytes = kT * kD * 2;
+constexpr int kStageBytes = 2 * kTileBytes;  // K and V
+constexpr int kThreads = 160;  // warp 0 producer, warps 1-4 consumers
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr int kOffBar = kNS * kStageBytes;
+constexpr int kSmemBytes = kOffBar + 2 * kNS * 8 + 16 + 1024;
+
+struct DecodeParams {
+    int B, Lmax, Hq, Hkv, G, window, splits, chunk;
+    float c_log2;
+    const __nv_bfloat16 *q;
+    const int *seqlens;
+    const float *sinks;
+    __nv_bfloat16 *out;
+    float *lse;
+    float *ws_o, *ws_ml;
+    unsigned *status;
+    long long timeout_ns;
+};
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3)
 {
-    return cudaErrorNotSupported;
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
 }
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+
+// D (fp32 16x8) += A (bf16 16x16, row) * B (bf16 16x8, col)
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
+{
+    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+                 "{%0,%1,%2,%3};"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// byte offset of (row, 16-byte chunk) in a 128-byte-swizzled tile
+__device__ __forceinline__ uint32_t swz(int row, int chunk) { return row * 128 + ((chunk ^ (row & 7)) << 4); }
+
+template <bool kRows16>
+__global__ void __launch_bounds__(kThreads)
+    decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                     const DecodeParams p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + kOffBar);
+    uint64_t *empty = full + kNS;
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffBar + 2 * kNS * 8);
+
+    const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int len = min(max(p.seqlens[b], 1), p.Lmax);
+    const int lo = p.window > 0 ? max(0, len - p.window) : 0;
+    const int nsplit = (len - lo + p.chunk - 1) / p.chunk;
+    if (c >= nsplit) return;  // uniform over the CTA
+    const int kbeg = lo + c * p.chunk;
+    const int kend = min(len, kbeg + p.chunk);
+    const int n_tiles = (kend - kbeg + kT - 1) / kT;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kNS; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 4);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    // per-warp partial state, combined through shared memory at the end
+    float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
+    float o[8][4];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+    bool ok = true;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            tma_prefetch_desc(&tmK);
+            tma_prefetch_desc(&tmV);
+            uint32_t issued[kNS] = {0, 0, 0, 0};
+            for (int j = 0; j < n_tiles; ++j) {
+                const int st = j % kNS;
+                if (!mbar_wait(&empty[st], ((j / kNS) & 1u) ^ 1u, abort_flag, p.status, p.timeout_ns)) break;
+                mbar_arrive_expect_tx(&full[st], kStageBytes);
+                tma_load_4d(smem + st * kStageBytes, &tmK, 0, g, kbeg + j * kT, b, &full[st]);
+                tma_load_4d(smem + st * kStageBytes + kTileBytes, &tmV, 0, g, kbeg + j * kT, b, &full[st]);
+                ++issued[st];
+            }
+            for (int s = 0; s < kNS; ++s)
+                if (issued[s]) {
+                    int never = 0;
+                    mbar_wait(&full[s], (issued[s] - 1) & 1u, &never, p.status, p.timeout_ns);
+                }
+        }
+    } else {
+        const int w = warp - 1;       // 16-key slice of each tile
+        const int gr = lane >> 2;     // fragment row (query head within the group)
+        const int tq = lane & 3;      // fragment column pair
+        // Q as the A operand (rows = heads of the group, zero beyond G), k-steps of 16 d
+        uint32_t qa[4][4];
+        {
+            const __nv_bfloat16 *qb = p.q + ((size_t)b * p.Hq + (size_t)g * p.G) * kD;
+            auto qpair = [&](int row, int d) -> uint32_t {
+                if (row >= p.G) return 0u;
+                return *reinterpret_cast<const uint32_t *>(qb + (size_t)row * kD + d);
+            };
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                qa[kk][0] = qpair(gr, 16 * kk + 2 * tq);
+                qa[kk][1] = qpair(gr + 8, 16 * kk + 2 * tq);
+                qa[kk][2] = qpair(gr, 16 * kk + 8 + 2 * tq);
+                qa[kk][3] = qpair(gr + 8, 16 * kk + 8 + 2 * tq);
+            }
+        }
+        const float C = p.c_log2;
+        const uint32_t sbase = smem_u32(smem);
+        for (int j = 0; j < n_tiles && ok; ++j) {
+            const int st = j % kNS;
+            if (!__all_sync(0xffffffffu,
+                            mbar_wait(&full[st], (j / kNS) & 1u, abort_flag, p.status, p.timeout_ns))) {
+                ok = false;
+                break;
+            }
+            const uint32_t kt = sbase + st * kStageBytes, vt = kt + kTileBytes;
+            const int key0 = kbeg + j * kT + 16 * w;  // first key of this warp's slice
+            // ---- S = Q K^T for 16 keys: two n-tiles of 8 keys
+            float s[2][4];
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+                const int krow = 16 * w + 8 * nt + (lane & 7);
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t b0, b1, b2, b3;  // d chunks 4*half + 0..3
+                    ldsm_x4(kt + swz(krow, 4 * half + (lane >> 3)), b0, b1, b2, b3);
+                    mma16816(s[nt], qa[2 * half], b0, b1);
+                    mma16816(s[nt], qa[2 * half + 1], b2, b3);
+                }
+            }
+            // ---- mask keys beyond the chunk; log2-domain logits
+            float x[2][4];
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int key = key0 + 8 * nt + 2 * tq + (e & 1);
+                    x[nt][e] = key < kend ? s[nt][e] * C : -INFINITY;
+                }
+            // ---- online softmax, row gr (elements 0,1) and row gr+8 (elements 2,3)
+            float mx_a = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
+            mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 1));
+            mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 2));
+            const float mn_a = fmaxf(m_a, mx_a);
+            const float al_a = (m_a == -INFINITY) ? 0.f : ex2(m_a - mn_a);
+            const float sub_a = (mn_a == -INFINITY) ? 0.f : mn_a;
+            m_a = mn_a;
+            float pv[2][4];
+            pv[0][0] = ex2(x[0][0] - sub_a);
+            pv[0][1] = ex2(x[0][1] - sub_a);
+            pv[1][0] = ex2(x[1][0] - sub_a);
+            pv[1][1] = ex2(x[1][1] - sub_a);
+            l_a = l_a * al_a + (pv[0][0] + pv[0][1]) + (pv[1][0] + pv[1][1]);
+            float al_b = 1.f;
+            if (kRows16) {
+                float mx_b = fmaxf(fmaxf(x[0][2], x[0][3]), fmaxf(x[1][2], x[1][3]));
+                mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 1));
+                mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 2));
+                const float mn_b = fmaxf(m_b, mx_b);
+                al_b = (m_b == -INFINITY) ? 0.f : ex2(m_b - mn_b);
+                const float sub_b = (mn_b == -INFINITY) ? 0.f : mn_b;
+                m_b = mn_b;
+                pv[0][2] = ex2(x[0][2] - sub_b);
+                pv[0][3] = ex2(x[0][3] - sub_b);
+                pv[1][2] = ex2(x[1][2] - sub_b);
+                pv[1][3] = ex2(x[1][3] - sub_b);
+                l_b = l_b * al_b + (pv[0][2] + pv[0][3]) + (pv[1][2] + pv[1][3]);
+            } else {
+                pv[0][2] = pv[0][3] = pv[1][2] = pv[1][3] = 0.f;
+            }
+#pragma unroll
+            for (int jn = 0; jn < 8; ++jn) {
+                o[jn][0] *= al_a;
+                o[jn][1] *= al_a;
+                o[jn][2] *= al_b;
+                o[jn][3] *= al_b;
+            }
+            // ---- O += P V: P from the score accumulators, V via transposing ldmatrix
+            uint32_t pa[4];
+            pa[0] = pack_bf16x2(pv[0][0], pv[0][1]);
+            pa[1] = pack_bf16x2(pv[0][2], pv[0][3]);
+            pa[2] = pack_bf16x2(pv[1][0], pv[1][1]);
+            pa[3] = pack_bf16x2(pv[1][2], pv[1][3]);
+            // rows of V past the chunk are zeroed in the operand (cache rows
+            // beyond the sequence may hold anything)
+            const bool tail = __any_sync(0xffffffffu, key0 + 15 >= kend);
+            const int vrow = 16 * w + ((lane >> 3) & 1) * 8 + (lane & 7);
+#pragma unroll
+            for (int jn = 0; jn < 8; jn += 2) {
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4_t(vt + swz(vrow, jn + (lane >> 4)), b0, b1, b2, b3);
+                if (tail) {
+                    // b0/b2: keys 2tq, 2tq+1 of the slice; b1/b3: keys 8 + 2tq, 8 + 2tq + 1
+                    const int k0 = key0 + 2 * tq, k8 = k0 + 8;
+                    const uint32_t m0 = (k0 < kend ? 0x0000FFFFu : 0u) | (k0 + 1 < kend ? 0xFFFF0000u : 0u);
+                    const uint32_t m8 = (k8 < kend ? 0x0000FFFFu : 0u) | (k8 + 1 < kend ? 0xFFFF0000u : 0u);
+                    b0 &= m0;
+                    b2 &= m0;
+                    b1 &= m8;
+                    b3 &= m8;
+                }
+                mma16816(o[jn], pa, b0, b1);
+                mma16816(o[jn + 1], pa, b2, b3);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[st]);
+        }
+        // row sums over the 4 lanes of a fragment row
+        l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
+        l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
+        l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
+        l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
+    }
+
+    // ---- combine the four consumer warps (ring buffers are idle now)
+    __syncthreads();
+    if (*abort_flag) return;
+    float *red = reinterpret_cast<float *>(smem);  // [4 warps][16 rows][66]: o[64], m, l
+    if (warp > 0) {
+        const int w = warp - 1, gr = lane >> 2, tq = lane & 3;
+        float *ra = red + ((size_t)w * 16 + gr) * 66;
+        float *rb = red + ((size_t)w * 16 + gr + 8) * 66;
+#pragma unroll
+        for (int jn = 0; jn < 8; ++jn) {
+            ra[8 * jn + 2 * tq] = o[jn][0];
+            ra[8 * jn + 2 * tq + 1] = o[jn][1];
+            rb[8 * jn + 2 * tq] = o[jn][2];
+            rb[8 * jn + 2 * tq + 1] = o[jn][3];
+        }
+        if (tq == 0) {
+            ra[64] = m_a;
+            ra[65] = l_a;
+            rb[64] = m_b;
+            rb[65] = l_b;
+        }
+    }
+    __syncthreads();
+    const int rows = kRows16 ? 16 : 8;
+    for (int e = threadIdx.x; e < rows * kD; e += kThreads) {
+        const int r = e / kD, d = e % kD;
+        if (r >= p.G) continue;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) M = fmaxf(M, red[((size_t)w * 16 + r) * 66 + 64]);
+        float L = 0.f, O = 0.f;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            const float *rr = red + ((size_t)w * 16 + r) * 66;
+            const float f = (rr[64] == -INFINITY) ? 0.f : ex2(rr[64] - M);
+            L += f * rr[65];
+            O += f * rr[d];
+        }
+        const int h = g * p.G + r;
+        if (nsplit == 1) {
+            // the only split of this sequence: the sink joins here, once
+            const float sk = p.sinks[h] * kLog2e;
+            const float M2 = fmaxf(M, sk);
+            const float fo = (M == -INFINITY) ? 0.f : ex2(M - M2);
+            const float fs = (sk == -INFINITY) ? 0.f : ex2(sk - M2);
+            const float Lt = L * fo + fs;
+            const float inv = Lt > 0.f ? 1.f / Lt : 0.f;
+            p.out[((size_t)b * p.Hq + h) * kD + d] = __float2bfloat16_rn(O * fo * inv);
+            if (d == 0) p.lse[(size_t)b * p.Hq + h] = Lt > 0.f ? (M2 + log2f(Lt)) * kLn2 : -INFINITY;
+        } else {
+            const size_t slot = ((size_t)b * p.Hq + h) * p.splits + c;
+            p.ws_o[slot * kD + d] = O;
+            if (d == 0) {
+                p.ws_ml[slot * 2 + 0] = M;
+                p.ws_ml[slot * 2 + 1] = L;
+            }
+        }
+    }
+}
+
+}  // namespace
+
+bool decode_bf16_supported(const DecodeShape &s)
+{
+    const int G = s.Hq / s.Hkv;
+    return s.D == kD && G >= 1 && G <= 16 && s.Hq % s.Hkv == 0 && s.splits <= 65535 && s.Hkv <= 65535 &&
+           s.B <= 65535;
+}
+
+cudaError_t launch_decode_bf16(const void *q, const void *kc, const void *vc, const int *seqlens,
+                               const float *sinks, void *out, float *lse, const DecodeShape &s, float *ws_o,
+                               float *ws_ml, cudaStream_t st)
+{
+    DecodeParams p;
+    p.B = s.B;
+    p.Lmax = s.Lmax;
+    p.Hq = s.Hq;
+    p.Hkv = s.Hkv;
+    p.G = s.Hq / s.Hkv;
+    p.window = s.window;
+    p.splits = s.splits;
+    p.chunk = s.chunk;
+    p.c_log2 = s.scale * kLog2e;
+    p.q = static_cast<const __nv_bfloat16 *>(q);
+    p.seqlens = seqlens;
+    p.sinks = sinks;
+    p.out = static_cast<__nv_bfloat16 *>(out);
+    p.lse = lse;
+    p.ws_o = ws_o;
+    p.ws_ml = ws_ml;
+    p.status = device_status_ptr();
+    p.timeout_ns = wait_timeout_ns();
+    alignas(64) CUtensorMap mk, mv;
+    const uint64_t dims[4] = {(uint64_t)kD, (uint64_t)s.Hkv, (uint64_t)s.Lmax, (uint64_t)s.B};
+    const uint64_t strides[3] = {(uint64_t)kD * 2, (uint64_t)s.Hkv * kD * 2, (uint64_t)s.Lmax * s.Hkv * kD * 2};
+    const uint32_t box[4] = {(uint32_t)kD, 1u, (uint32_t)kT, 1u};
+    if (!encode_tensor_map_4d(&mk, const_cast<void *>(kc), 2, dims, strides, box, true) ||
+        !encode_tensor_map_4d(&mv, const_cast<void *>(vc), 2, dims, strides, box, true))
+        return cudaErrorInvalidValue;
+    const dim3 grid(s.splits, s.Hkv, s.B);
+    cudaError_t e;
+    if (p.G > 8) {
+        e = cudaFuncSetAttribute(decode_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        if (e != cudaSuccess) return e;
+        decode_tc_kernel<true><<<grid, kThreads, kSmemBytes, st>>>(mk, mv, p);
+    } else {
+        e = cudaFuncSetAttribute(decode_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        if (e != cudaSuccess) return e;
+        decode_tc_kernel<false><<<grid, kThreads, kSmemBytes, st>>>(mk, mv, p);
+    }
+    return cudaGetLastError();
+}
+
 }  // namespace attn_sink

@@ -49,6 +49,11 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
+// Tile configurations (keys per tile BN, K/V stages NS, EMU = which pair of
+// every 4 uses the FMA-pipe exp2, -1 for none), chosen per layer type from
+// measurements on the gpt-oss-20b prefill: the dense causal layer runs best
+// with BN = 96 and a quarter of the exponentials off the MUFU unit, the
+// window-128 layer with BN = 64 and all exponentials on MUFU.
 template <int BN, int NS>
 struct FwdCfg {
     static constexpr int kQBytes = kM * kD * 2;
@@ -61,9 +66,12 @@ struct FwdCfg {
     // s_full[2], p_full[2], o_done, o_free, drain
     static constexpr int kNumBar = 4 + 4 * NS + 4 + 3;
     static constexpr int kOffMisc = kOffBar + kNumBar * 8;
-    static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + slack for 1024-byte alignment
     static constexpr int kTmemCols = (2 * BN + kD <= 256) ? 256 : 512;
     static constexpr int kCtasPerSm = kTmemCols == 256 ? 2 : 1;
+    // + slack for 1024-byte alignment; a CTA that takes all 512 TMEM columns
+    // also takes enough shared memory that no second CTA lands on its SM
+    static constexpr int kSmemUsed = kOffMisc + 16 + 1024;
+    static constexpr int kSmemBytes = (kCtasPerSm == 1 && kSmemUsed < 116 * 1024) ? 116 * 1024 : kSmemUsed;
     static constexpr int kTmS0 = 0;
     static constexpr int kTmO = 2 * BN;
 };
@@ -112,7 +120,7 @@ __device__ __forceinline__ bool wait_noabort(uint64_t *bar, uint32_t parity, uns
     return mbar_wait(bar, parity, &never, status, tmo);
 }
 
-template <int BN, int NS>
+template <int BN, int NS, int EMU>
 __global__ void __launch_bounds__(192, FwdCfg<BN, NS>::kCtasPerSm)
     fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdTcParams p)
@@ -322,17 +330,24 @@ __global__ void __launch_bounds__(192, FwdCfg<BN, NS>::kCtasPerSm)
                 // visible columns of this tile: c in [c_lo, c_hi] (32-bit, tile-relative)
                 const int c_hi = (int)max(-1L, min((long)BN - 1, vis_hi - j0));
                 const int c_lo = (int)max(0L, min((long)BN, vis_lo - j0));
-                if (__any_sync(0xffffffffu, c_lo > 0 || c_hi < BN - 1)) {
+                const bool need_mask = __any_sync(0xffffffffu, c_lo > 0 || c_hi < BN - 1);
+                if (need_mask) {
 #pragma unroll
                     for (int c = 0; c < BN; ++c) sv[c] = (c >= c_lo && c <= c_hi) ? sv[c] : -INFINITY;
                 }
+                // row max: four independent chains of 3-input max over columns
+                // 0-3 | 4..BN-1 in steps of 8 | the remaining 4 when (BN - 4) % 8 == 4
+                static_assert(BN % 32 == 0, "BN must be a multiple of 32");
                 float mx[4];
 #pragma unroll
-                for (int k = 0; k < 4; ++k) mx[k] = fmax3(sv[k], sv[k + 4], sv[k + 8]);
+                for (int k = 0; k < 4; ++k) mx[k] = sv[k];
+                constexpr int kFull = 4 + ((BN - 4) / 8) * 8;
 #pragma unroll
-                for (int c = 12; c < BN; c += 8)
+                for (int c = 4; c < kFull; c += 8)
 #pragma unroll
                     for (int k = 0; k < 4; ++k) mx[k] = fmax3(mx[k], sv[c + k], sv[c + 4 + k]);
+#pragma unroll
+                for (int k = 0; k < 4 && kFull + k < BN; ++k) mx[k] = fmaxf(mx[k], sv[kFull + k]);
                 const float tmax = fmax3(mx[0], mx[1], fmaxf(mx[2], mx[3]));
                 const float m_new = fmaxf(m, tmax * C);
                 const bool rescale = m_new > m + kRescaleThreshold;
@@ -342,18 +357,36 @@ __global__ void __launch_bounds__(192, FwdCfg<BN, NS>::kCtasPerSm)
                 const float2 C2 = make_float2(C, C), M2 = make_float2(neg_m, neg_m);
                 float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
                 // P (bf16 pairs) overwrites the first BN/2 columns of this S
-                // buffer, which has been read in full already; 32 scores per store.
+                // buffer, which has been read in full already; 32 scores per
+                // store.  On tiles with no masked element, pair EMU of every 4
+                // runs on the FMA pipe (fast_exp2x2) to offload the MUFU unit
+                // (two separate loops, so each element takes one path only).
+                if (!need_mask) {
 #pragma unroll
-                for (int c = 0; c < BN / 32; ++c) {
-                    uint32_t pk[16];
+                    for (int c = 0; c < BN / 32; ++c) {
+                        uint32_t pk[16];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const float2 x = ffma2(make_float2(sv[32 * c + 2 * e], sv[32 * c + 2 * e + 1]), C2, M2);
-                        const float2 pe = make_float2(ex2(x.x), ex2(x.y));
-                        acc[e & 1] = fadd2(acc[e & 1], pe);
-                        pk[e] = pack_bf16x2(pe.x, pe.y);
+                        for (int e = 0; e < 16; ++e) {
+                            const float2 x = ffma2(make_float2(sv[32 * c + 2 * e], sv[32 * c + 2 * e + 1]), C2, M2);
+                            const float2 pe = ((e & 3) == EMU) ? fast_exp2x2(x) : make_float2(ex2(x.x), ex2(x.y));
+                            acc[e & 1] = fadd2(acc[e & 1], pe);
+                            pk[e] = pack_bf16x2(pe.x, pe.y);
+                        }
+                        tmem_st16(trow + Cfg::kTmS0 + sb * BN + c * 16, pk);
                     }
-                    tmem_st16(trow + Cfg::kTmS0 + sb * BN + c * 16, pk);
+                } else {
+#pragma unroll
+                    for (int c = 0; c < BN / 32; ++c) {
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) {
+                            const float2 x = ffma2(make_float2(sv[32 * c + 2 * e], sv[32 * c + 2 * e + 1]), C2, M2);
+                            const float2 pe = make_float2(ex2(x.x), ex2(x.y));
+                            acc[e & 1] = fadd2(acc[e & 1], pe);
+                            pk[e] = pack_bf16x2(pe.x, pe.y);
+                        }
+                        tmem_st16(trow + Cfg::kTmS0 + sb * BN + c * 16, pk);
+                    }
                 }
                 l = l * alpha + ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y));
                 if (jt > 0) {
@@ -427,7 +460,7 @@ __global__ void __launch_bounds__(192, FwdCfg<BN, NS>::kCtasPerSm)
     }
 }
 
-template <int BN, int NS>
+template <int BN, int NS, int EMU>
 cudaError_t launch_cfg(const void *q, const void *k, const void *v, const float *sinks, void *out, float *lse,
                        const AttnShape &s, cudaStream_t st)
 {
@@ -473,7 +506,7 @@ cudaError_t launch_cfg(const void *q, const void *k, const void *v, const float 
         if (!encode_tensor_map_4d(&mv, const_cast<void *>(v), 2, dims, strides, box, true))
             return cudaErrorInvalidValue;
     }
-    auto kern = fwd_tc_kernel<BN, NS>;
+    auto kern = fwd_tc_kernel<BN, NS, EMU>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 0;
@@ -496,7 +529,8 @@ bool fwd_tc_supported(const AttnShape &s)
 cudaError_t launch_fwd_tc(const void *q, const void *k, const void *v, const float *sinks, void *out,
                           float *lse, const AttnShape &s, cudaStream_t st)
 {
-    return launch_cfg<64, 4>(q, k, v, sinks, out, lse, s, st);
+    if (s.window > 0 && s.window <= 1024) return launch_cfg<64, 4, -1>(q, k, v, sinks, out, lse, s, st);
+    return launch_cfg<96, 3, 3>(q, k, v, sinks, out, lse, s, st);
 }
 
 }  // namespace attn_sink

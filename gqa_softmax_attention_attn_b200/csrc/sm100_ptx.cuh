@@ -63,7 +63,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
 // Bounded wait for the phase with the given parity.  Gives up (returning
 // false) when *abort becomes non-zero or after timeout_ns; on a timeout it
 // raises the CTA's abort flag and the device status word so that every other
-// role of the CTA winds down too.
+// role of the CTA winds down too.  (A suspend-time hint on try_wait was
+// measured slower here: the woken thread resumes late.)
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
                                           unsigned *status, long long timeout_ns)
 {
@@ -263,6 +264,37 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b)
         : "=l"(*reinterpret_cast<unsigned long long *>(&d))
         : "l"(*reinterpret_cast<unsigned long long *>(&a)), "l"(*reinterpret_cast<unsigned long long *>(&b)));
     return d;
+}
+
+__device__ __forceinline__ float2 fsub2(float2 a, float2 b)
+{
+    float2 d;
+    asm("sub.rn.f32x2 %0, %1, %2;"
+        : "=l"(*reinterpret_cast<unsigned long long *>(&d))
+        : "l"(*reinterpret_cast<unsigned long long *>(&a)), "l"(*reinterpret_cast<unsigned long long *>(&b)));
+    return d;
+}
+
+// 2^x for two lanes on the FMA pipe, leaving the MUFU unit free.  Range
+// reduction x = n + f with n = round(x) (adding 1.5 * 2^23 rounds to an
+// integer in fp32) and |f| <= 1/2; 2^f by the degree-3 minimax polynomial
+// for relative error on [-1/2, 1/2] (coefficients from exp2_poly.py, max
+// relative error 7.5e-5); n enters the exponent field by an integer add of
+// n << 23, which is the bit pattern of the rounded value shifted by 23.
+// Valid for x in [-126, 126]; x below -126 is clamped (2^-126 ~ 1.2e-38),
+// so callers must not rely on it for exact zeros.
+__device__ __forceinline__ float2 fast_exp2x2(float2 x)
+{
+    x.x = fmaxf(x.x, -126.f);
+    x.y = fmaxf(x.y, -126.f);
+    const float2 magic = make_float2(12582912.f, 12582912.f);
+    const float2 t = fadd2(x, magic);
+    const float2 f = fsub2(x, fsub2(t, magic));
+    float2 q = ffma2(f, make_float2(0.05517167f, 0.05517167f), make_float2(0.24261113f, 0.24261113f));
+    q = ffma2(q, f, make_float2(0.69326097f, 0.69326097f));
+    q = ffma2(q, f, make_float2(0.99992806f, 0.99992806f));
+    return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
+                       __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
 }
 
 __device__ __forceinline__ float ex2(float x)

@@ -161,9 +161,10 @@ bool encode_tensor_map_4d(void *map, void *gaddr, int elem_bytes, const uint64_t
         else
             cudaGetLastError();
     });
-    if (!g_encode || elem_bytes != 2) return false;
+    if (!g_encode || (elem_bytes != 2 && elem_bytes != 4)) return false;
     const cuuint32_t estr[4] = {1, 1, 1, 1};
-    const CUresult r = g_encode(static_cast<CUtensorMap *>(map), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, gaddr,
+    const CUtensorMapDataType dt = elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    const CUresult r = g_encode(static_cast<CUtensorMap *>(map), dt, 4, gaddr,
                                 reinterpret_cast<const cuuint64_t *>(dims),
                                 reinterpret_cast<const cuuint64_t *>(strides_bytes),
                                 reinterpret_cast<const cuuint32_t *>(box), estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -274,11 +275,20 @@ int attn_sink_decode(const void *q, const void *k_cache, const void *v_cache, co
     return launch_status(e);
 }
 
+namespace {
+// bf16 backward workspace: [D_i][dsink terms] (as the exact path) + fp32 dQ accumulator
+size_t bwd_ws_bytes(const AttnShape &s, int dtype)
+{
+    const size_t base = (bwd_simt_workspace_bytes(s) + 255) / 256 * 256;
+    return dtype == ATTN_SINK_DTYPE_F32 ? bwd_simt_workspace_bytes(s) : base + bwd_tc_dq_acc_bytes(s);
+}
+}  // namespace
+
 size_t attn_sink_bwd_workspace_size(int B, int Lq, int Lk, int Hq, int Hkv, int D, int dtype)
 {
     if (check_common(B, Lq, Lk, Hq, Hkv, D, dtype) != ATTN_SINK_OK) return 0;
     AttnShape s{B, Lq, Lk, Hq, Hkv, D, 0, 1.f};
-    return bwd_simt_workspace_bytes(s);
+    return bwd_ws_bytes(s, dtype);
 }
 
 int attn_sink_bwd(const void *q, const void *k, const void *v, const float *sinks, const void *out,
@@ -294,7 +304,7 @@ int attn_sink_bwd(const void *q, const void *k, const void *v, const float *sink
     for (const void *p : ptrs)
         if (!aligned16(p)) return ATTN_SINK_ERR_MISALIGNED;
     AttnShape s{B, Lq, Lk, Hq, Hkv, D, window, scale};
-    const size_t need = bwd_simt_workspace_bytes(s);
+    const size_t need = bwd_ws_bytes(s, dtype);
     if (!workspace || ws_bytes < need) return ATTN_SINK_ERR_WORKSPACE;
     if (!aligned16(workspace)) return ATTN_SINK_ERR_MISALIGNED;
     rc = ensure_device();
@@ -306,10 +316,17 @@ int attn_sink_bwd(const void *q, const void *k, const void *v, const float *sink
             static_cast<const float *>(out), static_cast<const float *>(dout), lse, static_cast<float *>(dq),
             static_cast<float *>(dk), static_cast<float *>(dv), dsinks, s, workspace, st));
     using bf = __nv_bfloat16;
-    return launch_status(launch_bwd_simt<bf>(
-        static_cast<const bf *>(q), static_cast<const bf *>(k), static_cast<const bf *>(v), sinks,
-        static_cast<const bf *>(out), static_cast<const bf *>(dout), lse, static_cast<bf *>(dq),
-        static_cast<bf *>(dk), static_cast<bf *>(dv), dsinks, s, workspace, st));
+    if (!bwd_tc_supported(s)) return ATTN_SINK_ERR_UNSUPPORTED;
+    const size_t rows = (size_t)B * Hq * Lq;
+    float *Drow = static_cast<float *>(workspace);
+    float *terms = Drow + rows;
+    float *dq_acc = reinterpret_cast<float *>(static_cast<char *>(workspace) +
+                                              (bwd_simt_workspace_bytes(s) + 255) / 256 * 256);
+    cudaError_t e = launch_bwd_rows<bf>(static_cast<const bf *>(out), static_cast<const bf *>(dout), lse, sinks, Drow,
+                                        terms, s, st);
+    if (e == cudaSuccess) e = launch_bwd_tc(q, k, v, dout, lse, Drow, dq_acc, dq, dk, dv, s, st);
+    if (e == cudaSuccess) e = launch_dsink_reduce(terms, dsinks, s, st);
+    return launch_status(e);
 }
 
 int attn_sink_get_device_status(void *stream)

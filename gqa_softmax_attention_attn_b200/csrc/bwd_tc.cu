@@ -1,0 +1,510 @@
+// bwd_tc.cu -- bf16 backward of sink-softmax GQA attention on the sm_100a
+// tensor cores (tcgen05 / TMEM / TMA).
+//
+// What it computes (derived from the forward's definition -- "GPT-OSS on
+// day 0", section "Sink Attention": the sink is one more logit with no value
+// row, so it adds nothing to dK, dV or dQ beyond its share of the softmax
+// denominator, which the saved log-sum-exp already carries):
+//   P_ij  = exp(s_ij - lse_i)            (lse includes the sink)
+//   dS_ij = P_ij (<dO_i, v_j> - D_i),    D_i = <dO_i, O_i>
+//   dV_j += P_ij dO_i,  dK_j += scale dS_ij q_i,  dQ_i += scale dS_ij k_j
+// D_i and dsink are produced by the row kernel in simt_kernels.cu.
+//
+// Design (B200), one CTA per (128-key tile, KV head g, batch b):
+//  * K and V of the tile stay in shared memory; the CTA walks every q tile
+//    (128 rows = positions x query heads of the group, as in the forward)
+//    that can see a key of the tile.  Q and dO tiles stream in by TMA (two
+//    stages); lse and D for the tile's 128 rows go to shared memory.
+//  * Warp 1 issues, from one thread: S^T = K Q^T and dP^T = V dO^T (keys as
+//    the M dimension, so a thread of the softmax-gradient warps owns a key
+//    row); then dV += P^T dO and dK += dS^T Q with P^T and dS^T read back
+//    from tensor memory; then dQ = dS K with dS from shared memory (written
+//    there in the MN-major layout by the same threads) into one of two TMEM
+//    buffers.
+//  * Warps 2-5 (one key row per thread): P and dS in fp32 from the two TMEM
+//    tiles, written back as bf16 (TMEM and shared memory).
+//  * Warps 6-9 move each dQ tile from TMEM to shared memory and add it into an
+//    fp32 dQ accumulator in global memory with a TMA reduce-add (L2 atomics;
+//    the summation order over key tiles is not fixed).  dK and dV of the tile
+//    are written once, at the end (deterministic).
+//  * Every wait is bounded; on expiry the CTA raises the device status bit,
+//    drains its own TMA and MMA work, frees tensor memory and exits.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include "kernels.h"
+#include "sm100_ptx.cuh"
+
+namespace attn_sink {
+namespace {
+
+constexpr int kM = 128;  // keys per tile (rows of the transposed score tile)
+constexpr int kD = 64;
+constexpr int kThreads = 320;
+constexpr float kLog2e = 1.4426950408889634f;
+
+constexpr int kTile = kM * kD * 2;  // 16 KB bf16 tile
+constexpr int kOffK = 0;
+constexpr int kOffV = kOffK + kTile;
+constexpr int kOffQ = kOffV + kTile;       // 2 stages
+constexpr int kOffDO = kOffQ + 2 * kTile;  // 2 stages
+constexpr int kOffDS = kOffDO + 2 * kTile;  // dS, MN-major: two 64-row atoms of 16 KB
+constexpr int kOffStg = kOffDS + 2 * kTile;  // fp32 dQ staging [128][64]
+constexpr int kOffLD = kOffStg + 128 * 64 * 4;  // [2 stages][lse2 | D][128] fp32
+constexpr int kOffBar = kOffLD + 2 * 2 * 128 * 4;
+// kv_full, qdo_full[2], qdo_empty[2], s_full, p_ready, ds_free, dq_full[2],
+// dq_free[2], stg_full, stg_free, dkv_done, drain
+constexpr int kNumBar = 16;
+constexpr int kOffMisc = kOffBar + kNumBar * 8;
+constexpr int kSmemBytes = kOffMisc + 16 + 1024;
+// TMEM columns
+constexpr int kTmST = 0, kTmDPT = 128, kTmDV = 256, kTmDK = 320, kTmDQ = 384;
+
+struct BwdParams {
+    int B, Lq, Lk, Hq, Hkv, window, G;
+    int P, n_htiles;  // positions per q tile, head tiles per group
+    float c_log2, scale;
+    const float *lse, *Drow;
+    __nv_bfloat16 *dk, *dv;
+    unsigned *status;
+    long long timeout_ns;
+};
+
+__device__ __forceinline__ bool wait_noabort(uint64_t *bar, uint32_t parity, unsigned *status, long long tmo)
+{
+    int never = 0;
+    return mbar_wait(bar, parity, &never, status, tmo);
+}
+
+template <int GP>  // query heads packed per q tile
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
+                  const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                  const __grid_constant__ CUtensorMap tmDQ, const BwdParams p)
+{
+    constexpr int P = kM / GP;  // positions per q tile
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
+    uint64_t *kv_full = bars + 0;
+    uint64_t *qdo_full = bars + 1;   // [2]
+    uint64_t *qdo_empty = bars + 3;  // [2]
+    uint64_t *s_full = bars + 5;
+    uint64_t *p_ready = bars + 6;
+    uint64_t *ds_free = bars + 7;
+    uint64_t *dq_full = bars + 8;    // [2]
+    uint64_t *dq_free = bars + 10;   // [2]
+    uint64_t *stg_full = bars + 12;
+    uint64_t *stg_free = bars + 13;
+    uint64_t *dkv_done = bars + 14;
+    uint64_t *drain = bars + 15;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffMisc);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffMisc + 4);
+    float *ld = reinterpret_cast<float *>(smem + kOffLD);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int kt = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+    const int k0 = kt * kM;
+    const long off = (long)p.Lk - p.Lq;
+    // query positions whose rows can see a key of [k0, k0 + 128)
+    const long pos_lo = max(0L, (long)k0 - off);
+    long pos_hi = (long)p.Lq - 1;
+    if (p.window > 0) pos_hi = min(pos_hi, (long)k0 + kM - 1 + p.window - 1 - off);
+    const int n_q = pos_hi >= pos_lo ? (int)(pos_hi / P - pos_lo / P + 1) : 0;
+    const int qt_lo = (int)(pos_lo / P);
+    const int n_iter = n_q * p.n_htiles;
+
+    if (threadIdx.x == 0) {
+        mbar_init(kv_full, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&qdo_full[s], 2);
+            mbar_init(&qdo_empty[s], 1);
+            mbar_init(&dq_full[s], 1);
+            mbar_init(&dq_free[s], 128);
+        }
+        mbar_init(s_full, 1);
+        mbar_init(p_ready, 128);
+        mbar_init(ds_free, 1);
+        mbar_init(stg_full, 128);
+        mbar_init(stg_free, 1);
+        mbar_init(dkv_done, 1);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    auto iter_head = [&](int i, int &h0, int &pos0) {
+        const int ht = i / n_q, qt = qt_lo + i % n_q;
+        h0 = g * p.G + ht * GP;
+        pos0 = qt * P;
+    };
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ loads
+        uint32_t issued_qdo[2] = {0, 0};
+        bool ok = true;
+        if (lane == 0 && n_iter > 0) {
+            tma_prefetch_desc(&tmQ);
+            tma_prefetch_desc(&tmDO);
+            mbar_arrive_expect_tx(kv_full, 2 * kTile);
+            tma_load_4d(smem + kOffK, &tmK, 0, g, k0, b, kv_full);
+            tma_load_4d(smem + kOffV, &tmV, 0, g, k0, b, kv_full);
+        }
+        for (int i = 0; i < n_iter && ok; ++i) {
+            const int st = i & 1;
+            int h0, pos0;
+            iter_head(i, h0, pos0);
+            if (lane == 0) {
+                ok = mbar_wait(&qdo_empty[st], ((i >> 1) & 1u) ^ 1u, abort_flag, p.status, p.timeout_ns);
+                if (ok) {
+                    mbar_arrive_expect_tx(&qdo_full[st], 2 * kTile);
+                    tma_load_4d(smem + kOffQ + st * kTile, &tmQ, 0, h0, pos0, b, &qdo_full[st]);
+                    tma_load_4d(smem + kOffDO + st * kTile, &tmDO, 0, h0, pos0, b, &qdo_full[st]);
+                    ++issued_qdo[st];
+                }
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            // log2-domain lse (+inf for rows that do not exist or see nothing) and D
+            for (int c = lane; c < kM; c += 32) {
+                const int pos = pos0 + c / GP, h = h0 + c % GP;
+                float l2 = INFINITY, dd = 0.f;
+                if (pos < p.Lq) {
+                    const size_t li = ((size_t)b * p.Hq + h) * p.Lq + pos;
+                    const float L = p.lse[li];
+                    l2 = (L == -INFINITY) ? INFINITY : L * kLog2e;
+                    dd = p.Drow[li];
+                }
+                ld[(st * 2 + 0) * kM + c] = l2;
+                ld[(st * 2 + 1) * kM + c] = dd;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&qdo_full[st]);
+        }
+        if (lane == 0) {
+            if (n_iter > 0) wait_noabort(kv_full, 0, p.status, p.timeout_ns);
+            for (int s = 0; s < 2; ++s)
+                if (issued_qdo[s]) wait_noabort(&qdo_full[s], (issued_qdo[s] - 1) & 1u, p.status, p.timeout_ns);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issue
+        if (lane == 0) {
+            const uint32_t id_t = idesc_bf16_f32(kM, kM, 0, 0);       // S^T, dP^T: N = 128 q rows
+            const uint32_t id_kv = idesc_bf16_f32(kM, kD, 1, 0);      // dV, dK: B MN-major
+            const uint32_t id_q = idesc_bf16_f32(kM, kD, 1, 1);       // dQ: A and B MN-major
+            const uint64_t d_k = smem_desc_sw128(smem_u32(smem + kOffK), 16, 1024);
+            const uint64_t d_v = smem_desc_sw128(smem_u32(smem + kOffV), 16, 1024);
+            const uint64_t d_q = smem_desc_sw128(smem_u32(smem + kOffQ), 16, 1024);
+            const uint64_t d_do = smem_desc_sw128(smem_u32(smem + kOffDO), 16, 1024);
+            const uint64_t d_ds = smem_desc_sw128(smem_u32(smem + kOffDS), kTile, 1024);
+            const uint64_t d_kmn = smem_desc_sw128(smem_u32(smem + kOffK), kTile, 1024);
+            bool ok = n_iter > 0 && mbar_wait(kv_full, 0, abort_flag, p.status, p.timeout_ns);
+            for (int i = 0; i < n_iter && ok; ++i) {
+                const int st = i & 1, db = i & 1;
+                if (!mbar_wait(&qdo_full[st], (i >> 1) & 1u, abort_flag, p.status, p.timeout_ns)) break;
+                tc_fence_after();
+                const uint64_t q_st = d_q + (uint64_t)((st * kTile) >> 4);
+                const uint64_t do_st = d_do + (uint64_t)((st * kTile) >> 4);
+#pragma unroll
+                for (int kk = 0; kk < kD / 16; ++kk) mma_ss(tmem + kTmST, d_k + 2 * kk, q_st + 2 * kk, id_t, kk > 0);
+#pragma unroll
+                for (int kk = 0; kk < kD / 16; ++kk)
+                    mma_ss(tmem + kTmDPT, d_v + 2 * kk, do_st + 2 * kk, id_t, kk > 0);
+                mma_commit(s_full);
+                if (!mbar_wait(p_ready, i & 1u, abort_flag, p.status, p.timeout_ns)) break;
+                tc_fence_after();
+                // dV += P^T dO and dK += dS^T Q: K = 128 q rows in steps of 16 (2048 bytes of the MN-major B)
+#pragma unroll
+                for (int kk = 0; kk < kM / 16; ++kk)
+                    mma_ts(tmem + kTmDV, tmem + kTmST + kk * 8, do_st + 128 * kk, id_kv, (i > 0 || kk > 0));
+#pragma unroll
+                for (int kk = 0; kk < kM / 16; ++kk)
+                    mma_ts(tmem + kTmDK, tmem + kTmDPT + kk * 8, q_st + 128 * kk, id_kv, (i > 0 || kk > 0));
+                mma_commit(&qdo_empty[st]);
+                if (!mbar_wait(&dq_free[db], ((i >> 1) & 1u) ^ 1u, abort_flag, p.status, p.timeout_ns)) break;
+                tc_fence_after();
+                // dQ = dS K: K = 128 keys in steps of 16
+#pragma unroll
+                for (int kk = 0; kk < kM / 16; ++kk)
+                    mma_ss(tmem + kTmDQ + db * kD, d_ds + 128 * kk, d_kmn + 128 * kk, id_q, kk > 0);
+                mma_commit(&dq_full[db]);
+                mma_commit(ds_free);
+            }
+            mma_commit(dkv_done);
+            mma_commit(drain);
+            wait_noabort(drain, 0, p.status, p.timeout_ns);
+        }
+    } else if (warp <= 5) {
+        // ------------------------------------------------------------ P and dS, one key row per thread
+        const int quad = warp & 3;
+        const int r = quad * 32 + lane;
+        const int j = k0 + r;
+        const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
+        const float C = p.c_log2;
+        bool ok = true;
+        for (int i = 0; i < n_iter; ++i) {
+            const int st = i & 1;
+            int h0, pos0;
+            iter_head(i, h0, pos0);
+            if (!__all_sync(0xffffffffu,
+                            mbar_wait(&qdo_full[st], (i >> 1) & 1u, abort_flag, p.status, p.timeout_ns) &&
+                                mbar_wait(s_full, i & 1u, abort_flag, p.status, p.timeout_ns) &&
+                                (i == 0 || mbar_wait(ds_free, (i - 1) & 1u, abort_flag, p.status, p.timeout_ns)))) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            // key j is visible to column c (position pos0 + c / GP) iff
+            // pl = c / GP lies in [pl_lo, pl_hi]: j <= pos + off and, with a
+            // window, j > pos + off - window (bounds exact in 64 bits, then
+            // clamped to [-1, P])
+            const long jrel = (long)j - pos0 - off;
+            long lo_l = max(jrel, 0L);
+            long hi_l = p.window > 0 ? jrel + p.window - 1 : (long)P - 1;
+            if (j >= p.Lk) lo_l = P;  // keys past Lk see nothing
+            const int pl_lo = (int)min(lo_l, (long)P);
+            const int pl_hi = (int)max(-1L, min(hi_l, (long)P - 1));
+            const bool need_mask = __any_sync(0xffffffffu, pl_lo > 0 || pl_hi < P - 1);
+            const float *l2 = ld + (st * 2 + 0) * kM;
+            const float *dd = ld + (st * 2 + 1) * kM;
+#pragma unroll
+            for (int c = 0; c < kM / 32; ++c) {
+                uint32_t sr[32], dr[32];
+                tmem_ld32(trow + kTmST + 32 * c, sr);
+                tmem_ld32(trow + kTmDPT + 32 * c, dr);
+                tmem_wait_ld();
+                uint32_t pk[16], dk[16];
+                float dsv[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int col = 32 * c + e;
+                    float pe = ex2(fmaf(__uint_as_float(sr[e]), C, -l2[col]));
+                    if (need_mask) {
+                        const int pl = col / GP;
+                        pe = (pl >= pl_lo && pl <= pl_hi) ? pe : 0.f;
+                    }
+                    dsv[e] = pe * (__uint_as_float(dr[e]) - dd[col]);
+                    if (e & 1) {
+                        pk[e / 2] = pack_bf16x2(__uint_as_float(sr[e - 1]), pe);
+                        dk[e / 2] = pack_bf16x2(dsv[e - 1], dsv[e]);
+                    } else {
+                        sr[e] = __float_as_uint(pe);  // keep P of the even column for the pair
+                    }
+                }
+                // P^T and dS^T (bf16 pairs) over the already-read columns of their tiles
+                tmem_st16(trow + kTmST + 16 * c, pk);
+                tmem_st16(trow + kTmDPT + 16 * c, dk);
+                // dS into shared memory, MN-major: atom (col / 64), key row r, 8 q rows per 16 bytes
+#pragma unroll
+                for (int q8 = 0; q8 < 4; ++q8) {
+                    const int chunk = 4 * c + q8;  // 8-column chunk index 0..15
+                    const int atom = chunk >> 3, cc = chunk & 7;
+                    uint4 v;
+                    v.x = dk[4 * q8 + 0];
+                    v.y = dk[4 * q8 + 1];
+                    v.z = dk[4 * q8 + 2];
+                    v.w = dk[4 * q8 + 3];
+                    *reinterpret_cast<uint4 *>(smem + kOffDS + atom * kTile + r * 128 + ((cc ^ (r & 7)) << 4)) = v;
+                }
+            }
+            tmem_wait_st();
+            fence_proxy_async_smem();  // dS in shared memory is read by the tensor core next
+            tc_fence_before();
+            mbar_arrive(p_ready);
+        }
+        // ---- dK, dV of this key row
+        float kv[2][64];
+        bool have = false;
+        if (ok && n_iter > 0 &&
+            __all_sync(0xffffffffu, mbar_wait(dkv_done, 0, abort_flag, p.status, p.timeout_ns))) {
+            tc_fence_after();
+            uint32_t a[32];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                tmem_ld32(trow + kTmDV + 32 * h, a);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) kv[0][32 * h + e] = __uint_as_float(a[e]);
+                tmem_ld32(trow + kTmDK + 32 * h, a);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) kv[1][32 * h + e] = __uint_as_float(a[e]) * p.scale;
+            }
+            have = true;
+        }
+        if ((have || (n_iter == 0 && !*abort_flag)) && j < p.Lk) {
+            const size_t base = (((size_t)b * p.Lk + j) * p.Hkv + g) * kD;
+            uint4 *dv4 = reinterpret_cast<uint4 *>(p.dv + base);
+            uint4 *dk4 = reinterpret_cast<uint4 *>(p.dk + base);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                uint4 a, bb;
+                if (have) {
+                    a.x = pack_bf16x2(kv[0][8 * c + 0], kv[0][8 * c + 1]);
+                    a.y = pack_bf16x2(kv[0][8 * c + 2], kv[0][8 * c + 3]);
+                    a.z = pack_bf16x2(kv[0][8 * c + 4], kv[0][8 * c + 5]);
+                    a.w = pack_bf16x2(kv[0][8 * c + 6], kv[0][8 * c + 7]);
+                    bb.x = pack_bf16x2(kv[1][8 * c + 0], kv[1][8 * c + 1]);
+                    bb.y = pack_bf16x2(kv[1][8 * c + 2], kv[1][8 * c + 3]);
+                    bb.z = pack_bf16x2(kv[1][8 * c + 4], kv[1][8 * c + 5]);
+                    bb.w = pack_bf16x2(kv[1][8 * c + 6], kv[1][8 * c + 7]);
+                } else {
+                    a = make_uint4(0, 0, 0, 0);
+                    bb = a;
+                }
+                dv4[c] = a;
+                dk4[c] = bb;
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ dQ: TMEM -> smem -> TMA reduce-add
+        const int quad = warp & 3;
+        const int row = quad * 32 + lane;
+        const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
+        const bool issuer = (warp == 6 && lane == 0);
+        float *stg = reinterpret_cast<float *>(smem + kOffStg);
+        for (int i = 0; i < n_iter; ++i) {
+            const int db = i & 1;
+            int h0, pos0;
+            iter_head(i, h0, pos0);
+            if (!__all_sync(0xffffffffu,
+                            mbar_wait(&dq_full[db], (i >> 1) & 1u, abort_flag, p.status, p.timeout_ns)))
+                break;
+            tc_fence_after();
+            uint32_t a[2][32];
+            tmem_ld32(trow + kTmDQ + db * kD, a[0]);
+            tmem_ld32(trow + kTmDQ + db * kD + 32, a[1]);
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(&dq_free[db]);
+            if (!__all_sync(0xffffffffu, mbar_wait(stg_free, (i & 1u) ^ 1u, abort_flag, p.status, p.timeout_ns)))
+                break;
+            // row-major [128 rows][64 fp32]; chunk order rotated by lane to spread banks
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                const int ck = (k + lane) & 15;
+                float4 v;
+                v.x = __uint_as_float(a[ck / 8][(ck % 8) * 4 + 0]) * p.scale;
+                v.y = __uint_as_float(a[ck / 8][(ck % 8) * 4 + 1]) * p.scale;
+                v.z = __uint_as_float(a[ck / 8][(ck % 8) * 4 + 2]) * p.scale;
+                v.w = __uint_as_float(a[ck / 8][(ck % 8) * 4 + 3]) * p.scale;
+                *reinterpret_cast<float4 *>(stg + row * 64 + ck * 4) = v;
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(stg_full);
+            if (issuer) {
+                if (!mbar_wait(stg_full, i & 1u, abort_flag, p.status, p.timeout_ns)) break;
+                tma_reduce_add_4d(&tmDQ, stg, 0, h0, pos0, b);
+                bulk_commit_group();
+                bulk_wait_read_all();
+                mbar_arrive(stg_free);
+            }
+        }
+        if (issuer) bulk_wait_all();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+__global__ void __launch_bounds__(256) dq_convert_kernel(const float *__restrict__ acc, __nv_bfloat16 *__restrict__ dq,
+                                                         size_t n)
+{
+    const size_t i = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) * 4;
+    if (i >= n) return;
+    const float4 v = *reinterpret_cast<const float4 *>(acc + i);
+    uint2 o;
+    o.x = pack_bf16x2(v.x, v.y);
+    o.y = pack_bf16x2(v.z, v.w);
+    *reinterpret_cast<uint2 *>(dq + i) = o;
+}
+
+template <int GP>
+cudaError_t launch_gp(const CUtensorMap &mq, const CUtensorMap &mdo, const CUtensorMap &mk, const CUtensorMap &mv,
+                      const CUtensorMap &mdq, const BwdParams &p, dim3 grid, cudaStream_t st)
+{
+    cudaError_t e = cudaFuncSetAttribute(bwd_tc_kernel<GP>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    bwd_tc_kernel<GP><<<grid, kThreads, kSmemBytes, st>>>(mq, mdo, mk, mv, mdq, p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t bwd_tc_dq_acc_bytes(const AttnShape &s) { return (size_t)s.B * s.Lq * s.Hq * s.D * sizeof(float); }
+
+cudaError_t launch_bwd_tc(const void *q, const void *k, const void *v, const void *dout, const float *lse,
+                          const float *Drow, float *dq_acc, void *dq, void *dk, void *dv, const AttnShape &s,
+                          cudaStream_t st)
+{
+    BwdParams p;
+    p.B = s.B;
+    p.Lq = s.Lq;
+    p.Lk = s.Lk;
+    p.Hq = s.Hq;
+    p.Hkv = s.Hkv;
+    p.window = s.window;
+    p.G = s.Hq / s.Hkv;
+    int gp = 1;
+    while (gp * 2 <= 16 && p.G % (gp * 2) == 0) gp *= 2;
+    p.P = kM / gp;
+    p.n_htiles = p.G / gp;
+    p.c_log2 = s.scale * kLog2e;
+    p.scale = s.scale;
+    p.lse = lse;
+    p.Drow = Drow;
+    p.dk = static_cast<__nv_bfloat16 *>(dk);
+    p.dv = static_cast<__nv_bfloat16 *>(dv);
+    p.status = device_status_ptr();
+    p.timeout_ns = wait_timeout_ns();
+
+    alignas(64) CUtensorMap mq, mdo, mk, mv, mdq;
+    const uint64_t qd[4] = {(uint64_t)kD, (uint64_t)s.Hq, (uint64_t)s.Lq, (uint64_t)s.B};
+    const uint64_t qs2[3] = {(uint64_t)kD * 2, (uint64_t)s.Hq * kD * 2, (uint64_t)s.Lq * s.Hq * kD * 2};
+    const uint64_t qs4[3] = {(uint64_t)kD * 4, (uint64_t)s.Hq * kD * 4, (uint64_t)s.Lq * s.Hq * kD * 4};
+    const uint32_t qbox[4] = {(uint32_t)kD, (uint32_t)gp, (uint32_t)p.P, 1u};
+    const uint64_t kd[4] = {(uint64_t)kD, (uint64_t)s.Hkv, (uint64_t)s.Lk, (uint64_t)s.B};
+    const uint64_t ks2[3] = {(uint64_t)kD * 2, (uint64_t)s.Hkv * kD * 2, (uint64_t)s.Lk * s.Hkv * kD * 2};
+    const uint32_t kbox[4] = {(uint32_t)kD, 1u, (uint32_t)kM, 1u};
+    if (!encode_tensor_map_4d(&mq, const_cast<void *>(q), 2, qd, qs2, qbox, true) ||
+        !encode_tensor_map_4d(&mdo, const_cast<void *>(dout), 2, qd, qs2, qbox, true) ||
+        !encode_tensor_map_4d(&mk, const_cast<void *>(k), 2, kd, ks2, kbox, true) ||
+        !encode_tensor_map_4d(&mv, const_cast<void *>(v), 2, kd, ks2, kbox, true) ||
+        !encode_tensor_map_4d(&mdq, dq_acc, 4, qd, qs4, qbox, false))
+        return cudaErrorInvalidValue;
+    cudaError_t e = cudaMemsetAsync(dq_acc, 0, bwd_tc_dq_acc_bytes(s), st);
+    if (e != cudaSuccess) return e;
+    const dim3 grid((s.Lk + kM - 1) / kM, s.Hkv, s.B);
+    switch (gp) {
+    case 1: e = launch_gp<1>(mq, mdo, mk, mv, mdq, p, grid, st); break;
+    case 2: e = launch_gp<2>(mq, mdo, mk, mv, mdq, p, grid, st); break;
+    case 4: e = launch_gp<4>(mq, mdo, mk, mv, mdq, p, grid, st); break;
+    case 8: e = launch_gp<8>(mq, mdo, mk, mv, mdq, p, grid, st); break;
+    default: e = launch_gp<16>(mq, mdo, mk, mv, mdq, p, grid, st); break;
+    }
+    if (e != cudaSuccess) return e;
+    const size_t n = (size_t)s.B * s.Lq * s.Hq * s.D;
+    dq_convert_kernel<<<(unsigned)((n / 4 + 255) / 256), 256, 0, st>>>(dq_acc, static_cast<__nv_bfloat16 *>(dq), n);
+    return cudaGetLastError();
+}
+
+bool bwd_tc_supported(const AttnShape &s)
+{
+    return s.D == kD && s.Hq % s.Hkv == 0 && s.B <= 65535 && s.Hkv <= 65535;
+}
+
+}  // namespace attn_sink

@@ -503,6 +503,21 @@ cudaError_t launch_bwd_simt(const T *q, const T *k, const T *v, const float *sin
 }
 
 template <typename T>
+cudaError_t launch_bwd_rows(const T *out, const T *dout, const float *lse, const float *sinks, float *Drow,
+                            float *terms, const AttnShape &s, cudaStream_t st)
+{
+    const size_t rows = (size_t)s.B * s.Hq * s.Lq;
+    bwd_pre_kernel<T><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(out, dout, lse, sinks, Drow, terms, s);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_dsink_reduce(const float *terms, float *dsinks, const AttnShape &s, cudaStream_t st)
+{
+    dsink_reduce_kernel<<<s.Hq, 256, 0, st>>>(terms, dsinks, (long)s.B * s.Lq);
+    return cudaGetLastError();
+}
+
+template <typename T>
 cudaError_t launch_decode_simt(const T *q, const T *kc, const T *vc, const int *seqlens, const float *sinks,
                                T *out, float *lse, const DecodeShape &s, float *ws_o, float *ws_ml,
                                cudaStream_t st)
@@ -527,6 +542,8 @@ cudaError_t launch_decode_combine(const int *seqlens, const float *sinks, T *out
     template cudaError_t launch_bwd_simt<T>(const T *, const T *, const T *, const float *, const T *,        \
                                             const T *, const float *, T *, T *, T *, float *,                 \
                                             const AttnShape &, void *, cudaStream_t);                         \
+    template cudaError_t launch_bwd_rows<T>(const T *, const T *, const float *, const float *, float *, float *, \
+                                            const AttnShape &, cudaStream_t);                                 \
     template cudaError_t launch_decode_simt<T>(const T *, const T *, const T *, const int *, const float *,   \
                                                T *, float *, const DecodeShape &, float *, float *,           \
                                                cudaStream_t);                                                 \

@@ -138,12 +138,13 @@ def traffic_from_profile(kernel_file: str, profile_json: str):
 
 def run_ours(args, rank, world, dev):
     import gqa_softmax_attention_attn_b200 as attn
+    from gqa_softmax_attention_attn_b200 import multirank
 
     hbm, tf_burst, tf_sust, peak_src = peaks()
     stream = torch.cuda.current_stream(dev)
     layers = []
     for li, window in enumerate((0, WIN)):
-        d, host = make_prefill(1002 + 7919 * rank + li, dev)
+        d, host = make_prefill(multirank.rank_seed(1002 + li, rank), dev)
         d["out"] = torch.empty_like(d["q"])
         d["lse"] = torch.empty(B, HQ, L, device=dev, dtype=torch.float32)
         d["window"] = window
@@ -167,8 +168,7 @@ def run_ours(args, rank, world, dev):
     if rank == 0:
         sampler.start()
         time.sleep(0.5)
-    if world > 1:
-        torch.distributed.barrier()
+    multirank.barrier()
     torch.cuda.synchronize(dev)
     t0 = time.time()
     for i in range(K):
@@ -180,8 +180,7 @@ def run_ours(args, rank, world, dev):
         ev[i][2].record(stream)
     torch.cuda.synchronize(dev)
     t1 = time.time()
-    if world > 1:
-        torch.distributed.barrier()
+    multirank.barrier()
     if rank == 0:
         time.sleep(0.3)
         sampler.stop()
@@ -190,12 +189,10 @@ def run_ours(args, rank, world, dev):
     step_ms = sum(dense_ms) + sum(band_ms)
     status = attn.attn_sink_get_device_status(stream)
     assert status == 0, f"device status {status}"
-    t_ms = torch.tensor([step_ms, sum(dense_ms), sum(band_ms)], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(t_ms, op=torch.distributed.ReduceOp.MAX)
-    step_ms, dense_tot, band_tot = (float(x) for x in t_ms.tolist())
+    # slowest rank's device times; whole-job rate = all ranks' work over that time
+    step_ms, dense_tot, band_tot = multirank.max_over_ranks([step_ms, sum(dense_ms), sum(band_ms)], dev)
     flops_step = fwd_flops(B, L, HQ, 0) + fwd_flops(B, L, HQ, WIN)
-    value = flops_step * K * world / (step_ms * 1e-3) / 1e12
+    value = multirank.job_throughput(flops_step * K, world, step_ms * 1e-3) / 1e12
 
     # e2e through the public API with host buffers: pinned H2D of each layer's inputs, D2H of its outputs
     e2e = None
@@ -222,10 +219,8 @@ def run_ours(args, rank, world, dev):
                 h["lse"].copy_(d["lse"], non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize(dev)
-        e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-        if world > 1:
-            torch.distributed.all_reduce(e_ms, op=torch.distributed.ReduceOp.MAX)
-        e2e = {"value": flops_step * Ke * world / (float(e_ms.item()) * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e_ms = multirank.max_over_ranks([e0.elapsed_time(e1)], dev)[0]
+        e2e = {"value": multirank.job_throughput(flops_step * Ke, world, e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     dense_avg = dense_tot / K
@@ -259,28 +254,29 @@ def banded_bytes():
     return (2 * B * L * HQ * D + 2 * 2 * B * L * HKV * D + 4 * HQ + 2 * B * L * HQ * D + 4 * B * HQ * L)
 
 
-def decode_legs(dev, reps=20):
+def decode_legs(dev, reps=20, warmup=3, batch=None):
     import gqa_softmax_attention_attn_b200 as attn
     from gqa_softmax_attention_attn_b200.inputs import DECODE, SEEDS, decode_inputs
 
     hbm, _, _, _ = peaks()
     w = DECODE
-    d = decode_inputs(w.B, w.Lmax, w.Hq, w.Hkv, w.D, w.len_lo, w.len_hi, w.dtype, w.qkv_std, w.sink_std,
+    nb = batch or w.B
+    d = decode_inputs(nb, w.Lmax, w.Hq, w.Hkv, w.D, w.len_lo, w.len_hi, w.dtype, w.qkv_std, w.sink_std,
                       seed=SEEDS["decode"])
     lens = d["seqlens"].tolist()
     d = {k: v.to(dev) for k, v in d.items()}
     out = torch.empty_like(d["q"])
-    lse = torch.empty(w.B, w.Hq, device=dev, dtype=torch.float32)
+    lse = torch.empty(nb, w.Hq, device=dev, dtype=torch.float32)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     legs = {}
     for name, window in (("decode_dense", 0), ("decode_window128", WIN)):
-        nbytes = attn.attn_sink_decode_workspace_size(w.B, w.Hq, w.D, w.Lmax, window, 0)
+        nbytes = attn.attn_sink_decode_workspace_size(nb, w.Hq, w.D, w.Lmax, window, 0)
         ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
         kv_rows = sum(min(n, window) if window > 0 else n for n in lens)
-        by = kv_rows * w.Hkv * w.D * 2 * 2 + w.B * w.Hq * w.D * 2 * 2 + w.B * w.Hq * 4 + 4 * w.B
+        by = kv_rows * w.Hkv * w.D * 2 * 2 + nb * w.Hq * w.D * 2 * 2 + nb * w.Hq * 4 + 4 * nb
         times = []
-        for it in range(reps + 3):
+        for it in range(reps + warmup):
             flush.zero_()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
@@ -288,7 +284,7 @@ def decode_legs(dev, reps=20):
                                   SCALE, 0, ws, stream)
             e1.record(stream)
             torch.cuda.synchronize(dev)
-            if it >= 3:
+            if it >= warmup:
                 times.append(e0.elapsed_time(e1))
         ms = statistics.median(times)
         gbs = by / (ms * 1e-3) / 1e9
@@ -297,7 +293,7 @@ def decode_legs(dev, reps=20):
     return legs
 
 
-def bwd_legs(dev, reps=5):
+def bwd_legs(dev, reps=5, warmup=2):
     import gqa_softmax_attention_attn_b200 as attn
 
     hbm, tf_burst, _, _ = peaks()
@@ -313,14 +309,14 @@ def bwd_legs(dev, reps=5):
     for name, window in (("bwd_dense", 0), ("bwd_window128", WIN)):
         attn.attn_sink_fwd(d["q"], d["k"], d["v"], d["sinks"], out, lse, window, SCALE, stream)
         times = []
-        for it in range(reps + 2):
+        for it in range(reps + warmup):
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
             attn.attn_sink_bwd(d["q"], d["k"], d["v"], d["sinks"], out, d["dout"], lse, dq, dk, dv, ds, window,
                                SCALE, ws, stream)
             e1.record(stream)
             torch.cuda.synchronize(dev)
-            if it >= 2:
+            if it >= warmup:
                 times.append(e0.elapsed_time(e1))
         ms = statistics.median(times)
         fl = 2.5 * fwd_flops(B, L, HQ, window)
@@ -389,12 +385,15 @@ def main():
     ap.add_argument("--no-legs", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", choices=["decode", "bwd"], default=None,
+                    help="run just one leg (reps = --steps, warm-up = --warmup); used for profiling")
+    ap.add_argument("--decode-batch", type=int, default=None, help="sequences in the decode leg (default 64)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    from gqa_softmax_attention_attn_b200 import multirank
+
+    rank, world, local = multirank.env_rank()
 
     if args.impl == "reference":
         res = run_reference(args, rank, world)
@@ -403,12 +402,15 @@ def main():
         return
 
     if world > 1:
-        import datetime
-
         torch.cuda.set_device(local)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        multirank.init("nccl", timeout_s=300)
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
+    if args.only is not None:
+        legs = (decode_legs(dev, args.steps, args.warmup, args.decode_batch) if args.only == "decode"
+                else bwd_legs(dev, args.steps, args.warmup))
+        print(json.dumps({"only": args.only, "legs": legs}), flush=True)
+        return
     res = run_ours(args, rank, world, dev)
     if rank == 0:
         if not args.no_legs and world == 1:
@@ -422,7 +424,7 @@ def main():
                          "torch": torch.__version__, "cuda": torch.version.cuda}
         print(json.dumps(res), flush=True)
     if world > 1:
-        torch.distributed.barrier()
+        multirank.barrier()
         torch.distributed.destroy_process_group()
 
 

@@ -71,10 +71,13 @@ struct BwdParams {
     long long timeout_ns;
 };
 
+// Drain wait used on the way out (after an abort too): ignores the abort flag
+// and allows at least 1 s whatever the caller's wait limit, so a CTA never
+// exits with its own TMA loads or MMAs still in flight.
 __device__ __forceinline__ bool wait_noabort(uint64_t *bar, uint32_t parity, unsigned *status, long long tmo)
 {
     int never = 0;
-    return mbar_wait(bar, parity, &never, status, tmo);
+    return mbar_wait(bar, parity, &never, status, tmo > 1000000000LL ? tmo : 1000000000LL);
 }
 
 template <int GP>  // query heads packed per q tile

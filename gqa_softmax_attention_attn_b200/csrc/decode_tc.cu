@@ -133,10 +133,12 @@ __global__ void __launch_bounds__(kThreads)
                 tma_load_4d(smem + st * kStageBytes + kTileBytes, &tmV, 0, g, kbeg + j * kT, b, &full[st]);
                 ++issued[st];
             }
+            // drain: every issued load lands before the CTA exits (>= 1 s limit, abort ignored)
             for (int s = 0; s < kNS; ++s)
                 if (issued[s]) {
                     int never = 0;
-                    mbar_wait(&full[s], (issued[s] - 1) & 1u, &never, p.status, p.timeout_ns);
+                    mbar_wait(&full[s], (issued[s] - 1) & 1u, &never, p.status,
+                              p.timeout_ns > 1000000000LL ? p.timeout_ns : 1000000000LL);
                 }
         }
     } else {

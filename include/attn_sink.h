@@ -176,10 +176,14 @@ ATTN_SINK_API int attn_sink_decode_noalloc(const void *q, const void *k_cache, c
  * attn_sink_fwd for the same arguments; dout [B, Lq, Hq, D] (dtype).
  * Outputs (overwritten, not accumulated): dq [B, Lq, Hq, D],
  * dk, dv [B, Lk, Hkv, D] (dtype); dsinks [Hq] fp32, summed over the batch.
- * The result is deterministic run to run.
+ * Determinism: dk, dv and dsinks are identical run to run, and so is dq for
+ * dtype F32.  For dtype BF16, dq is summed over 128-key tiles by fp32 atomic
+ * adds in L2 (a TMA reduce-add), so its fp32 sum -- and rarely its bf16
+ * rounding -- may differ in the last bit between runs.
  *   workspace  device scratch of at least
  *              attn_sink_bwd_workspace_size(B, Lq, Lk, Hq, Hkv, D, dtype)
- *              bytes; contents on entry do not matter.
+ *              bytes (for BF16 it holds an fp32 copy of dq); contents on
+ *              entry do not matter.
  */
 ATTN_SINK_API int attn_sink_bwd(const void *q, const void *k, const void *v, const float *sinks,
                   const void *out, const void *dout, const float *lse,

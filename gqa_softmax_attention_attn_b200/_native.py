@@ -31,7 +31,18 @@ class AttnSinkLibraryMissing(RuntimeError):
 class AttnSinkError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: status {status} ({strerror(status)})")
+        msg = f"{where}: status {status} ({strerror(status)})"
+        if status == -6:
+            code = attn_sink_last_cuda_error()
+            try:
+                import ctypes.util
+
+                rt = torch.cuda.cudart()
+                name = rt.cudaGetErrorString(code) if hasattr(rt, "cudaGetErrorString") else ""
+            except Exception:
+                name = ""
+            msg += f"; CUDA error {code} {name}"
+        super().__init__(msg)
 
 
 def load():
@@ -66,6 +77,8 @@ def load():
         lib.attn_sink_strerror.restype = ctypes.c_char_p
         lib.attn_sink_version.argtypes = []
         lib.attn_sink_version.restype = I
+        lib.attn_sink_last_cuda_error.argtypes = []
+        lib.attn_sink_last_cuda_error.restype = I
         _lib = lib
         return lib
 
@@ -183,3 +196,7 @@ def attn_sink_set_wait_timeout_ns(ns: int) -> int:
 
 def attn_sink_version() -> int:
     return int(load().attn_sink_version())
+
+
+def attn_sink_last_cuda_error() -> int:
+    return int(load().attn_sink_last_cuda_error())

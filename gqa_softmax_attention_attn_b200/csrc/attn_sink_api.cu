@@ -96,9 +96,12 @@ int check_common(int B, int Lq, int Lk, int Hq, int Hkv, int D, int dtype)
     return ATTN_SINK_OK;
 }
 
+thread_local int g_last_cuda_error = 0;
+
 int launch_status(cudaError_t e)
 {
     if (e == cudaSuccess) return ATTN_SINK_OK;
+    g_last_cuda_error = (int)e;
     cudaGetLastError();
     return ATTN_SINK_ERR_CUDA;
 }
@@ -180,6 +183,8 @@ using namespace attn_sink;
 extern "C" {
 
 int attn_sink_version(void) { return 100; }
+
+int attn_sink_last_cuda_error(void) { return g_last_cuda_error; }
 
 const char *attn_sink_strerror(int status)
 {

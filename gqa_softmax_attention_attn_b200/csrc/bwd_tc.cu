@@ -19,10 +19,12 @@
 //    the M dimension, so a thread of the softmax-gradient warps owns a key
 //    row); then dV += P^T dO and dK += dS^T Q with P^T and dS^T read back
 //    from tensor memory; then dQ = dS K with dS from shared memory (written
-//    there in the MN-major layout by the same threads) into one of two TMEM
-//    buffers.
-//  * Warps 2-5 (one key row per thread): P and dS in fp32 from the two TMEM
-//    tiles, written back as bf16 (TMEM and shared memory).
+//    there in the MN-major layout by the same threads).  S^T of the next q
+//    tile is issued as soon as the current S^T has been read, so it overlaps
+//    the rest of the gradient pass and the dV / dK / dQ products.
+//  * Warps 2-5 (one key row per thread), in two phases: P from S^T (kept as
+//    bf16 pairs in registers, releasing S^T), then dS = P (dP - D) from dP^T;
+//    dS^T and P^T go back to tensor memory as bf16, dS to shared memory.
 //  * Warps 6-9 move each dQ tile from TMEM to shared memory and add it into an
 //    fp32 dQ accumulator in global memory with a TMA reduce-add (L2 atomics;
 //    the summation order over key tiles is not fixed).  dK and dV of the tile
@@ -53,13 +55,13 @@ constexpr int kOffDS = kOffDO + 2 * kTile;  // dS, MN-major: two 64-row atoms of
 constexpr int kOffStg = kOffDS + 2 * kTile;  // fp32 dQ staging [128][64]
 constexpr int kOffLD = kOffStg + 128 * 64 * 4;  // [2 stages][lse2 | D][128] fp32
 constexpr int kOffBar = kOffLD + 2 * 2 * 128 * 4;
-// kv_full, qdo_full[2], qdo_empty[2], s_full, p_ready, ds_free, dq_full[2],
-// dq_free[2], stg_full, stg_free, dkv_done, drain
-constexpr int kNumBar = 16;
+// kv_full, qdo_full[2], qdo_empty[2], s_full, s_consumed, dp_full, p_ready,
+// pt_free, ds_free, dq_full, dq_free, stg_full, stg_free, dkv_done, drain
+constexpr int kNumBar = 17;
 constexpr int kOffMisc = kOffBar + kNumBar * 8;
 constexpr int kSmemBytes = kOffMisc + 16 + 1024;
-// TMEM columns
-constexpr int kTmST = 0, kTmDPT = 128, kTmDV = 256, kTmDK = 320, kTmDQ = 384;
+// TMEM columns: S^T | P^T (bf16 pairs) | dP^T (dS^T bf16 pairs over its first half) | dV | dK | dQ
+constexpr int kTmST = 0, kTmPT = 128, kTmDPT = 192, kTmDV = 320, kTmDK = 384, kTmDQ = 448;
 
 struct BwdParams {
     int B, Lq, Lk, Hq, Hkv, window, G;
@@ -94,20 +96,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *qdo_full = bars + 1;   // [2]
     uint64_t *qdo_empty = bars + 3;  // [2]
     uint64_t *s_full = bars + 5;
-    uint64_t *p_ready = bars + 6;
-    uint64_t *ds_free = bars + 7;
-    uint64_t *dq_full = bars + 8;    // [2]
-    uint64_t *dq_free = bars + 10;   // [2]
-    uint64_t *stg_full = bars + 12;
-    uint64_t *stg_free = bars + 13;
-    uint64_t *dkv_done = bars + 14;
-    uint64_t *drain = bars + 15;
+    uint64_t *s_consumed = bars + 6;
+    uint64_t *dp_full = bars + 7;
+    uint64_t *p_ready = bars + 8;
+    uint64_t *pt_free = bars + 9;
+    uint64_t *ds_free = bars + 10;
+    uint64_t *dq_full = bars + 11;
+    uint64_t *dq_free = bars + 12;
+    uint64_t *stg_full = bars + 13;
+    uint64_t *stg_free = bars + 14;
+    uint64_t *dkv_done = bars + 15;
+    uint64_t *drain = bars + 16;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffMisc + 4);
     float *ld = reinterpret_cast<float *>(smem + kOffLD);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int kt = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+    // 1-D grid, key tile slowest: under a causal mask the first key tiles see
+    // the most q tiles, so every head's and batch's longest CTAs start first
+    const int per_kt = p.Hkv * p.B;
+    const int kt = (int)blockIdx.x / per_kt;
+    const int g = ((int)blockIdx.x % per_kt) % p.Hkv, b = ((int)blockIdx.x % per_kt) / p.Hkv;
     const int k0 = kt * kM;
     const long off = (long)p.Lk - p.Lq;
     // query positions whose rows can see a key of [k0, k0 + 128)
@@ -123,12 +132,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < 2; ++s) {
             mbar_init(&qdo_full[s], 2);
             mbar_init(&qdo_empty[s], 1);
-            mbar_init(&dq_full[s], 1);
-            mbar_init(&dq_free[s], 128);
         }
         mbar_init(s_full, 1);
+        mbar_init(s_consumed, 128);
+        mbar_init(dp_full, 1);
         mbar_init(p_ready, 128);
+        mbar_init(pt_free, 1);
         mbar_init(ds_free, 1);
+        mbar_init(dq_full, 1);
+        mbar_init(dq_free, 128);
         mbar_init(stg_full, 128);
         mbar_init(stg_free, 1);
         mbar_init(dkv_done, 1);
@@ -177,18 +189,33 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
-            // log2-domain lse (+inf for rows that do not exist or see nothing) and D
-            for (int c = lane; c < kM; c += 32) {
-                const int pos = pos0 + c / GP, h = h0 + c % GP;
-                float l2 = INFINITY, dd = 0.f;
-                if (pos < p.Lq) {
-                    const size_t li = ((size_t)b * p.Hq + h) * p.Lq + pos;
-                    const float L = p.lse[li];
-                    l2 = (L == -INFINITY) ? INFINITY : L * kLog2e;
-                    dd = p.Drow[li];
+            // log2-domain lse (+inf for rows that do not exist or see nothing) and
+            // D: lane l reads 4 consecutive positions of one head (16-byte loads
+            // when aligned) and scatters them to columns pos * GP + head
+            for (int e = lane * 4; e < kM; e += 128) {
+                const int hl = e / P, pl0 = e % P;  // head within the tile, first position
+                const int h = h0 + hl;
+                const size_t li0 = ((size_t)b * p.Hq + h) * p.Lq + pos0 + pl0;
+                float L4[4], D4[4];
+                if (pos0 + pl0 + 3 < p.Lq && (li0 & 3) == 0) {
+                    const float4 a = *reinterpret_cast<const float4 *>(p.lse + li0);
+                    const float4 d = *reinterpret_cast<const float4 *>(p.Drow + li0);
+                    L4[0] = a.x; L4[1] = a.y; L4[2] = a.z; L4[3] = a.w;
+                    D4[0] = d.x; D4[1] = d.y; D4[2] = d.z; D4[3] = d.w;
+                } else {
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const bool in = pos0 + pl0 + u < p.Lq;
+                        L4[u] = in ? p.lse[li0 + u] : -INFINITY;
+                        D4[u] = in ? p.Drow[li0 + u] : 0.f;
+                    }
                 }
-                ld[(st * 2 + 0) * kM + c] = l2;
-                ld[(st * 2 + 1) * kM + c] = dd;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int c = (pl0 + u) * GP + hl;
+                    ld[(st * 2 + 0) * kM + c] = (L4[u] == -INFINITY) ? INFINITY : L4[u] * kLog2e;
+                    ld[(st * 2 + 1) * kM + c] = D4[u];
+                }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&qdo_full[st]);
@@ -211,35 +238,61 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t d_ds = smem_desc_sw128(smem_u32(smem + kOffDS), kTile, 1024);
             const uint64_t d_kmn = smem_desc_sw128(smem_u32(smem + kOffK), kTile, 1024);
             bool ok = n_iter > 0 && mbar_wait(kv_full, 0, abort_flag, p.status, p.timeout_ns);
-            for (int i = 0; i < n_iter && ok; ++i) {
-                const int st = i & 1, db = i & 1;
-                if (!mbar_wait(&qdo_full[st], (i >> 1) & 1u, abort_flag, p.status, p.timeout_ns)) break;
+            // S^T(i) = K Q(i)^T into its own TMEM tile; issued for tile i+1 as
+            // soon as the softmax-gradient threads have read S^T(i) out.
+            auto issue_st = [&](int i) -> bool {
+                const int st = i & 1;
+                if (!mbar_wait(&qdo_full[st], (i >> 1) & 1u, abort_flag, p.status, p.timeout_ns)) return false;
+                if (i > 0 && !mbar_wait(s_consumed, (i - 1) & 1u, abort_flag, p.status, p.timeout_ns)) return false;
                 tc_fence_after();
                 const uint64_t q_st = d_q + (uint64_t)((st * kTile) >> 4);
-                const uint64_t do_st = d_do + (uint64_t)((st * kTile) >> 4);
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk) mma_ss(tmem + kTmST, d_k + 2 * kk, q_st + 2 * kk, id_t, kk > 0);
+                mma_commit(s_full);
+                return true;
+            };
+            // dP^T(i) = V dO(i)^T; its columns held dS^T(i-1), read by dK(i-1),
+            // which was issued before it (tcgen05 MMAs of one thread run in order)
+            auto issue_dpt = [&](int i) {
+                const uint64_t do_st = d_do + (uint64_t)(((i & 1) * kTile) >> 4);
+                tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk)
                     mma_ss(tmem + kTmDPT, d_v + 2 * kk, do_st + 2 * kk, id_t, kk > 0);
-                mma_commit(s_full);
+                mma_commit(dp_full);
+            };
+            if (ok) ok = issue_st(0);
+            if (ok) issue_dpt(0);
+            for (int i = 0; i < n_iter && ok; ++i) {
+                const int st = i & 1;
+                const uint64_t q_st = d_q + (uint64_t)((st * kTile) >> 4);
+                const uint64_t do_st = d_do + (uint64_t)((st * kTile) >> 4);
+                // scores of the next q tile, as soon as S^T(i) has been read
+                if (i + 1 < n_iter && !issue_st(i + 1)) break;
                 if (!mbar_wait(p_ready, i & 1u, abort_flag, p.status, p.timeout_ns)) break;
                 tc_fence_after();
                 // dV += P^T dO and dK += dS^T Q: K = 128 q rows in steps of 16 (2048 bytes of the MN-major B)
 #pragma unroll
                 for (int kk = 0; kk < kM / 16; ++kk)
-                    mma_ts(tmem + kTmDV, tmem + kTmST + kk * 8, do_st + 128 * kk, id_kv, (i > 0 || kk > 0));
+                    mma_ts(tmem + kTmDV, tmem + kTmPT + kk * 8, do_st + 128 * kk, id_kv, (i > 0 || kk > 0));
+                mma_commit(pt_free);
 #pragma unroll
                 for (int kk = 0; kk < kM / 16; ++kk)
                     mma_ts(tmem + kTmDK, tmem + kTmDPT + kk * 8, q_st + 128 * kk, id_kv, (i > 0 || kk > 0));
                 mma_commit(&qdo_empty[st]);
-                if (!mbar_wait(&dq_free[db], ((i >> 1) & 1u) ^ 1u, abort_flag, p.status, p.timeout_ns)) break;
+                // dP^T of the next q tile ahead of dQ(i), which only the dQ epilogue waits for
+                if (i + 1 < n_iter) {
+                    if (!mbar_wait(&qdo_full[(i + 1) & 1], ((i + 1) >> 1) & 1u, abort_flag, p.status, p.timeout_ns))
+                        break;
+                    issue_dpt(i + 1);
+                }
+                if (!mbar_wait(dq_free, (i & 1u) ^ 1u, abort_flag, p.status, p.timeout_ns)) break;
                 tc_fence_after();
                 // dQ = dS K: K = 128 keys in steps of 16
 #pragma unroll
                 for (int kk = 0; kk < kM / 16; ++kk)
-                    mma_ss(tmem + kTmDQ + db * kD, d_ds + 128 * kk, d_kmn + 128 * kk, id_q, kk > 0);
-                mma_commit(&dq_full[db]);
+                    mma_ss(tmem + kTmDQ, d_ds + 128 * kk, d_kmn + 128 * kk, id_q, kk > 0);
+                mma_commit(dq_full);
                 mma_commit(ds_free);
             }
             mma_commit(dkv_done);
@@ -260,8 +313,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             iter_head(i, h0, pos0);
             if (!__all_sync(0xffffffffu,
                             mbar_wait(&qdo_full[st], (i >> 1) & 1u, abort_flag, p.status, p.timeout_ns) &&
-                                mbar_wait(s_full, i & 1u, abort_flag, p.status, p.timeout_ns) &&
-                                (i == 0 || mbar_wait(ds_free, (i - 1) & 1u, abort_flag, p.status, p.timeout_ns)))) {
+                                mbar_wait(s_full, i & 1u, abort_flag, p.status, p.timeout_ns))) {
                 ok = false;
                 break;
             }
@@ -277,48 +329,83 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int pl_lo = (int)min(lo_l, (long)P);
             const int pl_hi = (int)max(-1L, min(hi_l, (long)P - 1));
             const bool need_mask = __any_sync(0xffffffffu, pl_lo > 0 || pl_hi < P - 1);
-            const float *l2 = ld + (st * 2 + 0) * kM;
-            const float *dd = ld + (st * 2 + 1) * kM;
+            const float4 *l2v = reinterpret_cast<const float4 *>(ld + (st * 2 + 0) * kM);
+            const float4 *ddv = reinterpret_cast<const float4 *>(ld + (st * 2 + 1) * kM);
+
+            // phase 1: P = exp2(S C - lse2) from S^T, kept as bf16 pairs; then S^T is free
+            uint32_t pk[kM / 2];
 #pragma unroll
-            for (int c = 0; c < kM / 32; ++c) {
-                uint32_t sr[32], dr[32];
-                tmem_ld32(trow + kTmST + 32 * c, sr);
-                tmem_ld32(trow + kTmDPT + 32 * c, dr);
+            for (int c = 0; c < kM / 16; ++c) {
+                uint32_t sr[16];
+                tmem_ld16(trow + kTmST + 16 * c, sr);
                 tmem_wait_ld();
-                uint32_t pk[16], dk[16];
-                float dsv[32];
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int col = 32 * c + e;
-                    float pe = ex2(fmaf(__uint_as_float(sr[e]), C, -l2[col]));
-                    if (need_mask) {
-                        const int pl = col / GP;
-                        pe = (pl >= pl_lo && pl <= pl_hi) ? pe : 0.f;
-                    }
-                    dsv[e] = pe * (__uint_as_float(dr[e]) - dd[col]);
-                    if (e & 1) {
-                        pk[e / 2] = pack_bf16x2(__uint_as_float(sr[e - 1]), pe);
-                        dk[e / 2] = pack_bf16x2(dsv[e - 1], dsv[e]);
-                    } else {
-                        sr[e] = __float_as_uint(pe);  // keep P of the even column for the pair
-                    }
-                }
-                // P^T and dS^T (bf16 pairs) over the already-read columns of their tiles
-                tmem_st16(trow + kTmST + 16 * c, pk);
-                tmem_st16(trow + kTmDPT + 16 * c, dk);
-                // dS into shared memory, MN-major: atom (col / 64), key row r, 8 q rows per 16 bytes
+                for (int e4 = 0; e4 < 4; ++e4) {
+                    const float4 l4 = l2v[4 * c + e4];
+                    const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+                    float pe[4];
 #pragma unroll
-                for (int q8 = 0; q8 < 4; ++q8) {
-                    const int chunk = 4 * c + q8;  // 8-column chunk index 0..15
-                    const int atom = chunk >> 3, cc = chunk & 7;
-                    uint4 v;
-                    v.x = dk[4 * q8 + 0];
-                    v.y = dk[4 * q8 + 1];
-                    v.z = dk[4 * q8 + 2];
-                    v.w = dk[4 * q8 + 3];
-                    *reinterpret_cast<uint4 *>(smem + kOffDS + atom * kTile + r * 128 + ((cc ^ (r & 7)) << 4)) = v;
+                    for (int u = 0; u < 4; ++u) {
+                        const int col = 16 * c + 4 * e4 + u;
+                        pe[u] = ex2(fmaf(__uint_as_float(sr[4 * e4 + u]), C, -lv[u]));
+                        if (need_mask) {
+                            const int pl = col / GP;
+                            pe[u] = (pl >= pl_lo && pl <= pl_hi) ? pe[u] : 0.f;
+                        }
+                    }
+                    pk[8 * c + 2 * e4] = pack_bf16x2(pe[0], pe[1]);
+                    pk[8 * c + 2 * e4 + 1] = pack_bf16x2(pe[2], pe[3]);
                 }
             }
+            tc_fence_before();
+            mbar_arrive(s_consumed);  // S^T(i+1) may be computed into these columns now
+
+            // phase 2: dS = P (dP - D) from dP^T; dS^T (bf16 pairs) over the read
+            // columns of dP^T, dS into shared memory (MN-major) for dQ
+            if (!__all_sync(0xffffffffu, mbar_wait(dp_full, i & 1u, abort_flag, p.status, p.timeout_ns) &&
+                                             (i == 0 || mbar_wait(ds_free, (i - 1) & 1u, abort_flag, p.status,
+                                                                  p.timeout_ns)))) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int c = 0; c < kM / 16; ++c) {
+                uint32_t dr[16];
+                tmem_ld16(trow + kTmDPT + 16 * c, dr);
+                tmem_wait_ld();
+                uint32_t dk[8];
+#pragma unroll
+                for (int e4 = 0; e4 < 4; ++e4) {
+                    const float4 d4 = ddv[4 * c + e4];
+                    const __nv_bfloat162 p01 = *reinterpret_cast<const __nv_bfloat162 *>(&pk[8 * c + 2 * e4]);
+                    const __nv_bfloat162 p23 = *reinterpret_cast<const __nv_bfloat162 *>(&pk[8 * c + 2 * e4 + 1]);
+                    const float ds0 = __low2float(p01) * (__uint_as_float(dr[4 * e4 + 0]) - d4.x);
+                    const float ds1 = __high2float(p01) * (__uint_as_float(dr[4 * e4 + 1]) - d4.y);
+                    const float ds2 = __low2float(p23) * (__uint_as_float(dr[4 * e4 + 2]) - d4.z);
+                    const float ds3 = __high2float(p23) * (__uint_as_float(dr[4 * e4 + 3]) - d4.w);
+                    dk[2 * e4] = pack_bf16x2(ds0, ds1);
+                    dk[2 * e4 + 1] = pack_bf16x2(ds2, ds3);
+                }
+                // dS^T over the 8 columns of dP^T just read (columns 8c .. 8c+7 of its first half)
+                tmem_st8(trow + kTmDPT + 8 * c, dk);
+#pragma unroll
+                for (int q8 = 0; q8 < 2; ++q8) {
+                    const int chunk = 2 * c + q8;  // 8-column chunk index 0..15
+                    const int atom = chunk >> 3, cc = chunk & 7;
+                    *reinterpret_cast<uint4 *>(smem + kOffDS + atom * kTile + r * 128 + ((cc ^ (r & 7)) << 4)) =
+                        make_uint4(dk[4 * q8], dk[4 * q8 + 1], dk[4 * q8 + 2], dk[4 * q8 + 3]);
+                }
+            }
+            // P^T into its columns once dV(i-1) has read the previous P^T
+            if (i > 0 &&
+                !__all_sync(0xffffffffu, mbar_wait(pt_free, (i - 1) & 1u, abort_flag, p.status, p.timeout_ns))) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int c = 0; c < kM / 32; ++c) tmem_st16(trow + kTmPT + 16 * c, &pk[16 * c]);
             tmem_wait_st();
             fence_proxy_async_smem();  // dS in shared memory is read by the tensor core next
             tc_fence_before();
@@ -376,19 +463,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool issuer = (warp == 6 && lane == 0);
         float *stg = reinterpret_cast<float *>(smem + kOffStg);
         for (int i = 0; i < n_iter; ++i) {
-            const int db = i & 1;
             int h0, pos0;
             iter_head(i, h0, pos0);
-            if (!__all_sync(0xffffffffu,
-                            mbar_wait(&dq_full[db], (i >> 1) & 1u, abort_flag, p.status, p.timeout_ns)))
+            if (!__all_sync(0xffffffffu, mbar_wait(dq_full, i & 1u, abort_flag, p.status, p.timeout_ns)))
                 break;
             tc_fence_after();
             uint32_t a[2][32];
-            tmem_ld32(trow + kTmDQ + db * kD, a[0]);
-            tmem_ld32(trow + kTmDQ + db * kD + 32, a[1]);
+            tmem_ld32(trow + kTmDQ, a[0]);
+            tmem_ld32(trow + kTmDQ + 32, a[1]);
             tmem_wait_ld();
             tc_fence_before();
-            mbar_arrive(&dq_free[db]);
+            mbar_arrive(dq_free);
             if (!__all_sync(0xffffffffu, mbar_wait(stg_free, (i & 1u) ^ 1u, abort_flag, p.status, p.timeout_ns)))
                 break;
             // row-major [128 rows][64 fp32]; chunk order rotated by lane to spread banks
@@ -491,7 +576,9 @@ cudaError_t launch_bwd_tc(const void *q, const void *k, const void *v, const voi
         return cudaErrorInvalidValue;
     cudaError_t e = cudaMemsetAsync(dq_acc, 0, bwd_tc_dq_acc_bytes(s), st);
     if (e != cudaSuccess) return e;
-    const dim3 grid((s.Lk + kM - 1) / kM, s.Hkv, s.B);
+    const long long n_cta = (long long)((s.Lk + kM - 1) / kM) * s.Hkv * s.B;
+    if (n_cta > 0x7fffffffLL) return cudaErrorInvalidValue;
+    const dim3 grid((unsigned)n_cta);
     switch (gp) {
     case 1: e = launch_gp<1>(mq, mdo, mk, mv, mdq, p, grid, st); break;
     case 2: e = launch_gp<2>(mq, mdo, mk, mv, mdq, p, grid, st); break;

@@ -49,12 +49,23 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
+// Banded-layer tile configuration (compile-time knob for measurements)
+// (measured on the window-128 layer of the gpt-oss-20b prefill: BN 32 with
+// three CTAs per SM 47 us, BN 64 with two 54 us, BN 32 with two 49 us)
+#ifndef ATTN_SINK_FWD_BAND_BN
+#define ATTN_SINK_FWD_BAND_BN 32
+#define ATTN_SINK_FWD_BAND_NS 4
+#define ATTN_SINK_FWD_BAND_CPS 3
+#endif
+
 // Tile configurations (keys per tile BN, K/V stages NS, EMU = which pair of
 // every 4 uses the FMA-pipe exp2, -1 for none), chosen per layer type from
 // measurements on the gpt-oss-20b prefill: the dense causal layer runs best
 // with BN = 96 and a quarter of the exponentials off the MUFU unit, the
 // window-128 layer with BN = 64 and all exponentials on MUFU.
-template <int BN, int NS>
+constexpr int pow2_at_least(int x) { return x <= 32 ? 32 : x <= 64 ? 64 : x <= 128 ? 128 : x <= 256 ? 256 : 512; }
+
+template <int BN, int NS, int CPS>
 struct FwdCfg {
     static constexpr int kQBytes = kM * kD * 2;
     static constexpr int kKVBytes = BN * kD * 2;
@@ -66,8 +77,9 @@ struct FwdCfg {
     // s_full[2], p_full[2], o_done, o_free, drain
     static constexpr int kNumBar = 4 + 4 * NS + 4 + 3;
     static constexpr int kOffMisc = kOffBar + kNumBar * 8;
-    static constexpr int kTmemCols = (2 * BN + kD <= 256) ? 256 : 512;
-    static constexpr int kCtasPerSm = kTmemCols == 256 ? 2 : 1;
+    static constexpr int kTmemCols = pow2_at_least(2 * BN + kD);
+    static constexpr int kCtasPerSm = CPS;  // CTAs resident per SM (TMEM, registers, shared memory)
+    static_assert(kTmemCols * CPS <= 512, "tensor memory over-subscribed");
     // + slack for 1024-byte alignment; a CTA that takes all 512 TMEM columns
     // also takes enough shared memory that no second CTA lands on its SM
     static constexpr int kSmemUsed = kOffMisc + 16 + 1024;
@@ -123,12 +135,12 @@ __device__ __forceinline__ bool wait_noabort(uint64_t *bar, uint32_t parity, uns
     return mbar_wait(bar, parity, &never, status, tmo > 1000000000LL ? tmo : 1000000000LL);
 }
 
-template <int BN, int NS, int EMU>
-__global__ void __launch_bounds__(192, FwdCfg<BN, NS>::kCtasPerSm)
+template <int BN, int NS, int EMU, int CPS>
+__global__ void __launch_bounds__(192, CPS)
     fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdTcParams p)
 {
-    using Cfg = FwdCfg<BN, NS>;
+    using Cfg = FwdCfg<BN, NS, CPS>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kOffBar);
@@ -463,11 +475,11 @@ __global__ void __launch_bounds__(192, FwdCfg<BN, NS>::kCtasPerSm)
     }
 }
 
-template <int BN, int NS, int EMU>
+template <int BN, int NS, int EMU, int CPS>
 cudaError_t launch_cfg(const void *q, const void *k, const void *v, const float *sinks, void *out, float *lse,
                        const AttnShape &s, cudaStream_t st)
 {
-    using Cfg = FwdCfg<BN, NS>;
+    using Cfg = FwdCfg<BN, NS, CPS>;
     FwdTcParams p;
     p.B = s.B;
     p.Lq = s.Lq;
@@ -509,7 +521,7 @@ cudaError_t launch_cfg(const void *q, const void *k, const void *v, const float 
         if (!encode_tensor_map_4d(&mv, const_cast<void *>(v), 2, dims, strides, box, true))
             return cudaErrorInvalidValue;
     }
-    auto kern = fwd_tc_kernel<BN, NS, EMU>;
+    auto kern = fwd_tc_kernel<BN, NS, EMU, CPS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 0;
@@ -532,8 +544,10 @@ bool fwd_tc_supported(const AttnShape &s)
 cudaError_t launch_fwd_tc(const void *q, const void *k, const void *v, const float *sinks, void *out,
                           float *lse, const AttnShape &s, cudaStream_t st)
 {
-    if (s.window > 0 && s.window <= 1024) return launch_cfg<64, 4, -1>(q, k, v, sinks, out, lse, s, st);
-    return launch_cfg<96, 3, 3>(q, k, v, sinks, out, lse, s, st);
+    if (s.window > 0 && s.window <= 1024)
+        return launch_cfg<ATTN_SINK_FWD_BAND_BN, ATTN_SINK_FWD_BAND_NS, -1, ATTN_SINK_FWD_BAND_CPS>(q, k, v, sinks, out,
+                                                                                                  lse, s, st);
+    return launch_cfg<96, 3, 3, 2>(q, k, v, sinks, out, lse, s, st);
 }
 
 }  // namespace attn_sink

@@ -211,6 +211,12 @@ ATTN_SINK_API long long attn_sink_set_wait_timeout_ns(long long ns);
 /* Static description of a status code. */
 ATTN_SINK_API const char *attn_sink_strerror(int status);
 
+/*
+ * The cudaError_t value behind the most recent ATTN_SINK_ERR_CUDA returned to
+ * the calling host thread (0 if none).  Not cleared by later successful calls.
+ */
+ATTN_SINK_API int attn_sink_last_cuda_error(void);
+
 /* Library version as 10000*major + 100*minor + patch. */
 ATTN_SINK_API int attn_sink_version(void);
 

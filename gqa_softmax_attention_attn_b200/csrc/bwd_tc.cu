@@ -22,9 +22,11 @@
 //    there in the MN-major layout by the same threads).  S^T of the next q
 //    tile is issued as soon as the current S^T has been read, so it overlaps
 //    the rest of the gradient pass and the dV / dK / dQ products.
-//  * Warps 2-5 (one key row per thread), in two phases: P from S^T (kept as
-//    bf16 pairs in registers, releasing S^T), then dS = P (dP - D) from dP^T;
-//    dS^T and P^T go back to tensor memory as bf16, dS to shared memory.
+//  * Warps 2-5 and 10-13: two warps per key row (one per 64-column half of
+//    the q tile, so each SM sub-partition runs two of them), in two phases:
+//    P from S^T (bf16 pairs into their own TMEM columns, releasing S^T), then
+//    dS = P (dP - D) from dP^T; dS^T goes back over the half's read columns
+//    of dP^T as bf16, dS to shared memory.
 //  * Warps 6-9 move each dQ tile from TMEM to shared memory and add it into an
 //    fp32 dQ accumulator in global memory with a TMA reduce-add (L2 atomics;
 //    the summation order over key tiles is not fixed).  dK and dV of the tile
@@ -43,7 +45,11 @@ namespace {
 
 constexpr int kM = 128;  // keys per tile (rows of the transposed score tile)
 constexpr int kD = 64;
-constexpr int kThreads = 320;
+constexpr int kThreads = 448;  // 14 warps: loads, MMA, 4 dQ, 8 gradient
+// 1: half of phase 1's exponentials on the FMA pipe (fast_exp2x2)
+#ifndef ATTN_SINK_BWD_EMU
+#define ATTN_SINK_BWD_EMU 0
+#endif
 constexpr float kLog2e = 1.4426950408889634f;
 
 constexpr int kTile = kM * kD * 2;  // 16 KB bf16 tile
@@ -52,7 +58,7 @@ constexpr int kOffV = kOffK + kTile;
 constexpr int kOffQ = kOffV + kTile;       // 2 stages
 constexpr int kOffDO = kOffQ + 2 * kTile;  // 2 stages
 constexpr int kOffDS = kOffDO + 2 * kTile;  // dS, MN-major: two 64-row atoms of 16 KB
-constexpr int kOffStg = kOffDS + 2 * kTile;  // fp32 dQ staging [128][64]
+constexpr int kOffStg = kOffDS + 2 * kTile;  // fp32 dQ staging: two [128][32] halves, 128-byte swizzle
 constexpr int kOffLD = kOffStg + 128 * 64 * 4;  // [2 stages][lse2 | D][128] fp32
 constexpr int kOffBar = kOffLD + 2 * 2 * 128 * 4;
 // kv_full, qdo_full[2], qdo_empty[2], s_full, s_consumed, dp_full, p_ready,
@@ -60,7 +66,9 @@ constexpr int kOffBar = kOffLD + 2 * 2 * 128 * 4;
 constexpr int kNumBar = 17;
 constexpr int kOffMisc = kOffBar + kNumBar * 8;
 constexpr int kSmemBytes = kOffMisc + 16 + 1024;
-// TMEM columns: S^T | P^T (bf16 pairs) | dP^T (dS^T bf16 pairs over its first half) | dV | dK | dQ
+// TMEM columns: S^T | P^T (bf16 pairs) | dP^T | dV | dK | dQ.  dS^T (bf16
+// pairs) goes over dP^T: q rows 0-63 at its columns 0-31, rows 64-127 at
+// 64-95, each inside the range its own warp has already read.
 constexpr int kTmST = 0, kTmPT = 128, kTmDPT = 192, kTmDV = 320, kTmDK = 384, kTmDQ = 448;
 
 struct BwdParams {
@@ -134,9 +142,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&qdo_empty[s], 1);
         }
         mbar_init(s_full, 1);
-        mbar_init(s_consumed, 128);
+        mbar_init(s_consumed, 256);
         mbar_init(dp_full, 1);
-        mbar_init(p_ready, 128);
+        mbar_init(p_ready, 256);
         mbar_init(pt_free, 1);
         mbar_init(ds_free, 1);
         mbar_init(dq_full, 1);
@@ -165,7 +173,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == 0) {
         // ------------------------------------------------------------ loads
-        uint32_t issued_qdo[2] = {0, 0};
+        uint32_t issued_qdo0 = 0, issued_qdo1 = 0;
         bool ok = true;
         if (lane == 0 && n_iter > 0) {
             tma_prefetch_desc(&tmQ);
@@ -184,7 +192,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mbar_arrive_expect_tx(&qdo_full[st], 2 * kTile);
                     tma_load_4d(smem + kOffQ + st * kTile, &tmQ, 0, h0, pos0, b, &qdo_full[st]);
                     tma_load_4d(smem + kOffDO + st * kTile, &tmDO, 0, h0, pos0, b, &qdo_full[st]);
-                    ++issued_qdo[st];
+                    if (st) ++issued_qdo1; else ++issued_qdo0;
                 }
             }
             ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -222,8 +230,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (lane == 0) {
             if (n_iter > 0) wait_noabort(kv_full, 0, p.status, p.timeout_ns);
-            for (int s = 0; s < 2; ++s)
-                if (issued_qdo[s]) wait_noabort(&qdo_full[s], (issued_qdo[s] - 1) & 1u, p.status, p.timeout_ns);
+            if (issued_qdo0) wait_noabort(&qdo_full[0], (issued_qdo0 - 1) & 1u, p.status, p.timeout_ns);
+            if (issued_qdo1) wait_noabort(&qdo_full[1], (issued_qdo1 - 1) & 1u, p.status, p.timeout_ns);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issue
@@ -278,7 +286,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mma_commit(pt_free);
 #pragma unroll
                 for (int kk = 0; kk < kM / 16; ++kk)
-                    mma_ts(tmem + kTmDK, tmem + kTmDPT + kk * 8, q_st + 128 * kk, id_kv, (i > 0 || kk > 0));
+                    mma_ts(tmem + kTmDK, tmem + kTmDPT + kk * 8 + (kk >= kM / 32 ? kM / 4 : 0), q_st + 128 * kk,
+                           id_kv, (i > 0 || kk > 0));
                 mma_commit(&qdo_empty[st]);
                 // dP^T of the next q tile ahead of dQ(i), which only the dQ epilogue waits for
                 if (i + 1 < n_iter) {
@@ -299,9 +308,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_commit(drain);
             wait_noabort(drain, 0, p.status, p.timeout_ns);
         }
-    } else if (warp <= 5) {
-        // ------------------------------------------------------------ P and dS, one key row per thread
+    } else if (warp <= 5 || warp >= 10) {
+        // ------------------------------------------------------------ P and dS, one key row per warp pair
+        constexpr int kCh = kM / 32;       // 16-column chunks per half
         const int quad = warp & 3;
+        const int half = warp >= 10;       // q columns [64 half, 64 half + 64)
+        const int c0 = half * kCh;
         const int r = quad * 32 + lane;
         const int j = k0 + r;
         const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
@@ -333,21 +345,33 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float4 *ddv = reinterpret_cast<const float4 *>(ld + (st * 2 + 1) * kM);
 
             // phase 1: P = exp2(S C - lse2) from S^T, kept as bf16 pairs; then S^T is free
-            uint32_t pk[kM / 2];
+            // TMEM loads are pipelined one 16-column chunk ahead of the arithmetic
+            uint32_t pk[kM / 4];
+            uint32_t sbuf[2][16];
+            tmem_ld16(trow + kTmST + 16 * c0, sbuf[0]);
+            tmem_wait_ld();
 #pragma unroll
-            for (int c = 0; c < kM / 16; ++c) {
-                uint32_t sr[16];
-                tmem_ld16(trow + kTmST + 16 * c, sr);
-                tmem_wait_ld();
+            for (int c = 0; c < kCh; ++c) {
+                if (c + 1 < kCh) tmem_ld16(trow + kTmST + 16 * (c0 + c + 1), sbuf[(c + 1) & 1]);
+                const uint32_t *sr = sbuf[c & 1];
 #pragma unroll
                 for (int e4 = 0; e4 < 4; ++e4) {
-                    const float4 l4 = l2v[4 * c + e4];
+                    const float4 l4 = l2v[4 * (c0 + c) + e4];
                     const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
                     float pe[4];
+                    if (ATTN_SINK_BWD_EMU && (e4 & 1)) {
+                        const float2 a = fast_exp2x2(make_float2(fmaf(__uint_as_float(sr[4 * e4 + 0]), C, -lv[0]),
+                                                                 fmaf(__uint_as_float(sr[4 * e4 + 1]), C, -lv[1])));
+                        const float2 bq = fast_exp2x2(make_float2(fmaf(__uint_as_float(sr[4 * e4 + 2]), C, -lv[2]),
+                                                                  fmaf(__uint_as_float(sr[4 * e4 + 3]), C, -lv[3])));
+                        pe[0] = a.x; pe[1] = a.y; pe[2] = bq.x; pe[3] = bq.y;
+                    } else {
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) pe[u] = ex2(fmaf(__uint_as_float(sr[4 * e4 + u]), C, -lv[u]));
+                    }
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
-                        const int col = 16 * c + 4 * e4 + u;
-                        pe[u] = ex2(fmaf(__uint_as_float(sr[4 * e4 + u]), C, -lv[u]));
+                        const int col = 16 * (c0 + c) + 4 * e4 + u;
                         if (need_mask) {
                             const int pl = col / GP;
                             pe[u] = (pl >= pl_lo && pl <= pl_hi) ? pe[u] : 0.f;
@@ -356,7 +380,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                     pk[8 * c + 2 * e4] = pack_bf16x2(pe[0], pe[1]);
                     pk[8 * c + 2 * e4 + 1] = pack_bf16x2(pe[2], pe[3]);
                 }
+                tmem_wait_ld();
             }
+            // P^T into its columns once dV(i-1) has read the previous P^T
+            if (i > 0 &&
+                !__all_sync(0xffffffffu, mbar_wait(pt_free, (i - 1) & 1u, abort_flag, p.status, p.timeout_ns))) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int c = 0; c < kCh / 2; ++c) tmem_st16(trow + kTmPT + kM / 4 * half + 16 * c, &pk[16 * c]);
             tc_fence_before();
             mbar_arrive(s_consumed);  // S^T(i+1) may be computed into these columns now
 
@@ -369,15 +403,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             tc_fence_after();
+            uint32_t dbuf[2][16];
+            tmem_ld16(trow + kTmDPT + 16 * c0, dbuf[0]);
+            tmem_wait_ld();
 #pragma unroll
-            for (int c = 0; c < kM / 16; ++c) {
-                uint32_t dr[16];
-                tmem_ld16(trow + kTmDPT + 16 * c, dr);
-                tmem_wait_ld();
+            for (int c = 0; c < kCh; ++c) {
+                if (c + 1 < kCh) tmem_ld16(trow + kTmDPT + 16 * (c0 + c + 1), dbuf[(c + 1) & 1]);
+                const uint32_t *dr = dbuf[c & 1];
                 uint32_t dk[8];
 #pragma unroll
                 for (int e4 = 0; e4 < 4; ++e4) {
-                    const float4 d4 = ddv[4 * c + e4];
+                    const float4 d4 = ddv[4 * (c0 + c) + e4];
                     const __nv_bfloat162 p01 = *reinterpret_cast<const __nv_bfloat162 *>(&pk[8 * c + 2 * e4]);
                     const __nv_bfloat162 p23 = *reinterpret_cast<const __nv_bfloat162 *>(&pk[8 * c + 2 * e4 + 1]);
                     const float ds0 = __low2float(p01) * (__uint_as_float(dr[4 * e4 + 0]) - d4.x);
@@ -387,72 +423,57 @@ __global__ void __launch_bounds__(kThreads, 1)
                     dk[2 * e4] = pack_bf16x2(ds0, ds1);
                     dk[2 * e4 + 1] = pack_bf16x2(ds2, ds3);
                 }
-                // dS^T over the 8 columns of dP^T just read (columns 8c .. 8c+7 of its first half)
-                tmem_st8(trow + kTmDPT + 8 * c, dk);
+                // dS^T over 8 columns of dP^T this warp has read (64 half + 8c .. + 7)
+                tmem_st8(trow + kTmDPT + 16 * c0 + 8 * c, dk);
 #pragma unroll
                 for (int q8 = 0; q8 < 2; ++q8) {
-                    const int chunk = 2 * c + q8;  // 8-column chunk index 0..15
+                    const int chunk = 2 * (c0 + c) + q8;  // 8-column chunk index 0..15
                     const int atom = chunk >> 3, cc = chunk & 7;
                     *reinterpret_cast<uint4 *>(smem + kOffDS + atom * kTile + r * 128 + ((cc ^ (r & 7)) << 4)) =
                         make_uint4(dk[4 * q8], dk[4 * q8 + 1], dk[4 * q8 + 2], dk[4 * q8 + 3]);
                 }
+                tmem_wait_ld();
             }
-            // P^T into its columns once dV(i-1) has read the previous P^T
-            if (i > 0 &&
-                !__all_sync(0xffffffffu, mbar_wait(pt_free, (i - 1) & 1u, abort_flag, p.status, p.timeout_ns))) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-#pragma unroll
-            for (int c = 0; c < kM / 32; ++c) tmem_st16(trow + kTmPT + 16 * c, &pk[16 * c]);
             tmem_wait_st();
             fence_proxy_async_smem();  // dS in shared memory is read by the tensor core next
             tc_fence_before();
             mbar_arrive(p_ready);
         }
-        // ---- dK, dV of this key row
-        float kv[2][64];
-        bool have = false;
-        if (ok && n_iter > 0 &&
-            __all_sync(0xffffffffu, mbar_wait(dkv_done, 0, abort_flag, p.status, p.timeout_ns))) {
-            tc_fence_after();
-            uint32_t a[32];
+        // ---- dK, dV of this key row, 16 columns at a time (32 per half)
+        const bool done = ok && n_iter > 0 &&
+                          __all_sync(0xffffffffu, mbar_wait(dkv_done, 0, abort_flag, p.status, p.timeout_ns));
+        if (done) tc_fence_after();
+        const bool write = (done || (n_iter == 0 && !*abort_flag)) && j < p.Lk;
+        const size_t base = (((size_t)b * p.Lk + (j < p.Lk ? j : 0)) * p.Hkv + g) * kD;
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                tmem_ld32(trow + kTmDV + 32 * h, a);
+        for (int cc = 0; cc < kD / 32; ++cc) {
+            const int c = half * (kD / 32) + cc;
+            uint32_t va[16], ka[16];
+            if (done) {  // warp-uniform
+                tmem_ld16(trow + kTmDV + 16 * c, va);
+                tmem_ld16(trow + kTmDK + 16 * c, ka);
                 tmem_wait_ld();
+            } else {
 #pragma unroll
-                for (int e = 0; e < 32; ++e) kv[0][32 * h + e] = __uint_as_float(a[e]);
-                tmem_ld32(trow + kTmDK + 32 * h, a);
-                tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 32; ++e) kv[1][32 * h + e] = __uint_as_float(a[e]) * p.scale;
+                for (int e = 0; e < 16; ++e) va[e] = ka[e] = 0u;
             }
-            have = true;
-        }
-        if ((have || (n_iter == 0 && !*abort_flag)) && j < p.Lk) {
-            const size_t base = (((size_t)b * p.Lk + j) * p.Hkv + g) * kD;
-            uint4 *dv4 = reinterpret_cast<uint4 *>(p.dv + base);
-            uint4 *dk4 = reinterpret_cast<uint4 *>(p.dk + base);
+            if (write) {
+                uint4 *dv4 = reinterpret_cast<uint4 *>(p.dv + base + 16 * c);
+                uint4 *dk4 = reinterpret_cast<uint4 *>(p.dk + base + 16 * c);
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                uint4 a, bb;
-                if (have) {
-                    a.x = pack_bf16x2(kv[0][8 * c + 0], kv[0][8 * c + 1]);
-                    a.y = pack_bf16x2(kv[0][8 * c + 2], kv[0][8 * c + 3]);
-                    a.z = pack_bf16x2(kv[0][8 * c + 4], kv[0][8 * c + 5]);
-                    a.w = pack_bf16x2(kv[0][8 * c + 6], kv[0][8 * c + 7]);
-                    bb.x = pack_bf16x2(kv[1][8 * c + 0], kv[1][8 * c + 1]);
-                    bb.y = pack_bf16x2(kv[1][8 * c + 2], kv[1][8 * c + 3]);
-                    bb.z = pack_bf16x2(kv[1][8 * c + 4], kv[1][8 * c + 5]);
-                    bb.w = pack_bf16x2(kv[1][8 * c + 6], kv[1][8 * c + 7]);
-                } else {
-                    a = make_uint4(0, 0, 0, 0);
-                    bb = a;
+                for (int h = 0; h < 2; ++h) {
+                    uint4 a, bb;
+                    a.x = pack_bf16x2(__uint_as_float(va[8 * h + 0]), __uint_as_float(va[8 * h + 1]));
+                    a.y = pack_bf16x2(__uint_as_float(va[8 * h + 2]), __uint_as_float(va[8 * h + 3]));
+                    a.z = pack_bf16x2(__uint_as_float(va[8 * h + 4]), __uint_as_float(va[8 * h + 5]));
+                    a.w = pack_bf16x2(__uint_as_float(va[8 * h + 6]), __uint_as_float(va[8 * h + 7]));
+                    bb.x = pack_bf16x2(__uint_as_float(ka[8 * h + 0]) * p.scale, __uint_as_float(ka[8 * h + 1]) * p.scale);
+                    bb.y = pack_bf16x2(__uint_as_float(ka[8 * h + 2]) * p.scale, __uint_as_float(ka[8 * h + 3]) * p.scale);
+                    bb.z = pack_bf16x2(__uint_as_float(ka[8 * h + 4]) * p.scale, __uint_as_float(ka[8 * h + 5]) * p.scale);
+                    bb.w = pack_bf16x2(__uint_as_float(ka[8 * h + 6]) * p.scale, __uint_as_float(ka[8 * h + 7]) * p.scale);
+                    dv4[h] = a;
+                    dk4[h] = bb;
                 }
-                dv4[c] = a;
-                dk4[c] = bb;
             }
         }
     } else {
@@ -476,22 +497,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive(dq_free);
             if (!__all_sync(0xffffffffu, mbar_wait(stg_free, (i & 1u) ^ 1u, abort_flag, p.status, p.timeout_ns)))
                 break;
-            // row-major [128 rows][64 fp32]; chunk order rotated by lane to spread banks
+            // columns 32 hh .. 32 hh + 31 of row `row` fill 128 bytes of half hh;
+            // 16-byte chunk j lands at chunk j ^ (row & 7) (the TMA 128-byte
+            // swizzle), so 8 consecutive rows hit 8 different bank groups
 #pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                const int ck = (k + lane) & 15;
-                float4 v;
-                v.x = __uint_as_float(a[ck / 8][(ck % 8) * 4 + 0]) * p.scale;
-                v.y = __uint_as_float(a[ck / 8][(ck % 8) * 4 + 1]) * p.scale;
-                v.z = __uint_as_float(a[ck / 8][(ck % 8) * 4 + 2]) * p.scale;
-                v.w = __uint_as_float(a[ck / 8][(ck % 8) * 4 + 3]) * p.scale;
-                *reinterpret_cast<float4 *>(stg + row * 64 + ck * 4) = v;
-            }
+            for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    float4 v;
+                    v.x = __uint_as_float(a[hh][4 * j + 0]) * p.scale;
+                    v.y = __uint_as_float(a[hh][4 * j + 1]) * p.scale;
+                    v.z = __uint_as_float(a[hh][4 * j + 2]) * p.scale;
+                    v.w = __uint_as_float(a[hh][4 * j + 3]) * p.scale;
+                    *reinterpret_cast<float4 *>(reinterpret_cast<uint8_t *>(stg) + hh * (kM * 128) + row * 128 +
+                                                ((j ^ (row & 7)) << 4)) = v;
+                }
             fence_proxy_async_smem();
             mbar_arrive(stg_full);
             if (issuer) {
                 if (!mbar_wait(stg_full, i & 1u, abort_flag, p.status, p.timeout_ns)) break;
                 tma_reduce_add_4d(&tmDQ, stg, 0, h0, pos0, b);
+                tma_reduce_add_4d(&tmDQ, reinterpret_cast<uint8_t *>(stg) + kM * 128, kD / 2, h0, pos0, b);
                 bulk_commit_group();
                 bulk_wait_read_all();
                 mbar_arrive(stg_free);
@@ -565,6 +591,7 @@ cudaError_t launch_bwd_tc(const void *q, const void *k, const void *v, const voi
     const uint64_t qs2[3] = {(uint64_t)kD * 2, (uint64_t)s.Hq * kD * 2, (uint64_t)s.Lq * s.Hq * kD * 2};
     const uint64_t qs4[3] = {(uint64_t)kD * 4, (uint64_t)s.Hq * kD * 4, (uint64_t)s.Lq * s.Hq * kD * 4};
     const uint32_t qbox[4] = {(uint32_t)kD, (uint32_t)gp, (uint32_t)p.P, 1u};
+    const uint32_t dqbox[4] = {(uint32_t)kD / 2, (uint32_t)gp, (uint32_t)p.P, 1u};  // 128-byte fp32 rows
     const uint64_t kd[4] = {(uint64_t)kD, (uint64_t)s.Hkv, (uint64_t)s.Lk, (uint64_t)s.B};
     const uint64_t ks2[3] = {(uint64_t)kD * 2, (uint64_t)s.Hkv * kD * 2, (uint64_t)s.Lk * s.Hkv * kD * 2};
     const uint32_t kbox[4] = {(uint32_t)kD, 1u, (uint32_t)kM, 1u};
@@ -572,7 +599,7 @@ cudaError_t launch_bwd_tc(const void *q, const void *k, const void *v, const voi
         !encode_tensor_map_4d(&mdo, const_cast<void *>(dout), 2, qd, qs2, qbox, true) ||
         !encode_tensor_map_4d(&mk, const_cast<void *>(k), 2, kd, ks2, kbox, true) ||
         !encode_tensor_map_4d(&mv, const_cast<void *>(v), 2, kd, ks2, kbox, true) ||
-        !encode_tensor_map_4d(&mdq, dq_acc, 4, qd, qs4, qbox, false))
+        !encode_tensor_map_4d(&mdq, dq_acc, 4, qd, qs4, dqbox, true))
         return cudaErrorInvalidValue;
     cudaError_t e = cudaMemsetAsync(dq_acc, 0, bwd_tc_dq_acc_bytes(s), st);
     if (e != cudaSuccess) return e;

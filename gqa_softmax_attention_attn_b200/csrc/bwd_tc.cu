@@ -46,9 +46,13 @@ namespace {
 constexpr int kM = 128;  // keys per tile (rows of the transposed score tile)
 constexpr int kD = 64;
 constexpr int kThreads = 448;  // 14 warps: loads, MMA, 4 dQ, 8 gradient
-// 1: half of phase 1's exponentials on the FMA pipe (fast_exp2x2)
+// exponentials of the first phase on the FMA pipe (fast_exp2x2): 0 none, 1 half, 2 a quarter
 #ifndef ATTN_SINK_BWD_EMU
 #define ATTN_SINK_BWD_EMU 0
+#endif
+// bf16 packing with integer rounding (pack_bf16x2_alu): bit 0 for P, bit 1 for dS
+#ifndef ATTN_SINK_BWD_PACK
+#define ATTN_SINK_BWD_PACK 0
 #endif
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -235,51 +239,62 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issue
-        if (lane == 0) {
-            const uint32_t id_t = idesc_bf16_f32(kM, kM, 0, 0);       // S^T, dP^T: N = 128 q rows
-            const uint32_t id_kv = idesc_bf16_f32(kM, kD, 1, 0);      // dV, dK: B MN-major
-            const uint32_t id_q = idesc_bf16_f32(kM, kD, 1, 1);       // dQ: A and B MN-major
-            const uint64_t d_k = smem_desc_sw128(smem_u32(smem + kOffK), 16, 1024);
-            const uint64_t d_v = smem_desc_sw128(smem_u32(smem + kOffV), 16, 1024);
-            const uint64_t d_q = smem_desc_sw128(smem_u32(smem + kOffQ), 16, 1024);
-            const uint64_t d_do = smem_desc_sw128(smem_u32(smem + kOffDO), 16, 1024);
-            const uint64_t d_ds = smem_desc_sw128(smem_u32(smem + kOffDS), kTile, 1024);
-            const uint64_t d_kmn = smem_desc_sw128(smem_u32(smem + kOffK), kTile, 1024);
-            bool ok = n_iter > 0 && mbar_wait(kv_full, 0, abort_flag, p.status, p.timeout_ns);
-            // S^T(i) = K Q(i)^T into its own TMEM tile; issued for tile i+1 as
-            // soon as the softmax-gradient threads have read S^T(i) out.
-            auto issue_st = [&](int i) -> bool {
-                const int st = i & 1;
-                if (!mbar_wait(&qdo_full[st], (i >> 1) & 1u, abort_flag, p.status, p.timeout_ns)) return false;
-                if (i > 0 && !mbar_wait(s_consumed, (i - 1) & 1u, abort_flag, p.status, p.timeout_ns)) return false;
-                tc_fence_after();
-                const uint64_t q_st = d_q + (uint64_t)((st * kTile) >> 4);
+        // The whole warp runs this loop (so every operand is warp-uniform) and
+        // one elected lane issues the MMAs and their commits.
+        const uint32_t id_t = idesc_bf16_f32(kM, kM, 0, 0);       // S^T, dP^T: N = 128 q rows
+        const uint32_t id_kv = idesc_bf16_f32(kM, kD, 1, 0);      // dV, dK: B MN-major
+        const uint32_t id_q = idesc_bf16_f32(kM, kD, 1, 1);       // dQ: A and B MN-major
+        const uint64_t d_k = smem_desc_sw128(smem_u32(smem + kOffK), 16, 1024);
+        const uint64_t d_v = smem_desc_sw128(smem_u32(smem + kOffV), 16, 1024);
+        const uint64_t d_q = smem_desc_sw128(smem_u32(smem + kOffQ), 16, 1024);
+        const uint64_t d_do = smem_desc_sw128(smem_u32(smem + kOffDO), 16, 1024);
+        const uint64_t d_ds = smem_desc_sw128(smem_u32(smem + kOffDS), kTile, 1024);
+        const uint64_t d_kmn = smem_desc_sw128(smem_u32(smem + kOffK), kTile, 1024);
+        auto wait_all = [&](uint64_t *bar, uint32_t parity) {
+            return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, p.status, p.timeout_ns));
+        };
+        bool ok = n_iter > 0 && wait_all(kv_full, 0);
+        // S^T(i) = K Q(i)^T into its own TMEM tile; issued for tile i+1 as
+        // soon as the softmax-gradient threads have read S^T(i) out.
+        auto issue_st = [&](int i) -> bool {
+            const int st = i & 1;
+            if (!wait_all(&qdo_full[st], (i >> 1) & 1u)) return false;
+            if (i > 0 && !wait_all(s_consumed, (i - 1) & 1u)) return false;
+            tc_fence_after();
+            const uint64_t q_st = d_q + (uint64_t)((st * kTile) >> 4);
+            if (elect_one()) {
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk) mma_ss(tmem + kTmST, d_k + 2 * kk, q_st + 2 * kk, id_t, kk > 0);
                 mma_commit(s_full);
-                return true;
-            };
-            // dP^T(i) = V dO(i)^T; its columns held dS^T(i-1), read by dK(i-1),
-            // which was issued before it (tcgen05 MMAs of one thread run in order)
-            auto issue_dpt = [&](int i) {
-                const uint64_t do_st = d_do + (uint64_t)(((i & 1) * kTile) >> 4);
-                tc_fence_after();
+            }
+            __syncwarp();
+            return true;
+        };
+        // dP^T(i) = V dO(i)^T; its columns held dS^T(i-1), read by dK(i-1),
+        // which was issued before it (tcgen05 MMAs of one thread run in order)
+        auto issue_dpt = [&](int i) {
+            const uint64_t do_st = d_do + (uint64_t)(((i & 1) * kTile) >> 4);
+            tc_fence_after();
+            if (elect_one()) {
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk)
                     mma_ss(tmem + kTmDPT, d_v + 2 * kk, do_st + 2 * kk, id_t, kk > 0);
                 mma_commit(dp_full);
-            };
-            if (ok) ok = issue_st(0);
-            if (ok) issue_dpt(0);
-            for (int i = 0; i < n_iter && ok; ++i) {
-                const int st = i & 1;
-                const uint64_t q_st = d_q + (uint64_t)((st * kTile) >> 4);
-                const uint64_t do_st = d_do + (uint64_t)((st * kTile) >> 4);
-                // scores of the next q tile, as soon as S^T(i) has been read
-                if (i + 1 < n_iter && !issue_st(i + 1)) break;
-                if (!mbar_wait(p_ready, i & 1u, abort_flag, p.status, p.timeout_ns)) break;
-                tc_fence_after();
-                // dV += P^T dO and dK += dS^T Q: K = 128 q rows in steps of 16 (2048 bytes of the MN-major B)
+            }
+            __syncwarp();
+        };
+        if (ok) ok = issue_st(0);
+        if (ok) issue_dpt(0);
+        for (int i = 0; i < n_iter && ok; ++i) {
+            const int st = i & 1;
+            const uint64_t q_st = d_q + (uint64_t)((st * kTile) >> 4);
+            const uint64_t do_st = d_do + (uint64_t)((st * kTile) >> 4);
+            // scores of the next q tile, as soon as S^T(i) has been read
+            if (i + 1 < n_iter && !issue_st(i + 1)) break;
+            if (!wait_all(p_ready, i & 1u)) break;
+            tc_fence_after();
+            // dV += P^T dO and dK += dS^T Q: K = 128 q rows in steps of 16 (2048 bytes of the MN-major B)
+            if (elect_one()) {
 #pragma unroll
                 for (int kk = 0; kk < kM / 16; ++kk)
                     mma_ts(tmem + kTmDV, tmem + kTmPT + kk * 8, do_st + 128 * kk, id_kv, (i > 0 || kk > 0));
@@ -289,25 +304,31 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mma_ts(tmem + kTmDK, tmem + kTmDPT + kk * 8 + (kk >= kM / 32 ? kM / 4 : 0), q_st + 128 * kk,
                            id_kv, (i > 0 || kk > 0));
                 mma_commit(&qdo_empty[st]);
-                // dP^T of the next q tile ahead of dQ(i), which only the dQ epilogue waits for
-                if (i + 1 < n_iter) {
-                    if (!mbar_wait(&qdo_full[(i + 1) & 1], ((i + 1) >> 1) & 1u, abort_flag, p.status, p.timeout_ns))
-                        break;
-                    issue_dpt(i + 1);
-                }
-                if (!mbar_wait(dq_free, (i & 1u) ^ 1u, abort_flag, p.status, p.timeout_ns)) break;
-                tc_fence_after();
-                // dQ = dS K: K = 128 keys in steps of 16
+            }
+            __syncwarp();
+            // dP^T of the next q tile ahead of dQ(i), which only the dQ epilogue waits for
+            if (i + 1 < n_iter) {
+                if (!wait_all(&qdo_full[(i + 1) & 1], ((i + 1) >> 1) & 1u)) break;
+                issue_dpt(i + 1);
+            }
+            if (!wait_all(dq_free, (i & 1u) ^ 1u)) break;
+            tc_fence_after();
+            // dQ = dS K: K = 128 keys in steps of 16
+            if (elect_one()) {
 #pragma unroll
                 for (int kk = 0; kk < kM / 16; ++kk)
                     mma_ss(tmem + kTmDQ, d_ds + 128 * kk, d_kmn + 128 * kk, id_q, kk > 0);
                 mma_commit(dq_full);
                 mma_commit(ds_free);
             }
+            __syncwarp();
+        }
+        if (elect_one()) {
             mma_commit(dkv_done);
             mma_commit(drain);
-            wait_noabort(drain, 0, p.status, p.timeout_ns);
         }
+        __syncwarp();
+        wait_noabort(drain, 0, p.status, p.timeout_ns);
     } else if (warp <= 5 || warp >= 10) {
         // ------------------------------------------------------------ P and dS, one key row per warp pair
         constexpr int kCh = kM / 32;       // 16-column chunks per half
@@ -359,7 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const float4 l4 = l2v[4 * (c0 + c) + e4];
                     const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
                     float pe[4];
-                    if (ATTN_SINK_BWD_EMU && (e4 & 1)) {
+                    if ((ATTN_SINK_BWD_EMU == 1 && (e4 & 1)) || (ATTN_SINK_BWD_EMU == 2 && e4 == 3)) {
                         const float2 a = fast_exp2x2(make_float2(fmaf(__uint_as_float(sr[4 * e4 + 0]), C, -lv[0]),
                                                                  fmaf(__uint_as_float(sr[4 * e4 + 1]), C, -lv[1])));
                         const float2 bq = fast_exp2x2(make_float2(fmaf(__uint_as_float(sr[4 * e4 + 2]), C, -lv[2]),
@@ -377,8 +398,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                             pe[u] = (pl >= pl_lo && pl <= pl_hi) ? pe[u] : 0.f;
                         }
                     }
-                    pk[8 * c + 2 * e4] = pack_bf16x2(pe[0], pe[1]);
-                    pk[8 * c + 2 * e4 + 1] = pack_bf16x2(pe[2], pe[3]);
+                    pk[8 * c + 2 * e4] = (ATTN_SINK_BWD_PACK & 1) ? pack_bf16x2_alu(pe[0], pe[1]) : pack_bf16x2(pe[0], pe[1]);
+                    pk[8 * c + 2 * e4 + 1] = (ATTN_SINK_BWD_PACK & 1) ? pack_bf16x2_alu(pe[2], pe[3]) : pack_bf16x2(pe[2], pe[3]);
                 }
                 tmem_wait_ld();
             }
@@ -420,8 +441,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const float ds1 = __high2float(p01) * (__uint_as_float(dr[4 * e4 + 1]) - d4.y);
                     const float ds2 = __low2float(p23) * (__uint_as_float(dr[4 * e4 + 2]) - d4.z);
                     const float ds3 = __high2float(p23) * (__uint_as_float(dr[4 * e4 + 3]) - d4.w);
-                    dk[2 * e4] = pack_bf16x2(ds0, ds1);
-                    dk[2 * e4 + 1] = pack_bf16x2(ds2, ds3);
+                    dk[2 * e4] = (ATTN_SINK_BWD_PACK & 2) ? pack_bf16x2_alu(ds0, ds1) : pack_bf16x2(ds0, ds1);
+                    dk[2 * e4 + 1] = (ATTN_SINK_BWD_PACK & 2) ? pack_bf16x2_alu(ds2, ds3) : pack_bf16x2(ds2, ds3);
                 }
                 // dS^T over 8 columns of dP^T this warp has read (64 half + 8c .. + 7)
                 tmem_st8(trow + kTmDPT + 16 * c0 + 8 * c, dk);

@@ -162,6 +162,20 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
         : "memory");
 }
 
+// One lane of a converged warp (the lowest active one) returns true.  Issuing
+// tcgen05.mma / commit under it from a warp that runs the issue loop together
+// keeps descriptors and TMEM addresses warp-uniform.
+__device__ __forceinline__ bool elect_one()
+{
+    uint32_t e;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "elect.sync _|p, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(e));
+    return e != 0;
+}
+
 // Arrive once on `bar` when every tcgen05 op issued so far by this thread completes.
 __device__ __forceinline__ void mma_commit(uint64_t *bar)
 {
@@ -277,6 +291,18 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// Same packing, rounded to nearest-even with integer ops (add 0x7FFF plus
+// the lowest kept bit, keep the upper half), so it runs on the ALU/FMA pipes
+// instead of the conversion unit.  Exact for every finite input; a NaN input
+// may come out as infinity.
+__device__ __forceinline__ uint32_t pack_bf16x2_alu(float lo, float hi)
+{
+    uint32_t a = __float_as_uint(lo), b = __float_as_uint(hi);
+    a += 0x7fffu + ((a >> 16) & 1u);
+    b += 0x7fffu + ((b >> 16) & 1u);
+    return __byte_perm(a, b, 0x7632);
 }
 
 // max of three floats in one instruction

@@ -16,8 +16,9 @@
 //    each) walk a static longest-first list of work items.
 //  * Warp 0: TMA producer -- Q (double-buffered, so the next item's Q lands
 //    while the current one finishes) and K/V tiles of BN keys into an
-//    NS-stage ring.  Warp 1: allocates tensor memory and issues tcgen05.mma
-//    from one thread: S = Q K^T into a double-buffered TMEM tile, O += P V
+//    NS-stage ring.  Warp 1: allocates tensor memory and runs the MMA issue
+//    loop as a whole warp (warp-uniform descriptors), one elected lane
+//    issuing tcgen05.mma: S = Q K^T into a double-buffered TMEM tile, O += P V
 //    with P read back from TMEM.  Warps 2-5: one thread per row --
 //    tcgen05.ld of S, masking, the exp2 softmax, P written over S as bf16,
 //    conditional rescale of O, epilogue.
@@ -238,23 +239,27 @@ __global__ void __launch_bounds__(192, CPS)
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            const uint32_t id_s = idesc_bf16_f32(kM, BN, 0);
-            const uint32_t id_pv = idesc_bf16_f32(kM, kD, 1);
-            const uint32_t k_addr = smem_u32(smem + Cfg::kOffK);
-            const uint32_t v_addr = smem_u32(smem + Cfg::kOffV);
-            uint32_t it = 0, item_n = 0;
-            bool ok = true;
-            // O += P(t) V(t); the first product of an item overwrites O, which
-            // must wait until the previous item's epilogue has read O out.
-            auto issue_pv = [&](uint32_t t, bool first) -> bool {
-                const int sb = t & 1, st = t % NS;
-                if (first && !mbar_wait(o_free, (item_n & 1u) ^ 1u, abort_flag, p.status, p.timeout_ns))
-                    return false;
-                if (!mbar_wait(&p_full[sb], (t >> 1) & 1u, abort_flag, p.status, p.timeout_ns)) return false;
-                if (!mbar_wait(&v_full[st], (t / NS) & 1u, abort_flag, p.status, p.timeout_ns)) return false;
-                tc_fence_after();
-                const uint32_t vb = v_addr + st * Cfg::kKVBytes;
+        // The whole warp runs this loop (so every operand is warp-uniform) and
+        // one elected lane issues the MMAs and their commits.
+        const uint32_t id_s = idesc_bf16_f32(kM, BN, 0);
+        const uint32_t id_pv = idesc_bf16_f32(kM, kD, 1);
+        const uint32_t k_addr = smem_u32(smem + Cfg::kOffK);
+        const uint32_t v_addr = smem_u32(smem + Cfg::kOffV);
+        auto wait_all = [&](uint64_t *bar, uint32_t parity) {
+            return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, p.status, p.timeout_ns));
+        };
+        uint32_t it = 0, item_n = 0;
+        bool ok = true;
+        // O += P(t) V(t); the first product of an item overwrites O, which
+        // must wait until the previous item's epilogue has read O out.
+        auto issue_pv = [&](uint32_t t, bool first) -> bool {
+            const int sb = t & 1, st = t % NS;
+            if (first && !wait_all(o_free, (item_n & 1u) ^ 1u)) return false;
+            if (!wait_all(&p_full[sb], (t >> 1) & 1u)) return false;
+            if (!wait_all(&v_full[st], (t / NS) & 1u)) return false;
+            tc_fence_after();
+            const uint32_t vb = v_addr + st * Cfg::kKVBytes;
+            if (elect_one()) {
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk) {
                     // V tile [BN keys][64 d] is the MN-major B operand: 16 keys = 2048 bytes per step
@@ -264,23 +269,26 @@ __global__ void __launch_bounds__(192, CPS)
                 }
                 mma_commit(o_done);
                 mma_commit(&v_empty[st]);
-                return true;
-            };
-            for (int w = blockIdx.x; w < p.n_items && ok; w += gridDim.x) {
-                const Item t = item_at<BN>(p, w);
-                if (t.n_tiles == 0) continue;
-                const int qb = item_n & 1;
-                if (!mbar_wait(&q_full[qb], (item_n >> 1) & 1u, abort_flag, p.status, p.timeout_ns)) break;
+            }
+            __syncwarp();
+            return true;
+        };
+        for (int w = blockIdx.x; w < p.n_items && ok; w += gridDim.x) {
+            const Item t = item_at<BN>(p, w);
+            if (t.n_tiles == 0) continue;
+            const int qb = item_n & 1;
+            if (!wait_all(&q_full[qb], (item_n >> 1) & 1u)) break;
+            tc_fence_after();
+            const uint32_t q_addr = smem_u32(smem + Cfg::kOffQ + qb * Cfg::kQBytes);
+            for (int jt = 0; jt < t.n_tiles; ++jt, ++it) {
+                const int st = it % NS, sb = it & 1;
+                if (!wait_all(&k_full[st], (it / NS) & 1u)) {
+                    ok = false;
+                    break;
+                }
                 tc_fence_after();
-                const uint32_t q_addr = smem_u32(smem + Cfg::kOffQ + qb * Cfg::kQBytes);
-                for (int jt = 0; jt < t.n_tiles; ++jt, ++it) {
-                    const int st = it % NS, sb = it & 1;
-                    if (!mbar_wait(&k_full[st], (it / NS) & 1u, abort_flag, p.status, p.timeout_ns)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t kb = k_addr + st * Cfg::kKVBytes;
+                const uint32_t kb = k_addr + st * Cfg::kKVBytes;
+                if (elect_one()) {
 #pragma unroll
                     for (int kk = 0; kk < kD / 16; ++kk) {
                         const uint64_t adesc = smem_desc_sw128(q_addr + kk * 32, 16, 1024);
@@ -290,20 +298,22 @@ __global__ void __launch_bounds__(192, CPS)
                     mma_commit(&s_full[sb]);
                     mma_commit(&k_empty[st]);
                     if (jt == t.n_tiles - 1) mma_commit(&q_empty[qb]);
-                    if (jt >= 1 && !issue_pv(it - 1, jt == 1)) {
-                        ok = false;
-                        break;
-                    }
                 }
-                if (!ok || !issue_pv(it - 1, t.n_tiles == 1)) {
+                __syncwarp();
+                if (jt >= 1 && !issue_pv(it - 1, jt == 1)) {
                     ok = false;
                     break;
                 }
-                ++item_n;
             }
-            mma_commit(drain);
-            wait_noabort(drain, 0, p.status, p.timeout_ns);
+            if (!ok || !issue_pv(it - 1, t.n_tiles == 1)) {
+                ok = false;
+                break;
+            }
+            ++item_n;
         }
+        if (elect_one()) mma_commit(drain);
+        __syncwarp();
+        wait_noabort(drain, 0, p.status, p.timeout_ns);
     } else {
         // ------------------------------------------------------------ softmax + epilogue
         const int quad = warp & 3;

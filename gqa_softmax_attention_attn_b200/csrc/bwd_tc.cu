@@ -37,6 +37,8 @@
 #include <cuda_bf16.h>
 #include <math.h>
 
+#include <type_traits>
+
 #include "kernels.h"
 #include "sm100_ptx.cuh"
 
@@ -46,14 +48,6 @@ namespace {
 constexpr int kM = 128;  // keys per tile (rows of the transposed score tile)
 constexpr int kD = 64;
 constexpr int kThreads = 448;  // 14 warps: loads, MMA, 4 dQ, 8 gradient
-// exponentials of the first phase on the FMA pipe (fast_exp2x2): 0 none, 1 half, 2 a quarter
-#ifndef ATTN_SINK_BWD_EMU
-#define ATTN_SINK_BWD_EMU 0
-#endif
-// bf16 packing with integer rounding (pack_bf16x2_alu): bit 0 for P, bit 1 for dS
-#ifndef ATTN_SINK_BWD_PACK
-#define ATTN_SINK_BWD_PACK 0
-#endif
 constexpr float kLog2e = 1.4426950408889634f;
 
 constexpr int kTile = kM * kD * 2;  // 16 KB bf16 tile
@@ -366,43 +360,42 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float4 *ddv = reinterpret_cast<const float4 *>(ld + (st * 2 + 1) * kM);
 
             // phase 1: P = exp2(S C - lse2) from S^T, kept as bf16 pairs; then S^T is free
-            // TMEM loads are pipelined one 16-column chunk ahead of the arithmetic
+            // TMEM loads are pipelined one 16-column chunk ahead of the arithmetic.
+            // Compiled twice: tiles with no masked element (most of them) run
+            // without the per-element visibility test.
             uint32_t pk[kM / 4];
-            uint32_t sbuf[2][16];
-            tmem_ld16(trow + kTmST + 16 * c0, sbuf[0]);
-            tmem_wait_ld();
-#pragma unroll
-            for (int c = 0; c < kCh; ++c) {
-                if (c + 1 < kCh) tmem_ld16(trow + kTmST + 16 * (c0 + c + 1), sbuf[(c + 1) & 1]);
-                const uint32_t *sr = sbuf[c & 1];
-#pragma unroll
-                for (int e4 = 0; e4 < 4; ++e4) {
-                    const float4 l4 = l2v[4 * (c0 + c) + e4];
-                    const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-                    float pe[4];
-                    if ((ATTN_SINK_BWD_EMU == 1 && (e4 & 1)) || (ATTN_SINK_BWD_EMU == 2 && e4 == 3)) {
-                        const float2 a = fast_exp2x2(make_float2(fmaf(__uint_as_float(sr[4 * e4 + 0]), C, -lv[0]),
-                                                                 fmaf(__uint_as_float(sr[4 * e4 + 1]), C, -lv[1])));
-                        const float2 bq = fast_exp2x2(make_float2(fmaf(__uint_as_float(sr[4 * e4 + 2]), C, -lv[2]),
-                                                                  fmaf(__uint_as_float(sr[4 * e4 + 3]), C, -lv[3])));
-                        pe[0] = a.x; pe[1] = a.y; pe[2] = bq.x; pe[3] = bq.y;
-                    } else {
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) pe[u] = ex2(fmaf(__uint_as_float(sr[4 * e4 + u]), C, -lv[u]));
-                    }
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int col = 16 * (c0 + c) + 4 * e4 + u;
-                        if (need_mask) {
-                            const int pl = col / GP;
-                            pe[u] = (pl >= pl_lo && pl <= pl_hi) ? pe[u] : 0.f;
-                        }
-                    }
-                    pk[8 * c + 2 * e4] = (ATTN_SINK_BWD_PACK & 1) ? pack_bf16x2_alu(pe[0], pe[1]) : pack_bf16x2(pe[0], pe[1]);
-                    pk[8 * c + 2 * e4 + 1] = (ATTN_SINK_BWD_PACK & 1) ? pack_bf16x2_alu(pe[2], pe[3]) : pack_bf16x2(pe[2], pe[3]);
-                }
+            auto phase1 = [&](auto masked_tag) {
+                constexpr bool kMasked = decltype(masked_tag)::value;
+                uint32_t sbuf[2][16];
+                tmem_ld16(trow + kTmST + 16 * c0, sbuf[0]);
                 tmem_wait_ld();
-            }
+#pragma unroll
+                for (int c = 0; c < kCh; ++c) {
+                    if (c + 1 < kCh) tmem_ld16(trow + kTmST + 16 * (c0 + c + 1), sbuf[(c + 1) & 1]);
+                    const uint32_t *sr = sbuf[c & 1];
+#pragma unroll
+                    for (int e4 = 0; e4 < 4; ++e4) {
+                        const float4 l4 = l2v[4 * (c0 + c) + e4];
+                        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+                        float pe[4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            pe[u] = ex2(fmaf(__uint_as_float(sr[4 * e4 + u]), C, -lv[u]));
+                            if (kMasked) {
+                                const int pl = (16 * (c0 + c) + 4 * e4 + u) / GP;
+                                pe[u] = (pl >= pl_lo && pl <= pl_hi) ? pe[u] : 0.f;
+                            }
+                        }
+                        pk[8 * c + 2 * e4] = pack_bf16x2(pe[0], pe[1]);
+                        pk[8 * c + 2 * e4 + 1] = pack_bf16x2(pe[2], pe[3]);
+                    }
+                    tmem_wait_ld();
+                }
+            };
+            if (need_mask)
+                phase1(std::true_type{});
+            else
+                phase1(std::false_type{});
             // P^T into its columns once dV(i-1) has read the previous P^T
             if (i > 0 &&
                 !__all_sync(0xffffffffu, mbar_wait(pt_free, (i - 1) & 1u, abort_flag, p.status, p.timeout_ns))) {
@@ -441,8 +434,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const float ds1 = __high2float(p01) * (__uint_as_float(dr[4 * e4 + 1]) - d4.y);
                     const float ds2 = __low2float(p23) * (__uint_as_float(dr[4 * e4 + 2]) - d4.z);
                     const float ds3 = __high2float(p23) * (__uint_as_float(dr[4 * e4 + 3]) - d4.w);
-                    dk[2 * e4] = (ATTN_SINK_BWD_PACK & 2) ? pack_bf16x2_alu(ds0, ds1) : pack_bf16x2(ds0, ds1);
-                    dk[2 * e4 + 1] = (ATTN_SINK_BWD_PACK & 2) ? pack_bf16x2_alu(ds2, ds3) : pack_bf16x2(ds2, ds3);
+                    dk[2 * e4] = pack_bf16x2(ds0, ds1);
+                    dk[2 * e4 + 1] = pack_bf16x2(ds2, ds3);
                 }
                 // dS^T over 8 columns of dP^T this warp has read (64 half + 8c .. + 7)
                 tmem_st8(trow + kTmDPT + 16 * c0 + 8 * c, dk);

@@ -21,7 +21,9 @@
 //    issuing tcgen05.mma: S = Q K^T into a double-buffered TMEM tile, O += P V
 //    with P read back from TMEM.  Warps 2-5: one thread per row --
 //    tcgen05.ld of S, masking, the exp2 softmax, P written over S as bf16,
-//    conditional rescale of O, epilogue.
+//    conditional rescale of O, epilogue.  (Compile-time option SPLIT = 2:
+//    warps 2-9, two per row on half the columns each, trading partial maxima
+//    and sums through shared memory under a per-quadrant mbarrier.)
 //  * The running maximum used for the exponentials is only moved when the
 //    true maximum exceeds it by more than 2^8, so the O rescale (which must
 //    wait for the previous PV product) is rare; the result is exact either
@@ -60,14 +62,35 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 #endif
 
 // Tile configurations (keys per tile BN, K/V stages NS, EMU = which pair of
-// every 4 uses the FMA-pipe exp2, -1 for none), chosen per layer type from
-// measurements on the gpt-oss-20b prefill: the dense causal layer runs best
-// with BN = 96 and a quarter of the exponentials off the MUFU unit, the
-// window-128 layer with BN = 64 and all exponentials on MUFU.
+// every 4 uses the FMA-pipe exp2 (4: every odd pair, -1: none), CTAs per
+// SM), chosen per layer type from measurements on the gpt-oss-20b prefill:
+// the dense causal layer runs best with BN = 96, two CTAs per SM and a
+// quarter of the exponentials off the MUFU unit (none: 3% slower, half: 4%
+// slower), the window-128 layer with the banded configuration above.
+#ifndef ATTN_SINK_FWD_DENSE_BN
+#define ATTN_SINK_FWD_DENSE_BN 96
+#define ATTN_SINK_FWD_DENSE_NS 3
+#endif
+#ifndef ATTN_SINK_FWD_DENSE_EMU
+#define ATTN_SINK_FWD_DENSE_EMU 3
+#endif
+// softmax warps per row (1 or 2) per layer type; two warps per row (half the
+// columns each, partial maxima traded every tile) measured slower on both
+// layers of the gpt-oss-20b prefill (dense 239 vs 212 us, banded 52 vs 47 us)
+#ifndef ATTN_SINK_FWD_DENSE_SPLIT
+#define ATTN_SINK_FWD_DENSE_SPLIT 1
+#endif
+#ifndef ATTN_SINK_FWD_BAND_SPLIT
+#define ATTN_SINK_FWD_BAND_SPLIT 1
+#endif
 constexpr int pow2_at_least(int x) { return x <= 32 ? 32 : x <= 64 ? 64 : x <= 128 ? 128 : x <= 256 ? 256 : 512; }
 
-template <int BN, int NS, int CPS>
+template <int BN, int NS, int CPS, int SPLIT>
 struct FwdCfg {
+    static_assert(SPLIT == 1 || SPLIT == 2, "one or two softmax warps per row");
+    static_assert(BN % (16 * SPLIT) == 0, "each softmax warp takes whole 16-column chunks");
+    static constexpr int kThreads = 64 + 128 * SPLIT;
+    static constexpr int kCols = BN / SPLIT;  // score columns per softmax thread
     static constexpr int kQBytes = kM * kD * 2;
     static constexpr int kKVBytes = BN * kD * 2;
     static constexpr int kOffQ = 0;  // two Q buffers
@@ -75,15 +98,17 @@ struct FwdCfg {
     static constexpr int kOffV = kOffK + NS * kKVBytes;
     static constexpr int kOffBar = kOffV + NS * kKVBytes;
     // q_full[2], q_empty[2], k_full[NS], k_empty[NS], v_full[NS], v_empty[NS],
-    // s_full[2], p_full[2], o_done, o_free, drain
-    static constexpr int kNumBar = 4 + 4 * NS + 4 + 3;
+    // s_full[2], p_full[2], o_done, o_free, drain, xchg[4]
+    static constexpr int kNumBar = 4 + 4 * NS + 4 + 3 + 4;
     static constexpr int kOffMisc = kOffBar + kNumBar * 8;
+    // row partials exchanged by the two softmax warps of a row: [2 slots][2 halves][128 rows]
+    static constexpr int kOffXchg = kOffMisc + 64;
     static constexpr int kTmemCols = pow2_at_least(2 * BN + kD);
     static constexpr int kCtasPerSm = CPS;  // CTAs resident per SM (TMEM, registers, shared memory)
     static_assert(kTmemCols * CPS <= 512, "tensor memory over-subscribed");
     // + slack for 1024-byte alignment; a CTA that takes all 512 TMEM columns
     // also takes enough shared memory that no second CTA lands on its SM
-    static constexpr int kSmemUsed = kOffMisc + 16 + 1024;
+    static constexpr int kSmemUsed = kOffXchg + 2 * 2 * kM * 4 + 1024;
     static constexpr int kSmemBytes = (kCtasPerSm == 1 && kSmemUsed < 116 * 1024) ? 116 * 1024 : kSmemUsed;
     static constexpr int kTmS0 = 0;
     static constexpr int kTmO = 2 * BN;
@@ -136,12 +161,12 @@ __device__ __forceinline__ bool wait_noabort(uint64_t *bar, uint32_t parity, uns
     return mbar_wait(bar, parity, &never, status, tmo > 1000000000LL ? tmo : 1000000000LL);
 }
 
-template <int BN, int NS, int EMU, int CPS>
-__global__ void __launch_bounds__(192, CPS)
+template <int BN, int NS, int EMU, int CPS, int SPLIT>
+__global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT>::kThreads, CPS)
     fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdTcParams p)
 {
-    using Cfg = FwdCfg<BN, NS, CPS>;
+    using Cfg = FwdCfg<BN, NS, CPS, SPLIT>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kOffBar);
@@ -156,6 +181,8 @@ __global__ void __launch_bounds__(192, CPS)
     uint64_t *o_done = p_full + 2;
     uint64_t *o_free = o_done + 1;
     uint64_t *drain = o_free + 1;
+    uint64_t *xchg = drain + 1;  // [4]: one per TMEM lane quadrant (SPLIT == 2)
+    float *xs = reinterpret_cast<float *>(smem + Cfg::kOffXchg);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Cfg::kOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Cfg::kOffMisc + 4);
 
@@ -166,7 +193,7 @@ __global__ void __launch_bounds__(192, CPS)
             mbar_init(&q_full[s], 1);
             mbar_init(&q_empty[s], 1);
             mbar_init(&s_full[s], 1);
-            mbar_init(&p_full[s], 128);
+            mbar_init(&p_full[s], 128 * SPLIT);
         }
         for (int s = 0; s < NS; ++s) {
             mbar_init(&k_full[s], 1);
@@ -175,8 +202,9 @@ __global__ void __launch_bounds__(192, CPS)
             mbar_init(&v_empty[s], 1);
         }
         mbar_init(o_done, 1);
-        mbar_init(o_free, 128);
+        mbar_init(o_free, 128 * SPLIT);
         mbar_init(drain, 1);
+        for (int qd = 0; qd < 4; ++qd) mbar_init(&xchg[qd], 64);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -264,7 +292,10 @@ __global__ void __launch_bounds__(192, CPS)
                 for (int kk = 0; kk < BN / 16; ++kk) {
                     // V tile [BN keys][64 d] is the MN-major B operand: 16 keys = 2048 bytes per step
                     const uint64_t bdesc = smem_desc_sw128(vb + kk * 2048, BN * 128, 1024);
-                    mma_ts(tmem + Cfg::kTmO, tmem + Cfg::kTmS0 + sb * BN + kk * 8, bdesc, id_pv,
+                    // P of keys 16kk..16kk+15: 8 packed columns; the softmax warp of
+                    // column half h writes its P at the start of its own S columns
+                    const int hcol = (16 * kk / Cfg::kCols) * (Cfg::kCols / 2);
+                    mma_ts(tmem + Cfg::kTmO, tmem + Cfg::kTmS0 + sb * BN + kk * 8 + hcol, bdesc, id_pv,
                            (!first || kk > 0) ? 1u : 0u);
                 }
                 mma_commit(o_done);
@@ -316,13 +347,33 @@ __global__ void __launch_bounds__(192, CPS)
         wait_noabort(drain, 0, p.status, p.timeout_ns);
     } else {
         // ------------------------------------------------------------ softmax + epilogue
+        // SPLIT warps per row: the warp of column half h (warps 2-5: h = 0,
+        // warps 6-9: h = 1) takes score columns [h kCols, (h + 1) kCols) of
+        // each tile and O columns [h 64 / SPLIT, ...).  The two halves of a row
+        // trade their partial maxima every tile (and their partial sums at the
+        // end of an item) through shared memory, ordered by the quadrant's
+        // exchange barrier, so both take the same reference maximum.
+        constexpr int kC = Cfg::kCols;
+        constexpr int kOC = kD / SPLIT;  // O columns per thread
         const int quad = warp & 3;
+        const int half = SPLIT == 2 ? (warp - 2) >> 2 : 0;
         const int r = quad * 32 + lane;
         const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
         const float C = p.c_log2;
         const long off = (long)p.Lk - p.Lq;
-        uint32_t it = 0;
+        uint32_t it = 0, xc = 0;
         bool ok = true;
+        // publish v, get the other half's value (bounded wait; false on abort)
+        auto trade = [&](float v, float &other) -> bool {
+            const int slot = xc & 1;
+            xs[(slot * 2 + half) * kM + r] = v;
+            mbar_arrive(&xchg[quad]);
+            const bool got =
+                __all_sync(0xffffffffu, mbar_wait(&xchg[quad], xc & 1u, abort_flag, p.status, p.timeout_ns));
+            other = xs[(slot * 2 + (half ^ 1)) * kM + r];
+            ++xc;
+            return got;
+        };
         for (int w = blockIdx.x; w < p.n_items && ok; w += gridDim.x) {
             const Item t = item_at<BN>(p, w);
             const int pos = t.pos0 + r / p.Gp;
@@ -331,49 +382,59 @@ __global__ void __launch_bounds__(192, CPS)
             const long pabs = pos + off;
             const float sink2 = p.sinks[h] * kLog2e;  // the sink logit in log2 units
             float m = sink2;                           // reference maximum, log2 units
-            float l = (sink2 == -INFINITY) ? 0.f : 1.f;  // running sum, seeded with the sink's mass
+            // running sum, seeded with the sink's mass (in column half 0 only)
+            float l = (sink2 == -INFINITY || half != 0) ? 0.f : 1.f;
             // rows beyond Lq only need finite, unused values
             const long vis_hi = row_valid ? min(pabs, (long)p.Lk - 1) : -1;   // last visible key
             const long vis_lo = p.window > 0 ? pabs - p.window + 1 : 0;     // first visible key
 
             for (int jt = 0; jt < t.n_tiles; ++jt, ++it) {
                 const int sb = it & 1;
-                const long j0 = (long)(t.t_lo + jt) * BN;
+                const long j0 = (long)(t.t_lo + jt) * BN + half * kC;  // first key of this thread's columns
                 if (!__all_sync(0xffffffffu,
                                 mbar_wait(&s_full[sb], (it >> 1) & 1u, abort_flag, p.status, p.timeout_ns))) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                uint32_t sr[BN / 32][32];
+                const uint32_t scol = Cfg::kTmS0 + sb * BN + half * kC;
+                uint32_t sr[kC / 16][16];
 #pragma unroll
-                for (int c = 0; c < BN / 32; ++c) tmem_ld32(trow + Cfg::kTmS0 + sb * BN + c * 32, sr[c]);
+                for (int c = 0; c < kC / 16; ++c) tmem_ld16(trow + scol + c * 16, sr[c]);
                 tmem_wait_ld();
-                float sv[BN];
+                float sv[kC];
 #pragma unroll
-                for (int c = 0; c < BN; ++c) sv[c] = __uint_as_float(sr[c / 32][c % 32]);
-                // visible columns of this tile: c in [c_lo, c_hi] (32-bit, tile-relative)
-                const int c_hi = (int)max(-1L, min((long)BN - 1, vis_hi - j0));
-                const int c_lo = (int)max(0L, min((long)BN, vis_lo - j0));
-                const bool need_mask = __any_sync(0xffffffffu, c_lo > 0 || c_hi < BN - 1);
+                for (int c = 0; c < kC; ++c) sv[c] = __uint_as_float(sr[c / 16][c % 16]);
+                // visible columns of this thread: c in [c_lo, c_hi] (32-bit, relative to j0)
+                const int c_hi = (int)max(-1L, min((long)kC - 1, vis_hi - j0));
+                const int c_lo = (int)max(0L, min((long)kC, vis_lo - j0));
+                const bool need_mask = __any_sync(0xffffffffu, c_lo > 0 || c_hi < kC - 1);
                 if (need_mask) {
 #pragma unroll
-                    for (int c = 0; c < BN; ++c) sv[c] = (c >= c_lo && c <= c_hi) ? sv[c] : -INFINITY;
+                    for (int c = 0; c < kC; ++c) sv[c] = (c >= c_lo && c <= c_hi) ? sv[c] : -INFINITY;
                 }
                 // row max: four independent chains of 3-input max over columns
-                // 0-3 | 4..BN-1 in steps of 8 | the remaining 4 when (BN - 4) % 8 == 4
-                static_assert(BN % 32 == 0, "BN must be a multiple of 32");
+                // 0-3 | 4..kC-1 in steps of 8 | the remaining 4 when (kC - 4) % 8 == 4
+                static_assert(kC % 16 == 0, "whole 16-column chunks per thread");
                 float mx[4];
 #pragma unroll
                 for (int k = 0; k < 4; ++k) mx[k] = sv[k];
-                constexpr int kFull = 4 + ((BN - 4) / 8) * 8;
+                constexpr int kFull = 4 + ((kC - 4) / 8) * 8;
 #pragma unroll
                 for (int c = 4; c < kFull; c += 8)
 #pragma unroll
                     for (int k = 0; k < 4; ++k) mx[k] = fmax3(mx[k], sv[c + k], sv[c + 4 + k]);
 #pragma unroll
-                for (int k = 0; k < 4 && kFull + k < BN; ++k) mx[k] = fmaxf(mx[k], sv[kFull + k]);
-                const float tmax = fmax3(mx[0], mx[1], fmaxf(mx[2], mx[3]));
+                for (int k = 0; k < 4 && kFull + k < kC; ++k) mx[k] = fmaxf(mx[k], sv[kFull + k]);
+                float tmax = fmax3(mx[0], mx[1], fmaxf(mx[2], mx[3]));
+                if (SPLIT == 2) {
+                    float other;
+                    if (!trade(tmax, other)) {
+                        ok = false;
+                        break;
+                    }
+                    tmax = fmaxf(tmax, other);
+                }
                 const float m_new = fmaxf(m, tmax * C);
                 const bool rescale = m_new > m + kRescaleThreshold;
                 const float alpha = rescale ? ((m == -INFINITY) ? 0.f : ex2(m - m_new)) : 1.f;
@@ -381,36 +442,37 @@ __global__ void __launch_bounds__(192, CPS)
                 const float neg_m = (m == -INFINITY) ? 0.f : -m;
                 const float2 C2 = make_float2(C, C), M2 = make_float2(neg_m, neg_m);
                 float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-                // P (bf16 pairs) overwrites the first BN/2 columns of this S
-                // buffer, which has been read in full already; 32 scores per
-                // store.  On tiles with no masked element, pair EMU of every 4
-                // runs on the FMA pipe (fast_exp2x2) to offload the MUFU unit
+                // P (bf16 pairs) overwrites the first kC/2 columns of this
+                // thread's part of the S buffer, read in full already; 16 scores
+                // per store.  On tiles with no masked element, pair EMU of every
+                // 4 runs on the FMA pipe (fast_exp2x2) to offload the MUFU unit
                 // (two separate loops, so each element takes one path only).
                 if (!need_mask) {
 #pragma unroll
-                    for (int c = 0; c < BN / 32; ++c) {
-                        uint32_t pk[16];
+                    for (int c = 0; c < kC / 16; ++c) {
+                        uint32_t pk[8];
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) {
-                            const float2 x = ffma2(make_float2(sv[32 * c + 2 * e], sv[32 * c + 2 * e + 1]), C2, M2);
-                            const float2 pe = ((e & 3) == EMU) ? fast_exp2x2(x) : make_float2(ex2(x.x), ex2(x.y));
+                        for (int e = 0; e < 8; ++e) {
+                            const float2 x = ffma2(make_float2(sv[16 * c + 2 * e], sv[16 * c + 2 * e + 1]), C2, M2);
+                            const bool emu = EMU == 4 ? (e & 1) != 0 : (e & 3) == EMU;
+                            const float2 pe = emu ? fast_exp2x2(x) : make_float2(ex2(x.x), ex2(x.y));
                             acc[e & 1] = fadd2(acc[e & 1], pe);
                             pk[e] = pack_bf16x2(pe.x, pe.y);
                         }
-                        tmem_st16(trow + Cfg::kTmS0 + sb * BN + c * 16, pk);
+                        tmem_st8(trow + scol + c * 8, pk);
                     }
                 } else {
 #pragma unroll
-                    for (int c = 0; c < BN / 32; ++c) {
-                        uint32_t pk[16];
+                    for (int c = 0; c < kC / 16; ++c) {
+                        uint32_t pk[8];
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) {
-                            const float2 x = ffma2(make_float2(sv[32 * c + 2 * e], sv[32 * c + 2 * e + 1]), C2, M2);
+                        for (int e = 0; e < 8; ++e) {
+                            const float2 x = ffma2(make_float2(sv[16 * c + 2 * e], sv[16 * c + 2 * e + 1]), C2, M2);
                             const float2 pe = make_float2(ex2(x.x), ex2(x.y));
                             acc[e & 1] = fadd2(acc[e & 1], pe);
                             pk[e] = pack_bf16x2(pe.x, pe.y);
                         }
-                        tmem_st16(trow + Cfg::kTmS0 + sb * BN + c * 16, pk);
+                        tmem_st8(trow + scol + c * 8, pk);
                     }
                 }
                 l = l * alpha + ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y));
@@ -423,15 +485,15 @@ __global__ void __launch_bounds__(192, CPS)
                     }
                     tc_fence_after();
                     if (__any_sync(0xffffffffu, rescale)) {
-                        uint32_t o[2][32];
-                        tmem_ld32(trow + Cfg::kTmO, o[0]);
-                        tmem_ld32(trow + Cfg::kTmO + 32, o[1]);
+                        uint32_t o[kOC / 32][32];
+#pragma unroll
+                        for (int c = 0; c < kOC / 32; ++c) tmem_ld32(trow + Cfg::kTmO + half * kOC + 32 * c, o[c]);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int c = 0; c < 64; ++c)
+                        for (int c = 0; c < kOC; ++c)
                             o[c / 32][c % 32] = __float_as_uint(__uint_as_float(o[c / 32][c % 32]) * alpha);
-                        tmem_st32(trow + Cfg::kTmO, o[0]);
-                        tmem_st32(trow + Cfg::kTmO + 32, o[1]);
+#pragma unroll
+                        for (int c = 0; c < kOC / 32; ++c) tmem_st32(trow + Cfg::kTmO + half * kOC + 32 * c, o[c]);
                     }
                 }
                 tmem_wait_st();
@@ -441,7 +503,7 @@ __global__ void __launch_bounds__(192, CPS)
             if (!ok) break;
 
             // -------------------------------------------------------- epilogue
-            uint32_t o[2][32];
+            uint32_t o[kOC / 32][32];
             if (t.n_tiles > 0) {
                 if (!__all_sync(0xffffffffu,
                                 mbar_wait(o_done, (it - 1) & 1u, abort_flag, p.status, p.timeout_ns))) {
@@ -449,20 +511,29 @@ __global__ void __launch_bounds__(192, CPS)
                     break;
                 }
                 tc_fence_after();
-                tmem_ld32(trow + Cfg::kTmO, o[0]);
-                tmem_ld32(trow + Cfg::kTmO + 32, o[1]);
+#pragma unroll
+                for (int c = 0; c < kOC / 32; ++c) tmem_ld32(trow + Cfg::kTmO + half * kOC + 32 * c, o[c]);
                 tmem_wait_ld();
                 tc_fence_before();
                 mbar_arrive(o_free);  // the next item's first PV may overwrite O now
             } else {
 #pragma unroll
-                for (int c = 0; c < 64; ++c) o[c / 32][c % 32] = 0u;
+                for (int c = 0; c < kOC; ++c) o[c / 32][c % 32] = 0u;
+            }
+            if (SPLIT == 2) {
+                float other;
+                if (!trade(l, other)) {
+                    ok = false;
+                    break;
+                }
+                l += other;
             }
             if (row_valid) {
                 const float inv = l > 0.f ? 1.f / l : 0.f;
-                uint4 *dst = reinterpret_cast<uint4 *>(p.out + (((size_t)t.b * p.Lq + pos) * p.Hq + h) * kD);
+                uint4 *dst =
+                    reinterpret_cast<uint4 *>(p.out + (((size_t)t.b * p.Lq + pos) * p.Hq + h) * kD + half * kOC);
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
+                for (int c = 0; c < kOC / 8; ++c) {
                     const uint32_t *src = &o[c / 4][(c % 4) * 8];
                     uint4 v;
                     v.x = pack_bf16x2(__uint_as_float(src[0]) * inv, __uint_as_float(src[1]) * inv);
@@ -471,7 +542,8 @@ __global__ void __launch_bounds__(192, CPS)
                     v.w = pack_bf16x2(__uint_as_float(src[6]) * inv, __uint_as_float(src[7]) * inv);
                     dst[c] = v;
                 }
-                p.lse[((size_t)t.b * p.Hq + h) * p.Lq + pos] = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
+                if (half == 0)
+                    p.lse[((size_t)t.b * p.Hq + h) * p.Lq + pos] = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
             }
         }
     }
@@ -485,11 +557,11 @@ __global__ void __launch_bounds__(192, CPS)
     }
 }
 
-template <int BN, int NS, int EMU, int CPS>
+template <int BN, int NS, int EMU, int CPS, int SPLIT>
 cudaError_t launch_cfg(const void *q, const void *k, const void *v, const float *sinks, void *out, float *lse,
                        const AttnShape &s, cudaStream_t st)
 {
-    using Cfg = FwdCfg<BN, NS, CPS>;
+    using Cfg = FwdCfg<BN, NS, CPS, SPLIT>;
     FwdTcParams p;
     p.B = s.B;
     p.Lq = s.Lq;
@@ -531,14 +603,14 @@ cudaError_t launch_cfg(const void *q, const void *k, const void *v, const float 
         if (!encode_tensor_map_4d(&mv, const_cast<void *>(v), 2, dims, strides, box, true))
             return cudaErrorInvalidValue;
     }
-    auto kern = fwd_tc_kernel<BN, NS, EMU, CPS>;
+    auto kern = fwd_tc_kernel<BN, NS, EMU, CPS, SPLIT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 0;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
     const int grid = (int)std::min<long long>(n_items, (long long)sms * Cfg::kCtasPerSm);
-    kern<<<grid, 192, Cfg::kSmemBytes, st>>>(mq, mk, mv, p);
+    kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, st>>>(mq, mk, mv, p);
     return cudaGetLastError();
 }
 
@@ -555,9 +627,10 @@ cudaError_t launch_fwd_tc(const void *q, const void *k, const void *v, const flo
                           float *lse, const AttnShape &s, cudaStream_t st)
 {
     if (s.window > 0 && s.window <= 1024)
-        return launch_cfg<ATTN_SINK_FWD_BAND_BN, ATTN_SINK_FWD_BAND_NS, -1, ATTN_SINK_FWD_BAND_CPS>(q, k, v, sinks, out,
-                                                                                                  lse, s, st);
-    return launch_cfg<96, 3, 3, 2>(q, k, v, sinks, out, lse, s, st);
+        return launch_cfg<ATTN_SINK_FWD_BAND_BN, ATTN_SINK_FWD_BAND_NS, -1, ATTN_SINK_FWD_BAND_CPS,
+                          ATTN_SINK_FWD_BAND_SPLIT>(q, k, v, sinks, out, lse, s, st);
+    return launch_cfg<ATTN_SINK_FWD_DENSE_BN, ATTN_SINK_FWD_DENSE_NS, ATTN_SINK_FWD_DENSE_EMU, 2,
+                      ATTN_SINK_FWD_DENSE_SPLIT>(q, k, v, sinks, out, lse, s, st);
 }
 
 }  // namespace attn_sink

@@ -293,18 +293,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
-// Same packing, rounded to nearest-even with integer ops (add 0x7FFF plus
-// the lowest kept bit, keep the upper half), so it runs on the ALU/FMA pipes
-// instead of the conversion unit.  Exact for every finite input; a NaN input
-// may come out as infinity.
-__device__ __forceinline__ uint32_t pack_bf16x2_alu(float lo, float hi)
-{
-    uint32_t a = __float_as_uint(lo), b = __float_as_uint(hi);
-    a += 0x7fffu + ((a >> 16) & 1u);
-    b += 0x7fffu + ((b >> 16) & 1u);
-    return __byte_perm(a, b, 0x7632);
-}
-
 // max of three floats in one instruction
 __device__ __forceinline__ float fmax3(float a, float b, float c)
 {

@@ -364,31 +364,34 @@ __global__ void __launch_bounds__(kThreads, 1)
             // Compiled twice: tiles with no masked element (most of them) run
             // without the per-element visibility test.
             uint32_t pk[kM / 4];
-            auto phase1 = [&](auto masked_tag) {
+            // 16 columns of chunk c (0..kCh-1 within the half) from S^T values sr -> 8 bf16 pairs
+            auto p_chunk = [&](auto masked_tag, const uint32_t *sr, int c, uint32_t *q) {
                 constexpr bool kMasked = decltype(masked_tag)::value;
+#pragma unroll
+                for (int e4 = 0; e4 < 4; ++e4) {
+                    const float4 l4 = l2v[4 * (c0 + c) + e4];
+                    const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+                    float pe[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        pe[u] = ex2(fmaf(__uint_as_float(sr[4 * e4 + u]), C, -lv[u]));
+                        if (kMasked) {
+                            const int pl = (16 * (c0 + c) + 4 * e4 + u) / GP;
+                            pe[u] = (pl >= pl_lo && pl <= pl_hi) ? pe[u] : 0.f;
+                        }
+                    }
+                    q[2 * e4] = pack_bf16x2(pe[0], pe[1]);
+                    q[2 * e4 + 1] = pack_bf16x2(pe[2], pe[3]);
+                }
+            };
+            auto phase1 = [&](auto masked_tag) {
                 uint32_t sbuf[2][16];
                 tmem_ld16(trow + kTmST + 16 * c0, sbuf[0]);
                 tmem_wait_ld();
 #pragma unroll
                 for (int c = 0; c < kCh; ++c) {
                     if (c + 1 < kCh) tmem_ld16(trow + kTmST + 16 * (c0 + c + 1), sbuf[(c + 1) & 1]);
-                    const uint32_t *sr = sbuf[c & 1];
-#pragma unroll
-                    for (int e4 = 0; e4 < 4; ++e4) {
-                        const float4 l4 = l2v[4 * (c0 + c) + e4];
-                        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-                        float pe[4];
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            pe[u] = ex2(fmaf(__uint_as_float(sr[4 * e4 + u]), C, -lv[u]));
-                            if (kMasked) {
-                                const int pl = (16 * (c0 + c) + 4 * e4 + u) / GP;
-                                pe[u] = (pl >= pl_lo && pl <= pl_hi) ? pe[u] : 0.f;
-                            }
-                        }
-                        pk[8 * c + 2 * e4] = pack_bf16x2(pe[0], pe[1]);
-                        pk[8 * c + 2 * e4 + 1] = pack_bf16x2(pe[2], pe[3]);
-                    }
+                    p_chunk(masked_tag, sbuf[c & 1], c, &pk[8 * c]);
                     tmem_wait_ld();
                 }
             };
@@ -417,19 +420,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             tc_fence_after();
-            uint32_t dbuf[2][16];
-            tmem_ld16(trow + kTmDPT + 16 * c0, dbuf[0]);
-            tmem_wait_ld();
-#pragma unroll
-            for (int c = 0; c < kCh; ++c) {
-                if (c + 1 < kCh) tmem_ld16(trow + kTmDPT + 16 * (c0 + c + 1), dbuf[(c + 1) & 1]);
-                const uint32_t *dr = dbuf[c & 1];
+            // chunk c: dS from dP^T values dr and P pairs pp; dS^T over 8 columns of
+            // dP^T this warp has read (64 half + 8c .. + 7), dS into shared memory
+            auto ds_chunk = [&](const uint32_t *dr, const uint32_t *pp, int c) {
                 uint32_t dk[8];
 #pragma unroll
                 for (int e4 = 0; e4 < 4; ++e4) {
                     const float4 d4 = ddv[4 * (c0 + c) + e4];
-                    const __nv_bfloat162 p01 = *reinterpret_cast<const __nv_bfloat162 *>(&pk[8 * c + 2 * e4]);
-                    const __nv_bfloat162 p23 = *reinterpret_cast<const __nv_bfloat162 *>(&pk[8 * c + 2 * e4 + 1]);
+                    const __nv_bfloat162 p01 = *reinterpret_cast<const __nv_bfloat162 *>(&pp[2 * e4]);
+                    const __nv_bfloat162 p23 = *reinterpret_cast<const __nv_bfloat162 *>(&pp[2 * e4 + 1]);
                     const float ds0 = __low2float(p01) * (__uint_as_float(dr[4 * e4 + 0]) - d4.x);
                     const float ds1 = __high2float(p01) * (__uint_as_float(dr[4 * e4 + 1]) - d4.y);
                     const float ds2 = __low2float(p23) * (__uint_as_float(dr[4 * e4 + 2]) - d4.z);
@@ -437,7 +436,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     dk[2 * e4] = pack_bf16x2(ds0, ds1);
                     dk[2 * e4 + 1] = pack_bf16x2(ds2, ds3);
                 }
-                // dS^T over 8 columns of dP^T this warp has read (64 half + 8c .. + 7)
                 tmem_st8(trow + kTmDPT + 16 * c0 + 8 * c, dk);
 #pragma unroll
                 for (int q8 = 0; q8 < 2; ++q8) {
@@ -446,6 +444,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     *reinterpret_cast<uint4 *>(smem + kOffDS + atom * kTile + r * 128 + ((cc ^ (r & 7)) << 4)) =
                         make_uint4(dk[4 * q8], dk[4 * q8 + 1], dk[4 * q8 + 2], dk[4 * q8 + 3]);
                 }
+            };
+            uint32_t dbuf[2][16];
+            tmem_ld16(trow + kTmDPT + 16 * c0, dbuf[0]);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < kCh; ++c) {
+                if (c + 1 < kCh) tmem_ld16(trow + kTmDPT + 16 * (c0 + c + 1), dbuf[(c + 1) & 1]);
+                ds_chunk(dbuf[c & 1], &pk[8 * c], c);
                 tmem_wait_ld();
             }
             tmem_wait_st();

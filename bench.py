@@ -122,14 +122,23 @@ def make_prefill(seed, dev):
     return {k: v.to(dev) for k, v in t.items()}, t
 
 
+def kernel_source_sha256(kernel_file: str) -> str:
+    """sha256 of a kernel's source file followed by the PTX helper header it includes."""
+    csrc = os.path.join(ROOT, "gqa_softmax_attention_attn_b200", "csrc")
+    h = hashlib.sha256()
+    for f in (kernel_file, "sm100_ptx.cuh"):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
 def traffic_from_profile(kernel_file: str, profile_json: str):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on
     the kernel source as it is now (else null)."""
     try:
         with open(os.path.join(ROOT, "profiles", profile_json)) as fh:
             pj = json.load(fh)
-        src = open(os.path.join(ROOT, "gqa_softmax_attention_attn_b200", "csrc", kernel_file), "rb").read()
-        if pj.get("source_sha256") != hashlib.sha256(src).hexdigest():
+        if pj.get("source_sha256") != kernel_source_sha256(kernel_file):
             return None
         return float(pj["dram_bytes_per_launch"])
     except Exception:

@@ -255,7 +255,35 @@ def run_ours(args, rank, world, dev):
     }
     if rank == 0:
         res["clocks"] = sampler.summary(t0, t1)
+        res["exp_roof"] = exp_roof(dev, res["clocks"])
     return res
+
+
+def exp_roof(dev, clocks):
+    """The third roof of the dense forward: MUFU ex2 results per second (measured
+    by the self-test library's microbenchmark) times the 4*D flop each visible
+    pair carries (one exponential per pair; the dense layer evaluates a quarter
+    of them on the FMA pipe, which lifts its exp roof by 4/3)."""
+    import ctypes
+
+    from gqa_softmax_attention_attn_b200 import build
+
+    try:
+        lib = ctypes.CDLL(build.SELFTEST_LIB)
+        lib.attn_sink_selftest_pipe_rate.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_double)]
+        rates = []
+        for which in (0, 1):
+            r = ctypes.c_double(0.0)
+            if lib.attn_sink_selftest_pipe_rate(which, ctypes.byref(r)) != 0:
+                return None
+            rates.append(r.value)
+    except OSError:
+        return None
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    mhz = (clocks or {}).get("sm_mhz") or (clocks or {}).get("sm_max_mhz") or 0.0
+    tf = rates[0] * sms * mhz * 1e6 * 4 * D / 1e12
+    return {"ex2_per_clk_per_sm": rates[0], "cvt_bf16x2_per_clk_per_sm": rates[1], "sm_mhz": mhz,
+            "exp_roof_tflops": tf, "exp_roof_tflops_dense_cfg": tf * 4 / 3}
 
 
 def banded_bytes():
@@ -299,6 +327,35 @@ def decode_legs(dev, reps=20, warmup=3, batch=None):
         gbs = by / (ms * 1e-3) / 1e9
         legs[name] = {"ms": ms, "GB/s": gbs, "frac_hbm": gbs / hbm, "bytes": by,
                       "flops": 4.0 * w.D * kv_rows * (w.Hq // w.Hkv) * w.Hkv}
+    # the same caches as a pool of 16-key pages in seeded random order, read
+    # through a page table (same compulsory bytes; the table is not credited)
+    ps = 16
+    maxp = w.Lmax // ps
+    n_pages = nb * maxp
+    perm = torch.randperm(n_pages, generator=torch.Generator().manual_seed(SEEDS["decode"] + ps)).to(dev)
+    kp = torch.empty((n_pages, ps, w.Hkv, w.D), dtype=d["k_cache"].dtype, device=dev)
+    vp = torch.empty_like(kp)
+    kp[perm] = d["k_cache"].reshape(n_pages, ps, w.Hkv, w.D)
+    vp[perm] = d["v_cache"].reshape(n_pages, ps, w.Hkv, w.D)
+    table = perm.view(nb, maxp).to(torch.int32).contiguous()
+    for name, window in (("decode_paged16_dense", 0), ("decode_paged16_window128", WIN)):
+        nbytes = attn.attn_sink_decode_paged_workspace_size(nb, w.Hq, w.D, maxp, ps, window, 0)
+        ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
+        by = legs[name.replace("paged16_", "")]["bytes"]
+        times = []
+        for it in range(reps + warmup):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            attn.attn_sink_decode_paged(d["q"], kp, vp, table, d["seqlens"], d["sinks"], out, lse, window, SCALE, 0,
+                                        ws, stream)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            if it >= warmup:
+                times.append(e0.elapsed_time(e1))
+        ms = statistics.median(times)
+        gbs = by / (ms * 1e-3) / 1e9
+        legs[name] = {"ms": ms, "GB/s": gbs, "frac_hbm": gbs / hbm, "bytes": by, "page_size": ps}
     return legs
 
 

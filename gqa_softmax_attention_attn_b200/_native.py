@@ -65,6 +65,10 @@ def load():
         lib.attn_sink_decode_noalloc.restype = I
         lib.attn_sink_decode_workspace_size.argtypes = [I] * 6
         lib.attn_sink_decode_workspace_size.restype = Z
+        lib.attn_sink_decode_paged.argtypes = [P] * 8 + [I] * 8 + [F, I, P, Z, I, P]
+        lib.attn_sink_decode_paged.restype = I
+        lib.attn_sink_decode_paged_workspace_size.argtypes = [I] * 7
+        lib.attn_sink_decode_paged_workspace_size.restype = Z
         lib.attn_sink_bwd.argtypes = [P] * 11 + [I] * 7 + [F, P, Z, I, P]
         lib.attn_sink_bwd.restype = I
         lib.attn_sink_bwd_workspace_size.argtypes = [I] * 7
@@ -149,6 +153,33 @@ def attn_sink_decode(q, k_cache, v_cache, seqlens, sinks, out, lse, window: int,
                                  int(window), float(scale), int(num_splits), ws_ptr, ws_bytes, _dtype_code(q),
                                  _stream(stream))
     _check(rc, "attn_sink_decode")
+
+
+def attn_sink_decode_paged_workspace_size(B: int, Hq: int, D: int, max_pages_per_seq: int, page_size: int,
+                                          window: int, num_splits: int) -> int:
+    return int(load().attn_sink_decode_paged_workspace_size(B, Hq, D, max_pages_per_seq, page_size, int(window),
+                                                            int(num_splits)))
+
+
+def attn_sink_decode_paged(q, k_pages, v_pages, page_table, seqlens, sinks, out, lse, window: int, scale: float,
+                           num_splits: int = 0, workspace=None, stream=None):
+    """q [B,Hq,D], page pools k/v [num_pages,page_size,Hkv,D] bf16, page_table [B,max_pages] int32,
+    seqlens [B] int32 -> writes out [B,Hq,D], lse [B,Hq]."""
+    B, Hq, D = q.shape
+    num_pages, page_size, Hkv = k_pages.shape[0], k_pages.shape[1], k_pages.shape[2]
+    max_pages = page_table.shape[1]
+    dt = q.dtype
+    ws_ptr, ws_bytes = 0, 0
+    if workspace is not None:
+        ws_ptr = _dev(workspace, "workspace")
+        ws_bytes = workspace.numel() * workspace.element_size()
+    rc = load().attn_sink_decode_paged(_dev(q, "q"), _dev(k_pages, "k_pages", dt), _dev(v_pages, "v_pages", dt),
+                                       _dev(page_table, "page_table", torch.int32),
+                                       _dev(seqlens, "seqlens", torch.int32), _dev(sinks, "sinks", torch.float32),
+                                       _dev(out, "out", dt), _dev(lse, "lse", torch.float32), B, max_pages, page_size,
+                                       num_pages, Hq, Hkv, D, int(window), float(scale), int(num_splits), ws_ptr,
+                                       ws_bytes, _dtype_code(q), _stream(stream))
+    _check(rc, "attn_sink_decode_paged")
 
 
 NOALLOC_SCRATCH_BYTES = 32 << 20  # ATTN_SINK_NOALLOC_SCRATCH_BYTES

@@ -117,7 +117,7 @@ int auto_splits(int Lmax, int window)
 
 DecodeShape decode_shape(int B, int Lmax, int Hq, int Hkv, int D, int window, float scale, int num_splits)
 {
-    DecodeShape s;
+    DecodeShape s{};
     s.B = B;
     s.Lmax = Lmax;
     s.Hq = Hq;
@@ -131,6 +131,42 @@ DecodeShape decode_shape(int B, int Lmax, int Hq, int Hkv, int D, int window, fl
     chunk = (chunk + 63) / 64 * 64;
     s.chunk = chunk;
     // splits that can actually be used by the longest visible range
+    s.splits = (lvis + chunk - 1) / chunk;
+    return s;
+}
+
+// Paged caches: tiles start on multiples of 64 keys, so a banded sequence's
+// split range can begin up to 63 keys before its visible start.
+bool paged_sizes_ok(int page_size, int max_pages, int num_pages)
+{
+    if (page_size <= 0 || max_pages <= 0 || num_pages <= 0) return false;
+    if (!(page_size % 64 == 0 || page_size == 8 || page_size == 16 || page_size == 32)) return false;
+    return (long long)max_pages * page_size <= 0x7fffffffLL;
+}
+
+DecodeShape decode_shape_paged(int B, int max_pages, int page_size, int num_pages, const int *page_table, int Hq,
+                               int Hkv, int D, int window, float scale, int num_splits)
+{
+    const int Lmax = max_pages * page_size;
+    DecodeShape s{};
+    s.B = B;
+    s.Lmax = Lmax;
+    s.Hq = Hq;
+    s.Hkv = Hkv;
+    s.D = D;
+    s.window = window;
+    s.scale = scale;
+    s.align = 64;
+    s.page_size = page_size;
+    s.max_pages = max_pages;
+    s.num_pages = num_pages;
+    s.page_table = page_table;
+    const long long lw = window > 0 ? (long long)window + 63 : (long long)Lmax;
+    const int lvis = (int)(lw < Lmax ? lw : Lmax);
+    s.splits = num_splits > 0 ? num_splits : auto_splits(Lmax, window);
+    int chunk = (lvis + s.splits - 1) / s.splits;
+    chunk = (chunk + 63) / 64 * 64;
+    s.chunk = chunk;
     s.splits = (lvis + chunk - 1) / chunk;
     return s;
 }
@@ -277,6 +313,48 @@ int attn_sink_decode(const void *q, const void *k_cache, const void *v_cache, co
             e = launch_decode_combine<__nv_bfloat16>(seqlens, sinks, static_cast<__nv_bfloat16 *>(out), lse, s,
                                                      ws_o, ws_ml, st);
     }
+    return launch_status(e);
+}
+
+size_t attn_sink_decode_paged_workspace_size(int B, int Hq, int D, int max_pages_per_seq, int page_size, int window,
+                                             int num_splits)
+{
+    if (B <= 0 || Hq <= 0 || D <= 0 || num_splits < 0 || num_splits > 32) return 0;
+    if (!paged_sizes_ok(page_size, max_pages_per_seq, 1)) return 0;
+    return decode_ws_bytes(
+        decode_shape_paged(B, max_pages_per_seq, page_size, 1, nullptr, Hq, 1, D, window, 1.f, num_splits));
+}
+
+int attn_sink_decode_paged(const void *q, const void *k_pages, const void *v_pages, const int *page_table,
+                           const int *seqlens, const float *sinks, void *out, float *lse, int B,
+                           int max_pages_per_seq, int page_size, int num_pages, int Hq, int Hkv, int D, int window,
+                           float scale, int num_splits, void *workspace, size_t ws_bytes, int dtype, void *stream)
+{
+    if (!q || !k_pages || !v_pages || !page_table || !seqlens || !sinks || !out || !lse)
+        return ATTN_SINK_ERR_INVALID_ARG;
+    if (num_splits < 0 || num_splits > 32) return ATTN_SINK_ERR_INVALID_ARG;
+    if (!paged_sizes_ok(page_size, max_pages_per_seq, num_pages)) return ATTN_SINK_ERR_INVALID_ARG;
+    int rc = check_common(B, 1, max_pages_per_seq * page_size, Hq, Hkv, D, dtype);
+    if (rc != ATTN_SINK_OK) return rc;
+    if (dtype != ATTN_SINK_DTYPE_BF16) return ATTN_SINK_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(page_table) || !aligned16(out) ||
+        !aligned16(lse) || !aligned16(sinks) || !aligned16(seqlens))
+        return ATTN_SINK_ERR_MISALIGNED;
+    const DecodeShape s = decode_shape_paged(B, max_pages_per_seq, page_size, num_pages, page_table, Hq, Hkv, D,
+                                             window, scale, num_splits);
+    if (!decode_bf16_supported(s)) return ATTN_SINK_ERR_UNSUPPORTED;
+    const size_t need = decode_ws_bytes(s);
+    if (need > 0 && (!workspace || ws_bytes < need)) return ATTN_SINK_ERR_WORKSPACE;
+    if (need > 0 && !aligned16(workspace)) return ATTN_SINK_ERR_MISALIGNED;
+    rc = ensure_device();
+    if (rc != ATTN_SINK_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    float *ws_o = static_cast<float *>(workspace);
+    float *ws_ml = need > 0 ? ws_o + (size_t)s.B * s.Hq * s.splits * s.D : nullptr;
+    cudaError_t e = launch_decode_bf16(q, k_pages, v_pages, seqlens, sinks, out, lse, s, ws_o, ws_ml, st);
+    if (e == cudaSuccess && s.splits > 1)
+        e = launch_decode_combine<__nv_bfloat16>(seqlens, sinks, static_cast<__nv_bfloat16 *>(out), lse, s, ws_o,
+                                                 ws_ml, st);
     return launch_status(e);
 }
 

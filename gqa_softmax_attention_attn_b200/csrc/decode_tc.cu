@@ -20,6 +20,12 @@
 //  * Keys past the chunk (ragged tail, cache rows beyond the sequence, or
 //    TMA zero fill past Lmax) are masked, and their V rows are zeroed in the
 //    operand registers so stale cache contents can never reach the output.
+//  * Paged caches (kPaged): K/V live in a pool of pages [num_pages,
+//    page_size, Hkv, D] addressed through a per-sequence page table.  Tiles
+//    then start on multiples of 64 keys (the split range begins at the
+//    visible start rounded down, the keys below it masked), so a tile lies in
+//    one page (page_size a multiple of 64) or is 64 / page_size whole pages
+//    (page_size 8, 16 or 32), each fetched with its own TMA box.
 //  * Every wait is bounded; on expiry the CTA raises the device status bit
 //    and winds down.
 #include <cuda.h>
@@ -44,6 +50,8 @@ constexpr int kOffBar = kNS * kStageBytes;
 constexpr int kSmemBytes = kOffBar + 2 * kNS * 8 + 16 + 1024;
 
 struct DecodeParams {
+    DecodeShape sh;  // split rule and (for kPaged) the page pool
+    int box_rows;    // rows per TMA box: 64, or page_size when the pages are smaller
     int B, Lmax, Hq, Hkv, G, window, splits, chunk;
     float c_log2;
     const __nv_bfloat16 *q;
@@ -82,7 +90,7 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
 // byte offset of (row, 16-byte chunk) in a 128-byte-swizzled tile
 __device__ __forceinline__ uint32_t swz(int row, int chunk) { return row * 128 + ((chunk ^ (row & 7)) << 4); }
 
-template <bool kRows16>
+template <bool kRows16, bool kPaged>
 __global__ void __launch_bounds__(kThreads)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                      const DecodeParams p)
@@ -96,10 +104,10 @@ __global__ void __launch_bounds__(kThreads)
     const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int len = min(max(p.seqlens[b], 1), p.Lmax);
-    const int lo = p.window > 0 ? max(0, len - p.window) : 0;
-    const int nsplit = (len - lo + p.chunk - 1) / p.chunk;
+    int lo, lo_al, nsplit;
+    decode_range(p.sh, len, lo, lo_al, nsplit);
     if (c >= nsplit) return;  // uniform over the CTA
-    const int kbeg = lo + c * p.chunk;
+    const int kbeg = lo_al + c * p.chunk;
     const int kend = min(len, kbeg + p.chunk);
     const int n_tiles = (kend - kbeg + kT - 1) / kT;
 
@@ -129,8 +137,25 @@ __global__ void __launch_bounds__(kThreads)
                 const int st = j % kNS;
                 if (!mbar_wait(&empty[st], ((j / kNS) & 1u) ^ 1u, abort_flag, p.status, p.timeout_ns)) break;
                 mbar_arrive_expect_tx(&full[st], kStageBytes);
-                tma_load_4d(smem + st * kStageBytes, &tmK, 0, g, kbeg + j * kT, b, &full[st]);
-                tma_load_4d(smem + st * kStageBytes + kTileBytes, &tmV, 0, g, kbeg + j * kT, b, &full[st]);
+                if (kPaged) {
+                    // the tile's keys in boxes of box_rows rows, each inside one page;
+                    // pages past the sequence (masked keys) reuse its last page, so the
+                    // page table is only read within this sequence's own entries
+                    const int ps = p.sh.page_size;
+                    const int npg = (len + ps - 1) / ps;
+                    for (int r0 = 0; r0 < kT; r0 += p.box_rows) {
+                        const int key = kbeg + j * kT + r0;
+                        const int lp = min(key / ps, npg - 1);
+                        const int phys = p.sh.page_table[(size_t)b * p.sh.max_pages + lp];
+                        const int slot = key % ps;
+                        tma_load_4d(smem + st * kStageBytes + r0 * 128, &tmK, 0, g, slot, phys, &full[st]);
+                        tma_load_4d(smem + st * kStageBytes + kTileBytes + r0 * 128, &tmV, 0, g, slot, phys,
+                                    &full[st]);
+                    }
+                } else {
+                    tma_load_4d(smem + st * kStageBytes, &tmK, 0, g, kbeg + j * kT, b, &full[st]);
+                    tma_load_4d(smem + st * kStageBytes + kTileBytes, &tmV, 0, g, kbeg + j * kT, b, &full[st]);
+                }
                 ++issued[st];
             }
             // drain: every issued load lands before the CTA exits (>= 1 s limit, abort ignored)
@@ -186,14 +211,14 @@ __global__ void __launch_bounds__(kThreads)
                     mma16816(s[nt], qa[2 * half + 1], b2, b3);
                 }
             }
-            // ---- mask keys beyond the chunk; log2-domain logits
+            // ---- mask keys outside [lo, kend); log2-domain logits
             float x[2][4];
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int key = key0 + 8 * nt + 2 * tq + (e & 1);
-                    x[nt][e] = key < kend ? s[nt][e] * C : -INFINITY;
+                    x[nt][e] = (key < kend && key >= lo) ? s[nt][e] * C : -INFINITY;
                 }
             // ---- online softmax, row gr (elements 0,1) and row gr+8 (elements 2,3)
             float mx_a = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
@@ -239,9 +264,9 @@ __global__ void __launch_bounds__(kThreads)
             pa[1] = pack_bf16x2(pv[0][2], pv[0][3]);
             pa[2] = pack_bf16x2(pv[1][0], pv[1][1]);
             pa[3] = pack_bf16x2(pv[1][2], pv[1][3]);
-            // rows of V past the chunk are zeroed in the operand (cache rows
+            // rows of V outside [lo, kend) are zeroed in the operand (cache rows
             // beyond the sequence may hold anything)
-            const bool tail = __any_sync(0xffffffffu, key0 + 15 >= kend);
+            const bool tail = __any_sync(0xffffffffu, key0 + 15 >= kend || key0 < lo);
             const int vrow = 16 * w + ((lane >> 3) & 1) * 8 + (lane & 7);
 #pragma unroll
             for (int jn = 0; jn < 8; jn += 2) {
@@ -250,8 +275,9 @@ __global__ void __launch_bounds__(kThreads)
                 if (tail) {
                     // b0/b2: keys 2tq, 2tq+1 of the slice; b1/b3: keys 8 + 2tq, 8 + 2tq + 1
                     const int k0 = key0 + 2 * tq, k8 = k0 + 8;
-                    const uint32_t m0 = (k0 < kend ? 0x0000FFFFu : 0u) | (k0 + 1 < kend ? 0xFFFF0000u : 0u);
-                    const uint32_t m8 = (k8 < kend ? 0x0000FFFFu : 0u) | (k8 + 1 < kend ? 0xFFFF0000u : 0u);
+                    auto in = [&](int k) { return k < kend && k >= lo; };
+                    const uint32_t m0 = (in(k0) ? 0x0000FFFFu : 0u) | (in(k0 + 1) ? 0xFFFF0000u : 0u);
+                    const uint32_t m8 = (in(k8) ? 0x0000FFFFu : 0u) | (in(k8 + 1) ? 0xFFFF0000u : 0u);
                     b0 &= m0;
                     b2 &= m0;
                     b1 &= m8;
@@ -344,6 +370,8 @@ cudaError_t launch_decode_bf16(const void *q, const void *kc, const void *vc, co
                                float *ws_ml, cudaStream_t st)
 {
     DecodeParams p;
+    p.sh = s;
+    p.box_rows = s.page_size > 0 && s.page_size < kT ? s.page_size : kT;
     p.B = s.B;
     p.Lmax = s.Lmax;
     p.Hq = s.Hq;
@@ -362,25 +390,27 @@ cudaError_t launch_decode_bf16(const void *q, const void *kc, const void *vc, co
     p.ws_ml = ws_ml;
     p.status = device_status_ptr();
     p.timeout_ns = wait_timeout_ns();
+    const bool paged = s.page_size > 0;
     alignas(64) CUtensorMap mk, mv;
-    const uint64_t dims[4] = {(uint64_t)kD, (uint64_t)s.Hkv, (uint64_t)s.Lmax, (uint64_t)s.B};
-    const uint64_t strides[3] = {(uint64_t)kD * 2, (uint64_t)s.Hkv * kD * 2, (uint64_t)s.Lmax * s.Hkv * kD * 2};
-    const uint32_t box[4] = {(uint32_t)kD, 1u, (uint32_t)kT, 1u};
+    // contiguous: [B][Lmax][Hkv][64]; paged pool: [num_pages][page_size][Hkv][64]
+    const uint64_t rows = paged ? (uint64_t)s.page_size : (uint64_t)s.Lmax;
+    const uint64_t outer = paged ? (uint64_t)s.num_pages : (uint64_t)s.B;
+    const uint64_t dims[4] = {(uint64_t)kD, (uint64_t)s.Hkv, rows, outer};
+    const uint64_t strides[3] = {(uint64_t)kD * 2, (uint64_t)s.Hkv * kD * 2, rows * s.Hkv * kD * 2};
+    const uint32_t box[4] = {(uint32_t)kD, 1u, (uint32_t)p.box_rows, 1u};
     if (!encode_tensor_map_4d(&mk, const_cast<void *>(kc), 2, dims, strides, box, true) ||
         !encode_tensor_map_4d(&mv, const_cast<void *>(vc), 2, dims, strides, box, true))
         return cudaErrorInvalidValue;
     const dim3 grid(s.splits, s.Hkv, s.B);
-    cudaError_t e;
-    if (p.G > 8) {
-        e = cudaFuncSetAttribute(decode_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    auto launch = [&](auto kern) -> cudaError_t {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
         if (e != cudaSuccess) return e;
-        decode_tc_kernel<true><<<grid, kThreads, kSmemBytes, st>>>(mk, mv, p);
-    } else {
-        e = cudaFuncSetAttribute(decode_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-        if (e != cudaSuccess) return e;
-        decode_tc_kernel<false><<<grid, kThreads, kSmemBytes, st>>>(mk, mv, p);
-    }
-    return cudaGetLastError();
+        kern<<<grid, kThreads, kSmemBytes, st>>>(mk, mv, p);
+        return cudaGetLastError();
+    };
+    if (p.G > 8)
+        return paged ? launch(decode_tc_kernel<true, true>) : launch(decode_tc_kernel<true, false>);
+    return paged ? launch(decode_tc_kernel<false, true>) : launch(decode_tc_kernel<false, false>);
 }
 
 }  // namespace attn_sink

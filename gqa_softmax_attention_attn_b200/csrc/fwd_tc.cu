@@ -71,6 +71,9 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 #define ATTN_SINK_FWD_DENSE_BN 96
 #define ATTN_SINK_FWD_DENSE_NS 3
 #endif
+#ifndef ATTN_SINK_FWD_DENSE_CPS
+#define ATTN_SINK_FWD_DENSE_CPS 2
+#endif
 #ifndef ATTN_SINK_FWD_DENSE_EMU
 #define ATTN_SINK_FWD_DENSE_EMU 3
 #endif
@@ -129,6 +132,18 @@ struct FwdTcParams {
 struct Item {
     int pos0, h0, b, t_lo, n_tiles;
 };
+
+// The r-th work item of this CTA, or -1 past the end: rounds of gridDim.x
+// items in snake order (even rounds ascending in blockIdx, odd rounds
+// descending), so that over the longest-first list every CTA gets a similar
+// total length (round-robin in one direction left the CTA that always takes
+// the longest item of a round 11-14% above the mean on a causal layer).
+__device__ __forceinline__ int cta_item(int r, int n_items)
+{
+    const long g = gridDim.x;
+    const long w = (long)r * g + ((r & 1) ? g - 1 - (long)blockIdx.x : (long)blockIdx.x);
+    return w < n_items ? (int)w : -1;
+}
 
 // Work item i of the longest-first order: q tiles from the last (most keys
 // under a causal mask) to the first, all head tiles and batches of one q tile
@@ -227,7 +242,7 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT>::kThreads, CPS)
             for (int s = 0; s < NS; ++s) k_issued[s] = v_issued[s] = 0;
             uint32_t it = 0, item_n = 0;
             bool ok = true;
-            for (int w = blockIdx.x; w < p.n_items && ok; w += gridDim.x) {
+            for (int r_it = 0, w = cta_item(0, p.n_items); w >= 0 && ok; w = cta_item(++r_it, p.n_items)) {
                 const Item t = item_at<BN>(p, w);
                 if (t.n_tiles == 0) continue;
                 const int qb = item_n & 1;
@@ -304,7 +319,7 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT>::kThreads, CPS)
             __syncwarp();
             return true;
         };
-        for (int w = blockIdx.x; w < p.n_items && ok; w += gridDim.x) {
+        for (int r_it = 0, w = cta_item(0, p.n_items); w >= 0 && ok; w = cta_item(++r_it, p.n_items)) {
             const Item t = item_at<BN>(p, w);
             if (t.n_tiles == 0) continue;
             const int qb = item_n & 1;
@@ -374,7 +389,7 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT>::kThreads, CPS)
             ++xc;
             return got;
         };
-        for (int w = blockIdx.x; w < p.n_items && ok; w += gridDim.x) {
+        for (int r_it = 0, w = cta_item(0, p.n_items); w >= 0 && ok; w = cta_item(++r_it, p.n_items)) {
             const Item t = item_at<BN>(p, w);
             const int pos = t.pos0 + r / p.Gp;
             const int h = t.h0 + r % p.Gp;
@@ -413,20 +428,19 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT>::kThreads, CPS)
 #pragma unroll
                     for (int c = 0; c < kC; ++c) sv[c] = (c >= c_lo && c <= c_hi) ? sv[c] : -INFINITY;
                 }
-                // row max: four independent chains of 3-input max over columns
-                // 0-3 | 4..kC-1 in steps of 8 | the remaining 4 when (kC - 4) % 8 == 4
+                // row max: eight independent chains of 3-input max over columns
+                // 0-7 | 8..kC-9 in steps of 16 | the last 8 (kC % 16 == 0)
                 static_assert(kC % 16 == 0, "whole 16-column chunks per thread");
-                float mx[4];
+                float mx[8];
 #pragma unroll
-                for (int k = 0; k < 4; ++k) mx[k] = sv[k];
-                constexpr int kFull = 4 + ((kC - 4) / 8) * 8;
+                for (int k = 0; k < 8; ++k) mx[k] = sv[k];
 #pragma unroll
-                for (int c = 4; c < kFull; c += 8)
+                for (int c = 8; c + 16 <= kC; c += 16)
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) mx[k] = fmax3(mx[k], sv[c + k], sv[c + 4 + k]);
+                    for (int k = 0; k < 8; ++k) mx[k] = fmax3(mx[k], sv[c + k], sv[c + 8 + k]);
 #pragma unroll
-                for (int k = 0; k < 4 && kFull + k < kC; ++k) mx[k] = fmaxf(mx[k], sv[kFull + k]);
-                float tmax = fmax3(mx[0], mx[1], fmaxf(mx[2], mx[3]));
+                for (int k = 0; k < 8; ++k) mx[k] = fmaxf(mx[k], sv[kC - 8 + k]);
+                float tmax = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
                 if (SPLIT == 2) {
                     float other;
                     if (!trade(tmax, other)) {
@@ -477,7 +491,10 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT>::kThreads, CPS)
                 }
                 l = l * alpha + ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y));
                 if (jt > 0) {
-                    // O holds sum_{t<jt} P_t V_t once PV(jt-1) completes
+                    // O holds sum_{t<jt} P_t V_t once PV(jt-1) completes.  Waited on
+                    // every tile, rescale or not: a parity wait is only unambiguous
+                    // while the barrier is at most one phase away, so no phase of
+                    // o_done may go unobserved.
                     if (!__all_sync(0xffffffffu,
                                     mbar_wait(o_done, (it - 1) & 1u, abort_flag, p.status, p.timeout_ns))) {
                         ok = false;
@@ -629,7 +646,7 @@ cudaError_t launch_fwd_tc(const void *q, const void *k, const void *v, const flo
     if (s.window > 0 && s.window <= 1024)
         return launch_cfg<ATTN_SINK_FWD_BAND_BN, ATTN_SINK_FWD_BAND_NS, -1, ATTN_SINK_FWD_BAND_CPS,
                           ATTN_SINK_FWD_BAND_SPLIT>(q, k, v, sinks, out, lse, s, st);
-    return launch_cfg<ATTN_SINK_FWD_DENSE_BN, ATTN_SINK_FWD_DENSE_NS, ATTN_SINK_FWD_DENSE_EMU, 2,
+    return launch_cfg<ATTN_SINK_FWD_DENSE_BN, ATTN_SINK_FWD_DENSE_NS, ATTN_SINK_FWD_DENSE_EMU, ATTN_SINK_FWD_DENSE_CPS,
                       ATTN_SINK_FWD_DENSE_SPLIT>(q, k, v, sinks, out, lse, s, st);
 }
 

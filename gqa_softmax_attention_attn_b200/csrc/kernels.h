@@ -21,7 +21,20 @@ struct DecodeShape {
     float scale;
     int splits;  // maximum number of chunks per sequence
     int chunk;   // keys per chunk (multiple of 64)
+    int align;   // 0, or 64: the split range starts at the visible start rounded down to this
+    // paged caches (pool [num_pages, page_size, Hkv, D]; page_table [B, max_pages]); 0 = contiguous
+    int page_size, max_pages, num_pages;
+    const int *page_table;
 };
+
+// First key of sequence b's split range and its number of splits (shared by the
+// split kernels and the combine kernel).
+__host__ __device__ inline void decode_range(const DecodeShape &s, int len, int &lo, int &lo_al, int &nsplit)
+{
+    lo = s.window > 0 ? (len - s.window > 0 ? len - s.window : 0) : 0;
+    lo_al = s.align > 0 ? lo / s.align * s.align : lo;
+    nsplit = (len - lo_al + s.chunk - 1) / s.chunk;
+}
 
 // Per-device status word (bit STATUS_TIMEOUT set by an expired bounded wait).
 unsigned *device_status_ptr();

@@ -446,8 +446,8 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const int *__restri
     if (bh >= (long)s.B * s.Hq) return;
     const int b = (int)(bh / s.Hq), h = (int)(bh % s.Hq);
     const int len = min(max(seqlens[b], 1), s.Lmax);
-    const int lo = s.window > 0 ? max(0, len - s.window) : 0;
-    const int nsplit = (len - lo + s.chunk - 1) / s.chunk;
+    int lo, lo_al, nsplit;
+    decode_range(s, len, lo, lo_al, nsplit);
     if (nsplit <= 1) return;  // written directly by the split kernel
     const size_t slot0 = (size_t)bh * s.splits;
     const float mc = lane < nsplit ? ws_ml[(slot0 + lane) * 2 + 0] : -INFINITY;

@@ -125,6 +125,43 @@ ATTN_SINK_API int attn_sink_decode(const void *q, const void *k_cache, const voi
 ATTN_SINK_API size_t attn_sink_decode_workspace_size(int B, int Hq, int D, int Lmax, int window, int num_splits);
 
 /*
+ * Split-KV decode over a paged KV cache: the same operation as
+ * attn_sink_decode, with each sequence's cached keys and values gathered
+ * through a page table instead of one contiguous [Lmax] slab per sequence
+ * (the pages name partitioned KV caches as the way to hold long contexts --
+ * "How much computing power is required for gpt-oss deployment?", the
+ * question on the KV cache and context length -- and split the attention
+ * along the KV length -- "GPT-OSS on day 0", section "Sink Attention").
+ *   k_pages, v_pages  [num_pages, page_size, Hkv, D] bf16: the page pool
+ *   page_table [B, max_pages_per_seq] int32, device: token t of sequence b
+ *              sits in slot t % page_size of page
+ *              page_table[b][t / page_size].  Only the first
+ *              ceil(seqlens[b] / page_size) entries of a row are read; the
+ *              rest may hold anything.  Entries outside [0, num_pages) read
+ *              zeros (no fault).  Pages may be shared between sequences.
+ *   page_size  8, 16, 32 or a multiple of 64.
+ *   seqlens    [B] int32 in [1, max_pages_per_seq * page_size] (clamped on
+ *              the device), with the query at position seqlens[b] - 1.
+ *   q, sinks, out, lse, window, scale, num_splits: as attn_sink_decode.
+ *   dtype      ATTN_SINK_DTYPE_BF16 only (F32 returns UNSUPPORTED).
+ *   workspace  at least attn_sink_decode_paged_workspace_size(B, Hq, D,
+ *              max_pages_per_seq, page_size, window, num_splits) bytes.
+ * Errors: INVALID_ARG for a null pointer, a page_size not listed above,
+ * non-positive sizes or max_pages_per_seq * page_size >= 2^31; otherwise as
+ * attn_sink_decode.  Nothing is allocated; the call is asynchronous on
+ * `stream`.
+ */
+ATTN_SINK_API int attn_sink_decode_paged(const void *q, const void *k_pages, const void *v_pages,
+                     const int *page_table, const int *seqlens, const float *sinks, void *out,
+                     float *lse, int B, int max_pages_per_seq, int page_size, int num_pages,
+                     int Hq, int Hkv, int D, int window, float scale, int num_splits,
+                     void *workspace, size_t ws_bytes, int dtype, void *stream);
+
+/* Bytes of paged-decode workspace for these sizes (0 when a single split suffices). */
+ATTN_SINK_API size_t attn_sink_decode_paged_workspace_size(int B, int Hq, int D, int max_pages_per_seq,
+                     int page_size, int window, int num_splits);
+
+/*
  * Size of the scratch buffer built into the library for
  * attn_sink_decode_noalloc: 32 MiB of device memory, reserved on every GPU
  * that loads the library and held until the process exits.

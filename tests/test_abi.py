@@ -73,6 +73,38 @@ def test_decode_host_checks():
     assert attn.attn_sink_decode_workspace_size(4, 8, 64, 4096, 128, 0) == 0
 
 
+def test_decode_paged_host_checks():
+    lib = attn.load()
+    q, kp, vp, pt, sl, s, o, l = _fake(8)
+    ws = _fake(9)[8]
+
+    def call(B=4, max_pages=256, page_size=16, num_pages=1024, Hq=8, Hkv=2, D=64, window=0, splits=0,
+             w=ws, wbytes=1 << 20, dtype=1, ptab=pt):
+        return lib.attn_sink_decode_paged(q, kp, vp, ptab, sl, s, o, l, B, max_pages, page_size, num_pages, Hq, Hkv,
+                                          D, window, 0.125, splits, w, wbytes, dtype, None)
+
+    for bad_ps in (0, -16, 4, 12, 24, 48, 100):
+        assert call(page_size=bad_ps) == INVALID, bad_ps
+    assert call(max_pages=0) == INVALID
+    assert call(num_pages=0) == INVALID
+    assert call(max_pages=1 << 25, page_size=64) == INVALID  # 2^31 keys per sequence
+    assert call(splits=33) == INVALID
+    assert call(ptab=None) == INVALID
+    assert call(dtype=0) == UNSUPPORTED  # bf16 only
+    assert call(D=128) == UNSUPPORTED
+    assert call(ptab=pt + 4) == MISALIGNED
+    # dense, 8 splits over 256 pages of 16 keys: chunk 512, 8 partials per (b, h)
+    need = attn.attn_sink_decode_paged_workspace_size(4, 8, 64, 256, 16, 0, 8)
+    assert need == 4 * 8 * 8 * (64 + 2) * 4
+    assert call(splits=8, w=None, wbytes=0) == WORKSPACE
+    assert call(splits=8, wbytes=need - 4) == WORKSPACE
+    # banded: the split range may start up to 63 keys early (64-key aligned tiles)
+    assert attn.attn_sink_decode_paged_workspace_size(4, 8, 64, 256, 16, 128, 0) == 0
+    # 4 splits asked over 191 keys: 64-key chunks, so 3 partials
+    assert attn.attn_sink_decode_paged_workspace_size(4, 8, 64, 256, 16, 128, 4) == 4 * 8 * 3 * 66 * 4
+    assert attn.attn_sink_decode_paged_workspace_size(4, 8, 64, 256, 12, 0, 8) == 0  # invalid page size
+
+
 def test_bwd_host_checks():
     lib = attn.load()
     p = _fake(12)

@@ -33,3 +33,19 @@ def test_fast_exp2_relative_error_bound():
     assert torch.isfinite(f).all() and (f >= 0).all()
     # results below 1e-37 (x < -122.9, and the clamp at x = -126) stay tiny and non-negative
     assert (f[~ok] <= 1.001e-37).all()
+
+
+def test_pipe_rate_microbenchmarks():
+    # measured results per clock per SM of MUFU ex2 and of the bf16x2 pack;
+    # the rates bench.py turns into the exponential roof
+    lib = ctypes.CDLL(build.SELFTEST_LIB)
+    lib.attn_sink_selftest_pipe_rate.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_double)]
+    rates = []
+    for which in (0, 1):
+        r = ctypes.c_double(0.0)
+        assert lib.attn_sink_selftest_pipe_rate(which, ctypes.byref(r)) == 0
+        rates.append(r.value)
+    assert 4.0 <= rates[0] <= 128.0, rates
+    assert 4.0 <= rates[1] <= 256.0, rates
+    r = ctypes.c_double(0.0)
+    assert lib.attn_sink_selftest_pipe_rate(7, ctypes.byref(r)) == -1

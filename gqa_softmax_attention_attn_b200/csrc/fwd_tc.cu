@@ -64,11 +64,14 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // Tile configurations (keys per tile BN, K/V stages NS, EMU = which pair of
 // every 4 uses the FMA-pipe exp2 (4: every odd pair, -1: none), CTAs per
 // SM), chosen per layer type from measurements on the gpt-oss-20b prefill:
-// the dense causal layer runs best with BN = 96, two CTAs per SM and a
-// quarter of the exponentials off the MUFU unit (none: 3% slower, half: 4%
+// the dense causal layer runs best with BN = 80, two CTAs per SM and a
+// quarter of the exponentials off the MUFU unit (none: 2% slower, half: 7%
 // slower), the window-128 layer with the banded configuration above.
+// dense layer: BN = 80 with three stages (two CTAs per SM) measured 203 us on
+// the gpt-oss-20b prefill's dense layer, against 209 us at BN = 96 and 233 us
+// at BN = 64 (and 255-270 us for BN = 32 at three or four CTAs per SM)
 #ifndef ATTN_SINK_FWD_DENSE_BN
-#define ATTN_SINK_FWD_DENSE_BN 96
+#define ATTN_SINK_FWD_DENSE_BN 80
 #define ATTN_SINK_FWD_DENSE_NS 3
 #endif
 #ifndef ATTN_SINK_FWD_DENSE_CPS

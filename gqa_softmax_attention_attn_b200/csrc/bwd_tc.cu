@@ -15,7 +15,8 @@
 //    (128 rows = positions x query heads of the group, as in the forward)
 //    that can see a key of the tile.  Q and dO tiles stream in by TMA (two
 //    stages); lse and D for the tile's 128 rows go to shared memory.
-//  * Warp 1 issues, from one thread: S^T = K Q^T and dP^T = V dO^T (keys as
+//  * Warp 1 runs the MMA issue loop as a whole warp (warp-uniform operands),
+//    one elected lane issuing: S^T = K Q^T and dP^T = V dO^T (keys as
 //    the M dimension, so a thread of the softmax-gradient warps owns a key
 //    row); then dV += P^T dO and dK += dS^T Q with P^T and dS^T read back
 //    from tensor memory; then dQ = dS K with dS from shared memory (written
@@ -27,10 +28,14 @@
 //    P from S^T (bf16 pairs into their own TMEM columns, releasing S^T), then
 //    dS = P (dP - D) from dP^T; dS^T goes back over the half's read columns
 //    of dP^T as bf16, dS to shared memory.
-//  * Warps 6-9 move each dQ tile from TMEM to shared memory and add it into an
-//    fp32 dQ accumulator in global memory with a TMA reduce-add (L2 atomics;
-//    the summation order over key tiles is not fixed).  dK and dV of the tile
-//    are written once, at the end (deterministic).
+//  * Warps 6-9 move each dQ tile from TMEM to shared memory (two 128-byte-
+//    swizzled fp32 halves) and add it into an fp32 dQ accumulator in global
+//    memory with TMA reduce-adds (L2 atomics; the summation order over key
+//    tiles is not fixed).  dK and dV of the tile are written once, at the end
+//    (deterministic).
+//  * One CTA per SM (512 TMEM columns); the 14 warps cap registers at 128 per
+//    thread.  The grid is 1-D with the key tile slowest, so the causally
+//    longest CTAs of every head and batch start first.
 //  * Every wait is bounded; on expiry the CTA raises the device status bit,
 //    drains its own TMA and MMA work, frees tensor memory and exits.
 #include <cuda.h>

@@ -13,7 +13,8 @@
 //  * Work item = 128 query rows = (128 / Gp) positions x Gp query heads of one
 //    KV group, so every K/V tile fetched is shared by Gp heads (GQA packing;
 //    no cluster multicast).  Persistent CTAs (two per SM, 256 TMEM columns
-//    each) walk a static longest-first list of work items.
+//    each) walk a static longest-first list of work items, dealt out in
+//    snake order (alternating direction every round of gridDim.x items).
 //  * Warp 0: TMA producer -- Q (double-buffered, so the next item's Q lands
 //    while the current one finishes) and K/V tiles of BN keys into an
 //    NS-stage ring.  Warp 1: allocates tensor memory and runs the MMA issue

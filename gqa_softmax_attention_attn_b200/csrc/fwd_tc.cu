@@ -13,9 +13,10 @@
 //  * Work item = 128 query rows = (128 / Gp) positions x Gp query heads of one
 //    KV group, so every K/V tile fetched is shared by Gp heads (GQA packing;
 //    no cluster multicast).  Persistent CTAs (two per SM, 256 TMEM columns
-//    each) walk a static longest-first list of work items, dealt out in
-//    snake order (alternating direction every round of gridDim.x items).
-//  * Warp 0: TMA producer -- Q (double-buffered, so the next item's Q lands
+//    each) take work items from a longest-first list through one atomic
+//    counter per launch (a CTA on a faster SM takes more of them).
+//  * Warp 0: item fetch (passed to the other warps through a shared-memory
+//    ring) and TMA producer -- Q (double-buffered, so the next item's Q lands
 //    while the current one finishes) and K/V tiles of BN keys into an
 //    NS-stage ring.  Warp 1: allocates tensor memory and runs the MMA issue
 //    loop as a whole warp (warp-uniform descriptors), one elected lane
@@ -40,6 +41,7 @@
 #include <math.h>
 
 #include <algorithm>
+#include <atomic>
 
 #include "kernels.h"
 #include "sm100_ptx.cuh"
@@ -105,8 +107,8 @@ struct FwdCfg {
     static constexpr int kOffV = kOffK + NS * kKVBytes;
     static constexpr int kOffBar = kOffV + NS * kKVBytes;
     // q_full[2], q_empty[2], k_full[NS], k_empty[NS], v_full[NS], v_empty[NS],
-    // s_full[2], p_full[2], o_done, o_free, drain, xchg[4]
-    static constexpr int kNumBar = 4 + 4 * NS + 4 + 3 + 4;
+    // s_full[2], p_full[2], o_done, o_free, drain, xchg[4], item_full[4], item_empty[4]
+    static constexpr int kNumBar = 4 + 4 * NS + 4 + 3 + 4 + 8;
     static constexpr int kOffMisc = kOffBar + kNumBar * 8;
     // row partials exchanged by the two softmax warps of a row: [2 slots][2 halves][128 rows]
     static constexpr int kOffXchg = kOffMisc + 64;
@@ -131,11 +133,33 @@ struct FwdTcParams {
     float *lse;
     unsigned *status;
     long long timeout_ns;
+    int sched_slot;  // this launch's counter in g_fwd_sched / g_fwd_done (dynamic item order)
 };
 
 struct Item {
     int pos0, h0, b, t_lo, n_tiles;
 };
+
+// Dynamic item order: the persistent CTAs take work items, longest first, from
+// one counter per launch (one atomic add per item), so a CTA on a faster SM
+// simply takes more of them (with a fixed assignment, CTAs given equal work
+// finished 182-209 us apart).  Launch number n uses counter n % kSchedSlots,
+// which is 0 when it starts: the last CTA of every launch (counted in
+// g_fwd_done) sets it back to 0, so replaying a captured launch starts
+// afresh.  Up to kSchedSlots forward launches may run at once on one device.
+#ifndef ATTN_SINK_FWD_DYNAMIC
+#define ATTN_SINK_FWD_DYNAMIC 1
+#endif
+constexpr int kSchedSlots = 64;
+__device__ unsigned g_fwd_sched[kSchedSlots];
+__device__ unsigned g_fwd_done[kSchedSlots];
+
+// Next item for this CTA from the launch's counter, or -1 when none is left.
+__device__ __forceinline__ int fetch_item(const FwdTcParams &p)
+{
+    const unsigned i = atomicAdd(&g_fwd_sched[p.sched_slot], 1u);
+    return i < (unsigned)p.n_items ? (int)i : -1;
+}
 
 // The r-th work item of this CTA, or -1 past the end: rounds of gridDim.x
 // items in snake order (even rounds ascending in blockIdx, odd rounds
@@ -201,6 +225,11 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT>::kThreads, CPS)
     uint64_t *o_free = o_done + 1;
     uint64_t *drain = o_free + 1;
     uint64_t *xchg = drain + 1;  // [4]: one per TMEM lane quadrant (SPLIT == 2)
+    // item ring (dynamic order): the producer warp fetches items and passes
+    // them to the MMA warp and the softmax warps through 4 slots
+    uint64_t *item_full = xchg + 4;        // [4]
+    uint64_t *item_empty = item_full + 4;  // [4]
+    volatile int *ring = reinterpret_cast<volatile int *>(smem + Cfg::kOffMisc + 16);
     float *xs = reinterpret_cast<float *>(smem + Cfg::kOffXchg);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Cfg::kOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Cfg::kOffMisc + 4);
@@ -224,6 +253,10 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT>::kThreads, CPS)
         mbar_init(o_free, 128 * SPLIT);
         mbar_init(drain, 1);
         for (int qd = 0; qd < 4; ++qd) mbar_init(&xchg[qd], 64);
+        for (int r = 0; r < 4; ++r) {
+            mbar_init(&item_full[r], 1);
+            mbar_init(&item_empty[r], 1 + 4 * SPLIT);  // the MMA warp and each softmax warp
+        }
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -236,6 +269,28 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT>::kThreads, CPS)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
+    // r-th item of this CTA: the producer (lane 0 of warp 0) fetches it and
+    // publishes it in the ring; every other warp reads it there (-1: no more)
+    auto producer_item = [&](int r) -> int {
+        if (!ATTN_SINK_FWD_DYNAMIC) return cta_item(r, p.n_items);
+        const int w = fetch_item(p);
+        const int sl = r & 3;
+        if (!mbar_wait(&item_empty[sl], ((r >> 2) & 1u) ^ 1u, abort_flag, p.status, p.timeout_ns)) return -1;
+        ring[sl] = w;
+        mbar_arrive(&item_full[sl]);
+        return w;
+    };
+    auto consumer_item = [&](int r) -> int {
+        if (!ATTN_SINK_FWD_DYNAMIC) return cta_item(r, p.n_items);
+        const int sl = r & 3;
+        if (!__all_sync(0xffffffffu, mbar_wait(&item_full[sl], (r >> 2) & 1u, abort_flag, p.status, p.timeout_ns)))
+            return -1;
+        const int w = ring[sl];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&item_empty[sl]);
+        return w;
+    };
+
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
@@ -246,7 +301,7 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT>::kThreads, CPS)
             for (int s = 0; s < NS; ++s) k_issued[s] = v_issued[s] = 0;
             uint32_t it = 0, item_n = 0;
             bool ok = true;
-            for (int r_it = 0, w = cta_item(0, p.n_items); w >= 0 && ok; w = cta_item(++r_it, p.n_items)) {
+            for (int r_it = 0, w = producer_item(0); w >= 0 && ok; w = producer_item(++r_it)) {
                 const Item t = item_at<BN>(p, w);
                 if (t.n_tiles == 0) continue;
                 const int qb = item_n & 1;
@@ -323,7 +378,7 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT>::kThreads, CPS)
             __syncwarp();
             return true;
         };
-        for (int r_it = 0, w = cta_item(0, p.n_items); w >= 0 && ok; w = cta_item(++r_it, p.n_items)) {
+        for (int r_it = 0, w = consumer_item(0); w >= 0 && ok; w = consumer_item(++r_it)) {
             const Item t = item_at<BN>(p, w);
             if (t.n_tiles == 0) continue;
             const int qb = item_n & 1;
@@ -393,7 +448,7 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT>::kThreads, CPS)
             ++xc;
             return got;
         };
-        for (int r_it = 0, w = cta_item(0, p.n_items); w >= 0 && ok; w = cta_item(++r_it, p.n_items)) {
+        for (int r_it = 0, w = consumer_item(0); w >= 0 && ok; w = consumer_item(++r_it)) {
             const Item t = item_at<BN>(p, w);
             const int pos = t.pos0 + r / p.Gp;
             const int h = t.h0 + r % p.Gp;
@@ -576,6 +631,14 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT>::kThreads, CPS)
         tc_fence_after();
         tmem_dealloc(tmem, Cfg::kTmemCols);
     }
+    if (ATTN_SINK_FWD_DYNAMIC && threadIdx.x == 0) {
+        // every CTA has taken its last item: the last one to finish resets the count
+        __threadfence();
+        if (atomicAdd(&g_fwd_done[p.sched_slot], 1u) == gridDim.x - 1) {
+            g_fwd_done[p.sched_slot] = 0;
+            atomicExch(&g_fwd_sched[p.sched_slot], 0u);
+        }
+    }
 }
 
 template <int BN, int NS, int EMU, int CPS, int SPLIT>
@@ -606,6 +669,8 @@ cudaError_t launch_cfg(const void *q, const void *k, const void *v, const float 
     p.lse = lse;
     p.status = device_status_ptr();
     p.timeout_ns = wait_timeout_ns();
+    static std::atomic<unsigned> launches{0};
+    p.sched_slot = (int)(launches.fetch_add(1u, std::memory_order_relaxed) % kSchedSlots);
 
     alignas(64) CUtensorMap mq, mk, mv;
     {

@@ -139,3 +139,40 @@ def test_deterministic_and_stream_ordered():
     o1, l1 = run_fwd(t, 0, 0.125)
     o2, l2 = run_fwd(t, 0, 0.125)
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_graph_replay_and_concurrent_streams():
+    # persistent CTAs take work items from a per-launch counter: replaying a
+    # captured launch, and launches running at once on two streams, must still
+    # each process every item exactly once
+    t = prefill_inputs(1, 2048, 2048, 64, 8, 64, torch.bfloat16, 0.5, 1.0, seed=12)
+    dev = "cuda"
+    q, k, v, s = (t[x].to(dev) for x in ("q", "k", "v", "sinks"))
+    ref_o, ref_l = run_fwd(t, 0, 0.125)
+    out = torch.empty_like(q)
+    lse = torch.empty(1, 64, 2048, device=dev)
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        attn_sink_fwd(q, k, v, s, out, lse, 0, 0.125, stream)  # outside the capture: one-time set-up
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream, capture_error_mode="thread_local"):
+        attn_sink_fwd(q, k, v, s, out, lse, 0, 0.125, stream)
+    for _ in range(3):
+        out.zero_()
+        lse.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref_o) and torch.equal(lse, ref_l)
+    del g
+    # two streams, several launches each, overlapping on the device
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    outs = [(torch.empty_like(q), torch.empty_like(lse)) for _ in range(6)]
+    torch.cuda.synchronize()
+    for i, (o, l) in enumerate(outs):
+        st = s1 if i % 2 == 0 else s2
+        with torch.cuda.stream(st):
+            attn_sink_fwd(q, k, v, s, o, l, 0, 0.125, st)
+    torch.cuda.synchronize()
+    for o, l in outs:
+        assert torch.equal(o, ref_o) and torch.equal(l, ref_l)

@@ -420,6 +420,38 @@ def oracle_sample(seconds_budget=12.0, seed=1002):
     return total_fl / total_s / 1e12, oracle.num_threads(), desc, total_fl, total_s
 
 
+_TINY_1CORE = r"""
+import json, sys, time
+sys.path.insert(0, sys.argv[1])
+import torch
+import oracle
+from gqa_softmax_attention_attn_b200.inputs import prefill_inputs
+t = prefill_inputs(1, 256, 256, 8, 2, 64, torch.float32, 1.0, 1.0, seed=1001)
+oracle.fwd(t["q"], t["k"], t["v"], t["sinks"], 0, 0.125)  # warm-up (load, first touch)
+t0 = time.perf_counter()
+for window in (0, 128):
+    oracle.fwd(t["q"], t["k"], t["v"], t["sinks"], window, 0.125)
+print(json.dumps({"seconds": time.perf_counter() - t0, "threads": oracle.num_threads()}))
+"""
+
+
+def oracle_tiny_1core():
+    """The oracle's forward on the tiny fp32 workload (B1 L256 Hq8 Hkv2 D64, dense and
+    window-128 layers) on one host core, in a child process with OMP_NUM_THREADS=1."""
+    import subprocess
+
+    env = dict(os.environ, OMP_NUM_THREADS="1")
+    try:
+        r = subprocess.run([sys.executable, "-c", _TINY_1CORE, ROOT], env=env, capture_output=True, text=True,
+                           timeout=300)
+        d = json.loads(r.stdout.strip().splitlines()[-1])
+    except Exception:
+        return None
+    flops = fwd_flops(1, 256, 8, 0) + fwd_flops(1, 256, 8, 128)
+    return {"workload": "B1 L256 Hq8 Hkv2 D64 fp32, dense + window-128 forward", "seconds": d["seconds"],
+            "value": flops / d["seconds"] / 1e12, "unit": "TFLOP/s", "cores": d["threads"]}
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return None
@@ -437,7 +469,8 @@ def run_reference(args, rank, world):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": {"workload": WORKLOAD, "global_batch": B, "seq_len": L,
                                              "parallelism": "cpu-oracle"},
-            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc,
+                             "tiny_1core": oracle_tiny_1core()},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
@@ -485,7 +518,8 @@ def main():
             res["legs"].update(bwd_legs(dev))
         if not args.no_cpu_baseline and world == 1:
             v, cores, desc, _, _ = oracle_sample(12.0)
-            res["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc}
+            res["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc,
+                                   "tiny_1core": oracle_tiny_1core()}
         res["device"] = {"name": torch.cuda.get_device_name(dev), "capability": list(torch.cuda.get_device_capability(dev)),
                          "torch": torch.__version__, "cuda": torch.version.cuda}
         print(json.dumps(res), flush=True)

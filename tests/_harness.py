@@ -4,7 +4,9 @@ import math
 import numpy as np
 import torch
 
-# Tolerances fixed by the benchmark spec for this path.
+# Parity tolerances: the exact fp32 path to 1e-5 max-abs; the bf16 path to
+# 2e-2 max-abs and 5e-3 relative L2 (bf16 rounding of P before the PV product
+# and of the stored output, against an fp64 reference).
 FP32_MAX_ABS = 1e-5
 BF16_MAX_ABS = 2e-2
 BF16_REL_L2 = 5e-3

@@ -72,8 +72,10 @@ def test_bf16_bwd_small(shape, window):
 
 @pytest.mark.parametrize("window", [0, WINDOW])
 def test_bf16_bwd_one_train_group(window):
-    """One (b, kv-group) slice of the training shape at full length L = 8192
-    (all 8 query heads of the group): the backward is separable per slice."""
+    """One (b, kv-group) slice with the training shape's group layout (all 8
+    query heads of one KV group) at L = 2048, the length the fp64 oracle's
+    full backward finishes in seconds: the backward is separable per (b,
+    group), so this runs the same per-tile code as the full shape."""
     w = TRAIN
     t = prefill_inputs(1, 2048, 2048, 8, 1, 64, torch.bfloat16, w.qkv_std, w.sink_std, w.dout_std,
                        seed=SEEDS["train"], with_dout=True)

@@ -2,9 +2,11 @@
 
 The attention path partitions into independent problems (a batch, a layer,
 a sequence), so N GPUs run as N ranks that each process their own batch with
-no collective on the data path (weak scaling).  The only cross-rank steps are
-host-side: a barrier around the timed region and the maximum of the ranks'
-device times, from which the whole-job throughput is computed.
+no collective on the data path (weak scaling).  The cross-rank steps are a
+barrier around the timed region and the maximum of the ranks' device times,
+from which the whole-job throughput is computed; and, for data-parallel
+training over batch shards, the sum of the ranks' sink gradients
+(allreduce_dsinks: attn_sink_bwd sums dsinks over its own batch only).
 """
 from __future__ import annotations
 
@@ -48,3 +50,14 @@ def job_throughput(units_per_rank: float, world: int, seconds: float) -> float:
 def barrier() -> None:
     if dist.is_initialized() and dist.get_world_size() > 1:
         dist.barrier()
+
+
+def allreduce_dsinks(dsinks: torch.Tensor) -> torch.Tensor:
+    """Sum the per-rank sink gradients in place (one all-reduce of Hq floats).
+
+    Each rank's attn_sink_bwd returns dsinks summed over that rank's batch
+    shard; the sink logits are shared by all ranks, so their gradient is the
+    sum over ranks.  Identity for one process."""
+    if dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(dsinks, op=dist.ReduceOp.SUM)
+    return dsinks

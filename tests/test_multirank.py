@@ -50,3 +50,37 @@ def test_two_gloo_ranks():
 def test_single_process_defaults():
     assert multirank.max_over_ranks([3.0, 4.0]) == [3.0, 4.0]
     assert multirank.rank_seed(5, 0) == 5
+
+
+def _dsink_worker(rank, world, port, out):
+    # rank r holds batch element r of a B = 2 problem and its own backward
+    os.environ.update({"MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port), "RANK": str(rank),
+                       "WORLD_SIZE": str(world), "LOCAL_RANK": str(rank)})
+    import oracle
+
+    multirank.init("gloo", timeout_s=60)
+    t = prefill_inputs(2, 24, 24, 4, 2, 64, torch.float32, 1.0, 1.0, 1.0, seed=77, with_dout=True)
+    sh = {k: (v[rank:rank + 1] if k in ("q", "k", "v", "dout") else v) for k, v in t.items()}
+    _, _, _, ds = oracle.bwd(sh["q"], sh["k"], sh["v"], sh["sinks"], sh["dout"], 0, 0.125)
+    local = torch.tensor(ds, dtype=torch.float64)
+    total = multirank.allreduce_dsinks(local.clone())
+    out[rank] = (local.tolist(), total.tolist())
+    torch.distributed.destroy_process_group()
+
+
+def test_dsinks_allreduce_over_batch_shards():
+    import numpy as np
+
+    import oracle
+
+    world, port = 2, _free_port()
+    manager = mp.Manager()
+    out = manager.dict()
+    mp.start_processes(_dsink_worker, args=(world, port, out), nprocs=world, join=True, start_method="spawn")
+    t = prefill_inputs(2, 24, 24, 4, 2, 64, torch.float32, 1.0, 1.0, 1.0, seed=77, with_dout=True)
+    _, _, _, full = oracle.bwd(t["q"], t["k"], t["v"], t["sinks"], t["dout"], 0, 0.125)
+    (l0, s0), (l1, s1) = out[0], out[1]
+    assert not np.allclose(l0, l1)                            # each rank saw only its shard
+    assert s0 == s1                                           # every rank holds the same sum
+    np.testing.assert_allclose(s0, full, rtol=1e-12, atol=1e-14)  # = dsinks of the whole batch
+

@@ -6,8 +6,11 @@ Hkv=8, D=64, bf16 -- as two layers run back to back, one dense causal and one
 causal banded to a window of 128 (forward: output bf16 + fp32 LSE).
 Metric: prefill TFLOP/s, counting only unmasked scores (4*D flops per visible
 (query, key) pair), whole job over all ranks.  Further legs measured in the
-same run (rank 0 only): split-KV decode (B=64 ragged sequences up to 32768,
-dense and window-128) in KV GB/s, and the backward.
+same run (rank 0 only), each against its own roof: split-KV decode (B=64
+ragged sequences up to 32768, dense and window-128, contiguous and paged) in
+KV GB/s; the backward at the prefill shape; forward and backward at the
+training shape (B8 L8192); the long-context layers (window 128 at L=131072,
+dense at L=32768).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--no-legs]
 
@@ -359,35 +362,103 @@ def decode_legs(dev, reps=20, warmup=3, batch=None):
     return legs
 
 
-def bwd_legs(dev, reps=5, warmup=2):
+def fwd_bytes(B_, L_, Hq_, Hkv_):
+    """Compulsory bytes of one forward: read q, k, v (bf16), sinks; write out (bf16) and lse (fp32)."""
+    return 2 * B_ * L_ * Hq_ * D * 2 + 2 * 2 * B_ * L_ * Hkv_ * D + 4 * Hq_ + 4 * B_ * Hq_ * L_
+
+
+def bwd_bytes(B_, L_, Hq_, Hkv_):
+    """Compulsory bytes of one backward: read q, out, dout (bf16), lse (fp32), k, v, sinks;
+    write dq (bf16), dk, dv (bf16), dsinks."""
+    return 4 * B_ * L_ * Hq_ * D * 2 + 4 * B_ * L_ * Hkv_ * D * 2 + 4 * B_ * Hq_ * L_ + 8 * Hq_
+
+
+def device_prefill(B_, L_, Hq_, Hkv_, sink_std, seed, dev, with_dout):
+    """Seeded synthetic prefill inputs drawn on the device (q, k, v ~ N(0,1)*0.5 bf16,
+    sinks ~ N(0, sink_std^2) fp32, dout ~ N(0,1)*0.1): the bench legs' timing inputs."""
+    g = torch.Generator(device=dev).manual_seed(seed)
+    t = {"q": (torch.randn(B_, L_, Hq_, D, device=dev, generator=g) * 0.5).to(torch.bfloat16),
+         "k": (torch.randn(B_, L_, Hkv_, D, device=dev, generator=g) * 0.5).to(torch.bfloat16),
+         "v": (torch.randn(B_, L_, Hkv_, D, device=dev, generator=g) * 0.5).to(torch.bfloat16),
+         "sinks": torch.randn(Hq_, device=dev, generator=g) * sink_std}
+    if with_dout:
+        t["dout"] = (torch.randn(B_, L_, Hq_, D, device=dev, generator=g) * 0.1).to(torch.bfloat16)
+    return t
+
+
+def timed(dev, fn, reps, warmup, flush):
+    """Median device time (ms) of fn() over `reps` runs after `warmup`, L2 flushed before each."""
+    stream = torch.cuda.current_stream(dev)
+    times = []
+    for it in range(reps + warmup):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        if it >= warmup:
+            times.append(e0.elapsed_time(e1))
+    return statistics.median(times)
+
+
+def leg_entry(ms, flops, nbytes, bound, shape):
+    hbm, tf_burst, _, _ = peaks()
+    tf = flops / (ms * 1e-3) / 1e12
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    e = {"ms": ms, "TFLOP/s": tf, "frac_tensor": tf / tf_burst, "GB/s": gbs, "frac_hbm": gbs / hbm,
+         "flops": flops, "bytes": nbytes, "bound": bound, "shape": shape}
+    e["frac"] = e["frac_hbm"] if bound == "hbm" else e["frac_tensor"]
+    return e
+
+
+def prefill_legs(dev, which=("bwd", "train", "long"), reps=5, warmup=2):
+    """Forward / backward legs beyond the headline step, each with its own roofline
+    fraction (dense layers against the tensor peak, window-128 layers against HBM),
+    L2 flushed before every timed run:
+      bwd:   the backward at the prefill shape (B1 L4096 Hq64 Hkv8);
+      train: forward and backward at the training shape (B8 L8192 Hq64 Hkv8);
+      long:  the long-context layers (window 128 at L = 131072, dense at L = 32768)."""
     import gqa_softmax_attention_attn_b200 as attn
 
-    hbm, tf_burst, _, _ = peaks()
-    d, _ = make_prefill(2002, dev)
     stream = torch.cuda.current_stream(dev)
-    out = torch.empty_like(d["q"])
-    lse = torch.empty(B, HQ, L, device=dev, dtype=torch.float32)
-    dq, dk, dv = torch.empty_like(d["q"]), torch.empty_like(d["k"]), torch.empty_like(d["v"])
-    ds = torch.empty(HQ, device=dev, dtype=torch.float32)
-    ws = torch.empty(attn.attn_sink_bwd_workspace_size(B, L, L, HQ, HKV, D, attn.DTYPE_BF16), dtype=torch.uint8,
-                     device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     legs = {}
-    for name, window in (("bwd_dense", 0), ("bwd_window128", WIN)):
-        attn.attn_sink_fwd(d["q"], d["k"], d["v"], d["sinks"], out, lse, window, SCALE, stream)
-        times = []
-        for it in range(reps + warmup):
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            attn.attn_sink_bwd(d["q"], d["k"], d["v"], d["sinks"], out, d["dout"], lse, dq, dk, dv, ds, window,
-                               SCALE, ws, stream)
-            e1.record(stream)
-            torch.cuda.synchronize(dev)
-            if it >= warmup:
-                times.append(e0.elapsed_time(e1))
-        ms = statistics.median(times)
-        fl = 2.5 * fwd_flops(B, L, HQ, window)
-        legs[name] = {"ms": ms, "TFLOP/s": fl / (ms * 1e-3) / 1e12, "frac_tensor": fl / (ms * 1e-3) / 1e12 / tf_burst,
-                      "shape": "B1 L4096 Hq64 Hkv8 D64"}
+
+    def run_shape(prefix, B_, L_, sink_std, seed, windows, do_bwd, do_fwd):
+        t = device_prefill(B_, L_, HQ, HKV, sink_std, seed, dev, do_bwd)
+        out = torch.empty_like(t["q"])
+        lse = torch.empty(B_, HQ, L_, device=dev, dtype=torch.float32)
+        shape = f"B{B_} L{L_} Hq{HQ} Hkv{HKV} D{D}"
+        if do_bwd:
+            dq, dk, dv = torch.empty_like(t["q"]), torch.empty_like(t["k"]), torch.empty_like(t["v"])
+            ds = torch.empty(HQ, device=dev, dtype=torch.float32)
+            ws = torch.empty(attn.attn_sink_bwd_workspace_size(B_, L_, L_, HQ, HKV, D, attn.DTYPE_BF16),
+                             dtype=torch.uint8, device=dev)
+        for window in windows:
+            tag = "dense" if window <= 0 else "window128"
+            bound = "tensor" if window <= 0 else "hbm"
+            fwd = lambda: attn.attn_sink_fwd(t["q"], t["k"], t["v"], t["sinks"], out, lse, window, SCALE, stream)
+            if do_fwd:
+                ms = timed(dev, fwd, reps, warmup, flush)
+                legs[f"{prefix}fwd_{tag}"] = leg_entry(ms, fwd_flops(B_, L_, HQ, window), fwd_bytes(B_, L_, HQ, HKV),
+                                                       bound, shape)
+            if do_bwd:
+                fwd()
+                bwd = lambda: attn.attn_sink_bwd(t["q"], t["k"], t["v"], t["sinks"], out, t["dout"], lse, dq, dk, dv,
+                                                 ds, window, SCALE, ws, stream)
+                ms = timed(dev, bwd, reps, warmup, flush)
+                legs[f"{prefix}bwd_{tag}"] = leg_entry(ms, 2.5 * fwd_flops(B_, L_, HQ, window),
+                                                       bwd_bytes(B_, L_, HQ, HKV), bound, shape)
+        assert attn.attn_sink_get_device_status(stream) == 0
+
+    if "bwd" in which:
+        run_shape("", B, L, 1.0, 2002, (0, WIN), True, False)
+    if "train" in which:
+        run_shape("train_", 8, 8192, 1.0, 2003, (0, WIN), True, True)
+    if "long" in which:
+        run_shape("long_", 1, 131072, 2.0, 2005, (WIN,), False, True)
+        run_shape("long_", 1, 32768, 2.0, 2006, (0,), False, True)
     return legs
 
 
@@ -484,7 +555,7 @@ def main():
     ap.add_argument("--no-legs", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["decode", "bwd"], default=None,
+    ap.add_argument("--only", choices=["decode", "bwd", "train", "long"], default=None,
                     help="run just one leg (reps = --steps, warm-up = --warmup); used for profiling")
     ap.add_argument("--decode-batch", type=int, default=None, help="sequences in the decode leg (default 64)")
     args = ap.parse_args()
@@ -507,7 +578,7 @@ def main():
     torch.cuda.set_device(dev)
     if args.only is not None:
         legs = (decode_legs(dev, args.steps, args.warmup, args.decode_batch) if args.only == "decode"
-                else bwd_legs(dev, args.steps, args.warmup))
+                else prefill_legs(dev, (args.only,), args.steps, args.warmup))
         print(json.dumps({"only": args.only, "legs": legs}), flush=True)
         return
     res = run_ours(args, rank, world, dev)
@@ -515,7 +586,7 @@ def main():
         if not args.no_legs and world == 1:
             res["legs"] = {}
             res["legs"].update(decode_legs(dev))
-            res["legs"].update(bwd_legs(dev))
+            res["legs"].update(prefill_legs(dev))
         if not args.no_cpu_baseline and world == 1:
             v, cores, desc, _, _ = oracle_sample(12.0)
             res["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc,

@@ -12,9 +12,11 @@
 // Design (B200):
 //  * Work item = 128 query rows = (128 / Gp) positions x Gp query heads of one
 //    KV group, so every K/V tile fetched is shared by Gp heads (GQA packing;
-//    no cluster multicast).  Persistent CTAs (two per SM, 256 TMEM columns
-//    each) take work items from a longest-first list through one atomic
-//    counter per launch (a CTA on a faster SM takes more of them).
+//    no cluster multicast).  The grid has one CTA per work item, numbered
+//    longest first; a running CTA (two per SM, 256 TMEM columns each) takes
+//    over the items of CTAs that have not started yet through cluster launch
+//    control (the hardware cancels their launch), so a CTA on a faster SM
+//    takes more items, and no counter or other state outlives the launch.
 //  * Warp 0: item fetch (passed to the other warps through a shared-memory
 //    ring) and TMA producer -- Q (double-buffered, so the next item's Q lands
 //    while the current one finishes) and K/V tiles of BN keys into an
@@ -41,7 +43,6 @@
 #include <math.h>
 
 #include <algorithm>
-#include <atomic>
 
 #include "kernels.h"
 #include "sm100_ptx.cuh"
@@ -107,9 +108,10 @@ struct FwdCfg {
     static constexpr int kOffV = kOffK + NS * kKVBytes;
     static constexpr int kOffBar = kOffV + NS * kKVBytes;
     // q_full[2], q_empty[2], k_full[NS], k_empty[NS], v_full[NS], v_empty[NS],
-    // s_full[2], p_full[2], o_done, o_free, drain, xchg[4], item_full[4], item_empty[4]
-    static constexpr int kNumBar = 4 + 4 * NS + 4 + 3 + 4 + 8;
-    static constexpr int kOffMisc = kOffBar + kNumBar * 8;
+    // s_full[2], p_full[2], o_done, o_free, drain, xchg[4], item_full[4], item_empty[4], clc
+    static constexpr int kNumBar = 4 + 4 * NS + 4 + 3 + 4 + 8 + 1;
+    // tmem slot (+0), abort flag (+4), item ring (+16, 4 ints), launch-control response (+32, 16 bytes)
+    static constexpr int kOffMisc = (kOffBar + kNumBar * 8 + 15) / 16 * 16;
     // row partials exchanged by the two softmax warps of a row: [2 slots][2 halves][128 rows]
     static constexpr int kOffXchg = kOffMisc + 64;
     static constexpr int kTmemCols = pow2_at_least(2 * BN + kD);
@@ -133,45 +135,11 @@ struct FwdTcParams {
     float *lse;
     unsigned *status;
     long long timeout_ns;
-    int sched_slot;  // this launch's counter in g_fwd_sched / g_fwd_done (dynamic item order)
 };
 
 struct Item {
     int pos0, h0, b, t_lo, n_tiles;
 };
-
-// Dynamic item order: the persistent CTAs take work items, longest first, from
-// one counter per launch (one atomic add per item), so a CTA on a faster SM
-// simply takes more of them (with a fixed assignment, CTAs given equal work
-// finished 182-209 us apart).  Launch number n uses counter n % kSchedSlots,
-// which is 0 when it starts: the last CTA of every launch (counted in
-// g_fwd_done) sets it back to 0, so replaying a captured launch starts
-// afresh.  Up to kSchedSlots forward launches may run at once on one device.
-#ifndef ATTN_SINK_FWD_DYNAMIC
-#define ATTN_SINK_FWD_DYNAMIC 1
-#endif
-constexpr int kSchedSlots = 64;
-__device__ unsigned g_fwd_sched[kSchedSlots];
-__device__ unsigned g_fwd_done[kSchedSlots];
-
-// Next item for this CTA from the launch's counter, or -1 when none is left.
-__device__ __forceinline__ int fetch_item(const FwdTcParams &p)
-{
-    const unsigned i = atomicAdd(&g_fwd_sched[p.sched_slot], 1u);
-    return i < (unsigned)p.n_items ? (int)i : -1;
-}
-
-// The r-th work item of this CTA, or -1 past the end: rounds of gridDim.x
-// items in snake order (even rounds ascending in blockIdx, odd rounds
-// descending), so that over the longest-first list every CTA gets a similar
-// total length (round-robin in one direction left the CTA that always takes
-// the longest item of a round 11-14% above the mean on a causal layer).
-__device__ __forceinline__ int cta_item(int r, int n_items)
-{
-    const long g = gridDim.x;
-    const long w = (long)r * g + ((r & 1) ? g - 1 - (long)blockIdx.x : (long)blockIdx.x);
-    return w < n_items ? (int)w : -1;
-}
 
 // Work item i of the longest-first order: q tiles from the last (most keys
 // under a causal mask) to the first, all head tiles and batches of one q tile
@@ -229,7 +197,9 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT>::kThreads, CPS)
     // them to the MMA warp and the softmax warps through 4 slots
     uint64_t *item_full = xchg + 4;        // [4]
     uint64_t *item_empty = item_full + 4;  // [4]
+    uint64_t *clc_full = item_empty + 4;   // launch-control response landed
     volatile int *ring = reinterpret_cast<volatile int *>(smem + Cfg::kOffMisc + 16);
+    void *clc_resp = smem + Cfg::kOffMisc + 32;
     float *xs = reinterpret_cast<float *>(smem + Cfg::kOffXchg);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Cfg::kOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Cfg::kOffMisc + 4);
@@ -257,6 +227,7 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT>::kThreads, CPS)
             mbar_init(&item_full[r], 1);
             mbar_init(&item_empty[r], 1 + 4 * SPLIT);  // the MMA warp and each softmax warp
         }
+        mbar_init(clc_full, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -269,11 +240,28 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT>::kThreads, CPS)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    // r-th item of this CTA: the producer (lane 0 of warp 0) fetches it and
-    // publishes it in the ring; every other warp reads it there (-1: no more)
+    // r-th item of this CTA: its own (blockIdx.x) first, then the items of the
+    // CTAs whose launch it cancels.  The producer (lane 0 of warp 0) learns
+    // it, requests the next one at once (so the request's latency hides behind
+    // the item) and publishes it in the ring; every other warp reads it there
+    // (-1: no more).
+    uint32_t clc_waits = 0;    // responses consumed
+    bool clc_pending = false;  // a request is in flight
     auto producer_item = [&](int r) -> int {
-        if (!ATTN_SINK_FWD_DYNAMIC) return cta_item(r, p.n_items);
-        const int w = fetch_item(p);
+        int w = -1;
+        if (r == 0) {
+            w = (int)blockIdx.x;
+        } else if (clc_pending) {
+            clc_pending = false;
+            if (!mbar_wait(clc_full, clc_waits & 1u, abort_flag, p.status, p.timeout_ns)) return -1;
+            ++clc_waits;
+            w = clc_cancelled_ctaid_x(clc_resp);
+        }
+        if (w >= 0) {  // an empty response ends the requests
+            mbar_arrive_expect_tx(clc_full, 16);
+            clc_try_cancel(clc_resp, clc_full);
+            clc_pending = true;
+        }
         const int sl = r & 3;
         if (!mbar_wait(&item_empty[sl], ((r >> 2) & 1u) ^ 1u, abort_flag, p.status, p.timeout_ns)) return -1;
         ring[sl] = w;
@@ -281,7 +269,6 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT>::kThreads, CPS)
         return w;
     };
     auto consumer_item = [&](int r) -> int {
-        if (!ATTN_SINK_FWD_DYNAMIC) return cta_item(r, p.n_items);
         const int sl = r & 3;
         if (!__all_sync(0xffffffffu, mbar_wait(&item_full[sl], (r >> 2) & 1u, abort_flag, p.status, p.timeout_ns)))
             return -1;
@@ -331,7 +318,9 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT>::kThreads, CPS)
                 }
                 ++item_n;
             }
-            // every load issued must land before the CTA may exit
+            // every load issued, and a launch-control request still in flight,
+            // must land before the CTA may exit
+            if (clc_pending) wait_noabort(clc_full, clc_waits & 1u, p.status, p.timeout_ns);
             for (int s = 0; s < 2; ++s)
                 if (q_issued[s]) wait_noabort(&q_full[s], (q_issued[s] - 1) & 1u, p.status, p.timeout_ns);
             for (int s = 0; s < NS; ++s) {
@@ -631,14 +620,6 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT>::kThreads, CPS)
         tc_fence_after();
         tmem_dealloc(tmem, Cfg::kTmemCols);
     }
-    if (ATTN_SINK_FWD_DYNAMIC && threadIdx.x == 0) {
-        // every CTA has taken its last item: the last one to finish resets the count
-        __threadfence();
-        if (atomicAdd(&g_fwd_done[p.sched_slot], 1u) == gridDim.x - 1) {
-            g_fwd_done[p.sched_slot] = 0;
-            atomicExch(&g_fwd_sched[p.sched_slot], 0u);
-        }
-    }
 }
 
 template <int BN, int NS, int EMU, int CPS, int SPLIT>
@@ -669,8 +650,6 @@ cudaError_t launch_cfg(const void *q, const void *k, const void *v, const float 
     p.lse = lse;
     p.status = device_status_ptr();
     p.timeout_ns = wait_timeout_ns();
-    static std::atomic<unsigned> launches{0};
-    p.sched_slot = (int)(launches.fetch_add(1u, std::memory_order_relaxed) % kSchedSlots);
 
     alignas(64) CUtensorMap mq, mk, mv;
     {
@@ -692,11 +671,9 @@ cudaError_t launch_cfg(const void *q, const void *k, const void *v, const float 
     auto kern = fwd_tc_kernel<BN, NS, EMU, CPS, SPLIT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
     if (e != cudaSuccess) return e;
-    int dev = 0, sms = 0;
-    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    const int grid = (int)std::min<long long>(n_items, (long long)sms * Cfg::kCtasPerSm);
-    kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, st>>>(mq, mk, mv, p);
+    // one CTA per item: as many start as fit (kCtasPerSm per SM), the rest are
+    // taken over by running CTAs before they launch
+    kern<<<p.n_items, Cfg::kThreads, Cfg::kSmemBytes, st>>>(mq, mk, mv, p);
     return cudaGetLastError();
 }
 

@@ -60,11 +60,32 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
     return ok != 0;
 }
 
+// try_wait with an explicit suspend-time limit (nanoseconds) instead of the
+// system-dependent one.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t *bar, uint32_t parity, uint32_t hint_ns)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
+// Waits shorter than this are polled with a suspend-time hint equal to the
+// limit and check the clock after every poll, so a short limit is honoured
+// even when one system-limited suspension would outlast the whole wait.
+constexpr long long kShortWaitNs = 1000000;
+
 // Bounded wait for the phase with the given parity.  Gives up (returning
 // false) when *abort becomes non-zero or after timeout_ns; on a timeout it
 // raises the CTA's abort flag and the device status word so that every other
 // role of the CTA winds down too.  (A suspend-time hint on try_wait was
-// measured slower here: the woken thread resumes late.)
+// measured slower at the default limit: the woken thread resumes late; it is
+// only used for limits below kShortWaitNs.)
 // The polling loop lives in one out-of-line function shared by every call
 // site: the kernels wait at a few dozen places, and a copy of the loop at each
 // one grew the code the SM's instruction cache has to hold (the backward
@@ -73,9 +94,11 @@ static __device__ __noinline__ bool mbar_wait_slow(uint64_t *bar, uint32_t parit
                                             long long timeout_ns)
 {
     const uint64_t t0 = globaltimer_ns();
+    const bool short_limit = timeout_ns < kShortWaitNs;
+    const uint32_t hint = short_limit ? (uint32_t)(timeout_ns > 0 ? timeout_ns : 1) : 0u;
     for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 63u) == 0) {
+        if (short_limit ? mbar_try_wait_hint(bar, parity, hint) : mbar_try_wait(bar, parity)) return true;
+        if (short_limit || (it & 63u) == 0) {
             if (*abort) return false;
             if ((long long)(globaltimer_ns() - t0) > timeout_ns) {
                 *abort = 1;
@@ -91,6 +114,39 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
 {
     if (mbar_try_wait(bar, parity)) return true;
     return mbar_wait_slow(bar, parity, abort, status, timeout_ns);
+}
+
+// ---------------------------------------------------------------- cluster launch control
+// Dynamic work distribution without any global counter: a running CTA asks
+// the hardware to cancel the launch of a CTA of the same grid that has not
+// started yet and takes over that CTA's work.  The 16-byte response is
+// written to shared memory (16-byte aligned) and completes 16 bytes of
+// transaction count on `bar`.  Once a request has come back empty (no CTA
+// left to cancel), the CTA must not issue another.
+__device__ __forceinline__ void clc_try_cancel(void *resp_smem, uint64_t *bar)
+{
+    asm volatile("clusterlaunchcontrol.try_cancel.async.shared::cta.mbarrier::complete_tx::bytes.b128 [%0], [%1];" ::"r"(
+                     smem_u32(resp_smem)),
+                 "r"(smem_u32(bar))
+                 : "memory");
+}
+
+// blockIdx.x of the CTA a completed request cancelled, or -1 if it cancelled
+// none.  Ends with a proxy fence, so the buffer may take the next request.
+__device__ __forceinline__ int clc_cancelled_ctaid_x(const void *resp_smem)
+{
+    uint32_t ok = 0, x = 0;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b128 r;\n\t"
+        "ld.shared.b128 r, [%2];\n\t"
+        "clusterlaunchcontrol.query_cancel.is_canceled.pred.b128 p, r;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t"
+        "@p clusterlaunchcontrol.query_cancel.get_first_ctaid::x.b32.b128 %1, r;\n\t}"
+        : "=r"(ok), "+r"(x)
+        : "r"(smem_u32(resp_smem))
+        : "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    return ok ? (int)x : -1;
 }
 
 // ---------------------------------------------------------------- TMA

@@ -87,11 +87,11 @@ enum { ATTN_SINK_DTYPE_F32 = 0, ATTN_SINK_DTYPE_BF16 = 1 };
  *   scale: multiplies <q, k> (usually 1/sqrt(D)).
  * Lq > Lk is allowed (leading rows then see no key).  B*Lq*Hq*D and
  * B*Lk*Hkv*D must stay below 2^31 elements per tensor for dtype F32.
- * For dtype BF16 the kernel's CTAs share out the work through a counter in
- * the library's static device memory (64 per device, used in turn, each
- * reset by the launch that used it): at most 64 attn_sink_fwd launches may
- * be running at the same time on one device.  Launches captured in a CUDA
- * graph may be replayed.
+ * For dtype BF16 the kernel's CTAs share out the work among themselves
+ * through the hardware's cluster launch control (a running CTA takes over
+ * the work of a CTA of the same launch that has not started); no state is
+ * kept between launches, so any number of launches may run at once, on any
+ * streams, and launches captured in a CUDA graph may be replayed.
  */
 ATTN_SINK_API int attn_sink_fwd(const void *q, const void *k, const void *v, const float *sinks,
                   void *out, float *lse, int B, int Lq, int Lk, int Hq, int Hkv, int D,

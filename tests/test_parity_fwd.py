@@ -7,6 +7,7 @@ import torch
 
 import oracle
 from _harness import assert_close_bf16, assert_close_fp32, assert_lse, errors
+import gqa_softmax_attention_attn_b200 as attn
 from gqa_softmax_attention_attn_b200 import attn_sink_fwd
 from gqa_softmax_attention_attn_b200.inputs import (LONG_BANDED, LONG_DENSE, PREFILL_20B, SEEDS, TINY_FP32, TRAIN,
                                                     WINDOW, prefill_inputs, sample_rows, workload_inputs)
@@ -142,13 +143,14 @@ def test_deterministic_and_stream_ordered():
 
 
 def test_graph_replay_and_concurrent_streams():
-    # persistent CTAs take work items from a per-launch counter: replaying a
-    # captured launch, and launches running at once on two streams, must still
-    # each process every item exactly once
+    # running CTAs take over the items of CTAs that have not started yet
+    # (cluster launch control): replaying a captured launch, and launches of
+    # both layer types running at once on two streams, must still each process
+    # every item exactly once
     t = prefill_inputs(1, 2048, 2048, 64, 8, 64, torch.bfloat16, 0.5, 1.0, seed=12)
     dev = "cuda"
     q, k, v, s = (t[x].to(dev) for x in ("q", "k", "v", "sinks"))
-    ref_o, ref_l = run_fwd(t, 0, 0.125)
+    refs = {w: run_fwd(t, w, 0.125) for w in (0, WINDOW)}
     out = torch.empty_like(q)
     lse = torch.empty(1, 64, 2048, device=dev)
     stream = torch.cuda.Stream()
@@ -163,16 +165,50 @@ def test_graph_replay_and_concurrent_streams():
         lse.zero_()
         g.replay()
         torch.cuda.synchronize()
-        assert torch.equal(out, ref_o) and torch.equal(lse, ref_l)
+        assert torch.equal(out, refs[0][0]) and torch.equal(lse, refs[0][1])
     del g
-    # two streams, several launches each, overlapping on the device
+    # two streams, dense launches on one and window-128 launches on the other,
+    # overlapping on the device
     s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
-    outs = [(torch.empty_like(q), torch.empty_like(lse)) for _ in range(6)]
+    outs = [(torch.empty_like(q), torch.empty_like(lse)) for _ in range(8)]
     torch.cuda.synchronize()
     for i, (o, l) in enumerate(outs):
-        st = s1 if i % 2 == 0 else s2
+        st, w = (s1, 0) if i % 2 == 0 else (s2, WINDOW)
         with torch.cuda.stream(st):
-            attn_sink_fwd(q, k, v, s, o, l, 0, 0.125, st)
+            attn_sink_fwd(q, k, v, s, o, l, w, 0.125, st)
     torch.cuda.synchronize()
-    for o, l in outs:
-        assert torch.equal(o, ref_o) and torch.equal(l, ref_l)
+    for i, (o, l) in enumerate(outs):
+        ro, rl = refs[0 if i % 2 == 0 else WINDOW]
+        assert torch.equal(o, ro) and torch.equal(l, rl), f"launch {i}"
+    assert attn.attn_sink_get_device_status() == 0
+
+
+def test_concurrent_replays_of_two_graphs():
+    """Two captured forwards (a dense and a banded layer) replayed at the same
+    time on two streams, many times: every replay complete and exact."""
+    t = prefill_inputs(1, 1024, 1024, 64, 8, 64, torch.bfloat16, 0.5, 1.0, seed=13)
+    dev = "cuda"
+    q, k, v, s = (t[x].to(dev) for x in ("q", "k", "v", "sinks"))
+    refs = {w: run_fwd(t, w, 0.125) for w in (0, WINDOW)}
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    bufs, graphs = {}, {}
+    for w, st in ((0, s1), (WINDOW, s2)):
+        bufs[w] = (torch.empty_like(q), torch.empty(1, 64, 1024, device=dev))
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=st, capture_error_mode="thread_local"):
+            attn_sink_fwd(q, k, v, s, bufs[w][0], bufs[w][1], w, 0.125, st)
+        graphs[w] = (g, st)
+    for _ in range(10):
+        for w in (0, WINDOW):
+            bufs[w][0].zero_()
+            bufs[w][1].zero_()
+        torch.cuda.synchronize()
+        for w in (0, WINDOW):
+            g, st = graphs[w]
+            with torch.cuda.stream(st):
+                g.replay()
+        torch.cuda.synchronize()
+        for w in (0, WINDOW):
+            assert torch.equal(bufs[w][0], refs[w][0]) and torch.equal(bufs[w][1], refs[w][1])
+    del graphs
+    assert attn.attn_sink_get_device_status() == 0

@@ -330,6 +330,31 @@ def decode_legs(dev, reps=20, warmup=3, batch=None):
         gbs = by / (ms * 1e-3) / 1e9
         legs[name] = {"ms": ms, "GB/s": gbs, "frac_hbm": gbs / hbm, "bytes": by,
                       "flops": 4.0 * w.D * kv_rows * (w.Hq // w.Hkv) * w.Hkv}
+    # the same caches in FP8 (e4m3 codes, one scale per KV head): half the bytes
+    from gqa_softmax_attention_attn_b200.inputs import quantize_e4m3_per_head
+
+    k8, ks = quantize_e4m3_per_head(d["k_cache"])
+    v8, vs = quantize_e4m3_per_head(d["v_cache"])
+    for name, window in (("decode_fp8_dense", 0), ("decode_fp8_window128", WIN)):
+        nbytes = attn.attn_sink_decode_workspace_size(nb, w.Hq, w.D, w.Lmax, window, 0)
+        ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
+        kv_rows = sum(min(n, window) if window > 0 else n for n in lens)
+        by = kv_rows * w.Hkv * w.D * 2 + nb * w.Hq * w.D * 2 * 2 + nb * w.Hq * 4 + 4 * nb + 2 * 4 * w.Hkv
+        times = []
+        for it in range(reps + warmup):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            attn.attn_sink_decode_fp8(d["q"], k8, v8, ks, vs, d["seqlens"], d["sinks"], out, lse, window, SCALE, 0,
+                                      ws, stream)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            if it >= warmup:
+                times.append(e0.elapsed_time(e1))
+        ms = statistics.median(times)
+        gbs = by / (ms * 1e-3) / 1e9
+        legs[name] = {"ms": ms, "GB/s": gbs, "frac_hbm": gbs / hbm, "bytes": by, "kv_dtype": "e4m3"}
+    del k8, v8
     # the same caches as a pool of 16-key pages in seeded random order, read
     # through a page table (same compulsory bytes; the table is not credited)
     ps = 16

@@ -65,6 +65,8 @@ def load():
         lib.attn_sink_decode_noalloc.restype = I
         lib.attn_sink_decode_workspace_size.argtypes = [I] * 6
         lib.attn_sink_decode_workspace_size.restype = Z
+        lib.attn_sink_decode_fp8.argtypes = [P] * 9 + [I] * 6 + [F, I, P, Z, P]
+        lib.attn_sink_decode_fp8.restype = I
         lib.attn_sink_decode_paged.argtypes = [P] * 8 + [I] * 8 + [F, I, P, Z, I, P]
         lib.attn_sink_decode_paged.restype = I
         lib.attn_sink_decode_paged_workspace_size.argtypes = [I] * 7
@@ -153,6 +155,28 @@ def attn_sink_decode(q, k_cache, v_cache, seqlens, sinks, out, lse, window: int,
                                  int(window), float(scale), int(num_splits), ws_ptr, ws_bytes, _dtype_code(q),
                                  _stream(stream))
     _check(rc, "attn_sink_decode")
+
+
+def attn_sink_decode_fp8(q, k_cache, v_cache, k_scale, v_scale, seqlens, sinks, out, lse, window: int,
+                         scale: float, num_splits: int = 0, workspace=None, stream=None):
+    """q [B,Hq,D] bf16, caches [B,Lmax,Hkv,D] e4m3 codes (uint8 or float8_e4m3fn), k_scale/v_scale [Hkv]
+    fp32, seqlens [B] int32 -> writes out [B,Hq,D] bf16, lse [B,Hq]."""
+    B, Hq, D = q.shape
+    Lmax, Hkv = k_cache.shape[1], k_cache.shape[2]
+    for name, c in (("k_cache", k_cache), ("v_cache", v_cache)):
+        if c.element_size() != 1:
+            raise TypeError(f"{name} must hold one-byte e4m3 codes, got {c.dtype}")
+    ws_ptr, ws_bytes = 0, 0
+    if workspace is not None:
+        ws_ptr = _dev(workspace, "workspace")
+        ws_bytes = workspace.numel() * workspace.element_size()
+    rc = load().attn_sink_decode_fp8(_dev(q, "q", torch.bfloat16), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+                                     _dev(k_scale, "k_scale", torch.float32), _dev(v_scale, "v_scale", torch.float32),
+                                     _dev(seqlens, "seqlens", torch.int32), _dev(sinks, "sinks", torch.float32),
+                                     _dev(out, "out", torch.bfloat16), _dev(lse, "lse", torch.float32), B, Lmax, Hq,
+                                     Hkv, D, int(window), float(scale), int(num_splits), ws_ptr, ws_bytes,
+                                     _stream(stream))
+    _check(rc, "attn_sink_decode_fp8")
 
 
 def attn_sink_decode_paged_workspace_size(B: int, Hq: int, D: int, max_pages_per_seq: int, page_size: int,

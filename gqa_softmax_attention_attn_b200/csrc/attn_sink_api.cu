@@ -200,9 +200,11 @@ bool encode_tensor_map_4d(void *map, void *gaddr, int elem_bytes, const uint64_t
         else
             cudaGetLastError();
     });
-    if (!g_encode || (elem_bytes != 2 && elem_bytes != 4)) return false;
+    if (!g_encode || (elem_bytes != 1 && elem_bytes != 2 && elem_bytes != 4)) return false;
     const cuuint32_t estr[4] = {1, 1, 1, 1};
-    const CUtensorMapDataType dt = elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    const CUtensorMapDataType dt = elem_bytes == 1   ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                   : elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                     : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
     const CUresult r = g_encode(static_cast<CUtensorMap *>(map), dt, 4, gaddr,
                                 reinterpret_cast<const cuuint64_t *>(dims),
                                 reinterpret_cast<const cuuint64_t *>(strides_bytes),
@@ -252,6 +254,9 @@ int attn_sink_fwd(const void *q, const void *k, const void *v, const float *sink
     if (!q || !k || !v || !sinks || !out || !lse) return ATTN_SINK_ERR_INVALID_ARG;
     int rc = check_common(B, Lq, Lk, Hq, Hkv, D, dtype);
     if (rc != ATTN_SINK_OK) return rc;
+    // the tensor-core forwards scale the row maximum of the raw scores, which
+    // is the maximum of the scaled scores only for a positive scale
+    if (dtype == ATTN_SINK_DTYPE_BF16 && !(scale > 0.f && scale < INFINITY)) return ATTN_SINK_ERR_UNSUPPORTED;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse) ||
         !aligned16(sinks))
         return ATTN_SINK_ERR_MISALIGNED;
@@ -313,6 +318,37 @@ int attn_sink_decode(const void *q, const void *k_cache, const void *v_cache, co
             e = launch_decode_combine<__nv_bfloat16>(seqlens, sinks, static_cast<__nv_bfloat16 *>(out), lse, s,
                                                      ws_o, ws_ml, st);
     }
+    return launch_status(e);
+}
+
+int attn_sink_decode_fp8(const void *q, const void *k_cache, const void *v_cache, const float *k_scale,
+                         const float *v_scale, const int *seqlens, const float *sinks, void *out, float *lse, int B,
+                         int Lmax, int Hq, int Hkv, int D, int window, float scale, int num_splits, void *workspace,
+                         size_t ws_bytes, void *stream)
+{
+    if (!q || !k_cache || !v_cache || !k_scale || !v_scale || !seqlens || !sinks || !out || !lse)
+        return ATTN_SINK_ERR_INVALID_ARG;
+    if (num_splits < 0 || num_splits > 32) return ATTN_SINK_ERR_INVALID_ARG;
+    int rc = check_common(B, 1, Lmax, Hq, Hkv, D, ATTN_SINK_DTYPE_BF16);
+    if (rc != ATTN_SINK_OK) return rc;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(k_scale) || !aligned16(v_scale) ||
+        !aligned16(out) || !aligned16(lse) || !aligned16(sinks) || !aligned16(seqlens))
+        return ATTN_SINK_ERR_MISALIGNED;
+    const DecodeShape s = decode_shape(B, Lmax, Hq, Hkv, D, window, scale, num_splits);
+    if (!decode_bf16_supported(s)) return ATTN_SINK_ERR_UNSUPPORTED;
+    const size_t need = decode_ws_bytes(s);
+    if (need > 0 && (!workspace || ws_bytes < need)) return ATTN_SINK_ERR_WORKSPACE;
+    if (need > 0 && !aligned16(workspace)) return ATTN_SINK_ERR_MISALIGNED;
+    rc = ensure_device();
+    if (rc != ATTN_SINK_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    float *ws_o = static_cast<float *>(workspace);
+    float *ws_ml = need > 0 ? ws_o + (size_t)s.B * s.Hq * s.splits * s.D : nullptr;
+    cudaError_t e = launch_decode_bf16(q, k_cache, v_cache, seqlens, sinks, out, lse, s, ws_o, ws_ml, st, k_scale,
+                                       v_scale);
+    if (e == cudaSuccess && s.splits > 1)
+        e = launch_decode_combine<__nv_bfloat16>(seqlens, sinks, static_cast<__nv_bfloat16 *>(out), lse, s, ws_o,
+                                                 ws_ml, st);
     return launch_status(e);
 }
 

@@ -30,6 +30,8 @@
 //    and winds down.
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <math.h>
 
 #include "kernels.h"
@@ -41,19 +43,31 @@ namespace {
 constexpr int kD = 64;
 constexpr int kT = 64;          // keys per tile
 constexpr int kNS = 4;          // ring stages
-constexpr int kTileBytes = kT * kD * 2;
-constexpr int kStageBytes = 2 * kTileBytes;  // K and V
 constexpr int kThreads = 160;  // warp 0 producer, warps 1-4 consumers
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
-constexpr int kOffBar = kNS * kStageBytes;
-constexpr int kSmemBytes = kOffBar + 2 * kNS * 8 + 16 + 1024;
+
+// Shared-memory layout; kFp8: K/V cached as e4m3 (one byte per element).
+template <bool kFp8>
+struct DecLayout {
+    static constexpr int kRowBytes = kFp8 ? kD : kD * 2;  // one cached K or V row
+    static constexpr int kTileBytes = kT * kRowBytes;
+    static constexpr int kStageBytes = 2 * kTileBytes;  // K and V
+    // e4m3 only: each consumer warp's 16 keys of K and of V as bf16, 128-byte swizzled
+    static constexpr int kOffStaging = kNS * kStageBytes;
+    static constexpr int kWarpStaging = 2 * 16 * kD * 2;
+    static constexpr int kOffBar = kOffStaging + (kFp8 ? 4 * kWarpStaging : 0);
+    static constexpr int kSmemBytes = kOffBar + 2 * kNS * 8 + 16 + 1024;
+    // the final reduction reuses [0, kOffBar): 4 warps x 16 rows x 66 floats
+    static_assert(4 * 16 * 66 * 4 <= kOffBar, "reduction buffer");
+};
 
 struct DecodeParams {
     DecodeShape sh;  // split rule and (for kPaged) the page pool
     int box_rows;    // rows per TMA box: 64, or page_size when the pages are smaller
     int B, Lmax, Hq, Hkv, G, window, splits, chunk;
     float c_log2;
+    const float *k_scale, *v_scale;  // e4m3 caches: per-KV-head dequantisation scales
     const __nv_bfloat16 *q;
     const int *seqlens;
     const float *sinks;
@@ -90,16 +104,36 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
 // byte offset of (row, 16-byte chunk) in a 128-byte-swizzled tile
 __device__ __forceinline__ uint32_t swz(int row, int chunk) { return row * 128 + ((chunk ^ (row & 7)) << 4); }
 
-template <bool kRows16, bool kPaged>
+// 16 e4m3 values (byte i = element i) -> 16 bf16, elements 0-7 in lo and 8-15
+// in hi (element 2m in the low half of word m).  Exact: every e4m3 value is a
+// half and a bf16 (e4m3 -> f16x2 by the hardware conversion, then f32, then
+// bf16 round-to-nearest, which changes nothing).
+__device__ __forceinline__ void e4m3x16_to_bf16(const uint4 &raw, uint4 &lo, uint4 &hi)
+{
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+    uint32_t o[8];
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+        const __nv_fp8x2_storage_t pr = (__nv_fp8x2_storage_t)((w[m >> 1] >> (16 * (m & 1))) & 0xffffu);
+        const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(pr, __NV_E4M3);
+        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&h));
+        o[m] = pack_bf16x2(f.x, f.y);
+    }
+    lo = make_uint4(o[0], o[1], o[2], o[3]);
+    hi = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
+template <bool kRows16, bool kPaged, bool kFp8>
 __global__ void __launch_bounds__(kThreads)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                      const DecodeParams p)
 {
+    using L = DecLayout<kFp8>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + kOffBar);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::kOffBar);
     uint64_t *empty = full + kNS;
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffBar + 2 * kNS * 8);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kOffBar + 2 * kNS * 8);
 
     const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -136,7 +170,7 @@ __global__ void __launch_bounds__(kThreads)
             for (int j = 0; j < n_tiles; ++j) {
                 const int st = j % kNS;
                 if (!mbar_wait(&empty[st], ((j / kNS) & 1u) ^ 1u, abort_flag, p.status, p.timeout_ns)) break;
-                mbar_arrive_expect_tx(&full[st], kStageBytes);
+                mbar_arrive_expect_tx(&full[st], L::kStageBytes);
                 if (kPaged) {
                     // the tile's keys in boxes of box_rows rows, each inside one page;
                     // pages past the sequence (masked keys) reuse its last page, so the
@@ -148,13 +182,15 @@ __global__ void __launch_bounds__(kThreads)
                         const int lp = min(key / ps, npg - 1);
                         const int phys = p.sh.page_table[(size_t)b * p.sh.max_pages + lp];
                         const int slot = key % ps;
-                        tma_load_4d(smem + st * kStageBytes + r0 * 128, &tmK, 0, g, slot, phys, &full[st]);
-                        tma_load_4d(smem + st * kStageBytes + kTileBytes + r0 * 128, &tmV, 0, g, slot, phys,
+                        tma_load_4d(smem + st * L::kStageBytes + r0 * L::kRowBytes, &tmK, 0, g, slot, phys,
                                     &full[st]);
+                        tma_load_4d(smem + st * L::kStageBytes + L::kTileBytes + r0 * L::kRowBytes, &tmV, 0, g,
+                                    slot, phys, &full[st]);
                     }
                 } else {
-                    tma_load_4d(smem + st * kStageBytes, &tmK, 0, g, kbeg + j * kT, b, &full[st]);
-                    tma_load_4d(smem + st * kStageBytes + kTileBytes, &tmV, 0, g, kbeg + j * kT, b, &full[st]);
+                    tma_load_4d(smem + st * L::kStageBytes, &tmK, 0, g, kbeg + j * kT, b, &full[st]);
+                    tma_load_4d(smem + st * L::kStageBytes + L::kTileBytes, &tmV, 0, g, kbeg + j * kT, b,
+                                &full[st]);
                 }
                 ++issued[st];
             }
@@ -186,7 +222,8 @@ __global__ void __launch_bounds__(kThreads)
                 qa[kk][3] = qpair(gr + 8, 16 * kk + 8 + 2 * tq);
             }
         }
-        const float C = p.c_log2;
+        // e4m3 caches: K's scale folds into the logit scale (V's into the output)
+        const float C = kFp8 ? p.c_log2 * p.k_scale[g] : p.c_log2;
         const uint32_t sbase = smem_u32(smem);
         for (int j = 0; j < n_tiles && ok; ++j) {
             const int st = j % kNS;
@@ -195,14 +232,40 @@ __global__ void __launch_bounds__(kThreads)
                 ok = false;
                 break;
             }
-            const uint32_t kt = sbase + st * kStageBytes, vt = kt + kTileBytes;
+            uint32_t kt = sbase + st * L::kStageBytes, vt = kt + L::kTileBytes;
+            int rw = 16 * w;  // first row of this warp's 16 keys in the tile it reads
+            if (kFp8) {
+                // this warp's 16 keys of K and V, e4m3 -> bf16 into its own staging
+                // (the layout of the bf16 tiles), then the raw stage is free again
+                const uint8_t *k8 = smem + st * L::kStageBytes + 16 * w * L::kRowBytes;
+                const uint8_t *v8 = k8 + L::kTileBytes;
+                uint8_t *ks = smem + L::kOffStaging + w * L::kWarpStaging;
+                uint8_t *vs = ks + L::kWarpStaging / 2;
+#pragma unroll
+                for (int it = 0; it < 2; ++it) {
+                    const int i = lane + 32 * it;
+                    const int row = i >> 2, ch = i & 3;  // 16 rows x 4 chunks of 16 values
+                    uint4 lo, hi;
+                    e4m3x16_to_bf16(*reinterpret_cast<const uint4 *>(k8 + row * L::kRowBytes + ch * 16), lo, hi);
+                    *reinterpret_cast<uint4 *>(ks + swz(row, 2 * ch)) = lo;
+                    *reinterpret_cast<uint4 *>(ks + swz(row, 2 * ch + 1)) = hi;
+                    e4m3x16_to_bf16(*reinterpret_cast<const uint4 *>(v8 + row * L::kRowBytes + ch * 16), lo, hi);
+                    *reinterpret_cast<uint4 *>(vs + swz(row, 2 * ch)) = lo;
+                    *reinterpret_cast<uint4 *>(vs + swz(row, 2 * ch + 1)) = hi;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[st]);
+                kt = smem_u32(ks);
+                vt = smem_u32(vs);
+                rw = 0;
+            }
             const int key0 = kbeg + j * kT + 16 * w;  // first key of this warp's slice
             // ---- S = Q K^T for 16 keys: two n-tiles of 8 keys
             float s[2][4];
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt) {
                 s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
-                const int krow = 16 * w + 8 * nt + (lane & 7);
+                const int krow = rw + 8 * nt + (lane & 7);
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     uint32_t b0, b1, b2, b3;  // d chunks 4*half + 0..3
@@ -267,7 +330,7 @@ __global__ void __launch_bounds__(kThreads)
             // rows of V outside [lo, kend) are zeroed in the operand (cache rows
             // beyond the sequence may hold anything)
             const bool tail = __any_sync(0xffffffffu, key0 + 15 >= kend || key0 < lo);
-            const int vrow = 16 * w + ((lane >> 3) & 1) * 8 + (lane & 7);
+            const int vrow = rw + ((lane >> 3) & 1) * 8 + (lane & 7);
 #pragma unroll
             for (int jn = 0; jn < 8; jn += 2) {
                 uint32_t b0, b1, b2, b3;
@@ -287,7 +350,7 @@ __global__ void __launch_bounds__(kThreads)
                 mma16816(o[jn + 1], pa, b2, b3);
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[st]);
+            if (!kFp8 && lane == 0) mbar_arrive(&empty[st]);
         }
         // row sums over the 4 lanes of a fragment row
         l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
@@ -320,6 +383,7 @@ __global__ void __launch_bounds__(kThreads)
     }
     __syncthreads();
     const int rows = kRows16 ? 16 : 8;
+    const float vsc = kFp8 ? p.v_scale[g] : 1.f;  // e4m3 caches: V's dequantisation scale
     for (int e = threadIdx.x; e < rows * kD; e += kThreads) {
         const int r = e / kD, d = e % kD;
         if (r >= p.G) continue;
@@ -343,11 +407,11 @@ __global__ void __launch_bounds__(kThreads)
             const float fs = (sk == -INFINITY) ? 0.f : ex2(sk - M2);
             const float Lt = L * fo + fs;
             const float inv = Lt > 0.f ? 1.f / Lt : 0.f;
-            p.out[((size_t)b * p.Hq + h) * kD + d] = __float2bfloat16_rn(O * fo * inv);
+            p.out[((size_t)b * p.Hq + h) * kD + d] = __float2bfloat16_rn(O * vsc * fo * inv);
             if (d == 0) p.lse[(size_t)b * p.Hq + h] = Lt > 0.f ? (M2 + log2f(Lt)) * kLn2 : -INFINITY;
         } else {
             const size_t slot = ((size_t)b * p.Hq + h) * p.splits + c;
-            p.ws_o[slot * kD + d] = O;
+            p.ws_o[slot * kD + d] = O * vsc;
             if (d == 0) {
                 p.ws_ml[slot * 2 + 0] = M;
                 p.ws_ml[slot * 2 + 1] = L;
@@ -367,9 +431,12 @@ bool decode_bf16_supported(const DecodeShape &s)
 
 cudaError_t launch_decode_bf16(const void *q, const void *kc, const void *vc, const int *seqlens,
                                const float *sinks, void *out, float *lse, const DecodeShape &s, float *ws_o,
-                               float *ws_ml, cudaStream_t st)
+                               float *ws_ml, cudaStream_t st, const float *k_scale, const float *v_scale)
 {
+    const bool fp8 = k_scale != nullptr;
     DecodeParams p;
+    p.k_scale = k_scale;
+    p.v_scale = v_scale;
     p.sh = s;
     p.box_rows = s.page_size > 0 && s.page_size < kT ? s.page_size : kT;
     p.B = s.B;
@@ -395,22 +462,31 @@ cudaError_t launch_decode_bf16(const void *q, const void *kc, const void *vc, co
     // contiguous: [B][Lmax][Hkv][64]; paged pool: [num_pages][page_size][Hkv][64]
     const uint64_t rows = paged ? (uint64_t)s.page_size : (uint64_t)s.Lmax;
     const uint64_t outer = paged ? (uint64_t)s.num_pages : (uint64_t)s.B;
+    // bf16 rows of 128 bytes (128-byte swizzle, the layout ldmatrix reads);
+    // e4m3 rows of 64 bytes, unswizzled (converted by the consumer warps)
+    const int eb = fp8 ? 1 : 2;
     const uint64_t dims[4] = {(uint64_t)kD, (uint64_t)s.Hkv, rows, outer};
-    const uint64_t strides[3] = {(uint64_t)kD * 2, (uint64_t)s.Hkv * kD * 2, rows * s.Hkv * kD * 2};
+    const uint64_t strides[3] = {(uint64_t)kD * eb, (uint64_t)s.Hkv * kD * eb, rows * s.Hkv * kD * eb};
     const uint32_t box[4] = {(uint32_t)kD, 1u, (uint32_t)p.box_rows, 1u};
-    if (!encode_tensor_map_4d(&mk, const_cast<void *>(kc), 2, dims, strides, box, true) ||
-        !encode_tensor_map_4d(&mv, const_cast<void *>(vc), 2, dims, strides, box, true))
+    if (!encode_tensor_map_4d(&mk, const_cast<void *>(kc), eb, dims, strides, box, !fp8) ||
+        !encode_tensor_map_4d(&mv, const_cast<void *>(vc), eb, dims, strides, box, !fp8))
         return cudaErrorInvalidValue;
     const dim3 grid(s.splits, s.Hkv, s.B);
-    auto launch = [&](auto kern) -> cudaError_t {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    auto launch = [&](auto kern, int smem_bytes) -> cudaError_t {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
         if (e != cudaSuccess) return e;
-        kern<<<grid, kThreads, kSmemBytes, st>>>(mk, mv, p);
+        kern<<<grid, kThreads, smem_bytes, st>>>(mk, mv, p);
         return cudaGetLastError();
     };
+    constexpr int sb = DecLayout<false>::kSmemBytes, s8 = DecLayout<true>::kSmemBytes;
+    if (fp8) {
+        if (p.G > 8)
+            return paged ? launch(decode_tc_kernel<true, true, true>, s8) : launch(decode_tc_kernel<true, false, true>, s8);
+        return paged ? launch(decode_tc_kernel<false, true, true>, s8) : launch(decode_tc_kernel<false, false, true>, s8);
+    }
     if (p.G > 8)
-        return paged ? launch(decode_tc_kernel<true, true>) : launch(decode_tc_kernel<true, false>);
-    return paged ? launch(decode_tc_kernel<false, true>) : launch(decode_tc_kernel<false, false>);
+        return paged ? launch(decode_tc_kernel<true, true, false>, sb) : launch(decode_tc_kernel<true, false, false>, sb);
+    return paged ? launch(decode_tc_kernel<false, true, false>, sb) : launch(decode_tc_kernel<false, false, false>, sb);
 }
 
 }  // namespace attn_sink

@@ -1,0 +1,491 @@
+// fwd_band.cu -- bf16 prefill forward of sink-softmax GQA attention for
+// causal layers banded to a short window (gpt-oss alternates dense layers
+// with layers banded to sliding_window = 128: "GPT-OSS 20B Egitimi: Unsloth,
+// A100 ve Hopper Uyumlulugu", section 1; "GPT-OSS-120B 4-bit ...", section 3).
+//
+// What it computes ("GPT-OSS on day 0", section "Sink Attention"): for each
+// query row, the softmax over its visible keys and the head's sink logit,
+// O = sum_j p_j v_j and the log-sum-exp including the sink.
+//
+// Design (B200).  A work item is 128 query rows = P positions x Gp query heads
+// of one KV group (GQA packing, as in the dense forward).  The rows of an item
+// see keys [pos0 + off - W + 1, pos0 + off + P - 1]: W + P - 1 keys, 143 for
+// W = 128 and P = 16.  So one K/V tile of KN >= W + P - 1 rows (144) holds
+// every key of the item, and the item is ONE score MMA (M = 128, N = KN), one
+// exact softmax (no running maximum, no rescale), and one P.V MMA -- instead
+// of a chain of online-softmax round trips over narrow tiles.
+//  * The grid has one CTA per item; two CTAs run per SM (KN <= 144 plus 64 TMEM
+//    columns in a 256-column allocation each; wider bands take the online-
+//    softmax kernel of fwd_tc.cu) and take over the items of CTAs that
+//    have not started yet through cluster launch control.
+//  * Warp 0: TMA producer.  Q (16 KB) and the K and V tiles (KN x 128 B each,
+//    starting at a negative row where the band reaches before key 0: the TMA
+//    fills rows outside the tensor with zeros) are double-buffered, so the
+//    next item's operands land while this one computes.
+//  * Warp 1: the MMA issue loop, run by the whole warp with one elected lane
+//    issuing: S = Q K^T into TMEM; after the softmax, O = P V with P (bf16)
+//    read from TMEM where it overwrote S.
+//  * Warps 2-5: one thread per row.  Pass 1 reads S from TMEM 16 columns at a
+//    time for the row maximum; pass 2 reads it again, takes exp2 of the
+//    log2-scaled logits against max(sink, row max), sums them, and writes P
+//    over S.  Columns outside the row's band are masked only in the 16-column
+//    chunks where some row of the warp needs it.  Then the epilogue: O / l
+//    and lse = m + log2(l) (natural units on output).
+//  * Every wait is bounded; on expiry the CTA raises a status bit, waits
+//    (bounded) for its own TMA loads and MMAs, frees tensor memory and exits.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include "kernels.h"
+#include "sm100_ptx.cuh"
+
+namespace attn_sink {
+namespace {
+
+constexpr int kM = 128;
+constexpr int kD = 64;
+constexpr int kThreads = 192;  // producer, MMA, 4 softmax warps
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr int kTmO = 192;        // O accumulator columns [192, 256)
+constexpr int kTmemCols = 256;   // S (KN <= 144 columns) + O
+constexpr int kCtasPerSm = 2;
+
+template <int KN>
+struct BandCfg {
+    static_assert(KN % 16 == 0 && KN >= 16 && KN <= 144, "KN: a multiple of 16 up to 144");
+    static constexpr int kQBytes = kM * kD * 2;
+    static constexpr int kKVBytes = KN * kD * 2;
+    static constexpr int kOffQ = 0;  // [2]
+    static constexpr int kOffK = 2 * kQBytes;  // [2]
+    static constexpr int kOffV = kOffK + 2 * kKVBytes;  // [2]
+    static constexpr int kOffBar = kOffV + 2 * kKVBytes;
+    // q_full[2] q_empty[2] k_full[2] k_empty[2] v_full[2] v_empty[2] s_full p_full o_done o_free drain
+    // item_full[4] item_empty[4] clc
+    static constexpr int kNumBar = 12 + 5 + 8 + 1;
+    static constexpr int kOffMisc = (kOffBar + kNumBar * 8 + 15) / 16 * 16;
+    // tmem slot (+0), abort flag (+4), item ring (+16), launch-control response (+32)
+    static constexpr int kSmemUsed = kOffMisc + 64 + 1024;  // + slack for 1024-byte alignment
+    // at least a third of the SM's 228 KB, so no third CTA (whose tensor-memory
+    // allocation would have to wait for one of the two others) lands on an SM
+    static constexpr int kSmemBytes = kSmemUsed < 80 * 1024 ? 80 * 1024 : kSmemUsed;
+    static_assert(2 * kSmemBytes <= 227 * 1024, "two CTAs per SM");
+};
+
+struct BandParams {
+    int B, Lq, Lk, Hq, Hkv, window;
+    int G, Gp, P;
+    int n_ptiles, n_htiles, n_items;
+    float c_log2;  // scale * log2(e)
+    const float *sinks;
+    __nv_bfloat16 *out;
+    float *lse;
+    unsigned *status;
+    long long timeout_ns;
+};
+
+struct BandItem {
+    int pos0, h0, b, js;  // first position, first head, batch, first key of the K/V tile
+};
+
+// Item i: head tiles fastest, then position tiles, then batches, so the CTAs
+// running at once cover neighbouring positions of every KV group and share
+// K/V rows through L2.
+__device__ __forceinline__ BandItem band_item(const BandParams &p, int i)
+{
+    BandItem it;
+    it.h0 = (i % p.n_htiles) * p.Gp;
+    const int r = i / p.n_htiles;
+    it.pos0 = (r % p.n_ptiles) * p.P;
+    it.b = r / p.n_ptiles;
+    it.js = it.pos0 + (p.Lk - p.Lq) - p.window + 1;
+    return it;
+}
+
+__device__ __forceinline__ bool wait_noabort(uint64_t *bar, uint32_t parity, unsigned *status, long long tmo)
+{
+    int never = 0;
+    return mbar_wait(bar, parity, &never, status, tmo > 1000000000LL ? tmo : 1000000000LL);
+}
+
+template <int KN>
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+    fwd_band_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const BandParams p)
+{
+    using Cfg = BandCfg<KN>;
+    constexpr int kChunks = KN / 16;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kOffBar);
+    uint64_t *q_full = bars, *q_empty = bars + 2;
+    uint64_t *k_full = bars + 4, *k_empty = bars + 6;
+    uint64_t *v_full = bars + 8, *v_empty = bars + 10;
+    uint64_t *s_full = bars + 12, *p_full = bars + 13, *o_done = bars + 14, *o_free = bars + 15;
+    uint64_t *drain = bars + 16;
+    uint64_t *item_full = bars + 17, *item_empty = bars + 21;
+    uint64_t *clc_full = bars + 25;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Cfg::kOffMisc);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Cfg::kOffMisc + 4);
+    volatile int *ring = reinterpret_cast<volatile int *>(smem + Cfg::kOffMisc + 16);
+    void *clc_resp = smem + Cfg::kOffMisc + 32;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&q_full[s], 1);
+            mbar_init(&q_empty[s], 1);
+            mbar_init(&k_full[s], 1);
+            mbar_init(&k_empty[s], 1);
+            mbar_init(&v_full[s], 1);
+            mbar_init(&v_empty[s], 1);
+        }
+        mbar_init(s_full, 1);
+        mbar_init(p_full, 128);
+        mbar_init(o_done, 1);
+        mbar_init(o_free, 128);
+        mbar_init(drain, 1);
+        for (int r = 0; r < 4; ++r) {
+            mbar_init(&item_full[r], 1);
+            mbar_init(&item_empty[r], 5);  // the MMA warp and the four softmax warps
+        }
+        mbar_init(clc_full, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    // r-th item of this CTA: its own (blockIdx.x), then those of the CTAs whose
+    // launch it cancels (requested one item ahead); published in a 4-slot ring.
+    uint32_t clc_waits = 0;
+    bool clc_pending = false;
+    auto producer_item = [&](int r) -> int {
+        int w = -1;
+        if (r == 0) {
+            w = (int)blockIdx.x;
+        } else if (clc_pending) {
+            clc_pending = false;
+            if (!mbar_wait(clc_full, clc_waits & 1u, abort_flag, p.status, p.timeout_ns)) return -1;
+            ++clc_waits;
+            w = clc_cancelled_ctaid_x(clc_resp);
+        }
+        if (w >= 0) {
+            mbar_arrive_expect_tx(clc_full, 16);
+            clc_try_cancel(clc_resp, clc_full);
+            clc_pending = true;
+        }
+        const int sl = r & 3;
+        if (!mbar_wait(&item_empty[sl], ((r >> 2) & 1u) ^ 1u, abort_flag, p.status, p.timeout_ns)) return -1;
+        ring[sl] = w;
+        mbar_arrive(&item_full[sl]);
+        return w;
+    };
+    auto consumer_item = [&](int r) -> int {
+        const int sl = r & 3;
+        if (!__all_sync(0xffffffffu, mbar_wait(&item_full[sl], (r >> 2) & 1u, abort_flag, p.status, p.timeout_ns)))
+            return -1;
+        const int w = ring[sl];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&item_empty[sl]);
+        return w;
+    };
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            tma_prefetch_desc(&tmQ);
+            tma_prefetch_desc(&tmK);
+            tma_prefetch_desc(&tmV);
+            uint32_t issued[6] = {0, 0, 0, 0, 0, 0};  // q, k, v loads per stage
+            int r = 0;
+            for (int w = producer_item(0); w >= 0; w = producer_item(++r)) {
+                const BandItem t = band_item(p, w);
+                const int st = r & 1;
+                const uint32_t ph = ((r >> 1) & 1u) ^ 1u;
+                const int g = t.h0 / p.G;
+                if (!mbar_wait(&q_empty[st], ph, abort_flag, p.status, p.timeout_ns)) break;
+                mbar_arrive_expect_tx(&q_full[st], Cfg::kQBytes);
+                tma_load_4d(smem + Cfg::kOffQ + st * Cfg::kQBytes, &tmQ, 0, t.h0, t.pos0, t.b, &q_full[st]);
+                ++issued[st];
+                if (!mbar_wait(&k_empty[st], ph, abort_flag, p.status, p.timeout_ns)) break;
+                mbar_arrive_expect_tx(&k_full[st], Cfg::kKVBytes);
+                tma_load_4d(smem + Cfg::kOffK + st * Cfg::kKVBytes, &tmK, 0, g, t.js, t.b, &k_full[st]);
+                ++issued[2 + st];
+                if (!mbar_wait(&v_empty[st], ph, abort_flag, p.status, p.timeout_ns)) break;
+                mbar_arrive_expect_tx(&v_full[st], Cfg::kKVBytes);
+                tma_load_4d(smem + Cfg::kOffV + st * Cfg::kKVBytes, &tmV, 0, g, t.js, t.b, &v_full[st]);
+                ++issued[4 + st];
+            }
+            // every load issued, and a launch-control request in flight, lands before the CTA exits
+            if (clc_pending) wait_noabort(clc_full, clc_waits & 1u, p.status, p.timeout_ns);
+            for (int s = 0; s < 2; ++s) {
+                if (issued[s]) wait_noabort(&q_full[s], (issued[s] - 1) & 1u, p.status, p.timeout_ns);
+                if (issued[2 + s]) wait_noabort(&k_full[s], (issued[2 + s] - 1) & 1u, p.status, p.timeout_ns);
+                if (issued[4 + s]) wait_noabort(&v_full[s], (issued[4 + s] - 1) & 1u, p.status, p.timeout_ns);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        const uint32_t id_s = idesc_bf16_f32(kM, KN, 0);
+        const uint32_t id_pv = idesc_bf16_f32(kM, kD, 1);
+        auto wait_all = [&](uint64_t *bar, uint32_t parity) {
+            return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, p.status, p.timeout_ns));
+        };
+        for (int r = 0, w = consumer_item(0); w >= 0; w = consumer_item(++r)) {
+            const int st = r & 1;
+            const uint32_t ph = (r >> 1) & 1u;
+            if (!wait_all(&q_full[st], ph) || !wait_all(&k_full[st], ph)) break;
+            tc_fence_after();
+            const uint32_t qa = smem_u32(smem + Cfg::kOffQ + st * Cfg::kQBytes);
+            const uint32_t kb = smem_u32(smem + Cfg::kOffK + st * Cfg::kKVBytes);
+            if (elect_one()) {
+#pragma unroll
+                for (int kk = 0; kk < kD / 16; ++kk)
+                    mma_ss(tmem, smem_desc_sw128(qa + kk * 32, 16, 1024), smem_desc_sw128(kb + kk * 32, 16, 1024),
+                           id_s, kk > 0 ? 1u : 0u);
+                mma_commit(s_full);
+                mma_commit(&k_empty[st]);
+                mma_commit(&q_empty[st]);
+            }
+            __syncwarp();
+            // O = P V once the softmax has written P, V has landed and the
+            // previous item's epilogue has read O out
+            if (!wait_all(p_full, r & 1u) || !wait_all(&v_full[st], ph) || !wait_all(o_free, (r & 1u) ^ 1u)) break;
+            tc_fence_after();
+            const uint32_t vb = smem_u32(smem + Cfg::kOffV + st * Cfg::kKVBytes);
+            if (elect_one()) {
+#pragma unroll
+                for (int kk = 0; kk < kChunks; ++kk)
+                    mma_ts(tmem + kTmO, tmem + kk * 8, smem_desc_sw128(vb + kk * 2048, KN * 128, 1024), id_pv,
+                           kk > 0 ? 1u : 0u);
+                mma_commit(o_done);
+                mma_commit(&v_empty[st]);
+            }
+            __syncwarp();
+        }
+        if (elect_one()) mma_commit(drain);
+        __syncwarp();
+        wait_noabort(drain, 0, p.status, p.timeout_ns);
+    } else {
+        // ------------------------------------------------------------ softmax + epilogue
+        const int quad = warp & 3;
+        const int row = quad * 32 + lane;
+        const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
+        const float C = p.c_log2;
+        for (int r = 0, w = consumer_item(0); w >= 0; w = consumer_item(++r)) {
+            const BandItem t = band_item(p, w);
+            const int dp = row / p.Gp;
+            const int pos = t.pos0 + dp;
+            const int h = t.h0 + row % p.Gp;
+            const bool row_valid = pos < p.Lq;
+            const float sink2 = p.sinks[h] * kLog2e;
+            // columns c of the tile (key js + c) this row sees: c in [c_lo, c_hi]
+            const int c_lo = max(dp, -t.js);
+            const int c_hi = row_valid ? min(dp + p.window - 1, p.Lk - 1 - t.js) : -1;
+            if (!__all_sync(0xffffffffu, mbar_wait(s_full, r & 1u, abort_flag, p.status, p.timeout_ns))) break;
+            tc_fence_after();
+            // a chunk needs element masks when some row of the warp does not see all of it
+            uint32_t mask_chunks = 0;
+#pragma unroll
+            for (int c = 0; c < kChunks; ++c)
+                if (__any_sync(0xffffffffu, 16 * c < c_lo || 16 * c + 15 > c_hi)) mask_chunks |= 1u << c;
+
+            // ---- pass 1: row maximum of the visible scores
+            float mx[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) mx[k] = -INFINITY;
+            {
+                // TMEM loads run one 16-column chunk ahead of the arithmetic
+                uint32_t sb[2][16];
+                tmem_ld16(trow, sb[0]);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < kChunks; ++c) {
+                    if (c + 1 < kChunks) tmem_ld16(trow + 16 * (c + 1), sb[(c + 1) & 1]);
+                    float v[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) v[e] = __uint_as_float(sb[c & 1][e]);
+                    if (mask_chunks & (1u << c)) {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) v[e] = (16 * c + e >= c_lo && 16 * c + e <= c_hi) ? v[e] : -INFINITY;
+                    }
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) mx[k] = fmax3(mx[k], v[k], v[8 + k]);
+                    tmem_wait_ld();
+                }
+            }
+            const float tmax = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
+            const float m = fmaxf(sink2, tmax * C);  // reference maximum, log2 units
+            const float neg_m = (m == -INFINITY) ? 0.f : -m;
+            float l = (sink2 == -INFINITY) ? 0.f : ex2(sink2 + neg_m);  // the sink's mass
+
+            // ---- pass 2: P = exp2(S C - m) as bf16 over S, and its row sum
+            {
+                const float2 C2 = make_float2(C, C), M2 = make_float2(neg_m, neg_m);
+                float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+                uint32_t sb[2][16];
+                tmem_ld16(trow, sb[0]);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < kChunks; ++c) {
+                    if (c + 1 < kChunks) tmem_ld16(trow + 16 * (c + 1), sb[(c + 1) & 1]);
+                    uint32_t pk[8];
+                    const bool msk = (mask_chunks & (1u << c)) != 0;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float2 x = ffma2(make_float2(__uint_as_float(sb[c & 1][2 * e]),
+                                                           __uint_as_float(sb[c & 1][2 * e + 1])),
+                                               C2, M2);
+                        float2 pe = make_float2(ex2(x.x), ex2(x.y));
+                        if (msk) {
+                            const int c0 = 16 * c + 2 * e;
+                            pe.x = (c0 >= c_lo && c0 <= c_hi) ? pe.x : 0.f;
+                            pe.y = (c0 + 1 >= c_lo && c0 + 1 <= c_hi) ? pe.y : 0.f;
+                        }
+                        acc[e & 1] = fadd2(acc[e & 1], pe);
+                        pk[e] = pack_bf16x2(pe.x, pe.y);
+                    }
+                    tmem_st8(trow + 8 * c, pk);
+                    tmem_wait_ld();
+                }
+                l += (acc[0].x + acc[0].y) + (acc[1].x + acc[1].y);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(p_full);
+
+            // ---- epilogue: O / l, lse
+            if (!__all_sync(0xffffffffu, mbar_wait(o_done, r & 1u, abort_flag, p.status, p.timeout_ns))) break;
+            tc_fence_after();
+            uint32_t o[2][32];
+            tmem_ld32(trow + kTmO, o[0]);
+            tmem_ld32(trow + kTmO + 32, o[1]);
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(o_free);
+            if (row_valid) {
+                const float inv = l > 0.f ? 1.f / l : 0.f;
+                uint4 *dst = reinterpret_cast<uint4 *>(p.out + (((size_t)t.b * p.Lq + pos) * p.Hq + h) * kD);
+#pragma unroll
+                for (int c = 0; c < kD / 8; ++c) {
+                    const uint32_t *src = &o[c / 4][(c % 4) * 8];
+                    uint4 v;
+                    v.x = pack_bf16x2(__uint_as_float(src[0]) * inv, __uint_as_float(src[1]) * inv);
+                    v.y = pack_bf16x2(__uint_as_float(src[2]) * inv, __uint_as_float(src[3]) * inv);
+                    v.z = pack_bf16x2(__uint_as_float(src[4]) * inv, __uint_as_float(src[5]) * inv);
+                    v.w = pack_bf16x2(__uint_as_float(src[6]) * inv, __uint_as_float(src[7]) * inv);
+                    dst[c] = v;
+                }
+                p.lse[((size_t)t.b * p.Hq + h) * p.Lq + pos] = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+template <int KN>
+cudaError_t launch_kn(const void *q, const void *k, const void *v, const BandParams &p, const AttnShape &s,
+                      cudaStream_t st)
+{
+    using Cfg = BandCfg<KN>;
+    alignas(64) CUtensorMap mq, mk, mv;
+    {
+        const uint64_t dims[4] = {(uint64_t)kD, (uint64_t)s.Hq, (uint64_t)s.Lq, (uint64_t)s.B};
+        const uint64_t strides[3] = {(uint64_t)kD * 2, (uint64_t)s.Hq * kD * 2, (uint64_t)s.Lq * s.Hq * kD * 2};
+        const uint32_t box[4] = {(uint32_t)kD, (uint32_t)p.Gp, (uint32_t)p.P, 1u};
+        if (!encode_tensor_map_4d(&mq, const_cast<void *>(q), 2, dims, strides, box, true))
+            return cudaErrorInvalidValue;
+    }
+    {
+        const uint64_t dims[4] = {(uint64_t)kD, (uint64_t)s.Hkv, (uint64_t)s.Lk, (uint64_t)s.B};
+        const uint64_t strides[3] = {(uint64_t)kD * 2, (uint64_t)s.Hkv * kD * 2, (uint64_t)s.Lk * s.Hkv * kD * 2};
+        const uint32_t box[4] = {(uint32_t)kD, 1u, (uint32_t)KN, 1u};
+        if (!encode_tensor_map_4d(&mk, const_cast<void *>(k), 2, dims, strides, box, true) ||
+            !encode_tensor_map_4d(&mv, const_cast<void *>(v), 2, dims, strides, box, true))
+            return cudaErrorInvalidValue;
+    }
+    auto kern = fwd_band_kernel<KN>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    kern<<<p.n_items, kThreads, Cfg::kSmemBytes, st>>>(mq, mk, mv, p);
+    return cudaGetLastError();
+}
+
+// query heads packed per item (a power of two dividing the group, at most 16)
+int packed_heads(const AttnShape &s)
+{
+    const int G = s.Hq / s.Hkv;
+    int gp = 1;
+    while (gp * 2 <= 16 && G % (gp * 2) == 0) gp *= 2;
+    return gp;
+}
+
+// Keys per tile the shape needs: the band plus the item's positions, rounded up
+// to a built tile width (0 when none is wide enough).
+int band_tile_keys(const AttnShape &s)
+{
+    if (s.window <= 0) return 0;
+    const long need = (long)s.window + kM / packed_heads(s) - 1;
+    const int widths[] = {32, 64, 96, 144};
+    for (int w : widths)
+        if (need <= w) return w;
+    return 0;
+}
+
+}  // namespace
+
+bool fwd_band_supported(const AttnShape &s)
+{
+    return s.D == kD && s.Hq % s.Hkv == 0 && s.window > 0 && band_tile_keys(s) > 0 && s.scale > 0.f;
+}
+
+cudaError_t launch_fwd_band(const void *q, const void *k, const void *v, const float *sinks, void *out, float *lse,
+                            const AttnShape &s, cudaStream_t st)
+{
+    BandParams p;
+    p.B = s.B;
+    p.Lq = s.Lq;
+    p.Lk = s.Lk;
+    p.Hq = s.Hq;
+    p.Hkv = s.Hkv;
+    p.window = s.window;
+    p.G = s.Hq / s.Hkv;
+    p.Gp = packed_heads(s);
+    p.P = kM / p.Gp;
+    p.n_ptiles = (s.Lq + p.P - 1) / p.P;
+    p.n_htiles = s.Hq / p.Gp;
+    const long long n_items = (long long)p.n_ptiles * p.n_htiles * s.B;
+    if (n_items > 0x7fffffffLL) return cudaErrorInvalidValue;
+    p.n_items = (int)n_items;
+    p.c_log2 = s.scale * kLog2e;
+    p.sinks = sinks;
+    p.out = static_cast<__nv_bfloat16 *>(out);
+    p.lse = lse;
+    p.status = device_status_ptr();
+    p.timeout_ns = wait_timeout_ns();
+    switch (band_tile_keys(s)) {
+    case 32: return launch_kn<32>(q, k, v, p, s, st);
+    case 64: return launch_kn<64>(q, k, v, p, s, st);
+    case 96: return launch_kn<96>(q, k, v, p, s, st);
+    case 144: return launch_kn<144>(q, k, v, p, s, st);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace attn_sink

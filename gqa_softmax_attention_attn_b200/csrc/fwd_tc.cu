@@ -689,6 +689,7 @@ bool fwd_tc_supported(const AttnShape &s)
 cudaError_t launch_fwd_tc(const void *q, const void *k, const void *v, const float *sinks, void *out,
                           float *lse, const AttnShape &s, cudaStream_t st)
 {
+    if (fwd_band_supported(s)) return launch_fwd_band(q, k, v, sinks, out, lse, s, st);
     if (s.window > 0 && s.window <= 1024)
         return launch_cfg<ATTN_SINK_FWD_BAND_BN, ATTN_SINK_FWD_BAND_NS, -1, ATTN_SINK_FWD_BAND_CPS,
                           ATTN_SINK_FWD_BAND_SPLIT>(q, k, v, sinks, out, lse, s, st);

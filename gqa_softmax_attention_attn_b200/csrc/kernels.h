@@ -70,15 +70,24 @@ template <typename T>
 cudaError_t launch_decode_combine(const int *seqlens, const float *sinks, T *out, float *lse,
                                   const DecodeShape &s, const float *ws_o, const float *ws_ml, cudaStream_t st);
 
+// Tensor-core bf16 prefill forward of short-window banded layers: one K/V tile
+// per work item, exact (single-pass) softmax.
+cudaError_t launch_fwd_band(const void *q, const void *k, const void *v, const float *sinks, void *out,
+                            float *lse, const AttnShape &s, cudaStream_t st);
+bool fwd_band_supported(const AttnShape &s);
+
 // Tensor-core (tcgen05 / TMEM / TMA) bf16 prefill forward.
 cudaError_t launch_fwd_tc(const void *q, const void *k, const void *v, const float *sinks, void *out,
                           float *lse, const AttnShape &s, cudaStream_t st);
 bool fwd_tc_supported(const AttnShape &s);
 
 // bf16 split-KV decode: TMA-staged K/V, tensor-core (mma.sync) group scores.
+// With k_scale / v_scale ([Hkv] fp32, device) the caches hold e4m3 values
+// whose real values are code * scale of their KV head.
 cudaError_t launch_decode_bf16(const void *q, const void *kc, const void *vc, const int *seqlens,
                                const float *sinks, void *out, float *lse, const DecodeShape &s, float *ws_o,
-                               float *ws_ml, cudaStream_t st);
+                               float *ws_ml, cudaStream_t st, const float *k_scale = nullptr,
+                               const float *v_scale = nullptr);
 bool decode_bf16_supported(const DecodeShape &s);
 
 // Driver entry point for cuTensorMapEncodeTiled (resolved once through the runtime).

@@ -114,3 +114,16 @@ def sample_rows(B, Hq, Lq, n, seed, window=0, sinks=None):
             pick = strong[torch.randint(0, len(strong), (k,), generator=g)]
             h[n1 + n2:n1 + n2 + k] = pick
     return b.int(), h.int(), i.int()
+
+
+def quantize_e4m3_per_head(x):
+    """A KV cache [B, L, Hkv, D] in FP8 e4m3 with one fp32 scale per KV head:
+    scale_g = max|x[..., g, :]| / 448 (448 is the largest e4m3 value), codes =
+    x / scale_g rounded to e4m3 by torch's cast.  Returns (codes as uint8, the
+    one-byte storage of the cache; scales [Hkv] fp32).  This only prepares
+    the input format; the attention arithmetic lives elsewhere."""
+    xf = x.float()
+    amax = xf.abs().amax(dim=(0, 1, 3)).clamp_min(1e-12)
+    scales = (amax / 448.0).float()
+    codes = (xf / scales[None, None, :, None]).to(torch.float8_e4m3fn).view(torch.uint8)
+    return codes.contiguous(), scales.contiguous()

@@ -84,7 +84,8 @@ enum { ATTN_SINK_DTYPE_F32 = 0, ATTN_SINK_DTYPE_BF16 = 1 };
  *   out   [B, Lq, Hq, D]   (dtype, written)
  *   lse   [B, Hq, Lq] fp32 (written; natural log, sink included)
  *   window <= 0: dense causal; window > 0: causal band of `window` keys.
- *   scale: multiplies <q, k> (usually 1/sqrt(D)).
+ *   scale: multiplies <q, k> (usually 1/sqrt(D)); for dtype BF16 it must be
+ *          positive and finite (ATTN_SINK_ERR_UNSUPPORTED otherwise).
  * Lq > Lk is allowed (leading rows then see no key).  B*Lq*Hq*D and
  * B*Lk*Hkv*D must stay below 2^31 elements per tensor for dtype F32.
  * For dtype BF16 the kernel's CTAs share out the work among themselves
@@ -128,6 +129,34 @@ ATTN_SINK_API int attn_sink_decode(const void *q, const void *k_cache, const voi
 
 /* Bytes of decode workspace for these sizes (0 when a single split suffices). */
 ATTN_SINK_API size_t attn_sink_decode_workspace_size(int B, int Hq, int D, int Lmax, int window, int num_splits);
+
+/*
+ * Split-KV decode over a KV cache stored in FP8 (e4m3): the operation of
+ * attn_sink_decode with the cached keys and values read at one byte per
+ * element, half the bytes of a bf16 cache.  The pages serve gpt-oss at FP8
+ * precision ("GPT-OSS on day 0", section "GPT-OSS a Hopper") and size the KV
+ * cache in proportion to its element size ("How much computing power is
+ * required for gpt-oss deployment?", the question on the KV cache and context
+ * length); the cache format and its scale granularity are not given there:
+ * here every KV head has one fp32 scale for K and one for V.
+ *   q        [B, Hq, D] bf16
+ *   k_cache, v_cache [B, Lmax, Hkv, D] e4m3 codes (OCP FP8 E4M3: bias 7,
+ *            3 mantissa bits, subnormals, no infinities, 0x7f / 0xff NaN);
+ *            the key (value) of head g is code * k_scale[g] (* v_scale[g]).
+ *   k_scale, v_scale [Hkv] fp32, device.
+ *   seqlens, sinks, window, scale, num_splits, workspace: as attn_sink_decode
+ *            (the workspace size is attn_sink_decode_workspace_size's).
+ *   out      [B, Hq, D] bf16           lse [B, Hq] fp32
+ * Each code is widened exactly (e4m3 -> bf16) and the scales are applied in
+ * fp32: K's to the logits, V's to the output.  Cache rows beyond a sequence's
+ * length may hold any bytes, NaN codes included.  Errors as attn_sink_decode;
+ * a null scale pointer is INVALID_ARG.
+ */
+ATTN_SINK_API int attn_sink_decode_fp8(const void *q, const void *k_cache, const void *v_cache,
+                     const float *k_scale, const float *v_scale, const int *seqlens,
+                     const float *sinks, void *out, float *lse, int B, int Lmax, int Hq, int Hkv,
+                     int D, int window, float scale, int num_splits, void *workspace,
+                     size_t ws_bytes, void *stream);
 
 /*
  * Split-KV decode over a paged KV cache: the same operation as

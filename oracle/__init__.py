@@ -11,8 +11,8 @@ definition it follows is stated in the C file's header ("GPT-OSS on day 0",
 sections "Attention: GQA with Attention Sinks" and "Sink Attention").
 
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
-against library routines (PyTorch CPU fp64 SDPA and autograd), closed forms,
-invariants, brute force and finite differences.  The pages print no worked
+against library routines (PyTorch CPU fp64 SDPA and autograd, torch's FP8
+widening), closed forms, invariants, brute force and finite differences.  The pages print no worked
 example, so no stored golden values from the pages exist.
 """
 from __future__ import annotations
@@ -158,3 +158,38 @@ def row_stats(q, k, v, sinks, dout, window: int, scale: float):
     _load().oracle_row_stats(_ptr(q), _ptr(k), _ptr(v), _ptr(sinks), _ptr(dout), _ptr(Dr), _ptr(Ps),
                              B, Lq, Lk, Hq, Hkv, D, int(window), float(scale))
     return Dr, Ps
+
+
+def _e4m3_from_fields(c):
+    """fp64 values of FP8 E4M3 codes c (OCP 8-bit floating point, E4M3: 1 sign
+    bit, 4 exponent bits with bias 7, 3 mantissa bits; exponent field 0 holds
+    the subnormals m * 2^-9; no infinities; codes 0x7f and 0xff are NaN),
+    computed field by field from that definition."""
+    c = np.asarray(c, dtype=np.int64)
+    sign = np.where((c >> 7) & 1, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 7).astype(np.float64)
+    normal = (1.0 + m / 8.0) * np.power(2.0, e.astype(np.float64) - 7.0)
+    sub = m * 2.0 ** -9
+    v = sign * np.where(e == 0, sub, normal)
+    return np.where((e == 15) & ((c & 7) == 7), np.nan, v)
+
+
+_E4M3 = _e4m3_from_fields(np.arange(256))  # the definition, once per code
+
+
+def e4m3_values(codes):
+    """fp64 values of an array of E4M3 codes (uint8), by the definition above."""
+    c = codes.detach().cpu().view(__import__("torch").uint8).numpy() if hasattr(codes, "detach") else codes
+    return _E4M3[np.asarray(c, dtype=np.uint8)]
+
+
+def decode_fp8(q, k_codes, v_codes, k_scale, v_scale, seqlens, sinks, window: int, scale: float):
+    """Decode over an e4m3 KV cache: every code is widened to its exact value
+    and multiplied by its KV head's scale in fp64, then the decode definition
+    runs unchanged.  Caches [B, Lmax, Hkv, D] of codes; scales [Hkv]."""
+    ks = np.asarray(_f64(k_scale))
+    vs = np.asarray(_f64(v_scale))
+    k = e4m3_values(k_codes) * ks[None, None, :, None]
+    v = e4m3_values(v_codes) * vs[None, None, :, None]
+    return decode(q, k, v, seqlens, sinks, window, scale)

@@ -58,6 +58,9 @@ def test_fwd_host_checks():
     assert lib.attn_sink_fwd(q, k, v, s, o, l, 1, 16, 16, 8, 2, 128, 0, 0.125, 1, None) == UNSUPPORTED
     assert lib.attn_sink_fwd(q, k, v, s, o, l, 1, 16, 16, 8, 2, 64, 0, 0.125, 7, None) == UNSUPPORTED
     assert lib.attn_sink_fwd(q + 2, k, v, s, o, l, 1, 16, 16, 8, 2, 64, 0, 0.125, 1, None) == MISALIGNED
+    # bf16: the scale must be positive and finite
+    for bad in (0.0, -0.125, float("inf"), float("nan")):
+        assert lib.attn_sink_fwd(q, k, v, s, o, l, 1, 16, 16, 8, 2, 64, 0, bad, 1, None) == UNSUPPORTED, bad
 
 
 def test_decode_host_checks():
@@ -71,6 +74,26 @@ def test_decode_host_checks():
     assert lib.attn_sink_decode(*args, 8, ws, need - 4, 1, None) == WORKSPACE
     # one split needs no workspace
     assert attn.attn_sink_decode_workspace_size(4, 8, 64, 4096, 128, 0) == 0
+
+
+def test_decode_fp8_host_checks():
+    lib = attn.load()
+    q, kc, vc, ks, vs, sl, s, o = _fake(8)
+    l, ws = _fake(10)[8:]
+
+    def call(k_scale=ks, v_scale=vs, B=4, Lmax=4096, Hq=8, Hkv=2, D=64, splits=8, w=ws, wbytes=1 << 20):
+        return lib.attn_sink_decode_fp8(q, kc, vc, k_scale, v_scale, sl, s, o, l, B, Lmax, Hq, Hkv, D, 0, 0.125,
+                                        splits, w, wbytes, None)
+
+    assert call(k_scale=None) == INVALID
+    assert call(v_scale=None) == INVALID
+    assert call(splits=33) == INVALID
+    assert call(Hkv=3) == INVALID
+    assert call(D=128) == UNSUPPORTED
+    assert call(k_scale=ks + 4) == MISALIGNED
+    assert call(w=None, wbytes=0) == WORKSPACE
+    need = attn.attn_sink_decode_workspace_size(4, 8, 64, 4096, 0, 8)
+    assert call(wbytes=need - 4) == WORKSPACE
 
 
 def test_decode_paged_host_checks():

@@ -310,3 +310,45 @@ def test_row_stats_reduce_to_dsink():
     _, _, _, ds = oracle.bwd(t["q"], t["k"], t["v"], t["sinks"], t["dout"], 6, 0.4)
     Dr, Ps = oracle.row_stats(t["q"], t["k"], t["v"], t["sinks"], t["dout"], 6, 0.4)
     assert np.abs(-(Ps * Dr).sum(axis=(0, 2)) - ds).max() < 1e-12
+
+
+# ----------------------------------------------------------------------------- FP8 (e4m3) K/V
+def test_e4m3_values_follow_the_format():
+    """The oracle's widening of E4M3 codes: closed-form values of the format
+    (zero, subnormals, smallest normal, one, largest finite, NaN codes), a
+    monotone order over the positive codes, and agreement with torch's
+    float8_e4m3fn widening on every one of the 256 codes."""
+    v = oracle.e4m3_values(np.arange(256, dtype=np.uint8))
+    assert v[0x00] == 0.0 and v[0x80] == 0.0 and np.signbit(v[0x80])
+    assert v[0x38] == 1.0 and v[0xB8] == -1.0
+    assert v[0x01] == 2.0 ** -9 and v[0x07] == 7 * 2.0 ** -9  # subnormals m * 2^-9
+    assert v[0x08] == 2.0 ** -6 and v[0x0F] == 1.875 * 2.0 ** -6  # smallest binade of normals
+    assert v[0x40] == 2.0 and v[0x3C] == 1.5
+    assert v[0x7E] == 448.0 and v[0xFE] == -448.0  # largest finite
+    nan = np.isnan(v)
+    assert nan[0x7F] and nan[0xFF] and nan.sum() == 2
+    assert (np.diff(v[:0x7F]) > 0).all()  # positive codes in increasing order
+    assert np.array_equal(v[0x80:0xFF], -v[:0x7F])  # the sign bit only flips the sign
+    t = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).double().numpy()
+    assert np.array_equal(np.isnan(t), nan) and np.array_equal(t[~nan], v[~nan])
+
+
+def test_decode_fp8_is_decode_of_the_scaled_codes():
+    """decode_fp8 = decode over code * scale per KV head: checked against the
+    bf16/fp32 decode of caches widened by torch, and by two invariances of the
+    scales (K's scale only rescales the logits, V's scale the output)."""
+    from gqa_softmax_attention_attn_b200.inputs import quantize_e4m3_per_head
+
+    d = decode_inputs(3, 40, 8, 2, 16, 5, 40, torch.float32, 0.5, 1.0, seed=81)
+    k8, ks = quantize_e4m3_per_head(d["k_cache"])
+    v8, vs = quantize_e4m3_per_head(d["v_cache"])
+    kw = k8.view(torch.float8_e4m3fn).double() * ks.double()[None, None, :, None]
+    vw = v8.view(torch.float8_e4m3fn).double() * vs.double()[None, None, :, None]
+    for window in (0, 7):
+        o, l = oracle.decode_fp8(d["q"], k8, v8, ks, vs, d["seqlens"], d["sinks"], window, 0.25)
+        ro, rl = oracle.decode(d["q"], kw, vw, d["seqlens"], d["sinks"], window, 0.25)
+        np.testing.assert_allclose(o, ro, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(l, rl, rtol=0, atol=1e-12)
+        o2, l2 = oracle.decode_fp8(d["q"], k8, v8, ks * 2, vs * 4, d["seqlens"], d["sinks"], window, 0.125)
+        np.testing.assert_allclose(o2, 4 * o, rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(l2, l, rtol=0, atol=1e-12)

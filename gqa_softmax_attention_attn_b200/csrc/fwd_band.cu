@@ -62,11 +62,12 @@ struct BandCfg {
     static constexpr int kOffV = kOffK + 2 * kKVBytes;  // [2]
     static constexpr int kOffBar = kOffV + 2 * kKVBytes;
     // q_full[2] q_empty[2] k_full[2] k_empty[2] v_full[2] v_empty[2] s_full p_full o_done o_free drain
-    // item_full[4] item_empty[4] clc
-    static constexpr int kNumBar = 12 + 5 + 8 + 1;
+    // item_full[4] item_empty[4] clc[kClcDepth]
+    static constexpr int kNumBar = 12 + 5 + 8 + kClcDepth;
     static constexpr int kOffMisc = (kOffBar + kNumBar * 8 + 15) / 16 * 16;
-    // tmem slot (+0), abort flag (+4), item ring (+16), launch-control response (+32)
-    static constexpr int kSmemUsed = kOffMisc + 64 + 1024;  // + slack for 1024-byte alignment
+    // tmem slot (+0), abort flag (+4), item ring (+16), launch-control responses (+32, 16 bytes each)
+    static_assert(32 + 16 * kClcDepth <= 128, "misc area");
+    static constexpr int kSmemUsed = kOffMisc + 128 + 1024;  // + slack for 1024-byte alignment
     // at least a third of the SM's 228 KB, so no third CTA (whose tensor-memory
     // allocation would have to wait for one of the two others) lands on an SM
     static constexpr int kSmemBytes = kSmemUsed < 80 * 1024 ? 80 * 1024 : kSmemUsed;
@@ -75,6 +76,9 @@ struct BandCfg {
 
 struct BandParams {
     int B, Lq, Lk, Hq, Hkv, window;
+    const int *cu_q, *cu_k;  // packed ragged sequences (else nullptr)
+    int total_q, total_k;
+    long long lse_hs;        // lse stride between heads: Lq, or total_q for packed sequences
     int G, Gp, P;
     int n_ptiles, n_htiles, n_items;
     float c_log2;  // scale * log2(e)
@@ -86,7 +90,12 @@ struct BandParams {
 };
 
 struct BandItem {
-    int pos0, h0, b, js;  // first position, first head, batch, first key of the K/V tile
+    int pos0, h0, b, js;  // first position, first head, batch, first key of the K/V tile (in the sequence)
+    int Lq, Lk;           // the sequence's query and key counts
+    int qrow0, krow0, tb; // tensor-map rows of its position 0 / key 0, outer coordinate
+    long long orow0;      // output row of its position 0
+    long long lrow0;      // lse index of (head 0, position 0)
+    bool empty;           // past the end of a shorter packed sequence
 };
 
 // Item i: head tiles fastest, then position tiles, then batches, so the CTAs
@@ -99,7 +108,17 @@ __device__ __forceinline__ BandItem band_item(const BandParams &p, int i)
     const int r = i / p.n_htiles;
     it.pos0 = (r % p.n_ptiles) * p.P;
     it.b = r / p.n_ptiles;
-    it.js = it.pos0 + (p.Lk - p.Lq) - p.window + 1;
+    const SeqRows sq = seq_rows(p.cu_q, it.b, p.Lq, p.total_q);
+    const SeqRows sk = seq_rows(p.cu_k, it.b, p.Lk, p.total_k);
+    it.Lq = sq.len;
+    it.Lk = sk.len;
+    it.qrow0 = sq.row0;
+    it.krow0 = sk.row0;
+    it.tb = p.cu_q ? 0 : it.b;
+    it.orow0 = p.cu_q ? (long long)sq.row0 : (long long)it.b * p.Lq;
+    it.lrow0 = p.cu_q ? (long long)sq.row0 : (long long)it.b * p.Hq * p.Lq;
+    it.empty = it.pos0 >= it.Lq;
+    it.js = it.pos0 + (it.Lk - it.Lq) - p.window + 1;
     return it;
 }
 
@@ -125,7 +144,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     uint64_t *s_full = bars + 12, *p_full = bars + 13, *o_done = bars + 14, *o_free = bars + 15;
     uint64_t *drain = bars + 16;
     uint64_t *item_full = bars + 17, *item_empty = bars + 21;
-    uint64_t *clc_full = bars + 25;
+    uint64_t *clc_bar = bars + 25;  // [kClcDepth]
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Cfg::kOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Cfg::kOffMisc + 4);
     volatile int *ring = reinterpret_cast<volatile int *>(smem + Cfg::kOffMisc + 16);
@@ -151,7 +170,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             mbar_init(&item_full[r], 1);
             mbar_init(&item_empty[r], 5);  // the MMA warp and the four softmax warps
         }
-        mbar_init(clc_full, 1);
+        for (int d = 0; d < kClcDepth; ++d) mbar_init(&clc_bar[d], 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -165,24 +184,18 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     const uint32_t tmem = *tmem_slot;
 
     // r-th item of this CTA: its own (blockIdx.x), then those of the CTAs whose
-    // launch it cancels (requested one item ahead); published in a 4-slot ring.
-    uint32_t clc_waits = 0;
-    bool clc_pending = false;
+    // launch it cancels (kClcDepth requests kept in flight); published in a
+    // 4-slot ring.
+    // Items past the end of a shorter packed sequence are passed over here.
+    ClcQueue<kClcDepth> clc{clc_bar, reinterpret_cast<uint8_t *>(clc_resp)};
     auto producer_item = [&](int r) -> int {
-        int w = -1;
-        if (r == 0) {
-            w = (int)blockIdx.x;
-        } else if (clc_pending) {
-            clc_pending = false;
-            if (!mbar_wait(clc_full, clc_waits & 1u, abort_flag, p.status, p.timeout_ns)) return -1;
-            ++clc_waits;
-            w = clc_cancelled_ctaid_x(clc_resp);
+        int w = r == 0 ? (int)blockIdx.x : clc.next(abort_flag, p.status, p.timeout_ns);
+        clc.fill();  // keep kClcDepth requests in flight
+        while (w >= 0 && band_item(p, w).empty) {
+            w = clc.next(abort_flag, p.status, p.timeout_ns);
+            clc.fill();
         }
-        if (w >= 0) {
-            mbar_arrive_expect_tx(clc_full, 16);
-            clc_try_cancel(clc_resp, clc_full);
-            clc_pending = true;
-        }
+        if (clc.failed) return -1;
         const int sl = r & 3;
         if (!mbar_wait(&item_empty[sl], ((r >> 2) & 1u) ^ 1u, abort_flag, p.status, p.timeout_ns)) return -1;
         ring[sl] = w;
@@ -214,19 +227,20 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                 const int g = t.h0 / p.G;
                 if (!mbar_wait(&q_empty[st], ph, abort_flag, p.status, p.timeout_ns)) break;
                 mbar_arrive_expect_tx(&q_full[st], Cfg::kQBytes);
-                tma_load_4d(smem + Cfg::kOffQ + st * Cfg::kQBytes, &tmQ, 0, t.h0, t.pos0, t.b, &q_full[st]);
+                tma_load_4d(smem + Cfg::kOffQ + st * Cfg::kQBytes, &tmQ, 0, t.h0, t.qrow0 + t.pos0, t.tb,
+                            &q_full[st]);
                 ++issued[st];
                 if (!mbar_wait(&k_empty[st], ph, abort_flag, p.status, p.timeout_ns)) break;
                 mbar_arrive_expect_tx(&k_full[st], Cfg::kKVBytes);
-                tma_load_4d(smem + Cfg::kOffK + st * Cfg::kKVBytes, &tmK, 0, g, t.js, t.b, &k_full[st]);
+                tma_load_4d(smem + Cfg::kOffK + st * Cfg::kKVBytes, &tmK, 0, g, t.krow0 + t.js, t.tb, &k_full[st]);
                 ++issued[2 + st];
                 if (!mbar_wait(&v_empty[st], ph, abort_flag, p.status, p.timeout_ns)) break;
                 mbar_arrive_expect_tx(&v_full[st], Cfg::kKVBytes);
-                tma_load_4d(smem + Cfg::kOffV + st * Cfg::kKVBytes, &tmV, 0, g, t.js, t.b, &v_full[st]);
+                tma_load_4d(smem + Cfg::kOffV + st * Cfg::kKVBytes, &tmV, 0, g, t.krow0 + t.js, t.tb, &v_full[st]);
                 ++issued[4 + st];
             }
             // every load issued, and a launch-control request in flight, lands before the CTA exits
-            if (clc_pending) wait_noabort(clc_full, clc_waits & 1u, p.status, p.timeout_ns);
+            clc.drain(p.status, p.timeout_ns);
             for (int s = 0; s < 2; ++s) {
                 if (issued[s]) wait_noabort(&q_full[s], (issued[s] - 1) & 1u, p.status, p.timeout_ns);
                 if (issued[2 + s]) wait_noabort(&k_full[s], (issued[2 + s] - 1) & 1u, p.status, p.timeout_ns);
@@ -286,11 +300,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             const int dp = row / p.Gp;
             const int pos = t.pos0 + dp;
             const int h = t.h0 + row % p.Gp;
-            const bool row_valid = pos < p.Lq;
+            const bool row_valid = pos < t.Lq;
             const float sink2 = p.sinks[h] * kLog2e;
             // columns c of the tile (key js + c) this row sees: c in [c_lo, c_hi]
             const int c_lo = max(dp, -t.js);
-            const int c_hi = row_valid ? min(dp + p.window - 1, p.Lk - 1 - t.js) : -1;
+            const int c_hi = row_valid ? min(dp + p.window - 1, t.Lk - 1 - t.js) : -1;
             if (!__all_sync(0xffffffffu, mbar_wait(s_full, r & 1u, abort_flag, p.status, p.timeout_ns))) break;
             tc_fence_after();
             // a chunk needs element masks when some row of the warp does not see all of it
@@ -374,7 +388,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             mbar_arrive(o_free);
             if (row_valid) {
                 const float inv = l > 0.f ? 1.f / l : 0.f;
-                uint4 *dst = reinterpret_cast<uint4 *>(p.out + (((size_t)t.b * p.Lq + pos) * p.Hq + h) * kD);
+                uint4 *dst = reinterpret_cast<uint4 *>(p.out + ((size_t)(t.orow0 + pos) * p.Hq + h) * kD);
 #pragma unroll
                 for (int c = 0; c < kD / 8; ++c) {
                     const uint32_t *src = &o[c / 4][(c % 4) * 8];
@@ -385,7 +399,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                     v.w = pack_bf16x2(__uint_as_float(src[6]) * inv, __uint_as_float(src[7]) * inv);
                     dst[c] = v;
                 }
-                p.lse[((size_t)t.b * p.Hq + h) * p.Lq + pos] = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
+                p.lse[(size_t)(t.lrow0 + (long long)h * p.lse_hs + pos)] = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
             }
         }
     }
@@ -405,16 +419,20 @@ cudaError_t launch_kn(const void *q, const void *k, const void *v, const BandPar
 {
     using Cfg = BandCfg<KN>;
     alignas(64) CUtensorMap mq, mk, mv;
+    // fixed-length batches: [B][L][H][D]; packed sequences: [1][total][H][D]
+    const uint64_t qrows = s.cu_q ? (uint64_t)s.total_q : (uint64_t)s.Lq;
+    const uint64_t krows = s.cu_q ? (uint64_t)s.total_k : (uint64_t)s.Lk;
+    const uint64_t outer = s.cu_q ? 1u : (uint64_t)s.B;
     {
-        const uint64_t dims[4] = {(uint64_t)kD, (uint64_t)s.Hq, (uint64_t)s.Lq, (uint64_t)s.B};
-        const uint64_t strides[3] = {(uint64_t)kD * 2, (uint64_t)s.Hq * kD * 2, (uint64_t)s.Lq * s.Hq * kD * 2};
+        const uint64_t dims[4] = {(uint64_t)kD, (uint64_t)s.Hq, qrows, outer};
+        const uint64_t strides[3] = {(uint64_t)kD * 2, (uint64_t)s.Hq * kD * 2, qrows * s.Hq * kD * 2};
         const uint32_t box[4] = {(uint32_t)kD, (uint32_t)p.Gp, (uint32_t)p.P, 1u};
         if (!encode_tensor_map_4d(&mq, const_cast<void *>(q), 2, dims, strides, box, true))
             return cudaErrorInvalidValue;
     }
     {
-        const uint64_t dims[4] = {(uint64_t)kD, (uint64_t)s.Hkv, (uint64_t)s.Lk, (uint64_t)s.B};
-        const uint64_t strides[3] = {(uint64_t)kD * 2, (uint64_t)s.Hkv * kD * 2, (uint64_t)s.Lk * s.Hkv * kD * 2};
+        const uint64_t dims[4] = {(uint64_t)kD, (uint64_t)s.Hkv, krows, outer};
+        const uint64_t strides[3] = {(uint64_t)kD * 2, (uint64_t)s.Hkv * kD * 2, krows * s.Hkv * kD * 2};
         const uint32_t box[4] = {(uint32_t)kD, 1u, (uint32_t)KN, 1u};
         if (!encode_tensor_map_4d(&mk, const_cast<void *>(k), 2, dims, strides, box, true) ||
             !encode_tensor_map_4d(&mv, const_cast<void *>(v), 2, dims, strides, box, true))
@@ -465,6 +483,11 @@ cudaError_t launch_fwd_band(const void *q, const void *k, const void *v, const f
     p.Hq = s.Hq;
     p.Hkv = s.Hkv;
     p.window = s.window;
+    p.cu_q = s.cu_q;
+    p.cu_k = s.cu_k;
+    p.total_q = s.total_q;
+    p.total_k = s.total_k;
+    p.lse_hs = s.cu_q ? s.total_q : s.Lq;
     p.G = s.Hq / s.Hkv;
     p.Gp = packed_heads(s);
     p.P = kM / p.Gp;

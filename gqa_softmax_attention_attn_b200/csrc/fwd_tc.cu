@@ -43,6 +43,7 @@
 #include <math.h>
 
 #include <algorithm>
+#include <type_traits>
 
 #include "kernels.h"
 #include "sm100_ptx.cuh"
@@ -93,6 +94,13 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 #ifndef ATTN_SINK_FWD_BAND_SPLIT
 #define ATTN_SINK_FWD_BAND_SPLIT 1
 #endif
+// 1: exponentials against the current reference maximum with the tile maximum
+// taken in the same pass (a rare second pass when it moves); 0: the tile
+// maximum first, then the exponentials
+#ifndef ATTN_SINK_FWD_SPEC
+#define ATTN_SINK_FWD_SPEC 1
+#endif
+constexpr bool FWD_SPEC = ATTN_SINK_FWD_SPEC != 0;
 constexpr int pow2_at_least(int x) { return x <= 32 ? 32 : x <= 64 ? 64 : x <= 128 ? 128 : x <= 256 ? 256 : 512; }
 
 template <int BN, int NS, int CPS, int SPLIT>
@@ -108,12 +116,13 @@ struct FwdCfg {
     static constexpr int kOffV = kOffK + NS * kKVBytes;
     static constexpr int kOffBar = kOffV + NS * kKVBytes;
     // q_full[2], q_empty[2], k_full[NS], k_empty[NS], v_full[NS], v_empty[NS],
-    // s_full[2], p_full[2], o_done, o_free, drain, xchg[4], item_full[4], item_empty[4], clc
-    static constexpr int kNumBar = 4 + 4 * NS + 4 + 3 + 4 + 8 + 1;
-    // tmem slot (+0), abort flag (+4), item ring (+16, 4 ints), launch-control response (+32, 16 bytes)
+    // s_full[2], p_full[2], o_done, o_free, drain, xchg[4], item_full[4], item_empty[4], clc[kClcDepth]
+    static constexpr int kNumBar = 4 + 4 * NS + 4 + 3 + 4 + 8 + kClcDepth;
+    // tmem slot (+0), abort flag (+4), item ring (+16, 4 ints), launch-control responses (+32, 16 bytes each)
     static constexpr int kOffMisc = (kOffBar + kNumBar * 8 + 15) / 16 * 16;
+    static_assert(32 + 16 * kClcDepth <= 128, "misc area");
     // row partials exchanged by the two softmax warps of a row: [2 slots][2 halves][128 rows]
-    static constexpr int kOffXchg = kOffMisc + 64;
+    static constexpr int kOffXchg = kOffMisc + 128;
     static constexpr int kTmemCols = pow2_at_least(2 * BN + kD);
     static constexpr int kCtasPerSm = CPS;  // CTAs resident per SM (TMEM, registers, shared memory)
     static_assert(kTmemCols * CPS <= 512, "tensor memory over-subscribed");
@@ -127,6 +136,9 @@ struct FwdCfg {
 
 struct FwdTcParams {
     int B, Lq, Lk, Hq, Hkv, window;
+    const int *cu_q, *cu_k;  // packed ragged sequences (else nullptr)
+    int total_q, total_k;
+    long long lse_hs;        // lse stride between heads: Lq, or total_q for packed sequences
     int G, Gp, P;  // group size, query heads packed per tile, positions per tile
     int n_ptiles, n_htiles, n_items;
     float c_log2;  // scale * log2(e)
@@ -139,6 +151,12 @@ struct FwdTcParams {
 
 struct Item {
     int pos0, h0, b, t_lo, n_tiles;
+    int Lq, Lk;        // the sequence's query and key counts
+    int qrow0, krow0;  // tensor-map row of its position 0 / key 0
+    int tb;            // tensor-map outer coordinate (batch; 0 for packed sequences)
+    long long orow0;   // output row of its position 0
+    long long lrow0;   // lse index of (head 0, position 0)
+    bool empty;        // the item lies past the end of a shorter packed sequence
 };
 
 // Work item i of the longest-first order: q tiles from the last (most keys
@@ -154,12 +172,22 @@ __device__ __forceinline__ Item item_at(const FwdTcParams &p, int i)
     it.h0 = (r % p.n_htiles) * p.Gp;
     it.b = r / p.n_htiles;
     it.pos0 = qt * p.P;
-    const long off = (long)p.Lk - p.Lq;
-    const int pos_last = min(it.pos0 + p.P - 1, p.Lq - 1);
+    const SeqRows sq = seq_rows(p.cu_q, it.b, p.Lq, p.total_q);
+    const SeqRows sk = seq_rows(p.cu_k, it.b, p.Lk, p.total_k);
+    it.Lq = sq.len;
+    it.Lk = sk.len;
+    it.qrow0 = sq.row0;
+    it.krow0 = sk.row0;
+    it.tb = p.cu_q ? 0 : it.b;
+    it.orow0 = p.cu_q ? (long long)sq.row0 : (long long)it.b * p.Lq;
+    it.lrow0 = p.cu_q ? (long long)sq.row0 : (long long)it.b * p.Hq * p.Lq;
+    it.empty = it.pos0 >= it.Lq;
+    const long off = (long)it.Lk - it.Lq;
+    const int pos_last = min(it.pos0 + p.P - 1, it.Lq - 1);
     const long lo = p.window > 0 ? max(0L, it.pos0 + off - p.window + 1) : 0L;
-    const long hi = min((long)p.Lk, pos_last + off + 1);  // exclusive
+    const long hi = min((long)it.Lk, pos_last + off + 1);  // exclusive
     it.t_lo = (int)(lo / BN);
-    it.n_tiles = hi > lo ? (int)((hi - 1) / BN) - it.t_lo + 1 : 0;
+    it.n_tiles = (hi > lo && !it.empty) ? (int)((hi - 1) / BN) - it.t_lo + 1 : 0;
     return it;
 }
 
@@ -197,7 +225,7 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT>::kThreads, CPS)
     // them to the MMA warp and the softmax warps through 4 slots
     uint64_t *item_full = xchg + 4;        // [4]
     uint64_t *item_empty = item_full + 4;  // [4]
-    uint64_t *clc_full = item_empty + 4;   // launch-control response landed
+    uint64_t *clc_bar = item_empty + 4;    // [kClcDepth]: launch-control responses landed
     volatile int *ring = reinterpret_cast<volatile int *>(smem + Cfg::kOffMisc + 16);
     void *clc_resp = smem + Cfg::kOffMisc + 32;
     float *xs = reinterpret_cast<float *>(smem + Cfg::kOffXchg);
@@ -227,7 +255,7 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT>::kThreads, CPS)
             mbar_init(&item_full[r], 1);
             mbar_init(&item_empty[r], 1 + 4 * SPLIT);  // the MMA warp and each softmax warp
         }
-        mbar_init(clc_full, 1);
+        for (int d = 0; d < kClcDepth; ++d) mbar_init(&clc_bar[d], 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -244,24 +272,17 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT>::kThreads, CPS)
     // CTAs whose launch it cancels.  The producer (lane 0 of warp 0) learns
     // it, requests the next one at once (so the request's latency hides behind
     // the item) and publishes it in the ring; every other warp reads it there
-    // (-1: no more).
-    uint32_t clc_waits = 0;    // responses consumed
-    bool clc_pending = false;  // a request is in flight
+    // (-1: no more).  Items past the end of a shorter packed sequence are
+    // passed over here, so the other warps never see them.
+    ClcQueue<kClcDepth> clc{clc_bar, reinterpret_cast<uint8_t *>(clc_resp)};
     auto producer_item = [&](int r) -> int {
-        int w = -1;
-        if (r == 0) {
-            w = (int)blockIdx.x;
-        } else if (clc_pending) {
-            clc_pending = false;
-            if (!mbar_wait(clc_full, clc_waits & 1u, abort_flag, p.status, p.timeout_ns)) return -1;
-            ++clc_waits;
-            w = clc_cancelled_ctaid_x(clc_resp);
+        int w = r == 0 ? (int)blockIdx.x : clc.next(abort_flag, p.status, p.timeout_ns);
+        clc.fill();  // keep kClcDepth requests in flight
+        while (w >= 0 && item_at<BN>(p, w).empty) {
+            w = clc.next(abort_flag, p.status, p.timeout_ns);
+            clc.fill();
         }
-        if (w >= 0) {  // an empty response ends the requests
-            mbar_arrive_expect_tx(clc_full, 16);
-            clc_try_cancel(clc_resp, clc_full);
-            clc_pending = true;
-        }
+        if (clc.failed) return -1;
         const int sl = r & 3;
         if (!mbar_wait(&item_empty[sl], ((r >> 2) & 1u) ^ 1u, abort_flag, p.status, p.timeout_ns)) return -1;
         ring[sl] = w;
@@ -294,7 +315,8 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT>::kThreads, CPS)
                 const int qb = item_n & 1;
                 if (!mbar_wait(&q_empty[qb], ((item_n >> 1) & 1u) ^ 1u, abort_flag, p.status, p.timeout_ns)) break;
                 mbar_arrive_expect_tx(&q_full[qb], Cfg::kQBytes);
-                tma_load_4d(smem + Cfg::kOffQ + qb * Cfg::kQBytes, &tmQ, 0, t.h0, t.pos0, t.b, &q_full[qb]);
+                tma_load_4d(smem + Cfg::kOffQ + qb * Cfg::kQBytes, &tmQ, 0, t.h0, t.qrow0 + t.pos0, t.tb,
+                            &q_full[qb]);
                 ++q_issued[qb];
                 const int g = t.h0 / p.G;
                 for (int jt = 0; jt < t.n_tiles; ++jt, ++it) {
@@ -306,21 +328,21 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT>::kThreads, CPS)
                         break;
                     }
                     mbar_arrive_expect_tx(&k_full[st], Cfg::kKVBytes);
-                    tma_load_4d(smem + Cfg::kOffK + st * Cfg::kKVBytes, &tmK, 0, g, j0, t.b, &k_full[st]);
+                    tma_load_4d(smem + Cfg::kOffK + st * Cfg::kKVBytes, &tmK, 0, g, t.krow0 + j0, t.tb, &k_full[st]);
                     ++k_issued[st];
                     if (!mbar_wait(&v_empty[st], ph ^ 1u, abort_flag, p.status, p.timeout_ns)) {
                         ok = false;
                         break;
                     }
                     mbar_arrive_expect_tx(&v_full[st], Cfg::kKVBytes);
-                    tma_load_4d(smem + Cfg::kOffV + st * Cfg::kKVBytes, &tmV, 0, g, j0, t.b, &v_full[st]);
+                    tma_load_4d(smem + Cfg::kOffV + st * Cfg::kKVBytes, &tmV, 0, g, t.krow0 + j0, t.tb, &v_full[st]);
                     ++v_issued[st];
                 }
                 ++item_n;
             }
             // every load issued, and a launch-control request still in flight,
             // must land before the CTA may exit
-            if (clc_pending) wait_noabort(clc_full, clc_waits & 1u, p.status, p.timeout_ns);
+            clc.drain(p.status, p.timeout_ns);
             for (int s = 0; s < 2; ++s)
                 if (q_issued[s]) wait_noabort(&q_full[s], (q_issued[s] - 1) & 1u, p.status, p.timeout_ns);
             for (int s = 0; s < NS; ++s) {
@@ -423,7 +445,6 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT>::kThreads, CPS)
         const int r = quad * 32 + lane;
         const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
         const float C = p.c_log2;
-        const long off = (long)p.Lk - p.Lq;
         uint32_t it = 0, xc = 0;
         bool ok = true;
         // publish v, get the other half's value (bounded wait; false on abort)
@@ -441,14 +462,14 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT>::kThreads, CPS)
             const Item t = item_at<BN>(p, w);
             const int pos = t.pos0 + r / p.Gp;
             const int h = t.h0 + r % p.Gp;
-            const bool row_valid = pos < p.Lq;
-            const long pabs = pos + off;
+            const bool row_valid = pos < t.Lq;
+            const long pabs = pos + ((long)t.Lk - t.Lq);
             const float sink2 = p.sinks[h] * kLog2e;  // the sink logit in log2 units
             float m = sink2;                           // reference maximum, log2 units
             // running sum, seeded with the sink's mass (in column half 0 only)
             float l = (sink2 == -INFINITY || half != 0) ? 0.f : 1.f;
             // rows beyond Lq only need finite, unused values
-            const long vis_hi = row_valid ? min(pabs, (long)p.Lk - 1) : -1;   // last visible key
+            const long vis_hi = row_valid ? min(pabs, (long)t.Lk - 1) : -1;   // last visible key
             const long vis_lo = p.window > 0 ? pabs - p.window + 1 : 0;     // first visible key
 
             for (int jt = 0; jt < t.n_tiles; ++jt, ++it) {
@@ -476,66 +497,88 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT>::kThreads, CPS)
 #pragma unroll
                     for (int c = 0; c < kC; ++c) sv[c] = (c >= c_lo && c <= c_hi) ? sv[c] : -INFINITY;
                 }
-                // row max: eight independent chains of 3-input max over columns
-                // 0-7 | 8..kC-9 in steps of 16 | the last 8 (kC % 16 == 0)
                 static_assert(kC % 16 == 0, "whole 16-column chunks per thread");
+                const float2 C2 = make_float2(C, C);
+                float2 acc[2];
                 float mx[8];
 #pragma unroll
-                for (int k = 0; k < 8; ++k) mx[k] = sv[k];
-#pragma unroll
-                for (int c = 8; c + 16 <= kC; c += 16)
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) mx[k] = fmax3(mx[k], sv[c + k], sv[c + 8 + k]);
-#pragma unroll
-                for (int k = 0; k < 8; ++k) mx[k] = fmaxf(mx[k], sv[kC - 8 + k]);
-                float tmax = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
-                if (SPLIT == 2) {
-                    float other;
-                    if (!trade(tmax, other)) {
-                        ok = false;
-                        break;
-                    }
-                    tmax = fmaxf(tmax, other);
-                }
-                const float m_new = fmaxf(m, tmax * C);
-                const bool rescale = m_new > m + kRescaleThreshold;
-                const float alpha = rescale ? ((m == -INFINITY) ? 0.f : ex2(m - m_new)) : 1.f;
-                if (rescale) m = m_new;
-                const float neg_m = (m == -INFINITY) ? 0.f : -m;
-                const float2 C2 = make_float2(C, C), M2 = make_float2(neg_m, neg_m);
-                float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-                // P (bf16 pairs) overwrites the first kC/2 columns of this
-                // thread's part of the S buffer, read in full already; 16 scores
-                // per store.  On tiles with no masked element, pair EMU of every
-                // 4 runs on the FMA pipe (fast_exp2x2) to offload the MUFU unit
-                // (two separate loops, so each element takes one path only).
-                if (!need_mask) {
+                for (int k = 0; k < 8; ++k) mx[k] = -INFINITY;
+                // One pass over the tile: P = exp2(S C - m) against the reference
+                // maximum m, written as bf16 pairs over the first kC/2 columns of
+                // this thread's part of the S buffer (read in full already), 16
+                // scores per store; with kTrack, the tile's row maximum too, in
+                // eight independent chains of 3-input max.  On tiles with no
+                // masked element, pair EMU of every 4 runs on the FMA pipe
+                // (fast_exp2x2) to offload the MUFU unit.
+                auto exp_pass = [&](float neg_m_, auto track_tag, auto emu_tag) {
+                    constexpr bool kTrack = decltype(track_tag)::value;
+                    constexpr bool kEmu = decltype(emu_tag)::value;
+                    const float2 M2 = make_float2(neg_m_, neg_m_);
+                    acc[0] = acc[1] = make_float2(0.f, 0.f);
 #pragma unroll
                     for (int c = 0; c < kC / 16; ++c) {
                         uint32_t pk[8];
 #pragma unroll
                         for (int e = 0; e < 8; ++e) {
                             const float2 x = ffma2(make_float2(sv[16 * c + 2 * e], sv[16 * c + 2 * e + 1]), C2, M2);
-                            const bool emu = EMU == 4 ? (e & 1) != 0 : (e & 3) == EMU;
+                            const bool emu = kEmu && (EMU == 4 ? (e & 1) != 0 : (e & 3) == EMU);
                             const float2 pe = emu ? fast_exp2x2(x) : make_float2(ex2(x.x), ex2(x.y));
                             acc[e & 1] = fadd2(acc[e & 1], pe);
                             pk[e] = pack_bf16x2(pe.x, pe.y);
                         }
-                        tmem_st8(trow + scol + c * 8, pk);
-                    }
-                } else {
+                        if (kTrack) {
 #pragma unroll
-                    for (int c = 0; c < kC / 16; ++c) {
-                        uint32_t pk[8];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const float2 x = ffma2(make_float2(sv[16 * c + 2 * e], sv[16 * c + 2 * e + 1]), C2, M2);
-                            const float2 pe = make_float2(ex2(x.x), ex2(x.y));
-                            acc[e & 1] = fadd2(acc[e & 1], pe);
-                            pk[e] = pack_bf16x2(pe.x, pe.y);
+                            for (int k = 0; k < 8; ++k) mx[k] = fmax3(mx[k], sv[16 * c + k], sv[16 * c + 8 + k]);
                         }
                         tmem_st8(trow + scol + c * 8, pk);
                     }
+                };
+                bool rescale = false;
+                float alpha = 1.f;
+                if (FWD_SPEC && SPLIT == 1) {
+                    // The exponentials first, against the current reference (it
+                    // only moves when the true maximum exceeds it by 2^8, so it
+                    // rarely does), with the tile maximum found in the same pass;
+                    // a row whose maximum did move redoes the pass (S is still in
+                    // registers, P not yet handed to the MMA).
+                    const float neg_m0 = (m == -INFINITY) ? 0.f : -m;
+                    if (need_mask)
+                        exp_pass(neg_m0, std::true_type{}, std::false_type{});
+                    else
+                        exp_pass(neg_m0, std::true_type{}, std::true_type{});
+                    const float tmax =
+                        fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
+                    const float m_new = fmaxf(m, tmax * C);
+                    rescale = m_new > m + kRescaleThreshold;
+                    if (__any_sync(0xffffffffu, rescale)) {
+                        alpha = rescale ? ((m == -INFINITY) ? 0.f : ex2(m - m_new)) : 1.f;
+                        if (rescale) m = m_new;
+                        exp_pass((m == -INFINITY) ? 0.f : -m, std::false_type{}, std::false_type{});
+                    }
+                } else {
+                    // the tile's row maximum first, then the exponentials
+#pragma unroll
+                    for (int c = 0; c < kC; c += 16)
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) mx[k] = fmax3(mx[k], sv[c + k], sv[c + 8 + k]);
+                    float tmax = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
+                    if (SPLIT == 2) {
+                        float other;
+                        if (!trade(tmax, other)) {
+                            ok = false;
+                            break;
+                        }
+                        tmax = fmaxf(tmax, other);
+                    }
+                    const float m_new = fmaxf(m, tmax * C);
+                    rescale = m_new > m + kRescaleThreshold;
+                    alpha = rescale ? ((m == -INFINITY) ? 0.f : ex2(m - m_new)) : 1.f;
+                    if (rescale) m = m_new;
+                    const float neg_m = (m == -INFINITY) ? 0.f : -m;
+                    if (need_mask)
+                        exp_pass(neg_m, std::false_type{}, std::false_type{});
+                    else
+                        exp_pass(neg_m, std::false_type{}, std::true_type{});
                 }
                 l = l * alpha + ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y));
                 if (jt > 0) {
@@ -596,7 +639,7 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT>::kThreads, CPS)
             if (row_valid) {
                 const float inv = l > 0.f ? 1.f / l : 0.f;
                 uint4 *dst =
-                    reinterpret_cast<uint4 *>(p.out + (((size_t)t.b * p.Lq + pos) * p.Hq + h) * kD + half * kOC);
+                    reinterpret_cast<uint4 *>(p.out + ((size_t)(t.orow0 + pos) * p.Hq + h) * kD + half * kOC);
 #pragma unroll
                 for (int c = 0; c < kOC / 8; ++c) {
                     const uint32_t *src = &o[c / 4][(c % 4) * 8];
@@ -608,7 +651,8 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT>::kThreads, CPS)
                     dst[c] = v;
                 }
                 if (half == 0)
-                    p.lse[((size_t)t.b * p.Hq + h) * p.Lq + pos] = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
+                    p.lse[(size_t)(t.lrow0 + (long long)h * p.lse_hs + pos)] =
+                        l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
             }
         }
     }
@@ -634,6 +678,11 @@ cudaError_t launch_cfg(const void *q, const void *k, const void *v, const float 
     p.Hq = s.Hq;
     p.Hkv = s.Hkv;
     p.window = s.window;
+    p.cu_q = s.cu_q;
+    p.cu_k = s.cu_k;
+    p.total_q = s.total_q;
+    p.total_k = s.total_k;
+    p.lse_hs = s.cu_q ? s.total_q : s.Lq;
     p.G = s.Hq / s.Hkv;
     int gp = 1;
     while (gp * 2 <= 16 && p.G % (gp * 2) == 0) gp *= 2;
@@ -652,16 +701,20 @@ cudaError_t launch_cfg(const void *q, const void *k, const void *v, const float 
     p.timeout_ns = wait_timeout_ns();
 
     alignas(64) CUtensorMap mq, mk, mv;
+    // fixed-length batches: [B][L][H][D]; packed sequences: [1][total][H][D]
+    const uint64_t qrows = s.cu_q ? (uint64_t)s.total_q : (uint64_t)s.Lq;
+    const uint64_t krows = s.cu_q ? (uint64_t)s.total_k : (uint64_t)s.Lk;
+    const uint64_t outer = s.cu_q ? 1u : (uint64_t)s.B;
     {
-        const uint64_t dims[4] = {(uint64_t)kD, (uint64_t)s.Hq, (uint64_t)s.Lq, (uint64_t)s.B};
-        const uint64_t strides[3] = {(uint64_t)kD * 2, (uint64_t)s.Hq * kD * 2, (uint64_t)s.Lq * s.Hq * kD * 2};
+        const uint64_t dims[4] = {(uint64_t)kD, (uint64_t)s.Hq, qrows, outer};
+        const uint64_t strides[3] = {(uint64_t)kD * 2, (uint64_t)s.Hq * kD * 2, qrows * s.Hq * kD * 2};
         const uint32_t box[4] = {(uint32_t)kD, (uint32_t)p.Gp, (uint32_t)p.P, 1u};
         if (!encode_tensor_map_4d(&mq, const_cast<void *>(q), 2, dims, strides, box, true))
             return cudaErrorInvalidValue;
     }
     {
-        const uint64_t dims[4] = {(uint64_t)kD, (uint64_t)s.Hkv, (uint64_t)s.Lk, (uint64_t)s.B};
-        const uint64_t strides[3] = {(uint64_t)kD * 2, (uint64_t)s.Hkv * kD * 2, (uint64_t)s.Lk * s.Hkv * kD * 2};
+        const uint64_t dims[4] = {(uint64_t)kD, (uint64_t)s.Hkv, krows, outer};
+        const uint64_t strides[3] = {(uint64_t)kD * 2, (uint64_t)s.Hkv * kD * 2, krows * s.Hkv * kD * 2};
         const uint32_t box[4] = {(uint32_t)kD, 1u, (uint32_t)BN, 1u};
         if (!encode_tensor_map_4d(&mk, const_cast<void *>(k), 2, dims, strides, box, true))
             return cudaErrorInvalidValue;

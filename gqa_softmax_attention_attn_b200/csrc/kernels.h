@@ -14,6 +14,11 @@ enum : unsigned { STATUS_TIMEOUT = 1u };
 struct AttnShape {
     int B, Lq, Lk, Hq, Hkv, D, window;
     float scale;
+    // packed ragged sequences (varlen): cu_q / cu_k [B + 1] device offsets into
+    // q [total_q, Hq, D] and k, v [total_k, Hkv, D]; Lq is then the longest
+    // sequence's query count (an upper bound).  nullptr: fixed-length batch.
+    const int *cu_q = nullptr, *cu_k = nullptr;
+    int total_q = 0, total_k = 0;
 };
 
 struct DecodeShape {
@@ -34,6 +39,22 @@ __host__ __device__ inline void decode_range(const DecodeShape &s, int len, int 
     lo = s.window > 0 ? (len - s.window > 0 ? len - s.window : 0) : 0;
     lo_al = s.align > 0 ? lo / s.align * s.align : lo;
     nsplit = (len - lo_al + s.chunk - 1) / s.chunk;
+}
+
+// Sequence b of a prefill batch: fixed-length sequences (cu == nullptr:
+// length fixed_len, its own batch slot) or packed ragged sequences whose rows
+// are [cu[b], cu[b + 1]) of one [total, H, D] tensor.  Offsets are clamped
+// into [0, total], so any cu array yields in-bounds rows.
+struct SeqRows {
+    int len;   // rows of the sequence
+    int row0;  // its first row in the packed tensor (0 for fixed-length batches)
+};
+__device__ __forceinline__ SeqRows seq_rows(const int *cu, int b, int fixed_len, int total)
+{
+    if (cu == nullptr) return {fixed_len, 0};
+    const int a = min(max(cu[b], 0), total);
+    const int e = min(max(cu[b + 1], a), total);
+    return {e - a, a};
 }
 
 // Per-device status word (bit STATUS_TIMEOUT set by an expired bounded wait).

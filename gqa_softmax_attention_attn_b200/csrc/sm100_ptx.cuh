@@ -149,6 +149,62 @@ __device__ __forceinline__ int clc_cancelled_ctaid_x(const void *resp_smem)
     return ok ? (int)x : -1;
 }
 
+// Launch-control requests a persistent CTA keeps in flight (so the round trip
+// to the hardware scheduler overlaps the items already claimed).
+#ifndef ATTN_SINK_CLC_DEPTH
+#define ATTN_SINK_CLC_DEPTH 2
+#endif
+constexpr int kClcDepth = ATTN_SINK_CLC_DEPTH;
+
+// Up to DEPTH launch-control requests in flight, answered in the order they
+// were issued; used by one thread (the producer).  bar: DEPTH mbarriers
+// initialised with count 1; resp: DEPTH 16-byte response slots.
+template <int DEPTH>
+struct ClcQueue {
+    uint64_t *bar;
+    uint8_t *resp;
+    uint32_t issued = 0, consumed = 0;
+    bool stop = false;    // an empty response came back (or a wait gave up): issue no more
+    bool failed = false;  // a wait for a response gave up
+
+    __device__ __forceinline__ void fill()
+    {
+        while (!stop && issued - consumed < (uint32_t)DEPTH) {
+            const int s = issued % DEPTH;
+            mbar_arrive_expect_tx(&bar[s], 16);
+            clc_try_cancel(resp + 16 * s, &bar[s]);
+            ++issued;
+        }
+    }
+    // blockIdx.x of the next CTA taken over, or -1 once every response in
+    // flight came back empty (or a wait gave up).  Responses are read in issue
+    // order; an empty one stops further requests, and the ones already in
+    // flight are still read, so no CTA that was taken over is ever dropped.
+    __device__ __forceinline__ int next(volatile int *abort, unsigned *status, long long timeout_ns)
+    {
+        while (consumed != issued) {
+            const int s = consumed % DEPTH;
+            if (!mbar_wait(&bar[s], (consumed / DEPTH) & 1u, abort, status, timeout_ns)) {
+                failed = stop = true;
+                return -1;
+            }
+            ++consumed;
+            const int x = clc_cancelled_ctaid_x(resp + 16 * s);
+            if (x >= 0) return x;
+            stop = true;
+        }
+        return -1;
+    }
+    // exit path: every response still in flight lands before the CTA may exit
+    __device__ __forceinline__ void drain(unsigned *status, long long timeout_ns)
+    {
+        int never = 0;
+        const long long tmo = timeout_ns > 1000000000LL ? timeout_ns : 1000000000LL;
+        for (; consumed != issued; ++consumed)
+            mbar_wait(&bar[consumed % DEPTH], (consumed / DEPTH) & 1u, &never, status, tmo);
+    }
+};
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map)
 {

@@ -437,12 +437,13 @@ def leg_entry(ms, flops, nbytes, bound, shape):
     return e
 
 
-def prefill_legs(dev, which=("bwd", "train", "long"), reps=5, warmup=2):
+def prefill_legs(dev, which=("bwd", "train", "varlen", "long"), reps=5, warmup=2):
     """Forward / backward legs beyond the headline step, each with its own roofline
     fraction (dense layers against the tensor peak, window-128 layers against HBM),
     L2 flushed before every timed run:
       bwd:   the backward at the prefill shape (B1 L4096 Hq64 Hkv8);
       train: forward and backward at the training shape (B8 L8192 Hq64 Hkv8);
+      varlen: a prefill batch of 12 packed sequences of mixed lengths;
       long:  the long-context layers (window 128 at L = 131072, dense at L = 32768)."""
     import gqa_softmax_attention_attn_b200 as attn
 
@@ -481,6 +482,27 @@ def prefill_legs(dev, which=("bwd", "train", "long"), reps=5, warmup=2):
         run_shape("", B, L, 1.0, 2002, (0, WIN), True, False)
     if "train" in which:
         run_shape("train_", 8, 8192, 1.0, 2003, (0, WIN), True, True)
+    if "varlen" in which:
+        # a prefill batch of mixed lengths packed back to back (seeded lengths in [256, 4096])
+        import numpy as np
+
+        lens = [int(x) for x in np.random.default_rng(1002).integers(256, 4097, 12)]
+        tot = sum(lens)
+        t = device_prefill(1, tot, HQ, HKV, 1.0, 2007, dev, False)
+        q, k, v = t["q"][0], t["k"][0], t["v"][0]
+        out = torch.empty_like(q)
+        lse = torch.empty(HQ, tot, device=dev, dtype=torch.float32)
+        cu = torch.tensor([0] + list(np.cumsum(lens)), dtype=torch.int32, device=dev)
+        shape = f"varlen {len(lens)} seqs, {tot} tokens Hq{HQ} Hkv{HKV} D{D}"
+        for window in (0, WIN):
+            fn = lambda: attn.attn_sink_fwd_varlen(q, k, v, t["sinks"], out, lse, cu, cu, max(lens), window, SCALE,
+                                                   stream)
+            ms = timed(dev, fn, reps, warmup, flush)
+            fl = sum(fwd_flops(1, n, HQ, window) for n in lens)
+            tag = "dense" if window <= 0 else "window128"
+            legs[f"varlen_fwd_{tag}"] = leg_entry(ms, fl, fwd_bytes(1, tot, HQ, HKV), "tensor" if window <= 0 else "hbm",
+                                                  shape)
+        assert attn.attn_sink_get_device_status(stream) == 0
     if "long" in which:
         run_shape("long_", 1, 131072, 2.0, 2005, (WIN,), False, True)
         run_shape("long_", 1, 32768, 2.0, 2006, (0,), False, True)
@@ -580,7 +602,7 @@ def main():
     ap.add_argument("--no-legs", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["decode", "bwd", "train", "long"], default=None,
+    ap.add_argument("--only", choices=["decode", "bwd", "train", "varlen", "long"], default=None,
                     help="run just one leg (reps = --steps, warm-up = --warmup); used for profiling")
     ap.add_argument("--decode-batch", type=int, default=None, help="sequences in the decode leg (default 64)")
     args = ap.parse_args()

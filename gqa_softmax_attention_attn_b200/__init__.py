@@ -19,6 +19,7 @@ from ._native import (  # noqa: F401
     attn_sink_decode_paged_workspace_size,
     attn_sink_decode_workspace_size,
     attn_sink_fwd,
+    attn_sink_fwd_varlen,
     attn_sink_get_device_status,
     attn_sink_set_wait_timeout_ns,
     attn_sink_version,

@@ -59,6 +59,8 @@ def load():
         P, I, F, Z, LL = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.c_longlong
         lib.attn_sink_fwd.argtypes = [P] * 6 + [I] * 7 + [F, I, P]
         lib.attn_sink_fwd.restype = I
+        lib.attn_sink_fwd_varlen.argtypes = [P] * 8 + [I] * 8 + [F, P]
+        lib.attn_sink_fwd_varlen.restype = I
         lib.attn_sink_decode.argtypes = [P] * 7 + [I] * 6 + [F, I, P, Z, I, P]
         lib.attn_sink_decode.restype = I
         lib.attn_sink_decode_noalloc.argtypes = [P] * 7 + [I] * 6 + [F, I, I, P]
@@ -133,6 +135,24 @@ def attn_sink_fwd(q, k, v, sinks, out, lse, window: int, scale: float, stream=No
                               _dev(out, "out", dt), _dev(lse, "lse", torch.float32), B, Lq, Lk, Hq, Hkv, D,
                               int(window), float(scale), _dtype_code(q), _stream(stream))
     _check(rc, "attn_sink_fwd")
+
+
+def attn_sink_fwd_varlen(q, k, v, sinks, out, lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, window: int,
+                         scale: float, stream=None):
+    """Packed ragged sequences: q [total_q,Hq,D], k/v [total_k,Hkv,D] bf16, cu_seqlens_q/k [B+1] int32
+    -> writes out [total_q,Hq,D], lse [Hq,total_q]."""
+    total_q, Hq, D = q.shape
+    total_k, Hkv = k.shape[0], k.shape[1]
+    B = cu_seqlens_q.shape[0] - 1
+    if cu_seqlens_k.shape[0] != B + 1:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must both hold B + 1 offsets")
+    rc = load().attn_sink_fwd_varlen(_dev(q, "q", torch.bfloat16), _dev(k, "k", torch.bfloat16),
+                                     _dev(v, "v", torch.bfloat16), _dev(sinks, "sinks", torch.float32),
+                                     _dev(out, "out", torch.bfloat16), _dev(lse, "lse", torch.float32),
+                                     _dev(cu_seqlens_q, "cu_seqlens_q", torch.int32),
+                                     _dev(cu_seqlens_k, "cu_seqlens_k", torch.int32), B, int(max_seqlen_q), total_q,
+                                     total_k, Hq, Hkv, D, int(window), float(scale), _stream(stream))
+    _check(rc, "attn_sink_fwd_varlen")
 
 
 def attn_sink_decode_workspace_size(B: int, Hq: int, D: int, Lmax: int, window: int, num_splits: int) -> int:

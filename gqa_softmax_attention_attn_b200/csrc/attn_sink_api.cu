@@ -272,6 +272,29 @@ int attn_sink_fwd(const void *q, const void *k, const void *v, const float *sink
     return launch_status(launch_fwd_tc(q, k, v, sinks, out, lse, s, st));
 }
 
+int attn_sink_fwd_varlen(const void *q, const void *k, const void *v, const float *sinks, void *out, float *lse,
+                         const int *cu_seqlens_q, const int *cu_seqlens_k, int B, int max_seqlen_q, int total_q,
+                         int total_k, int Hq, int Hkv, int D, int window, float scale, void *stream)
+{
+    if (!q || !k || !v || !sinks || !out || !lse || !cu_seqlens_q || !cu_seqlens_k) return ATTN_SINK_ERR_INVALID_ARG;
+    int rc = check_common(B, max_seqlen_q, 1, Hq, Hkv, D, ATTN_SINK_DTYPE_BF16);
+    if (rc != ATTN_SINK_OK) return rc;
+    if (total_q <= 0 || total_k <= 0) return ATTN_SINK_ERR_INVALID_ARG;
+    if (!(scale > 0.f && scale < INFINITY)) return ATTN_SINK_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse) || !aligned16(sinks) ||
+        !aligned16(cu_seqlens_q) || !aligned16(cu_seqlens_k))
+        return ATTN_SINK_ERR_MISALIGNED;
+    rc = ensure_device();
+    if (rc != ATTN_SINK_OK) return rc;
+    AttnShape s{B, max_seqlen_q, max_seqlen_q, Hq, Hkv, D, window, scale};
+    s.cu_q = cu_seqlens_q;
+    s.cu_k = cu_seqlens_k;
+    s.total_q = total_q;
+    s.total_k = total_k;
+    if (!fwd_tc_supported(s)) return ATTN_SINK_ERR_UNSUPPORTED;
+    return launch_status(launch_fwd_tc(q, k, v, sinks, out, lse, s, static_cast<cudaStream_t>(stream)));
+}
+
 size_t attn_sink_decode_workspace_size(int B, int Hq, int D, int Lmax, int window, int num_splits)
 {
     if (B <= 0 || Hq <= 0 || D <= 0 || Lmax <= 0 || num_splits < 0 || num_splits > 32) return 0;

@@ -42,7 +42,11 @@ namespace {
 
 constexpr int kD = 64;
 constexpr int kT = 64;          // keys per tile
-constexpr int kNS = 4;          // ring stages
+// K/V ring stages: the loads in flight per SM must cover the HBM latency at
+// full bandwidth, so the e4m3 ring (half the bytes per stage) is deeper
+#ifndef ATTN_SINK_DEC_FP8_STAGES
+#define ATTN_SINK_DEC_FP8_STAGES 8
+#endif
 constexpr int kThreads = 160;  // warp 0 producer, warps 1-4 consumers
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -50,6 +54,7 @@ constexpr float kLn2 = 0.6931471805599453f;
 // Shared-memory layout; kFp8: K/V cached as e4m3 (one byte per element).
 template <bool kFp8>
 struct DecLayout {
+    static constexpr int kNS = kFp8 ? ATTN_SINK_DEC_FP8_STAGES : 4;
     static constexpr int kRowBytes = kFp8 ? kD : kD * 2;  // one cached K or V row
     static constexpr int kTileBytes = kT * kRowBytes;
     static constexpr int kStageBytes = 2 * kTileBytes;  // K and V
@@ -131,6 +136,7 @@ __global__ void __launch_bounds__(kThreads)
     using L = DecLayout<kFp8>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    constexpr int kNS = L::kNS;
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::kOffBar);
     uint64_t *empty = full + kNS;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kOffBar + 2 * kNS * 8);
@@ -166,7 +172,9 @@ __global__ void __launch_bounds__(kThreads)
         if (lane == 0) {
             tma_prefetch_desc(&tmK);
             tma_prefetch_desc(&tmV);
-            uint32_t issued[kNS] = {0, 0, 0, 0};
+            uint32_t issued[kNS];
+#pragma unroll
+            for (int s = 0; s < kNS; ++s) issued[s] = 0;
             for (int j = 0; j < n_tiles; ++j) {
                 const int st = j % kNS;
                 if (!mbar_wait(&empty[st], ((j / kNS) & 1u) ^ 1u, abort_flag, p.status, p.timeout_ns)) break;

@@ -101,6 +101,11 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 #define ATTN_SINK_FWD_SPEC 1
 #endif
 constexpr bool FWD_SPEC = ATTN_SINK_FWD_SPEC != 0;
+// launch-control requests in flight: dense items are long, so one hides the
+// round trip (measured on the gpt-oss-20b prefill's dense layer: 205.6 us at
+// one, 206.8 at two, 230.5 at four, where CTAs hold on to items others could
+// have taken)
+constexpr int kClcDepthDense = 1;
 constexpr int pow2_at_least(int x) { return x <= 32 ? 32 : x <= 64 ? 64 : x <= 128 ? 128 : x <= 256 ? 256 : 512; }
 
 template <int BN, int NS, int CPS, int SPLIT>
@@ -116,11 +121,11 @@ struct FwdCfg {
     static constexpr int kOffV = kOffK + NS * kKVBytes;
     static constexpr int kOffBar = kOffV + NS * kKVBytes;
     // q_full[2], q_empty[2], k_full[NS], k_empty[NS], v_full[NS], v_empty[NS],
-    // s_full[2], p_full[2], o_done, o_free, drain, xchg[4], item_full[4], item_empty[4], clc[kClcDepth]
-    static constexpr int kNumBar = 4 + 4 * NS + 4 + 3 + 4 + 8 + kClcDepth;
+    // s_full[2], p_full[2], o_done, o_free, drain, xchg[4], item_full[4], item_empty[4], clc[kClcDepthDense]
+    static constexpr int kNumBar = 4 + 4 * NS + 4 + 3 + 4 + 8 + kClcDepthDense;
     // tmem slot (+0), abort flag (+4), item ring (+16, 4 ints), launch-control responses (+32, 16 bytes each)
     static constexpr int kOffMisc = (kOffBar + kNumBar * 8 + 15) / 16 * 16;
-    static_assert(32 + 16 * kClcDepth <= 128, "misc area");
+    static_assert(32 + 16 * kClcDepthDense <= 128, "misc area");
     // row partials exchanged by the two softmax warps of a row: [2 slots][2 halves][128 rows]
     static constexpr int kOffXchg = kOffMisc + 128;
     static constexpr int kTmemCols = pow2_at_least(2 * BN + kD);
@@ -225,7 +230,7 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT>::kThreads, CPS)
     // them to the MMA warp and the softmax warps through 4 slots
     uint64_t *item_full = xchg + 4;        // [4]
     uint64_t *item_empty = item_full + 4;  // [4]
-    uint64_t *clc_bar = item_empty + 4;    // [kClcDepth]: launch-control responses landed
+    uint64_t *clc_bar = item_empty + 4;    // [kClcDepthDense]: launch-control responses landed
     volatile int *ring = reinterpret_cast<volatile int *>(smem + Cfg::kOffMisc + 16);
     void *clc_resp = smem + Cfg::kOffMisc + 32;
     float *xs = reinterpret_cast<float *>(smem + Cfg::kOffXchg);
@@ -255,7 +260,7 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT>::kThreads, CPS)
             mbar_init(&item_full[r], 1);
             mbar_init(&item_empty[r], 1 + 4 * SPLIT);  // the MMA warp and each softmax warp
         }
-        for (int d = 0; d < kClcDepth; ++d) mbar_init(&clc_bar[d], 1);
+        for (int d = 0; d < kClcDepthDense; ++d) mbar_init(&clc_bar[d], 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -274,10 +279,10 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT>::kThreads, CPS)
     // the item) and publishes it in the ring; every other warp reads it there
     // (-1: no more).  Items past the end of a shorter packed sequence are
     // passed over here, so the other warps never see them.
-    ClcQueue<kClcDepth> clc{clc_bar, reinterpret_cast<uint8_t *>(clc_resp)};
+    ClcQueue<kClcDepthDense> clc{clc_bar, reinterpret_cast<uint8_t *>(clc_resp)};
     auto producer_item = [&](int r) -> int {
         int w = r == 0 ? (int)blockIdx.x : clc.next(abort_flag, p.status, p.timeout_ns);
-        clc.fill();  // keep kClcDepth requests in flight
+        clc.fill();  // keep kClcDepthDense requests in flight
         while (w >= 0 && item_at<BN>(p, w).empty) {
             w = clc.next(abort_flag, p.status, p.timeout_ns);
             clc.fill();

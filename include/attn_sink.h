@@ -99,6 +99,33 @@ ATTN_SINK_API int attn_sink_fwd(const void *q, const void *k, const void *v, con
                   int window, float scale, int dtype, void *stream);
 
 /*
+ * Prefill forward over packed ragged sequences ("varlen"): a batch of B
+ * sequences of different lengths stored back to back, as a prefill server
+ * that gathers requests of any length receives them (the pages separate the
+ * prefill of requests from their decode -- "GPT-OSS on day 0", section "Cost
+ * i rendiment" -- and measure prefill over batches of mixed sizes).  Each
+ * sequence is an independent problem with the operation of attn_sink_fwd.
+ *   q, out [total_q, Hq, D] bf16     k, v [total_k, Hkv, D] bf16
+ *   cu_seqlens_q, cu_seqlens_k [B + 1] int32, device: sequence b owns query
+ *           rows [cu_seqlens_q[b], cu_seqlens_q[b+1]) and key rows
+ *           [cu_seqlens_k[b], cu_seqlens_k[b+1]); its query i sits at
+ *           position i + (Lk_b - Lq_b) (bottom-right causal alignment, so a
+ *           sequence with a cached prefix has Lk_b > Lq_b).  Offsets must be
+ *           non-decreasing from 0; they are clamped into [0, total] on the
+ *           device, so no bad offset reads or writes out of bounds.
+ *   max_seqlen_q  host-side upper bound on every Lq_b (rows past it are not
+ *           computed).  A sequence may be empty.
+ *   lse     [Hq, total_q] fp32 (natural log, sink included).
+ *   sinks, window, scale: as attn_sink_fwd (scale positive and finite).
+ * bf16 only.  Errors: INVALID_ARG for null pointers or non-positive sizes,
+ * otherwise as attn_sink_fwd.  Nothing is allocated; asynchronous on stream.
+ */
+ATTN_SINK_API int attn_sink_fwd_varlen(const void *q, const void *k, const void *v, const float *sinks,
+                  void *out, float *lse, const int *cu_seqlens_q, const int *cu_seqlens_k,
+                  int B, int max_seqlen_q, int total_q, int total_k, int Hq, int Hkv, int D,
+                  int window, float scale, void *stream);
+
+/*
  * Split-KV decode over a contiguous per-sequence KV cache with ragged
  * lengths ("GPT-OSS on day 0", section "Sink Attention": attention is split
  * along the KV length as well as across heads, and the sink must be counted

@@ -193,3 +193,24 @@ def decode_fp8(q, k_codes, v_codes, k_scale, v_scale, seqlens, sinks, window: in
     k = e4m3_values(k_codes) * ks[None, None, :, None]
     v = e4m3_values(v_codes) * vs[None, None, :, None]
     return decode(q, k, v, seqlens, sinks, window, scale)
+
+
+def fwd_varlen(q, k, v, sinks, cu_q, cu_k, window: int, scale: float):
+    """Packed ragged sequences: sequence b is the independent problem
+    q[cu_q[b]:cu_q[b+1]] against k, v[cu_k[b]:cu_k[b+1]], run through fwd with
+    B = 1.  q [total_q, Hq, D], k/v [total_k, Hkv, D] -> (out [total_q, Hq, D],
+    lse [Hq, total_q]); empty sequences contribute nothing."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    cq = [int(x) for x in (cu_q.tolist() if hasattr(cu_q, "tolist") else cu_q)]
+    ck = [int(x) for x in (cu_k.tolist() if hasattr(cu_k, "tolist") else cu_k)]
+    total_q, Hq, D = q.shape
+    out = np.zeros((total_q, Hq, D))
+    lse = np.zeros((Hq, total_q))
+    for b in range(len(cq) - 1):
+        a, e = cq[b], cq[b + 1]
+        if e <= a:
+            continue
+        o, l = fwd(q[None, a:e], k[None, ck[b]:ck[b + 1]], v[None, ck[b]:ck[b + 1]], sinks, window, scale)
+        out[a:e] = o[0]
+        lse[:, a:e] = l[0]
+    return out, lse

@@ -76,6 +76,26 @@ def test_decode_host_checks():
     assert attn.attn_sink_decode_workspace_size(4, 8, 64, 4096, 128, 0) == 0
 
 
+def test_fwd_varlen_host_checks():
+    lib = attn.load()
+    q, k, v, s, o, l, cq, ck = _fake(8)
+
+    def call(cu_q=cq, cu_k=ck, B=3, max_q=100, total_q=200, total_k=200, Hq=8, Hkv=2, D=64, scale=0.125):
+        return lib.attn_sink_fwd_varlen(q, k, v, s, o, l, cu_q, cu_k, B, max_q, total_q, total_k, Hq, Hkv, D, 0,
+                                        scale, None)
+
+    assert call(cu_q=None) == INVALID
+    assert call(cu_k=None) == INVALID
+    assert call(B=0) == INVALID
+    assert call(max_q=0) == INVALID
+    assert call(total_q=0) == INVALID
+    assert call(total_k=0) == INVALID
+    assert call(Hkv=3) == INVALID
+    assert call(D=128) == UNSUPPORTED
+    assert call(scale=0.0) == UNSUPPORTED
+    assert call(cu_q=cq + 4) == MISALIGNED
+
+
 def test_decode_fp8_host_checks():
     lib = attn.load()
     q, kc, vc, ks, vs, sl, s, o = _fake(8)

@@ -352,3 +352,24 @@ def test_decode_fp8_is_decode_of_the_scaled_codes():
         o2, l2 = oracle.decode_fp8(d["q"], k8, v8, ks * 2, vs * 4, d["seqlens"], d["sinks"], window, 0.125)
         np.testing.assert_allclose(o2, 4 * o, rtol=1e-12, atol=1e-14)
         np.testing.assert_allclose(l2, l, rtol=0, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------- packed ragged sequences
+def test_fwd_varlen_is_the_batch_when_lengths_agree_and_skips_empty_sequences():
+    """fwd_varlen over B equal-length sequences packed back to back equals fwd
+    on the [B, L] batch (out row for row; lse [Hq, total] = the batch's
+    [B, Hq, L] laid head-major), and an empty sequence between them changes
+    nothing for the others."""
+    B, L, Hq, Hkv = 3, 37, 8, 2
+    t = prefill_inputs(B, L, L, Hq, Hkv, 16, torch.float32, 0.5, 1.0, seed=91)
+    for window in (0, 5):
+        ro, rl = oracle.fwd(t["q"], t["k"], t["v"], t["sinks"], window, 0.25)
+        cu = [0, L, 2 * L, 3 * L]
+        o, l = oracle.fwd_varlen(t["q"].reshape(B * L, Hq, 16), t["k"].reshape(B * L, Hkv, 16),
+                                 t["v"].reshape(B * L, Hkv, 16), t["sinks"], cu, cu, window, 0.25)
+        assert np.array_equal(o, ro.reshape(B * L, Hq, 16))
+        assert np.array_equal(l, np.concatenate(list(rl), axis=1))
+        cu_e = [0, L, L, 2 * L, 3 * L]  # sequence 1 is empty
+        o2, l2 = oracle.fwd_varlen(t["q"].reshape(B * L, Hq, 16), t["k"].reshape(B * L, Hkv, 16),
+                                   t["v"].reshape(B * L, Hkv, 16), t["sinks"], cu_e, cu_e, window, 0.25)
+        assert np.array_equal(o2, o) and np.array_equal(l2, l)

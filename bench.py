@@ -437,13 +437,14 @@ def leg_entry(ms, flops, nbytes, bound, shape):
     return e
 
 
-def prefill_legs(dev, which=("bwd", "train", "varlen", "long"), reps=5, warmup=2):
+def prefill_legs(dev, which=("bwd", "train", "varlen", "prologue", "long"), reps=5, warmup=2):
     """Forward / backward legs beyond the headline step, each with its own roofline
     fraction (dense layers against the tensor peak, window-128 layers against HBM),
     L2 flushed before every timed run:
       bwd:   the backward at the prefill shape (B1 L4096 Hq64 Hkv8);
       train: forward and backward at the training shape (B8 L8192 Hq64 Hkv8);
       varlen: a prefill batch of 12 packed sequences of mixed lengths;
+      prologue: bias + YaRN rotary embedding + split of the prefill's QKV rows;
       long:  the long-context layers (window 128 at L = 131072, dense at L = 32768)."""
     import gqa_softmax_attention_attn_b200 as attn
 
@@ -502,6 +503,22 @@ def prefill_legs(dev, which=("bwd", "train", "varlen", "long"), reps=5, warmup=2
             tag = "dense" if window <= 0 else "window128"
             legs[f"varlen_fwd_{tag}"] = leg_entry(ms, fl, fwd_bytes(1, tot, HQ, HKV), "tensor" if window <= 0 else "hbm",
                                                   shape)
+        assert attn.attn_sink_get_device_status(stream) == 0
+    if "prologue" in which:
+        # bias + YaRN rotary embedding + split of the prefill's QKV rows (B1 L4096 Hq64 Hkv8)
+        width = (HQ + 2 * HKV) * D
+        g = torch.Generator(device=dev).manual_seed(2008)
+        qkv = (torch.randn(L, width, device=dev, generator=g) * 0.5).to(torch.bfloat16)
+        bias = torch.randn(width, device=dev, generator=g) * 0.1
+        pos = torch.arange(L, device=dev, dtype=torch.int32)
+        qo = torch.empty(L, HQ, D, dtype=torch.bfloat16, device=dev)
+        ko = torch.empty(L, HKV, D, dtype=torch.bfloat16, device=dev)
+        vo = torch.empty_like(ko)
+        fn = lambda: attn.attn_sink_qkv_prologue(qkv, bias, pos, qo, ko, vo, 150000.0, 32.0, 4096, 32.0, 1.0,
+                                                 stream=stream)
+        ms = timed(dev, fn, reps, warmup, flush)
+        nbytes = 2 * L * width * 2 + 4 * width + 4 * L
+        legs["prologue_qkv"] = leg_entry(ms, 0.0, nbytes, "hbm", f"T{L} Hq{HQ} Hkv{HKV} D{D}, YaRN factor 32")
         assert attn.attn_sink_get_device_status(stream) == 0
     if "long" in which:
         run_shape("long_", 1, 131072, 2.0, 2005, (WIN,), False, True)
@@ -602,7 +619,7 @@ def main():
     ap.add_argument("--no-legs", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["decode", "bwd", "train", "varlen", "long"], default=None,
+    ap.add_argument("--only", choices=["decode", "bwd", "train", "varlen", "prologue", "long"], default=None,
                     help="run just one leg (reps = --steps, warm-up = --warmup); used for profiling")
     ap.add_argument("--decode-batch", type=int, default=None, help="sequences in the decode leg (default 64)")
     args = ap.parse_args()

@@ -21,6 +21,7 @@ from ._native import (  # noqa: F401
     attn_sink_fwd,
     attn_sink_fwd_varlen,
     attn_sink_get_device_status,
+    attn_sink_qkv_prologue,
     attn_sink_set_wait_timeout_ns,
     attn_sink_version,
     load,

@@ -59,6 +59,8 @@ def load():
         P, I, F, Z, LL = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.c_longlong
         lib.attn_sink_fwd.argtypes = [P] * 6 + [I] * 7 + [F, I, P]
         lib.attn_sink_fwd.restype = I
+        lib.attn_sink_qkv_prologue.argtypes = [P] * 7 + [I] * 5 + [F, F, I, F, F, I, P]
+        lib.attn_sink_qkv_prologue.restype = I
         lib.attn_sink_fwd_varlen.argtypes = [P] * 8 + [I] * 8 + [F, P]
         lib.attn_sink_fwd_varlen.restype = I
         lib.attn_sink_decode.argtypes = [P] * 7 + [I] * 6 + [F, I, P, Z, I, P]
@@ -135,6 +137,26 @@ def attn_sink_fwd(q, k, v, sinks, out, lse, window: int, scale: float, stream=No
                               _dev(out, "out", dt), _dev(lse, "lse", torch.float32), B, Lq, Lk, Hq, Hkv, D,
                               int(window), float(scale), _dtype_code(q), _stream(stream))
     _check(rc, "attn_sink_fwd")
+
+
+def attn_sink_qkv_prologue(qkv, bias, positions, q_out, k_out, v_out, rope_theta: float, rope_factor: float = 1.0,
+                           rope_original_max_pos: int = 0, beta_fast: float = 32.0, beta_slow: float = 1.0,
+                           interleaved: bool = False, kv_rows=None, stream=None):
+    """qkv [T,(Hq+2Hkv)*D] bf16, bias [(Hq+2Hkv)*D] fp32 or None, positions [T] int32 -> writes
+    q_out [T,Hq,D], k_out/v_out [rows,Hkv,D] (row kv_rows[t], or t) with bias and YaRN rotary embedding."""
+    T, Hq, D = q_out.shape
+    rows, Hkv = k_out.shape[0], k_out.shape[1]
+    if qkv.shape != (T, (Hq + 2 * Hkv) * D):
+        raise ValueError(f"qkv must be [{T}, {(Hq + 2 * Hkv) * D}]")
+    rc = load().attn_sink_qkv_prologue(_dev(qkv, "qkv", torch.bfloat16),
+                                       _dev(bias, "bias", torch.float32) if bias is not None else None,
+                                       _dev(positions, "positions", torch.int32),
+                                       _dev(kv_rows, "kv_rows", torch.int32) if kv_rows is not None else None,
+                                       _dev(q_out, "q_out", torch.bfloat16), _dev(k_out, "k_out", torch.bfloat16),
+                                       _dev(v_out, "v_out", torch.bfloat16), T, Hq, Hkv, D, rows, float(rope_theta),
+                                       float(rope_factor), int(rope_original_max_pos), float(beta_fast),
+                                       float(beta_slow), int(bool(interleaved)), _stream(stream))
+    _check(rc, "attn_sink_qkv_prologue")
 
 
 def attn_sink_fwd_varlen(q, k, v, sinks, out, lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, window: int,

@@ -295,6 +295,31 @@ int attn_sink_fwd_varlen(const void *q, const void *k, const void *v, const floa
     return launch_status(launch_fwd_tc(q, k, v, sinks, out, lse, s, static_cast<cudaStream_t>(stream)));
 }
 
+int attn_sink_qkv_prologue(const void *qkv, const float *bias, const int *positions, const int *kv_rows, void *q_out,
+                           void *k_out, void *v_out, int T, int Hq, int Hkv, int D, int kv_rows_total,
+                           float rope_theta, float rope_factor, int rope_original_max_pos, float beta_fast,
+                           float beta_slow, int interleaved, void *stream)
+{
+    if (!qkv || !positions || !q_out || !k_out || !v_out) return ATTN_SINK_ERR_INVALID_ARG;
+    if (T <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || kv_rows_total <= 0 || Hq % Hkv != 0)
+        return ATTN_SINK_ERR_INVALID_ARG;
+    if (D != 64) return ATTN_SINK_ERR_UNSUPPORTED;
+    if (!kv_rows && kv_rows_total < T) return ATTN_SINK_ERR_INVALID_ARG;
+    if (!(rope_theta > 1.f && rope_theta < INFINITY) || !(rope_factor > 0.f && rope_factor < INFINITY))
+        return ATTN_SINK_ERR_INVALID_ARG;
+    if (rope_factor > 1.f && (rope_original_max_pos <= 0 || !(beta_fast > beta_slow) || !(beta_slow > 0.f)))
+        return ATTN_SINK_ERR_INVALID_ARG;
+    if (interleaved != 0 && interleaved != 1) return ATTN_SINK_ERR_INVALID_ARG;
+    if (!aligned16(qkv) || !aligned16(positions) || !aligned16(q_out) || !aligned16(k_out) || !aligned16(v_out) ||
+        (bias && !aligned16(bias)) || (kv_rows && !aligned16(kv_rows)))
+        return ATTN_SINK_ERR_MISALIGNED;
+    int rc = ensure_device();
+    if (rc != ATTN_SINK_OK) return rc;
+    const RopeParams r{rope_theta, rope_factor, (double)rope_original_max_pos, beta_fast, beta_slow, interleaved};
+    return launch_status(launch_qkv_prologue(qkv, bias, positions, kv_rows, q_out, k_out, v_out, T, Hq, Hkv,
+                                             kv_rows_total, r, static_cast<cudaStream_t>(stream)));
+}
+
 size_t attn_sink_decode_workspace_size(int B, int Hq, int D, int Lmax, int window, int num_splits)
 {
     if (B <= 0 || Hq <= 0 || D <= 0 || Lmax <= 0 || num_splits < 0 || num_splits > 32) return 0;

@@ -111,6 +111,15 @@ cudaError_t launch_decode_bf16(const void *q, const void *kc, const void *vc, co
                                const float *v_scale = nullptr);
 bool decode_bf16_supported(const DecodeShape &s);
 
+// QKV prologue: bias, YaRN rotary embedding of q and k, split into q / k / v.
+struct RopeParams {
+    double base, factor, original_max_pos, beta_fast, beta_slow;
+    int interleaved;  // 0: pairs (i, i + D/2); 1: pairs (2i, 2i + 1)
+};
+cudaError_t launch_qkv_prologue(const void *qkv, const float *bias, const int *positions, const int *kv_rows,
+                                void *q, void *k, void *v, int T, int Hq, int Hkv, int kv_rows_total,
+                                const RopeParams &r, cudaStream_t st);
+
 // Driver entry point for cuTensorMapEncodeTiled (resolved once through the runtime).
 bool encode_tensor_map_4d(void *map, void *gaddr, int elem_bytes, const uint64_t dims[4],
                           const uint64_t strides_bytes[3], const uint32_t box[4], bool swizzle128);

@@ -1,0 +1,206 @@
+// prologue.cu -- the step just before attention: the QKV projection's output
+// gets its bias, q and k are rotated by YaRN-scaled rotary position embeddings,
+// and the three are written in the layouts the attention calls read
+// ("GPT-OSS on day 0", section "Attention: GQA with Attention Sinks": the QKV
+// projections carry biases and positions use YaRN encoding, as in DeepSeek-V3;
+// "GPT-OSS-120B 4-bit ...", section 3: YaRN-type RoPE scaling extends the
+// context to 131072 tokens).
+//
+// Per token t at position p, with frequencies for pair i (D/2 pairs):
+//   f_i    = base^(-2i/D)                             (plain rotary frequency)
+//   lo, hi = the dimensions where a full wavelength fits beta_fast and
+//            beta_slow times into the original context L0:
+//            d(n) = D ln(L0 / (2 pi n)) / (2 ln base)
+//   e_i    = 1 - clamp((i - lo) / (hi - lo), 0, 1)    (1: keep f_i, 0: interpolate)
+//   f'_i   = f_i e_i + (f_i / factor) (1 - e_i)
+//   a      = 0.1 ln(factor) + 1 (1 when factor <= 1), multiplying cos and sin
+//   rotate-half pairs (i, i + D/2) or interleaved pairs (2i, 2i + 1):
+//   x'_lo = a (x_lo cos(p f'_i) - x_hi sin(p f'_i)),  x'_hi = a (x_hi cos + x_lo sin)
+// v only gets its bias.  The angles are formed and reduced in fp64 (positions
+// up to 131072 times frequencies near 1 leave fp32 with too few bits of phase).
+//
+// Design: HBM-bound (one read and one write of the QKV rows).  A CTA takes one
+// token: 32 threads compute the D/2 cos/sin pairs into shared memory, then all
+// threads move 16-byte chunks of q, k and v, eight pairs (or eight v values)
+// per thread-step.  k and v rows can be written to any row of their outputs
+// (kv_rows), which appends them to a decode cache in the same pass.
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include "kernels.h"
+#include "sm100_ptx.cuh"
+
+namespace attn_sink {
+namespace {
+
+constexpr int kD = 64;
+constexpr int kPairs = kD / 2;
+constexpr int kThreads = 256;
+
+struct ProParams {
+    const __nv_bfloat16 *qkv;  // [T, (Hq + 2 Hkv) * D]
+    const float *bias;         // [(Hq + 2 Hkv) * D] or nullptr
+    const int *pos;            // [T]
+    const int *kv_rows;        // [T] or nullptr (row t)
+    __nv_bfloat16 *q, *k, *v;
+    int T, Hq, Hkv, interleaved;
+    int kv_rows_total;         // rows of k / v (a kv_rows entry outside [0, rows) writes nothing)
+    double base, factor, L0, beta_fast, beta_slow, attn_factor;
+};
+
+// rotary frequency of pair i after the YaRN correction
+__device__ double yarn_freq(const ProParams &p, int i)
+{
+    const double f = pow(p.base, -2.0 * i / kD);
+    if (!(p.factor > 1.0)) return f;
+    const double lo = kD * log(p.L0 / (2.0 * M_PI * p.beta_fast)) / (2.0 * log(p.base));
+    const double hi = kD * log(p.L0 / (2.0 * M_PI * p.beta_slow)) / (2.0 * log(p.base));
+    double ramp = hi > lo ? (i - lo) / (hi - lo) : (i >= lo ? 1.0 : 0.0);
+    ramp = ramp < 0.0 ? 0.0 : (ramp > 1.0 ? 1.0 : ramp);
+    const double keep = 1.0 - ramp;
+    return f * keep + (f / p.factor) * (1.0 - keep);
+}
+
+__device__ __forceinline__ float2 bf2(uint32_t w)
+{
+    const __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162 *>(&w);
+    return __bfloat1622float2(h);
+}
+
+__global__ void __launch_bounds__(kThreads) prologue_kernel(const ProParams p)
+{
+    __shared__ float cs[kPairs], sn[kPairs];
+    const int t = blockIdx.x;
+    const int width = (p.Hq + 2 * p.Hkv) * kD;
+    if (threadIdx.x < kPairs) {
+        const int i = threadIdx.x;
+        const double ang = fmod((double)p.pos[t] * yarn_freq(p, i), 2.0 * M_PI);
+        double s, c;
+        sincos(ang, &s, &c);
+        cs[i] = (float)(c * p.attn_factor);
+        sn[i] = (float)(s * p.attn_factor);
+    }
+    __syncthreads();
+    const __nv_bfloat16 *row = p.qkv + (size_t)t * width;
+    const int kr = p.kv_rows ? p.kv_rows[t] : t;
+    const bool kv_ok = kr >= 0 && kr < p.kv_rows_total;
+    // rotated heads (q then k): each step takes 8 pairs of one head
+    const int rot_heads = p.Hq + p.Hkv;
+    for (int u = threadIdx.x; u < rot_heads * (kPairs / 8); u += kThreads) {
+        const int h = u / (kPairs / 8), i0 = (u % (kPairs / 8)) * 8;
+        const int col = h * kD;
+        float xa[8], xb[8];  // the two members of pairs i0 .. i0 + 7
+        if (!p.interleaved) {
+            const uint4 a = *reinterpret_cast<const uint4 *>(row + col + i0);
+            const uint4 b = *reinterpret_cast<const uint4 *>(row + col + kPairs + i0);
+            const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float2 fa = bf2(aw[j]), fb = bf2(bw[j]);
+                xa[2 * j] = fa.x;
+                xa[2 * j + 1] = fa.y;
+                xb[2 * j] = fb.x;
+                xb[2 * j + 1] = fb.y;
+            }
+        } else {
+            const uint4 a = *reinterpret_cast<const uint4 *>(row + col + 2 * i0);
+            const uint4 b = *reinterpret_cast<const uint4 *>(row + col + 2 * i0 + 8);
+            const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const float2 f = bf2(w[j]);
+                xa[j] = f.x;
+                xb[j] = f.y;
+            }
+        }
+        if (p.bias) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int da = p.interleaved ? 2 * (i0 + j) : i0 + j;
+                const int db = p.interleaved ? da + 1 : i0 + j + kPairs;
+                xa[j] += p.bias[col + da];
+                xb[j] += p.bias[col + db];
+            }
+        }
+        uint32_t oa[4], ob[4], oi[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float c = cs[i0 + j], s = sn[i0 + j];
+            const float ra = xa[j] * c - xb[j] * s;
+            const float rb = xb[j] * c + xa[j] * s;
+            xa[j] = ra;
+            xb[j] = rb;
+        }
+        __nv_bfloat16 *dst;
+        if (h < p.Hq) {
+            dst = p.q + ((size_t)t * p.Hq + h) * kD;
+        } else {
+            if (!kv_ok) continue;
+            dst = p.k + ((size_t)kr * p.Hkv + (h - p.Hq)) * kD;
+        }
+        if (!p.interleaved) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                oa[j] = pack_bf16x2(xa[2 * j], xa[2 * j + 1]);
+                ob[j] = pack_bf16x2(xb[2 * j], xb[2 * j + 1]);
+            }
+            *reinterpret_cast<uint4 *>(dst + i0) = make_uint4(oa[0], oa[1], oa[2], oa[3]);
+            *reinterpret_cast<uint4 *>(dst + kPairs + i0) = make_uint4(ob[0], ob[1], ob[2], ob[3]);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) oi[j] = pack_bf16x2(xa[j], xb[j]);
+            *reinterpret_cast<uint4 *>(dst + 2 * i0) = make_uint4(oi[0], oi[1], oi[2], oi[3]);
+            *reinterpret_cast<uint4 *>(dst + 2 * i0 + 8) = make_uint4(oi[4], oi[5], oi[6], oi[7]);
+        }
+    }
+    // v: bias only, 8 values per step
+    if (!kv_ok) return;
+    for (int u = threadIdx.x; u < p.Hkv * (kD / 8); u += kThreads) {
+        const int h = u / (kD / 8), d0 = (u % (kD / 8)) * 8;
+        const int col = (p.Hq + p.Hkv + h) * kD + d0;
+        const uint4 a = *reinterpret_cast<const uint4 *>(row + col);
+        const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            float2 f = bf2(w[j]);
+            if (p.bias) {
+                f.x += p.bias[col + 2 * j];
+                f.y += p.bias[col + 2 * j + 1];
+            }
+            o[j] = pack_bf16x2(f.x, f.y);
+        }
+        *reinterpret_cast<uint4 *>(p.v + ((size_t)kr * p.Hkv + h) * kD + d0) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_qkv_prologue(const void *qkv, const float *bias, const int *positions, const int *kv_rows,
+                                void *q, void *k, void *v, int T, int Hq, int Hkv, int kv_rows_total,
+                                const RopeParams &r, cudaStream_t st)
+{
+    ProParams p;
+    p.qkv = static_cast<const __nv_bfloat16 *>(qkv);
+    p.bias = bias;
+    p.pos = positions;
+    p.kv_rows = kv_rows;
+    p.q = static_cast<__nv_bfloat16 *>(q);
+    p.k = static_cast<__nv_bfloat16 *>(k);
+    p.v = static_cast<__nv_bfloat16 *>(v);
+    p.T = T;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.interleaved = r.interleaved;
+    p.kv_rows_total = kv_rows_total;
+    p.base = r.base;
+    p.factor = r.factor;
+    p.L0 = r.original_max_pos;
+    p.beta_fast = r.beta_fast;
+    p.beta_slow = r.beta_slow;
+    p.attn_factor = r.factor > 1.0 ? 0.1 * log(r.factor) + 1.0 : 1.0;
+    prologue_kernel<<<T, kThreads, 0, st>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace attn_sink

@@ -126,6 +126,45 @@ ATTN_SINK_API int attn_sink_fwd_varlen(const void *q, const void *k, const void 
                   int window, float scale, void *stream);
 
 /*
+ * QKV prologue: the step just before attention, in one pass over the QKV
+ * projection's output.  The pages give gpt-oss QKV projections with biases
+ * and YaRN rotary position encoding "as in DeepSeek-V3" ("GPT-OSS on day 0",
+ * section "Attention: GQA with Attention Sinks"), extended to 131072 tokens
+ * ("GPT-OSS-120B 4-bit ...", section 3); they give no parameter values, so
+ * the rotation's parameters are arguments.  For token t at position p:
+ *   y = qkv[t] + bias (fp32), split into q (Hq heads), k (Hkv), v (Hkv);
+ *   q and k are rotated pair by pair, with rotary frequency f_i =
+ *   rope_theta^(-2i/D) for pair i of D/2, corrected by YaRN when
+ *   rope_factor > 1: with d(n) = D ln(L0 / (2 pi n)) / (2 ln rope_theta),
+ *   L0 = rope_original_max_pos, the weight e_i = 1 - clamp((i - d(beta_fast))
+ *   / (d(beta_slow) - d(beta_fast)), 0, 1) keeps f_i where a wavelength fits
+ *   many times into L0 and interpolates to f_i / rope_factor where it does
+ *   not: f'_i = e_i f_i + (1 - e_i) f_i / rope_factor; cos and sin of
+ *   p f'_i are scaled by the attention factor 0.1 ln(rope_factor) + 1.
+ *   Pair i is (i, i + D/2) (interleaved = 0) or (2i, 2i + 1) (interleaved = 1);
+ *   (x, y) -> (x cos - y sin, y cos + x sin).  v gets its bias only.
+ *   rope_factor <= 1 is plain rotary embedding (no correction, factor 1).
+ *   qkv     [T, (Hq + 2 Hkv) * D] bf16, q columns first, then k, then v
+ *   bias    [(Hq + 2 Hkv) * D] fp32, or NULL for none
+ *   positions [T] int32, device
+ *   kv_rows [T] int32, device, or NULL: token t's k and v go to row
+ *           kv_rows[t] (row t) of k_out / v_out, so a decode step can append
+ *           them to a cache laid out [B, Lmax, Hkv, D] (row b * Lmax + p) in
+ *           the same pass; a row outside [0, kv_rows_total) is not written.
+ *   q_out   [T, Hq, D] bf16     k_out, v_out [kv_rows_total, Hkv, D] bf16
+ * Angles are formed and reduced in fp64.  D must be 64.  Errors:
+ * INVALID_ARG for null pointers, non-positive sizes, kv_rows NULL with
+ * kv_rows_total < T, rope_theta <= 1, rope_factor <= 0, or (rope_factor > 1)
+ * rope_original_max_pos <= 0 or not beta_fast > beta_slow > 0;
+ * UNSUPPORTED for D != 64.  Nothing is allocated; asynchronous on stream.
+ */
+ATTN_SINK_API int attn_sink_qkv_prologue(const void *qkv, const float *bias, const int *positions,
+                  const int *kv_rows, void *q_out, void *k_out, void *v_out, int T, int Hq,
+                  int Hkv, int D, int kv_rows_total, float rope_theta, float rope_factor,
+                  int rope_original_max_pos, float beta_fast, float beta_slow, int interleaved,
+                  void *stream);
+
+/*
  * Split-KV decode over a contiguous per-sequence KV cache with ragged
  * lengths ("GPT-OSS on day 0", section "Sink Attention": attention is split
  * along the KV length as well as across heads, and the sink must be counted

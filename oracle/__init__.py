@@ -214,3 +214,62 @@ def fwd_varlen(q, k, v, sinks, cu_q, cu_k, window: int, scale: float):
         out[a:e] = o[0]
         lse[:, a:e] = l[0]
     return out, lse
+
+
+def yarn_frequencies(D: int, base: float, factor: float = 1.0, original_max_pos: float = 0.0,
+                     beta_fast: float = 32.0, beta_slow: float = 1.0):
+    """Rotary frequencies of the D/2 pairs and the attention factor, in fp64.
+
+    Plain rotary embedding: f_i = base^(-2i/D).  YaRN (factor > 1), in the
+    DeepSeek-V3 form the pages point to ("GPT-OSS on day 0", section
+    "Attention: GQA with Attention Sinks"): d(n) = D ln(L0 / (2 pi n)) /
+    (2 ln base) is the pair index at which a full wavelength fits n times
+    into the original context L0; between d(beta_fast) and d(beta_slow) a
+    ramp linear in the pair index moves the frequency from f_i (kept) to
+    f_i / factor (interpolated); the attention factor is 0.1 ln(factor) + 1."""
+    i = np.arange(D // 2, dtype=np.float64)
+    f = np.power(float(base), -2.0 * i / D)
+    if not factor > 1.0:
+        return f, 1.0
+    d = lambda n: D * np.log(original_max_pos / (2.0 * np.pi * n)) / (2.0 * np.log(base))
+    lo, hi = d(beta_fast), d(beta_slow)
+    ramp = np.clip((i - lo) / (hi - lo), 0.0, 1.0) if hi > lo else (i >= lo).astype(np.float64)
+    keep = 1.0 - ramp
+    return f * keep + (f / factor) * (1.0 - keep), 0.1 * np.log(factor) + 1.0
+
+
+def rotate(x, positions, freqs, attn_factor, interleaved=False):
+    """Rotary embedding of x [T, H, D] (fp64): pair i of token t turns by the
+    angle positions[t] * freqs[i], scaled by attn_factor.  Pairs are
+    (i, i + D/2), or (2i, 2i + 1) when interleaved."""
+    x = np.asarray(x, dtype=np.float64)
+    D = x.shape[-1]
+    ang = np.asarray(positions, dtype=np.float64)[:, None] * freqs[None, :]
+    c = (np.cos(ang) * attn_factor)[:, None, :]
+    s = (np.sin(ang) * attn_factor)[:, None, :]
+    a, b = (x[..., 0::2], x[..., 1::2]) if interleaved else (x[..., :D // 2], x[..., D // 2:])
+    out = np.empty_like(x)
+    ra, rb = a * c - b * s, b * c + a * s
+    if interleaved:
+        out[..., 0::2], out[..., 1::2] = ra, rb
+    else:
+        out[..., :D // 2], out[..., D // 2:] = ra, rb
+    return out
+
+
+def qkv_prologue(qkv, bias, positions, Hq: int, Hkv: int, D: int, base: float, factor: float = 1.0,
+                 original_max_pos: float = 0.0, beta_fast: float = 32.0, beta_slow: float = 1.0,
+                 interleaved: bool = False):
+    """The step before attention: y = qkv + bias, split into q [T, Hq, D],
+    k [T, Hkv, D], v [T, Hkv, D]; q and k rotated at their token's position.
+    Returns (q, k, v) in fp64."""
+    y = _f64(qkv)
+    if bias is not None:
+        y = y + _f64(bias)[None, :]
+    T = y.shape[0]
+    y = y.reshape(T, Hq + 2 * Hkv, D)
+    pos = np.asarray(positions.cpu() if hasattr(positions, "cpu") else positions, dtype=np.float64)
+    f, a = yarn_frequencies(D, base, factor, original_max_pos, beta_fast, beta_slow)
+    q = rotate(y[:, :Hq], pos, f, a, interleaved)
+    k = rotate(y[:, Hq:Hq + Hkv], pos, f, a, interleaved)
+    return q, k, y[:, Hq + Hkv:].copy()

@@ -174,3 +174,26 @@ def test_no_device_is_reported_cleanly():
 def test_wait_timeout_setting_round_trips():
     old = attn.attn_sink_set_wait_timeout_ns(123456789)
     assert attn.attn_sink_set_wait_timeout_ns(old) == 123456789
+
+
+def test_qkv_prologue_host_checks():
+    lib = attn.load()
+    qkv, b, pos, rows, q, k, v = _fake(7)
+
+    def call(qkv_=qkv, pos_=pos, rows_=rows, T=10, Hq=8, Hkv=2, D=64, nrows=10, theta=10000.0, factor=32.0, L0=4096,
+             bf=32.0, bs=1.0, inter=0):
+        return lib.attn_sink_qkv_prologue(qkv_, b, pos_, rows_, q, k, v, T, Hq, Hkv, D, nrows, theta, factor, L0, bf,
+                                          bs, inter, None)
+
+    assert call(qkv_=None) == INVALID
+    assert call(pos_=None) == INVALID
+    assert call(T=0) == INVALID
+    assert call(Hkv=3) == INVALID
+    assert call(D=128) == UNSUPPORTED
+    assert call(rows_=None, nrows=5) == INVALID  # row t must exist without a row map
+    assert call(theta=1.0) == INVALID
+    assert call(factor=0.0) == INVALID
+    assert call(L0=0) == INVALID  # YaRN needs the original context
+    assert call(bf=1.0, bs=1.0) == INVALID
+    assert call(inter=2) == INVALID
+    assert call(pos_=pos + 4) == MISALIGNED

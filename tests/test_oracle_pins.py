@@ -373,3 +373,72 @@ def test_fwd_varlen_is_the_batch_when_lengths_agree_and_skips_empty_sequences():
         o2, l2 = oracle.fwd_varlen(t["q"].reshape(B * L, Hq, 16), t["k"].reshape(B * L, Hkv, 16),
                                    t["v"].reshape(B * L, Hkv, 16), t["sinks"], cu_e, cu_e, window, 0.25)
         assert np.array_equal(o2, o) and np.array_equal(l2, l)
+
+
+# ----------------------------------------------------------------------------- QKV prologue (YaRN rotary embedding)
+YARN = dict(base=150000.0, factor=32.0, original_max_pos=4096, beta_fast=32.0, beta_slow=1.0)
+
+
+def test_yarn_frequencies_closed_forms():
+    """The correction dimension d(n) is where the wavelength 2 pi / f fits n
+    times into L0; pairs below d(beta_fast) keep f_i exactly, pairs above
+    d(beta_slow) take f_i / factor exactly, pairs between lie strictly between;
+    the attention factor is 0.1 ln(factor) + 1; factor 1 is plain rotary."""
+    D, base, L0 = 64, 10000.0, 4096
+    f0, a0 = oracle.yarn_frequencies(D, base)
+    assert a0 == 1.0 and np.array_equal(f0, base ** (-np.arange(32) * 2.0 / D))
+    f, a = oracle.yarn_frequencies(D, base, 32.0, L0, 32.0, 1.0)
+    lo = D * math.log(L0 / (2 * math.pi * 32.0)) / (2 * math.log(base))
+    hi = D * math.log(L0 / (2 * math.pi * 1.0)) / (2 * math.log(base))
+    # the wavelength at the (fractional) pair index lo fits beta_fast = 32 times into L0
+    assert abs(L0 * base ** (-2 * lo / D) / (2 * math.pi) - 32.0) < 1e-9
+    i = np.arange(32)
+    keep, interp = i <= math.floor(lo), i >= math.ceil(hi)
+    assert keep.any() and interp.any()
+    assert np.array_equal(f[keep], f0[keep])
+    np.testing.assert_allclose(f[interp], f0[interp] / 32.0, rtol=1e-15)
+    mid = ~keep & ~interp
+    assert (f[mid] < f0[mid]).all() and (f[mid] > f0[mid] / 32.0).all()
+    assert abs(a - (0.1 * math.log(32.0) + 1.0)) < 1e-15
+    _, a_e = oracle.yarn_frequencies(D, base, math.exp(10.0), L0)
+    assert abs(a_e - 2.0) < 1e-12
+
+
+@pytest.mark.parametrize("interleaved", [False, True])
+def test_rotation_is_complex_multiplication(interleaved):
+    """Each pair (a, b) turned by angle t is the complex number a + ib times
+    attn_factor * e^{it} (written with numpy complex arithmetic here)."""
+    g = np.random.default_rng(5)
+    x = g.standard_normal((7, 3, 16))
+    pos = g.integers(0, 131072, 7)
+    f, a = oracle.yarn_frequencies(16, YARN["base"], YARN["factor"], YARN["original_max_pos"])
+    r = oracle.rotate(x, pos, f, a, interleaved)
+    pa, pb = (slice(0, None, 2), slice(1, None, 2)) if interleaved else (slice(0, 8), slice(8, 16))
+    z = (x[..., pa] + 1j * x[..., pb]) * (a * np.exp(1j * pos[:, None, None] * f[None, None, :]))
+    np.testing.assert_allclose(r[..., pa], z.real, atol=1e-12)
+    np.testing.assert_allclose(r[..., pb], z.imag, atol=1e-12)
+
+
+def test_rotation_depends_only_on_relative_position_and_scales_norms():
+    g = np.random.default_rng(6)
+    q, k = g.standard_normal((1, 1, 64)), g.standard_normal((1, 1, 64))
+    f, a = oracle.yarn_frequencies(64, YARN["base"], YARN["factor"], YARN["original_max_pos"])
+    dots = [float((oracle.rotate(q, [p + 1000], f, a) * oracle.rotate(k, [p], f, a)).sum()) for p in (0, 77, 50000)]
+    np.testing.assert_allclose(dots, dots[0], rtol=1e-9)
+    np.testing.assert_allclose(np.linalg.norm(oracle.rotate(q, [123456], f, a)), a * np.linalg.norm(q), rtol=1e-12)
+
+
+def test_qkv_prologue_splits_adds_bias_and_rotates_q_and_k_only():
+    g = np.random.default_rng(7)
+    T, Hq, Hkv, D = 5, 4, 2, 16
+    qkv = g.standard_normal((T, (Hq + 2 * Hkv) * D))
+    bias = g.standard_normal((Hq + 2 * Hkv) * D)
+    pos = g.integers(0, 5000, T)
+    q, k, v = oracle.qkv_prologue(qkv, bias, pos, Hq, Hkv, D, **YARN)
+    y = (qkv + bias).reshape(T, Hq + 2 * Hkv, D)
+    np.testing.assert_array_equal(v, y[:, Hq + Hkv:])
+    f, a = oracle.yarn_frequencies(D, **{k_: YARN[k_] for k_ in YARN if k_ != "base"}, base=YARN["base"])
+    np.testing.assert_array_equal(q, oracle.rotate(y[:, :Hq], pos, f, a))
+    np.testing.assert_array_equal(k, oracle.rotate(y[:, Hq:Hq + Hkv], pos, f, a))
+    q0, _, _ = oracle.qkv_prologue(qkv, bias, np.zeros(T), Hq, Hkv, D, **YARN)  # position 0: scaling only
+    np.testing.assert_allclose(q0, a * y[:, :Hq], rtol=1e-15)

@@ -45,7 +45,7 @@ constexpr int kT = 64;          // keys per tile
 // K/V ring stages: the loads in flight per SM must cover the HBM latency at
 // full bandwidth, so the e4m3 ring (half the bytes per stage) is deeper
 #ifndef ATTN_SINK_DEC_FP8_STAGES
-#define ATTN_SINK_DEC_FP8_STAGES 8
+#define ATTN_SINK_DEC_FP8_STAGES 6
 #endif
 constexpr int kThreads = 160;  // warp 0 producer, warps 1-4 consumers
 constexpr float kLog2e = 1.4426950408889634f;
@@ -58,9 +58,10 @@ struct DecLayout {
     static constexpr int kRowBytes = kFp8 ? kD : kD * 2;  // one cached K or V row
     static constexpr int kTileBytes = kT * kRowBytes;
     static constexpr int kStageBytes = 2 * kTileBytes;  // K and V
-    // e4m3 only: each consumer warp's 16 keys of K and of V as bf16, 128-byte swizzled
+    // e4m3 only: each consumer warp's 16 keys of V as f16, 128-byte swizzled
+    // (K is read straight from the e4m3 tile)
     static constexpr int kOffStaging = kNS * kStageBytes;
-    static constexpr int kWarpStaging = 2 * 16 * kD * 2;
+    static constexpr int kWarpStaging = 16 * kD * 2;
     static constexpr int kOffBar = kOffStaging + (kFp8 ? 4 * kWarpStaging : 0);
     static constexpr int kSmemBytes = kOffBar + 2 * kNS * 8 + 16 + 1024;
     // the final reduction reuses [0, kOffBar): 4 warps x 16 rows x 66 floats
@@ -106,24 +107,39 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
                  : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// D (fp32 16x8) += A (f16 16x16, row) * B (f16 16x8, col)
+__device__ __forceinline__ void mma16816_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
+{
+    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+                 "{%0,%1,%2,%3};"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// two e4m3 codes (low byte first) -> their exact values as an f16 pair
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes)
+{
+    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two_codes & 0xffffu), __NV_E4M3);
+    return (uint32_t)h.x | ((uint32_t)h.y << 16);
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi)
+{
+    const __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&v);
+}
+
 // byte offset of (row, 16-byte chunk) in a 128-byte-swizzled tile
 __device__ __forceinline__ uint32_t swz(int row, int chunk) { return row * 128 + ((chunk ^ (row & 7)) << 4); }
 
-// 16 e4m3 values (byte i = element i) -> 16 bf16, elements 0-7 in lo and 8-15
-// in hi (element 2m in the low half of word m).  Exact: every e4m3 value is a
-// half and a bf16 (e4m3 -> f16x2 by the hardware conversion, then f32, then
-// bf16 round-to-nearest, which changes nothing).
-__device__ __forceinline__ void e4m3x16_to_bf16(const uint4 &raw, uint4 &lo, uint4 &hi)
+// 16 e4m3 codes (byte i = element i) -> their 16 exact f16 values, elements
+// 0-7 in lo and 8-15 in hi (element 2m in the low half of word m)
+__device__ __forceinline__ void e4m3x16_to_f16(const uint4 &raw, uint4 &lo, uint4 &hi)
 {
     const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
     uint32_t o[8];
 #pragma unroll
-    for (int m = 0; m < 8; ++m) {
-        const __nv_fp8x2_storage_t pr = (__nv_fp8x2_storage_t)((w[m >> 1] >> (16 * (m & 1))) & 0xffffu);
-        const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(pr, __NV_E4M3);
-        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&h));
-        o[m] = pack_bf16x2(f.x, f.y);
-    }
+    for (int m = 0; m < 8; ++m) o[m] = e4m3x2_to_f16x2(w[m >> 1] >> (16 * (m & 1)));
     lo = make_uint4(o[0], o[1], o[2], o[3]);
     hi = make_uint4(o[4], o[5], o[6], o[7]);
 }
@@ -216,22 +232,62 @@ __global__ void __launch_bounds__(kThreads)
         const int tq = lane & 3;      // fragment column pair
         // Q as the A operand (rows = heads of the group, zero beyond G), k-steps of 16 d
         uint32_t qa[4][4];
+        float qscale_inv = 1.f;
         {
             const __nv_bfloat16 *qb = p.q + ((size_t)b * p.Hq + (size_t)g * p.G) * kD;
             auto qpair = [&](int row, int d) -> uint32_t {
                 if (row >= p.G) return 0u;
                 return *reinterpret_cast<const uint32_t *>(qb + (size_t)row * kD + d);
             };
+            if (!kFp8) {
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                qa[kk][0] = qpair(gr, 16 * kk + 2 * tq);
-                qa[kk][1] = qpair(gr + 8, 16 * kk + 2 * tq);
-                qa[kk][2] = qpair(gr, 16 * kk + 8 + 2 * tq);
-                qa[kk][3] = qpair(gr + 8, 16 * kk + 8 + 2 * tq);
+                for (int kk = 0; kk < 4; ++kk) {
+                    qa[kk][0] = qpair(gr, 16 * kk + 2 * tq);
+                    qa[kk][1] = qpair(gr + 8, 16 * kk + 2 * tq);
+                    qa[kk][2] = qpair(gr, 16 * kk + 8 + 2 * tq);
+                    qa[kk][3] = qpair(gr + 8, 16 * kk + 8 + 2 * tq);
+                }
+            } else {
+                // e4m3 caches: f16 MMAs (every e4m3 value is an f16).  q goes to f16
+                // times 2^e, the power of two that puts max|q| of the group in
+                // [2^14, 2^15), so no element overflows; 2^-e joins the logit scale.
+                // The head dimension is visited in the order that lets a lane take
+                // K's fragments from 16 consecutive bytes of a key row: in k-step
+                // kk, fragment columns 2t, 2t+1 (8+2t, 9+2t) are dimensions
+                // 16t + 4kk + 0, 1 (2, 3); q and k use the same order.
+                uint32_t raw[4][4];
+                float amax = 0.f;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    const int d0 = 16 * tq + 4 * kk;
+                    raw[kk][0] = qpair(gr, d0);
+                    raw[kk][1] = qpair(gr + 8, d0);
+                    raw[kk][2] = qpair(gr, d0 + 2);
+                    raw[kk][3] = qpair(gr + 8, d0 + 2);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162 *>(&raw[kk][u]);
+                        amax = fmaxf(amax, fmaxf(fabsf(__low2float(h)), fabsf(__high2float(h))));
+                    }
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+                const int e = amax > 0.f ? 141 - (int)((__float_as_uint(amax) >> 23) & 0xffu) : 0;
+                const int ec = max(-100, min(100, e));
+                const float qsc = __uint_as_float((uint32_t)(ec + 127) << 23);
+                qscale_inv = __uint_as_float((uint32_t)(127 - ec) << 23);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162 *>(&raw[kk][u]);
+                        qa[kk][u] = pack_f16x2(__low2float(h) * qsc, __high2float(h) * qsc);
+                    }
             }
         }
-        // e4m3 caches: K's scale folds into the logit scale (V's into the output)
-        const float C = kFp8 ? p.c_log2 * p.k_scale[g] : p.c_log2;
+        // e4m3 caches: K's scale (and q's power of two) fold into the logit
+        // scale, V's scale into the output
+        const float C = kFp8 ? p.c_log2 * p.k_scale[g] * qscale_inv : p.c_log2;
         const uint32_t sbase = smem_u32(smem);
         for (int j = 0; j < n_tiles && ok; ++j) {
             const int st = j % kNS;
@@ -242,28 +298,28 @@ __global__ void __launch_bounds__(kThreads)
             }
             uint32_t kt = sbase + st * L::kStageBytes, vt = kt + L::kTileBytes;
             int rw = 16 * w;  // first row of this warp's 16 keys in the tile it reads
+            uint4 k8r[2];  // e4m3 only: this lane's 16 bytes of key row (16w + 8nt + gr), nt = 0, 1
             if (kFp8) {
-                // this warp's 16 keys of K and V, e4m3 -> bf16 into its own staging
-                // (the layout of the bf16 tiles), then the raw stage is free again
+                // this warp's 16 keys: K's fragments straight from the e4m3 tile,
+                // V widened to f16 into the warp's own staging (the layout the
+                // transposing ldmatrix reads); then the raw stage is free again
                 const uint8_t *k8 = smem + st * L::kStageBytes + 16 * w * L::kRowBytes;
                 const uint8_t *v8 = k8 + L::kTileBytes;
-                uint8_t *ks = smem + L::kOffStaging + w * L::kWarpStaging;
-                uint8_t *vs = ks + L::kWarpStaging / 2;
+                uint8_t *vs = smem + L::kOffStaging + w * L::kWarpStaging;
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+                    k8r[nt] = *reinterpret_cast<const uint4 *>(k8 + (8 * nt + gr) * L::kRowBytes + 16 * tq);
 #pragma unroll
                 for (int it = 0; it < 2; ++it) {
                     const int i = lane + 32 * it;
                     const int row = i >> 2, ch = i & 3;  // 16 rows x 4 chunks of 16 values
                     uint4 lo, hi;
-                    e4m3x16_to_bf16(*reinterpret_cast<const uint4 *>(k8 + row * L::kRowBytes + ch * 16), lo, hi);
-                    *reinterpret_cast<uint4 *>(ks + swz(row, 2 * ch)) = lo;
-                    *reinterpret_cast<uint4 *>(ks + swz(row, 2 * ch + 1)) = hi;
-                    e4m3x16_to_bf16(*reinterpret_cast<const uint4 *>(v8 + row * L::kRowBytes + ch * 16), lo, hi);
+                    e4m3x16_to_f16(*reinterpret_cast<const uint4 *>(v8 + row * L::kRowBytes + ch * 16), lo, hi);
                     *reinterpret_cast<uint4 *>(vs + swz(row, 2 * ch)) = lo;
                     *reinterpret_cast<uint4 *>(vs + swz(row, 2 * ch + 1)) = hi;
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&empty[st]);
-                kt = smem_u32(ks);
                 vt = smem_u32(vs);
                 rw = 0;
             }
@@ -273,13 +329,20 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt) {
                 s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
-                const int krow = rw + 8 * nt + (lane & 7);
+                if (kFp8) {
+                    const uint32_t w4[4] = {k8r[nt].x, k8r[nt].y, k8r[nt].z, k8r[nt].w};
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t b0, b1, b2, b3;  // d chunks 4*half + 0..3
-                    ldsm_x4(kt + swz(krow, 4 * half + (lane >> 3)), b0, b1, b2, b3);
-                    mma16816(s[nt], qa[2 * half], b0, b1);
-                    mma16816(s[nt], qa[2 * half + 1], b2, b3);
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma16816_f16(s[nt], qa[kk], e4m3x2_to_f16x2(w4[kk]), e4m3x2_to_f16x2(w4[kk] >> 16));
+                } else {
+                    const int krow = rw + 8 * nt + (lane & 7);
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        uint32_t b0, b1, b2, b3;  // d chunks 4*half + 0..3
+                        ldsm_x4(kt + swz(krow, 4 * half + (lane >> 3)), b0, b1, b2, b3);
+                        mma16816(s[nt], qa[2 * half], b0, b1);
+                        mma16816(s[nt], qa[2 * half + 1], b2, b3);
+                    }
                 }
             }
             // ---- mask keys outside [lo, kend); log2-domain logits
@@ -331,10 +394,17 @@ __global__ void __launch_bounds__(kThreads)
             }
             // ---- O += P V: P from the score accumulators, V via transposing ldmatrix
             uint32_t pa[4];
-            pa[0] = pack_bf16x2(pv[0][0], pv[0][1]);
-            pa[1] = pack_bf16x2(pv[0][2], pv[0][3]);
-            pa[2] = pack_bf16x2(pv[1][0], pv[1][1]);
-            pa[3] = pack_bf16x2(pv[1][2], pv[1][3]);
+            if (kFp8) {
+                pa[0] = pack_f16x2(pv[0][0], pv[0][1]);
+                pa[1] = pack_f16x2(pv[0][2], pv[0][3]);
+                pa[2] = pack_f16x2(pv[1][0], pv[1][1]);
+                pa[3] = pack_f16x2(pv[1][2], pv[1][3]);
+            } else {
+                pa[0] = pack_bf16x2(pv[0][0], pv[0][1]);
+                pa[1] = pack_bf16x2(pv[0][2], pv[0][3]);
+                pa[2] = pack_bf16x2(pv[1][0], pv[1][1]);
+                pa[3] = pack_bf16x2(pv[1][2], pv[1][3]);
+            }
             // rows of V outside [lo, kend) are zeroed in the operand (cache rows
             // beyond the sequence may hold anything)
             const bool tail = __any_sync(0xffffffffu, key0 + 15 >= kend || key0 < lo);
@@ -354,8 +424,13 @@ __global__ void __launch_bounds__(kThreads)
                     b1 &= m8;
                     b3 &= m8;
                 }
-                mma16816(o[jn], pa, b0, b1);
-                mma16816(o[jn + 1], pa, b2, b3);
+                if (kFp8) {
+                    mma16816_f16(o[jn], pa, b0, b1);
+                    mma16816_f16(o[jn + 1], pa, b2, b3);
+                } else {
+                    mma16816(o[jn], pa, b0, b1);
+                    mma16816(o[jn + 1], pa, b2, b3);
+                }
             }
             __syncwarp();
             if (!kFp8 && lane == 0) mbar_arrive(&empty[st]);

@@ -318,23 +318,31 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 #pragma unroll
             for (int k = 0; k < 8; ++k) mx[k] = -INFINITY;
             {
-                // TMEM loads run one 16-column chunk ahead of the arithmetic
-                uint32_t sb[2][16];
-                tmem_ld16(trow, sb[0]);
-                tmem_wait_ld();
+                // three 16-column loads, then one wait: a TMEM load round trip
+                // costs more than the maxima of 16 columns, so it is paid per 48
+                constexpr int kGroup = 3;
 #pragma unroll
-                for (int c = 0; c < kChunks; ++c) {
-                    if (c + 1 < kChunks) tmem_ld16(trow + 16 * (c + 1), sb[(c + 1) & 1]);
-                    float v[16];
+                for (int c0 = 0; c0 < kChunks; c0 += kGroup) {
+                    uint32_t sb[kGroup][16];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) v[e] = __uint_as_float(sb[c & 1][e]);
-                    if (mask_chunks & (1u << c)) {
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) v[e] = (16 * c + e >= c_lo && 16 * c + e <= c_hi) ? v[e] : -INFINITY;
-                    }
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) mx[k] = fmax3(mx[k], v[k], v[8 + k]);
+                    for (int u = 0; u < kGroup; ++u)
+                        if (c0 + u < kChunks) tmem_ld16(trow + 16 * (c0 + u), sb[u]);
                     tmem_wait_ld();
+#pragma unroll
+                    for (int u = 0; u < kGroup; ++u) {
+                        const int c = c0 + u;
+                        if (c >= kChunks) break;
+                        float v[16];
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) v[e] = __uint_as_float(sb[u][e]);
+                        if (mask_chunks & (1u << c)) {
+#pragma unroll
+                            for (int e = 0; e < 16; ++e)
+                                v[e] = (16 * c + e >= c_lo && 16 * c + e <= c_hi) ? v[e] : -INFINITY;
+                        }
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) mx[k] = fmax3(mx[k], v[k], v[8 + k]);
+                    }
                 }
             }
             const float tmax = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
@@ -388,7 +396,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             mbar_arrive(o_free);
             if (row_valid) {
                 const float inv = l > 0.f ? 1.f / l : 0.f;
-                uint4 *dst = reinterpret_cast<uint4 *>(p.out + ((size_t)(t.orow0 + pos) * p.Hq + h) * kD);
+                // the item's output rows, looked up again here rather than kept
+                // live (in registers) through both softmax passes
+                const BandItem te = band_item(p, w);
+                uint4 *dst = reinterpret_cast<uint4 *>(p.out + ((size_t)(te.orow0 + pos) * p.Hq + h) * kD);
 #pragma unroll
                 for (int c = 0; c < kD / 8; ++c) {
                     const uint32_t *src = &o[c / 4][(c % 4) * 8];
@@ -399,7 +410,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                     v.w = pack_bf16x2(__uint_as_float(src[6]) * inv, __uint_as_float(src[7]) * inv);
                     dst[c] = v;
                 }
-                p.lse[(size_t)(t.lrow0 + (long long)h * p.lse_hs + pos)] = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
+                p.lse[(size_t)(te.lrow0 + (long long)h * p.lse_hs + pos)] = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
             }
         }
     }

@@ -16,14 +16,16 @@
 //   a      = 0.1 ln(factor) + 1 (1 when factor <= 1), multiplying cos and sin
 //   rotate-half pairs (i, i + D/2) or interleaved pairs (2i, 2i + 1):
 //   x'_lo = a (x_lo cos(p f'_i) - x_hi sin(p f'_i)),  x'_hi = a (x_hi cos + x_lo sin)
-// v only gets its bias.  The angles are formed and reduced in fp64 (positions
-// up to 131072 times frequencies near 1 leave fp32 with too few bits of phase).
+// v only gets its bias.  The angles are formed and their sine and cosine taken
+// in fp64 (positions up to 131072 times frequencies near 1 leave fp32 with too
+// few bits of phase).
 //
-// Design: HBM-bound (one read and one write of the QKV rows).  A CTA takes one
-// token: 32 threads compute the D/2 cos/sin pairs into shared memory, then all
-// threads move 16-byte chunks of q, k and v, eight pairs (or eight v values)
-// per thread-step.  k and v rows can be written to any row of their outputs
-// (kv_rows), which appends them to a decode cache in the same pass.
+// Design: HBM-bound (one read and one write of the QKV rows).  A CTA takes
+// eight tokens: the D/2 pair frequencies once, one fp64 angle per thread into
+// shared memory, then all threads move 16-byte chunks of q, k and v, eight
+// pairs (or eight v values) per thread-step.  k and v rows can be written to
+// any row of their outputs (kv_rows), which appends them to a decode cache in
+// the same pass.
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -38,11 +40,11 @@ constexpr int kPairs = kD / 2;
 constexpr int kThreads = 256;
 
 struct ProParams {
-    const __nv_bfloat16 *qkv;  // [T, (Hq + 2 Hkv) * D]
+    const __nv_bfloat16 *__restrict__ qkv;  // [T, (Hq + 2 Hkv) * D]
     const float *bias;         // [(Hq + 2 Hkv) * D] or nullptr
     const int *pos;            // [T]
     const int *kv_rows;        // [T] or nullptr (row t)
-    __nv_bfloat16 *q, *k, *v;
+    __nv_bfloat16 *__restrict__ q, *__restrict__ k, *__restrict__ v;
     int T, Hq, Hkv, interleaved;
     int kv_rows_total;         // rows of k / v (a kv_rows entry outside [0, rows) writes nothing)
     double base, factor, L0, beta_fast, beta_slow, attn_factor;
@@ -67,29 +69,20 @@ __device__ __forceinline__ float2 bf2(uint32_t w)
     return __bfloat1622float2(h);
 }
 
-__global__ void __launch_bounds__(kThreads) prologue_kernel(const ProParams p)
+// One 8-pair (or, for v, 8-value) step of token tt's row.
+__device__ __forceinline__ void prologue_step(const ProParams &p, int t, int u, const float *cs, const float *sn)
 {
-    __shared__ float cs[kPairs], sn[kPairs];
-    const int t = blockIdx.x;
     const int width = (p.Hq + 2 * p.Hkv) * kD;
-    if (threadIdx.x < kPairs) {
-        const int i = threadIdx.x;
-        const double ang = fmod((double)p.pos[t] * yarn_freq(p, i), 2.0 * M_PI);
-        double s, c;
-        sincos(ang, &s, &c);
-        cs[i] = (float)(c * p.attn_factor);
-        sn[i] = (float)(s * p.attn_factor);
-    }
-    __syncthreads();
-    const __nv_bfloat16 *row = p.qkv + (size_t)t * width;
+    const int rot_units = (p.Hq + p.Hkv) * (kPairs / 8);
+    const __nv_bfloat16 *__restrict__ row = p.qkv + (size_t)t * width;
     const int kr = p.kv_rows ? p.kv_rows[t] : t;
     const bool kv_ok = kr >= 0 && kr < p.kv_rows_total;
-    // rotated heads (q then k): each step takes 8 pairs of one head
-    const int rot_heads = p.Hq + p.Hkv;
-    for (int u = threadIdx.x; u < rot_heads * (kPairs / 8); u += kThreads) {
+    if (u < rot_units) {
+        // rotated heads (q then k): pairs i0 .. i0 + 7 of head h
         const int h = u / (kPairs / 8), i0 = (u % (kPairs / 8)) * 8;
+        if (h >= p.Hq && !kv_ok) return;
         const int col = h * kD;
-        float xa[8], xb[8];  // the two members of pairs i0 .. i0 + 7
+        float xa[8], xb[8];
         if (!p.interleaved) {
             const uint4 a = *reinterpret_cast<const uint4 *>(row + col + i0);
             const uint4 b = *reinterpret_cast<const uint4 *>(row + col + kPairs + i0);
@@ -122,23 +115,18 @@ __global__ void __launch_bounds__(kThreads) prologue_kernel(const ProParams p)
                 xb[j] += p.bias[col + db];
             }
         }
-        uint32_t oa[4], ob[4], oi[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-            const float c = cs[i0 + j], s = sn[i0 + j];
-            const float ra = xa[j] * c - xb[j] * s;
-            const float rb = xb[j] * c + xa[j] * s;
+            const float c = cs[i0 + j], sv = sn[i0 + j];
+            const float ra = xa[j] * c - xb[j] * sv;
+            const float rb = xb[j] * c + xa[j] * sv;
             xa[j] = ra;
             xb[j] = rb;
         }
-        __nv_bfloat16 *dst;
-        if (h < p.Hq) {
-            dst = p.q + ((size_t)t * p.Hq + h) * kD;
-        } else {
-            if (!kv_ok) continue;
-            dst = p.k + ((size_t)kr * p.Hkv + (h - p.Hq)) * kD;
-        }
+        __nv_bfloat16 *__restrict__ dst =
+            h < p.Hq ? p.q + ((size_t)t * p.Hq + h) * kD : p.k + ((size_t)kr * p.Hkv + (h - p.Hq)) * kD;
         if (!p.interleaved) {
+            uint32_t oa[4], ob[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 oa[j] = pack_bf16x2(xa[2 * j], xa[2 * j + 1]);
@@ -147,16 +135,17 @@ __global__ void __launch_bounds__(kThreads) prologue_kernel(const ProParams p)
             *reinterpret_cast<uint4 *>(dst + i0) = make_uint4(oa[0], oa[1], oa[2], oa[3]);
             *reinterpret_cast<uint4 *>(dst + kPairs + i0) = make_uint4(ob[0], ob[1], ob[2], ob[3]);
         } else {
+            uint32_t oi[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) oi[j] = pack_bf16x2(xa[j], xb[j]);
             *reinterpret_cast<uint4 *>(dst + 2 * i0) = make_uint4(oi[0], oi[1], oi[2], oi[3]);
             *reinterpret_cast<uint4 *>(dst + 2 * i0 + 8) = make_uint4(oi[4], oi[5], oi[6], oi[7]);
         }
-    }
-    // v: bias only, 8 values per step
-    if (!kv_ok) return;
-    for (int u = threadIdx.x; u < p.Hkv * (kD / 8); u += kThreads) {
-        const int h = u / (kD / 8), d0 = (u % (kD / 8)) * 8;
+    } else {
+        // v: bias only, values d0 .. d0 + 7 of head h
+        if (!kv_ok) return;
+        const int vu = u - rot_units;
+        const int h = vu / (kD / 8), d0 = (vu % (kD / 8)) * 8;
         const int col = (p.Hq + p.Hkv + h) * kD + d0;
         const uint4 a = *reinterpret_cast<const uint4 *>(row + col);
         const uint32_t w[4] = {a.x, a.y, a.z, a.w};
@@ -171,6 +160,36 @@ __global__ void __launch_bounds__(kThreads) prologue_kernel(const ProParams p)
             o[j] = pack_bf16x2(f.x, f.y);
         }
         *reinterpret_cast<uint4 *>(p.v + ((size_t)kr * p.Hkv + h) * kD + d0) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+}
+
+// kTok tokens per CTA: the pair frequencies once, then one angle per thread
+// (kTok x 32 = 256), then every thread moves 16-byte chunks of the tokens' rows.
+constexpr int kTok = kThreads / kPairs;
+
+__global__ void __launch_bounds__(kThreads) prologue_kernel(const ProParams p)
+{
+    __shared__ double freq[kPairs];
+    __shared__ float cs[kTok][kPairs], sn[kTok][kPairs];
+    const int t0 = blockIdx.x * kTok;
+    if (threadIdx.x < kPairs) freq[threadIdx.x] = yarn_freq(p, threadIdx.x);
+    __syncthreads();
+    {
+        const int tt = threadIdx.x / kPairs, i = threadIdx.x % kPairs;
+        if (t0 + tt < p.T) {
+            double sv, cv;
+            sincos((double)p.pos[t0 + tt] * freq[i], &sv, &cv);
+            cs[tt][i] = (float)(cv * p.attn_factor);
+            sn[tt][i] = (float)(sv * p.attn_factor);
+        }
+    }
+    __syncthreads();
+    const int units = (p.Hq + p.Hkv) * (kPairs / 8) + p.Hkv * (kD / 8);
+    const int ntok = min(kTok, p.T - t0);
+#pragma unroll 2
+    for (int x = threadIdx.x; x < ntok * units; x += kThreads) {
+        const int tt = x / units;
+        prologue_step(p, t0 + tt, x - tt * units, cs[tt], sn[tt]);
     }
 }
 
@@ -199,7 +218,7 @@ cudaError_t launch_qkv_prologue(const void *qkv, const float *bias, const int *p
     p.beta_fast = r.beta_fast;
     p.beta_slow = r.beta_slow;
     p.attn_factor = r.factor > 1.0 ? 0.1 * log(r.factor) + 1.0 : 1.0;
-    prologue_kernel<<<T, kThreads, 0, st>>>(p);
+    prologue_kernel<<<(T + kTok - 1) / kTok, kThreads, 0, st>>>(p);
     return cudaGetLastError();
 }
 

@@ -382,7 +382,12 @@ int attn_sink_decode_fp8(const void *q, const void *k_cache, const void *v_cache
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(k_scale) || !aligned16(v_scale) ||
         !aligned16(out) || !aligned16(lse) || !aligned16(sinks) || !aligned16(seqlens))
         return ATTN_SINK_ERR_MISALIGNED;
-    const DecodeShape s = decode_shape(B, Lmax, Hq, Hkv, D, window, scale, num_splits);
+    DecodeShape s = decode_shape(B, Lmax, Hq, Hkv, D, window, scale, num_splits);
+    // the e4m3 kernel's tiles are 128 keys: chunks of whole tiles (never more
+    // splits than the bf16 rule, so the same workspace size suffices)
+    const int lvis = window > 0 ? (window < Lmax ? window : Lmax) : Lmax;
+    s.chunk = (s.chunk + 127) / 128 * 128;
+    s.splits = (lvis + s.chunk - 1) / s.chunk;
     if (!decode_bf16_supported(s)) return ATTN_SINK_ERR_UNSUPPORTED;
     const size_t need = decode_ws_bytes(s);
     if (need > 0 && (!workspace || ws_bytes < need)) return ATTN_SINK_ERR_WORKSPACE;

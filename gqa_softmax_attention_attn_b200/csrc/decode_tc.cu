@@ -41,11 +41,10 @@ namespace attn_sink {
 namespace {
 
 constexpr int kD = 64;
-constexpr int kT = 64;          // keys per tile
 // K/V ring stages: the loads in flight per SM must cover the HBM latency at
 // full bandwidth, so the e4m3 ring (half the bytes per stage) is deeper
 #ifndef ATTN_SINK_DEC_FP8_STAGES
-#define ATTN_SINK_DEC_FP8_STAGES 6
+#define ATTN_SINK_DEC_FP8_STAGES 3
 #endif
 constexpr int kThreads = 160;  // warp 0 producer, warps 1-4 consumers
 constexpr float kLog2e = 1.4426950408889634f;
@@ -54,14 +53,18 @@ constexpr float kLn2 = 0.6931471805599453f;
 // Shared-memory layout; kFp8: K/V cached as e4m3 (one byte per element).
 template <bool kFp8>
 struct DecLayout {
+    // keys per tile: the e4m3 tile spans twice the keys, so a tile's bytes (and
+    // its fixed costs: TMA issue, barrier round trips) are those of a bf16 tile
+    static constexpr int kT = kFp8 ? 128 : 64;
+    static constexpr int kSlices = kT / 64;  // 16-key slices per consumer warp and tile
     static constexpr int kNS = kFp8 ? ATTN_SINK_DEC_FP8_STAGES : 4;
     static constexpr int kRowBytes = kFp8 ? kD : kD * 2;  // one cached K or V row
     static constexpr int kTileBytes = kT * kRowBytes;
     static constexpr int kStageBytes = 2 * kTileBytes;  // K and V
-    // e4m3 only: each consumer warp's 16 keys of V as f16, 128-byte swizzled
+    // e4m3 only: each consumer warp's keys of V as f16, 128-byte swizzled
     // (K is read straight from the e4m3 tile)
     static constexpr int kOffStaging = kNS * kStageBytes;
-    static constexpr int kWarpStaging = 16 * kD * 2;
+    static constexpr int kWarpStaging = kSlices * 16 * kD * 2;
     static constexpr int kOffBar = kOffStaging + (kFp8 ? 4 * kWarpStaging : 0);
     static constexpr int kSmemBytes = kOffBar + 2 * kNS * 8 + 16 + 1024;
     // the final reduction reuses [0, kOffBar): 4 warps x 16 rows x 66 floats
@@ -150,6 +153,8 @@ __global__ void __launch_bounds__(kThreads)
                      const DecodeParams p)
 {
     using L = DecLayout<kFp8>;
+    constexpr int kT = L::kT;
+    static_assert(!(kPaged && kFp8), "paged caches are bf16 only");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     constexpr int kNS = L::kNS;
@@ -296,25 +301,31 @@ __global__ void __launch_bounds__(kThreads)
                 ok = false;
                 break;
             }
-            uint32_t kt = sbase + st * L::kStageBytes, vt = kt + L::kTileBytes;
+            const uint32_t kt = sbase + st * L::kStageBytes;
+            uint32_t vt = kt + L::kTileBytes;
             int rw = 16 * w;  // first row of this warp's 16 keys in the tile it reads
-            uint4 k8r[2];  // e4m3 only: this lane's 16 bytes of key row (16w + 8nt + gr), nt = 0, 1
+            uint4 k8r[L::kSlices][2];  // e4m3 only: this lane's 16 bytes of key row (16w + 64 sl + 8nt + gr)
             if (kFp8) {
-                // this warp's 16 keys: K's fragments straight from the e4m3 tile,
-                // V widened to f16 into the warp's own staging (the layout the
-                // transposing ldmatrix reads); then the raw stage is free again
-                const uint8_t *k8 = smem + st * L::kStageBytes + 16 * w * L::kRowBytes;
+                // this warp's keys (16w + 64 sl .. + 15 for each slice sl): K's
+                // fragments straight from the e4m3 tile, V widened to f16 into the
+                // warp's own staging (the layout the transposing ldmatrix reads);
+                // then the raw stage is free again
+                const uint8_t *k8 = smem + st * L::kStageBytes;
                 const uint8_t *v8 = k8 + L::kTileBytes;
                 uint8_t *vs = smem + L::kOffStaging + w * L::kWarpStaging;
 #pragma unroll
-                for (int nt = 0; nt < 2; ++nt)
-                    k8r[nt] = *reinterpret_cast<const uint4 *>(k8 + (8 * nt + gr) * L::kRowBytes + 16 * tq);
+                for (int sl = 0; sl < L::kSlices; ++sl)
 #pragma unroll
-                for (int it = 0; it < 2; ++it) {
+                    for (int nt = 0; nt < 2; ++nt)
+                        k8r[sl][nt] = *reinterpret_cast<const uint4 *>(
+                            k8 + (64 * sl + 16 * w + 8 * nt + gr) * L::kRowBytes + 16 * tq);
+#pragma unroll
+                for (int it = 0; it < 2 * L::kSlices; ++it) {
                     const int i = lane + 32 * it;
-                    const int row = i >> 2, ch = i & 3;  // 16 rows x 4 chunks of 16 values
+                    const int row = i >> 2, ch = i & 3;  // 16 rows per slice x 4 chunks of 16 values
+                    const int trow_ = 64 * (row >> 4) + 16 * w + (row & 15);
                     uint4 lo, hi;
-                    e4m3x16_to_f16(*reinterpret_cast<const uint4 *>(v8 + row * L::kRowBytes + ch * 16), lo, hi);
+                    e4m3x16_to_f16(*reinterpret_cast<const uint4 *>(v8 + trow_ * L::kRowBytes + ch * 16), lo, hi);
                     *reinterpret_cast<uint4 *>(vs + swz(row, 2 * ch)) = lo;
                     *reinterpret_cast<uint4 *>(vs + swz(row, 2 * ch + 1)) = hi;
                 }
@@ -323,14 +334,16 @@ __global__ void __launch_bounds__(kThreads)
                 vt = smem_u32(vs);
                 rw = 0;
             }
-            const int key0 = kbeg + j * kT + 16 * w;  // first key of this warp's slice
+#pragma unroll
+            for (int sl = 0; sl < L::kSlices; ++sl) {
+            const int key0 = kbeg + j * kT + 64 * sl + 16 * w;  // first key of this warp's slice
             // ---- S = Q K^T for 16 keys: two n-tiles of 8 keys
             float s[2][4];
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt) {
                 s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
                 if (kFp8) {
-                    const uint32_t w4[4] = {k8r[nt].x, k8r[nt].y, k8r[nt].z, k8r[nt].w};
+                    const uint32_t w4[4] = {k8r[sl][nt].x, k8r[sl][nt].y, k8r[sl][nt].z, k8r[sl][nt].w};
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         mma16816_f16(s[nt], qa[kk], e4m3x2_to_f16x2(w4[kk]), e4m3x2_to_f16x2(w4[kk] >> 16));
@@ -408,7 +421,7 @@ __global__ void __launch_bounds__(kThreads)
             // rows of V outside [lo, kend) are zeroed in the operand (cache rows
             // beyond the sequence may hold anything)
             const bool tail = __any_sync(0xffffffffu, key0 + 15 >= kend || key0 < lo);
-            const int vrow = rw + ((lane >> 3) & 1) * 8 + (lane & 7);
+            const int vrow = rw + 16 * sl + ((lane >> 3) & 1) * 8 + (lane & 7);
 #pragma unroll
             for (int jn = 0; jn < 8; jn += 2) {
                 uint32_t b0, b1, b2, b3;
@@ -432,6 +445,7 @@ __global__ void __launch_bounds__(kThreads)
                     mma16816(o[jn + 1], pa, b2, b3);
                 }
             }
+            }  // slices
             __syncwarp();
             if (!kFp8 && lane == 0) mbar_arrive(&empty[st]);
         }
@@ -521,6 +535,7 @@ cudaError_t launch_decode_bf16(const void *q, const void *kc, const void *vc, co
     p.k_scale = k_scale;
     p.v_scale = v_scale;
     p.sh = s;
+    const int kT = fp8 ? DecLayout<true>::kT : DecLayout<false>::kT;
     p.box_rows = s.page_size > 0 && s.page_size < kT ? s.page_size : kT;
     p.B = s.B;
     p.Lmax = s.Lmax;
@@ -563,9 +578,8 @@ cudaError_t launch_decode_bf16(const void *q, const void *kc, const void *vc, co
     };
     constexpr int sb = DecLayout<false>::kSmemBytes, s8 = DecLayout<true>::kSmemBytes;
     if (fp8) {
-        if (p.G > 8)
-            return paged ? launch(decode_tc_kernel<true, true, true>, s8) : launch(decode_tc_kernel<true, false, true>, s8);
-        return paged ? launch(decode_tc_kernel<false, true, true>, s8) : launch(decode_tc_kernel<false, false, true>, s8);
+        if (paged) return cudaErrorInvalidValue;  // e4m3 caches are contiguous only
+        return p.G > 8 ? launch(decode_tc_kernel<true, false, true>, s8) : launch(decode_tc_kernel<false, false, true>, s8);
     }
     if (p.G > 8)
         return paged ? launch(decode_tc_kernel<true, true, false>, sb) : launch(decode_tc_kernel<true, false, false>, sb);

@@ -12,27 +12,30 @@
 // see keys [pos0 + off - W + 1, pos0 + off + P - 1]: W + P - 1 keys, 143 for
 // W = 128 and P = 16.  So one K/V tile of KN >= W + P - 1 rows (144) holds
 // every key of the item, and the item is ONE score MMA (M = 128, N = KN), one
-// exact softmax (no running maximum, no rescale), and one P.V MMA -- instead
-// of a chain of online-softmax round trips over narrow tiles.
-//  * The grid has one CTA per item; two CTAs run per SM (KN <= 144 plus 64 TMEM
-//    columns in a 256-column allocation each; wider bands take the online-
-//    softmax kernel of fwd_tc.cu) and take over the items of CTAs that
-//    have not started yet through cluster launch control.
+// exact softmax (no running maximum, no rescale), and one P.V MMA.
+//  * One CTA per SM (all 512 TMEM columns), two softmax warpgroups that take
+//    alternate items, so one item's softmax overlaps the other's MMAs, loads
+//    and epilogue.  The grid has one CTA per item; running CTAs take over the
+//    items of CTAs that have not started through cluster launch control.
 //  * Warp 0: TMA producer.  Q (16 KB) and the K and V tiles (KN x 128 B each,
 //    starting at a negative row where the band reaches before key 0: the TMA
-//    fills rows outside the tensor with zeros) are double-buffered, so the
-//    next item's operands land while this one computes.
-//  * Warp 1: the MMA issue loop, run by the whole warp with one elected lane
-//    issuing: S = Q K^T into TMEM; after the softmax, O = P V with P (bf16)
-//    read from TMEM where it overwrote S.
-//  * Warps 2-5: one thread per row.  Pass 1 reads S from TMEM 16 columns at a
-//    time for the row maximum; pass 2 reads it again, takes exp2 of the
-//    log2-scaled logits against max(sink, row max), sums them, and writes P
-//    over S.  Columns outside the row's band are masked only in the 16-column
-//    chunks where some row of the warp needs it.  Then the epilogue: O / l
-//    and lse = m + log2(l) (natural units on output).
+//    fills rows outside the tensor with zeros) in four stages, so items ahead
+//    of the two being computed are in flight.
+//  * Warp 1: the MMA issue loop (whole warp, one elected lane issuing):
+//    S = Q K^T of item r + 2 goes right after P.V of item r, into the TMEM
+//    half of item r's warpgroup (the tensor pipe runs them in order).
+//  * Warps 4-7 and 8-11 (registers moved to them from warpgroup 0 with
+//    setmaxnreg), one thread per row: the whole score row (KN columns)
+//    comes out of TMEM in one go into registers; masks only on the 16-column
+//    chunks where some row of the warp needs them; m = max(sink, row max);
+//    P = exp2(S C - m) as bf16 over S; l.  Epilogue: O / l written into the
+//    item's K buffer (its Q buffer for narrow bands; either is dead once S is
+//    done) in the 128-byte-swizzled layout of an output box, and stored with
+//    one TMA tensor store (a box that would run into the next packed sequence
+//    is stored row by row instead); lse row by row.
 //  * Every wait is bounded; on expiry the CTA raises a status bit, waits
-//    (bounded) for its own TMA loads and MMAs, frees tensor memory and exits.
+//    (bounded) for its own TMA loads, stores and MMAs, frees tensor memory and
+//    exits.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <math.h>
@@ -45,33 +48,44 @@ namespace {
 
 constexpr int kM = 128;
 constexpr int kD = 64;
-constexpr int kThreads = 192;  // producer, MMA, 4 softmax warps
+constexpr int kThreads = 384;  // warpgroup 0: producer, MMA (2 warps idle); warpgroups 1, 2: softmax
+// Registers: launched at 168 per thread (384 threads, one CTA per SM); warpgroup
+// 0 then gives up all but 56 and the softmax warpgroups take 224 each, so the
+// score row of a thread stays in registers: 128 x 56 + 256 x 224 = 384 x 168.
+// (Each SM sub-partition holds one warp of every warpgroup: 56 + 2 x 224 fits
+// its 16K registers as 3 x 168 does.)
+constexpr int kRegsLaunch = 168, kRegsCtl = 56, kRegsSoftmax = 224;
+static_assert(128 * kRegsCtl + 256 * kRegsSoftmax <= kThreads * kRegsLaunch, "register split");
+constexpr int kNS = 4;         // Q/K/V stages
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
-constexpr int kTmO = 192;        // O accumulator columns [192, 256)
-constexpr int kTmemCols = 256;   // S (KN <= 144 columns) + O
-constexpr int kCtasPerSm = 2;
+constexpr int kTmemCols = 512;  // warpgroup w: S at [256 w, 256 w + KN), O at [256 w + 192, 256 w + 256)
+constexpr int kTmO = 192;
 
 template <int KN>
 struct BandCfg {
     static_assert(KN % 16 == 0 && KN >= 16 && KN <= 144, "KN: a multiple of 16 up to 144");
     static constexpr int kQBytes = kM * kD * 2;
     static constexpr int kKVBytes = KN * kD * 2;
-    static constexpr int kOffQ = 0;  // [2]
-    static constexpr int kOffK = 2 * kQBytes;  // [2]
-    static constexpr int kOffV = kOffK + 2 * kKVBytes;  // [2]
-    static constexpr int kOffBar = kOffV + 2 * kKVBytes;
-    // q_full[2] q_empty[2] k_full[2] k_empty[2] v_full[2] v_empty[2] s_full p_full o_done o_free drain
-    // item_full[4] item_empty[4] clc[kClcDepth]
-    static constexpr int kNumBar = 12 + 5 + 8 + kClcDepth;
+    static constexpr int kOffQ = 0;                       // [kNS]
+    static constexpr int kOffK = kNS * kQBytes;           // [kNS]
+    static constexpr int kOffV = kOffK + kNS * kKVBytes;  // [kNS]
+    static constexpr int kOffBar = kOffV + kNS * kKVBytes;
+    // The item's O is staged in its K buffer when that holds 16 KB (K is dead
+    // once S is done and is only needed again two items of this warpgroup
+    // later), else in its Q buffer.
+    static constexpr bool kStageInK = kKVBytes >= kQBytes;
+    // q_full q_empty k_full k_empty v_full v_empty [kNS each]; s_full p_full o_done o_free stg_ready [2 each];
+    // drain; item_full[4] item_empty[4]; clc[kClcDepth]
+    static constexpr int kNumBar = 6 * kNS + 10 + 1 + 8 + kClcDepth;
     static constexpr int kOffMisc = (kOffBar + kNumBar * 8 + 15) / 16 * 16;
     // tmem slot (+0), abort flag (+4), item ring (+16), launch-control responses (+32, 16 bytes each)
     static_assert(32 + 16 * kClcDepth <= 128, "misc area");
     static constexpr int kSmemUsed = kOffMisc + 128 + 1024;  // + slack for 1024-byte alignment
-    // at least a third of the SM's 228 KB, so no third CTA (whose tensor-memory
-    // allocation would have to wait for one of the two others) lands on an SM
-    static constexpr int kSmemBytes = kSmemUsed < 80 * 1024 ? 80 * 1024 : kSmemUsed;
-    static_assert(2 * kSmemBytes <= 227 * 1024, "two CTAs per SM");
+    // more than half the SM's shared memory even for narrow bands: a second
+    // CTA on the SM would only wait for the first one's tensor memory
+    static constexpr int kSmemBytes = kSmemUsed < 116 * 1024 ? 116 * 1024 : kSmemUsed;
+    static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
 
 struct BandParams {
@@ -90,12 +104,12 @@ struct BandParams {
 };
 
 struct BandItem {
-    int pos0, h0, b, js;  // first position, first head, batch, first key of the K/V tile (in the sequence)
-    int Lq, Lk;           // the sequence's query and key counts
-    int qrow0, krow0, tb; // tensor-map rows of its position 0 / key 0, outer coordinate
-    long long orow0;      // output row of its position 0
-    long long lrow0;      // lse index of (head 0, position 0)
-    bool empty;           // past the end of a shorter packed sequence
+    int pos0, h0, b, js;   // first position, first head, batch, first key of the K/V tile (in the sequence)
+    int Lq, Lk;            // the sequence's query and key counts
+    int qrow0, krow0, tb;  // tensor-map rows of its position 0 / key 0, outer coordinate
+    long long orow0;       // output row of its position 0
+    long long lrow0;       // lse index of (head 0, position 0)
+    bool empty;            // past the end of a shorter packed sequence
 };
 
 // Item i: head tiles fastest, then position tiles, then batches, so the CTAs
@@ -125,50 +139,58 @@ __device__ __forceinline__ BandItem band_item(const BandParams &p, int i)
 __device__ __forceinline__ bool wait_noabort(uint64_t *bar, uint32_t parity, unsigned *status, long long tmo)
 {
     int never = 0;
-    return mbar_wait(bar, parity, &never, status, tmo > 1000000000LL ? tmo : 1000000000LL);
+    return mbar_wait<false>(bar, parity, &never, status, tmo > 1000000000LL ? tmo : 1000000000LL);
 }
 
 template <int KN>
-__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+__global__ void __launch_bounds__(kThreads, 1)
     fwd_band_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                    const __grid_constant__ CUtensorMap tmV, const BandParams p)
+                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                    const BandParams p)
 {
     using Cfg = BandCfg<KN>;
     constexpr int kChunks = KN / 16;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kOffBar);
-    uint64_t *q_full = bars, *q_empty = bars + 2;
-    uint64_t *k_full = bars + 4, *k_empty = bars + 6;
-    uint64_t *v_full = bars + 8, *v_empty = bars + 10;
-    uint64_t *s_full = bars + 12, *p_full = bars + 13, *o_done = bars + 14, *o_free = bars + 15;
-    uint64_t *drain = bars + 16;
-    uint64_t *item_full = bars + 17, *item_empty = bars + 21;
-    uint64_t *clc_bar = bars + 25;  // [kClcDepth]
+    uint64_t *q_full = bars, *q_empty = bars + kNS;
+    uint64_t *k_full = bars + 2 * kNS, *k_empty = bars + 3 * kNS;
+    uint64_t *v_full = bars + 4 * kNS, *v_empty = bars + 5 * kNS;
+    uint64_t *s_full = bars + 6 * kNS;  // [2]: one per warpgroup
+    uint64_t *p_full = s_full + 2;      // [2]
+    uint64_t *o_done = p_full + 2;      // [2]
+    uint64_t *o_free = o_done + 2;      // [2]
+    uint64_t *stg_ready = o_free + 2;   // [2]: every row of the item staged for its tensor store
+    uint64_t *drain = stg_ready + 2;
+    uint64_t *item_full = drain + 1, *item_empty = item_full + 4;
+    uint64_t *clc_bar = item_empty + 4;  // [kClcDepth]
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Cfg::kOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Cfg::kOffMisc + 4);
     volatile int *ring = reinterpret_cast<volatile int *>(smem + Cfg::kOffMisc + 16);
-    void *clc_resp = smem + Cfg::kOffMisc + 32;
+    uint8_t *clc_resp = smem + Cfg::kOffMisc + 32;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < kNS; ++s) {
             mbar_init(&q_full[s], 1);
-            mbar_init(&q_empty[s], 1);
+            mbar_init(&q_empty[s], 1);  // S, or the epilogue once the O store has read the buffer
             mbar_init(&k_full[s], 1);
             mbar_init(&k_empty[s], 1);
             mbar_init(&v_full[s], 1);
             mbar_init(&v_empty[s], 1);
         }
-        mbar_init(s_full, 1);
-        mbar_init(p_full, 128);
-        mbar_init(o_done, 1);
-        mbar_init(o_free, 128);
+        for (int w = 0; w < 2; ++w) {
+            mbar_init(&s_full[w], 1);
+            mbar_init(&p_full[w], 128);
+            mbar_init(&o_done[w], 1);
+            mbar_init(&o_free[w], 128);
+            mbar_init(&stg_ready[w], 128);
+        }
         mbar_init(drain, 1);
         for (int r = 0; r < 4; ++r) {
             mbar_init(&item_full[r], 1);
-            mbar_init(&item_empty[r], 5);  // the MMA warp and the four softmax warps
+            mbar_init(&item_empty[r], 5);  // the MMA warp and the four warps of the item's warpgroup
         }
         for (int d = 0; d < kClcDepth; ++d) mbar_init(&clc_bar[d], 1);
         *abort_flag = 0;
@@ -185,9 +207,16 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 
     // r-th item of this CTA: its own (blockIdx.x), then those of the CTAs whose
     // launch it cancels (kClcDepth requests kept in flight); published in a
-    // 4-slot ring.
-    // Items past the end of a shorter packed sequence are passed over here.
-    ClcQueue<kClcDepth> clc{clc_bar, reinterpret_cast<uint8_t *>(clc_resp)};
+    // 4-slot ring, and -1 twice at the end (once for each warpgroup).  Items
+    // past the end of a shorter packed sequence are passed over here.
+    ClcQueue<kClcDepth, false> clc{clc_bar, clc_resp};
+    auto publish = [&](int r, int w) -> bool {
+        const int sl = r & 3;
+        if (!mbar_wait<false>(&item_empty[sl], ((r >> 2) & 1u) ^ 1u, abort_flag, p.status, p.timeout_ns)) return false;
+        ring[sl] = w;
+        mbar_arrive(&item_full[sl]);
+        return true;
+    };
     auto producer_item = [&](int r) -> int {
         int w = r == 0 ? (int)blockIdx.x : clc.next(abort_flag, p.status, p.timeout_ns);
         clc.fill();  // keep kClcDepth requests in flight
@@ -196,15 +225,13 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             clc.fill();
         }
         if (clc.failed) return -1;
-        const int sl = r & 3;
-        if (!mbar_wait(&item_empty[sl], ((r >> 2) & 1u) ^ 1u, abort_flag, p.status, p.timeout_ns)) return -1;
-        ring[sl] = w;
-        mbar_arrive(&item_full[sl]);
+        if (!publish(r, w)) return -1;
+        if (w < 0) publish(r + 1, -1);
         return w;
     };
     auto consumer_item = [&](int r) -> int {
         const int sl = r & 3;
-        if (!__all_sync(0xffffffffu, mbar_wait(&item_full[sl], (r >> 2) & 1u, abort_flag, p.status, p.timeout_ns)))
+        if (!__all_sync(0xffffffffu, mbar_wait<false>(&item_full[sl], (r >> 2) & 1u, abort_flag, p.status, p.timeout_ns)))
             return -1;
         const int w = ring[sl];
         __syncwarp();
@@ -212,91 +239,120 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         return w;
     };
 
+    if (warp < 4) {
+    regs_release<kRegsCtl>();  // the whole warpgroup; warps 2 and 3 have no role
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             tma_prefetch_desc(&tmQ);
             tma_prefetch_desc(&tmK);
             tma_prefetch_desc(&tmV);
-            uint32_t issued[6] = {0, 0, 0, 0, 0, 0};  // q, k, v loads per stage
+            tma_prefetch_desc(&tmO);
+            uint32_t nq = 0, nk = 0, nv = 0;  // loads issued (the stage of load n is n % kNS)
             int r = 0;
             for (int w = producer_item(0); w >= 0; w = producer_item(++r)) {
                 const BandItem t = band_item(p, w);
-                const int st = r & 1;
-                const uint32_t ph = ((r >> 1) & 1u) ^ 1u;
+                const int st = r % kNS;
+                const uint32_t ph = ((r / kNS) & 1u) ^ 1u;
                 const int g = t.h0 / p.G;
-                if (!mbar_wait(&q_empty[st], ph, abort_flag, p.status, p.timeout_ns)) break;
+                if (!mbar_wait<false>(&q_empty[st], ph, abort_flag, p.status, p.timeout_ns)) break;
                 mbar_arrive_expect_tx(&q_full[st], Cfg::kQBytes);
                 tma_load_4d(smem + Cfg::kOffQ + st * Cfg::kQBytes, &tmQ, 0, t.h0, t.qrow0 + t.pos0, t.tb,
                             &q_full[st]);
-                ++issued[st];
-                if (!mbar_wait(&k_empty[st], ph, abort_flag, p.status, p.timeout_ns)) break;
+                ++nq;
+                if (!mbar_wait<false>(&k_empty[st], ph, abort_flag, p.status, p.timeout_ns)) break;
                 mbar_arrive_expect_tx(&k_full[st], Cfg::kKVBytes);
                 tma_load_4d(smem + Cfg::kOffK + st * Cfg::kKVBytes, &tmK, 0, g, t.krow0 + t.js, t.tb, &k_full[st]);
-                ++issued[2 + st];
-                if (!mbar_wait(&v_empty[st], ph, abort_flag, p.status, p.timeout_ns)) break;
+                ++nk;
+                if (!mbar_wait<false>(&v_empty[st], ph, abort_flag, p.status, p.timeout_ns)) break;
                 mbar_arrive_expect_tx(&v_full[st], Cfg::kKVBytes);
                 tma_load_4d(smem + Cfg::kOffV + st * Cfg::kKVBytes, &tmV, 0, g, t.krow0 + t.js, t.tb, &v_full[st]);
-                ++issued[4 + st];
+                ++nv;
             }
             // every load issued, and a launch-control request in flight, lands before the CTA exits
             clc.drain(p.status, p.timeout_ns);
-            for (int s = 0; s < 2; ++s) {
-                if (issued[s]) wait_noabort(&q_full[s], (issued[s] - 1) & 1u, p.status, p.timeout_ns);
-                if (issued[2 + s]) wait_noabort(&k_full[s], (issued[2 + s] - 1) & 1u, p.status, p.timeout_ns);
-                if (issued[4 + s]) wait_noabort(&v_full[s], (issued[4 + s] - 1) & 1u, p.status, p.timeout_ns);
-            }
+            for (uint32_t n = nq > kNS ? nq - kNS : 0; n < nq; ++n)
+                wait_noabort(&q_full[n % kNS], (n / kNS) & 1u, p.status, p.timeout_ns);
+            for (uint32_t n = nk > kNS ? nk - kNS : 0; n < nk; ++n)
+                wait_noabort(&k_full[n % kNS], (n / kNS) & 1u, p.status, p.timeout_ns);
+            for (uint32_t n = nv > kNS ? nv - kNS : 0; n < nv; ++n)
+                wait_noabort(&v_full[n % kNS], (n / kNS) & 1u, p.status, p.timeout_ns);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         const uint32_t id_s = idesc_bf16_f32(kM, KN, 0);
         const uint32_t id_pv = idesc_bf16_f32(kM, kD, 1);
         auto wait_all = [&](uint64_t *bar, uint32_t parity) {
-            return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, p.status, p.timeout_ns));
+            return __all_sync(0xffffffffu, mbar_wait<false>(bar, parity, abort_flag, p.status, p.timeout_ns));
         };
-        for (int r = 0, w = consumer_item(0); w >= 0; w = consumer_item(++r)) {
-            const int st = r & 1;
-            const uint32_t ph = (r >> 1) & 1u;
-            if (!wait_all(&q_full[st], ph) || !wait_all(&k_full[st], ph)) break;
+        // S = Q K^T of item r into its warpgroup's TMEM half; false on abort
+        auto issue_s = [&](int r) -> bool {
+            const int st = r % kNS;
+            const uint32_t ph = (r / kNS) & 1u;
+            if (!wait_all(&q_full[st], ph) || !wait_all(&k_full[st], ph)) return false;
             tc_fence_after();
             const uint32_t qa = smem_u32(smem + Cfg::kOffQ + st * Cfg::kQBytes);
             const uint32_t kb = smem_u32(smem + Cfg::kOffK + st * Cfg::kKVBytes);
             if (elect_one()) {
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk)
-                    mma_ss(tmem, smem_desc_sw128(qa + kk * 32, 16, 1024), smem_desc_sw128(kb + kk * 32, 16, 1024),
-                           id_s, kk > 0 ? 1u : 0u);
-                mma_commit(s_full);
-                mma_commit(&k_empty[st]);
-                mma_commit(&q_empty[st]);
+                    mma_ss(tmem + 256 * (r & 1), smem_desc_sw128(qa + kk * 32, 16, 1024),
+                           smem_desc_sw128(kb + kk * 32, 16, 1024), id_s, kk > 0 ? 1u : 0u);
+                mma_commit(&s_full[r & 1]);
+                mma_commit(Cfg::kStageInK ? &q_empty[st] : &k_empty[st]);  // the other one stages O
             }
             __syncwarp();
-            // O = P V once the softmax has written P, V has landed and the
-            // previous item's epilogue has read O out
-            if (!wait_all(p_full, r & 1u) || !wait_all(&v_full[st], ph) || !wait_all(o_free, (r & 1u) ^ 1u)) break;
+            return true;
+        };
+        // O = P V of item r, once its warpgroup has written P, V has landed and
+        // the warpgroup's previous epilogue has read its O out
+        auto issue_pv = [&](int r) -> bool {
+            const int st = r % kNS, wg = r & 1;
+            if (!wait_all(&p_full[wg], (r >> 1) & 1u) || !wait_all(&v_full[st], (r / kNS) & 1u) ||
+                !wait_all(&o_free[wg], ((r >> 1) & 1u) ^ 1u))
+                return false;
             tc_fence_after();
             const uint32_t vb = smem_u32(smem + Cfg::kOffV + st * Cfg::kKVBytes);
             if (elect_one()) {
 #pragma unroll
                 for (int kk = 0; kk < kChunks; ++kk)
-                    mma_ts(tmem + kTmO, tmem + kk * 8, smem_desc_sw128(vb + kk * 2048, KN * 128, 1024), id_pv,
-                           kk > 0 ? 1u : 0u);
-                mma_commit(o_done);
+                    mma_ts(tmem + 256 * wg + kTmO, tmem + 256 * wg + kk * 8,
+                           smem_desc_sw128(vb + kk * 2048, KN * 128, 1024), id_pv, kk > 0 ? 1u : 0u);
+                mma_commit(&o_done[wg]);
                 mma_commit(&v_empty[st]);
             }
             __syncwarp();
+            return true;
+        };
+        int w_cur = consumer_item(0);
+        int w_nxt = w_cur >= 0 ? consumer_item(1) : -1;
+        bool ok = (w_cur < 0 || issue_s(0)) && (w_nxt < 0 || issue_s(1));
+        for (int r = 0; ok && w_cur >= 0; ++r) {
+            if (!issue_pv(r)) break;
+            const int w2 = w_nxt >= 0 ? consumer_item(r + 2) : -1;
+            if (w2 >= 0 && !issue_s(r + 2)) break;
+            w_cur = w_nxt;
+            w_nxt = w2;
         }
         if (elect_one()) mma_commit(drain);
         __syncwarp();
         wait_noabort(drain, 0, p.status, p.timeout_ns);
+    }
     } else {
+        regs_claim<kRegsSoftmax>();
         // ------------------------------------------------------------ softmax + epilogue
-        const int quad = warp & 3;
+        const int wg = (warp - 4) >> 2;  // softmax warpgroup: items r with r % 2 == wg
+        const int quad = warp & 3;       // TMEM lane quadrant of this warp
         const int row = quad * 32 + lane;
-        const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
+        const uint32_t trow = tmem + 256 * wg + ((uint32_t)(quad * 32) << 16);
         const float C = p.c_log2;
-        for (int r = 0, w = consumer_item(0); w >= 0; w = consumer_item(++r)) {
+        const bool storer = (warp == 4 + 4 * wg) && lane == 0;  // issues the warpgroup's tensor stores
+        bool stores_issued = false;
+        for (int r = wg;; r += 2) {
+            const int w = consumer_item(r);
+            if (w < 0) break;
             const BandItem t = band_item(p, w);
+            const int st = r % kNS;
             const int dp = row / p.Gp;
             const int pos = t.pos0 + dp;
             const int h = t.h0 + row % p.Gp;
@@ -305,114 +361,116 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             // columns c of the tile (key js + c) this row sees: c in [c_lo, c_hi]
             const int c_lo = max(dp, -t.js);
             const int c_hi = row_valid ? min(dp + p.window - 1, t.Lk - 1 - t.js) : -1;
-            if (!__all_sync(0xffffffffu, mbar_wait(s_full, r & 1u, abort_flag, p.status, p.timeout_ns))) break;
+            if (!__all_sync(0xffffffffu, mbar_wait<false>(&s_full[wg], (r >> 1) & 1u, abort_flag, p.status, p.timeout_ns)))
+                break;
             tc_fence_after();
-            // a chunk needs element masks when some row of the warp does not see all of it
-            uint32_t mask_chunks = 0;
-#pragma unroll
-            for (int c = 0; c < kChunks; ++c)
-                if (__any_sync(0xffffffffu, 16 * c < c_lo || 16 * c + 15 > c_hi)) mask_chunks |= 1u << c;
 
-            // ---- pass 1: row maximum of the visible scores
+            // ---- the score row, all KN columns, in one TMEM read
+            uint32_t sr[kChunks][16];
+#pragma unroll
+            for (int c = 0; c < kChunks; ++c) tmem_ld16(trow + 16 * c, sr[c]);
+            tmem_wait_ld();
             float mx[8];
 #pragma unroll
             for (int k = 0; k < 8; ++k) mx[k] = -INFINITY;
-            {
-                // three 16-column loads, then one wait: a TMEM load round trip
-                // costs more than the maxima of 16 columns, so it is paid per 48
-                constexpr int kGroup = 3;
 #pragma unroll
-                for (int c0 = 0; c0 < kChunks; c0 += kGroup) {
-                    uint32_t sb[kGroup][16];
+            for (int c = 0; c < kChunks; ++c) {
+                // masks only where some row of the warp does not see the whole chunk
+                if (__any_sync(0xffffffffu, 16 * c < c_lo || 16 * c + 15 > c_hi)) {
 #pragma unroll
-                    for (int u = 0; u < kGroup; ++u)
-                        if (c0 + u < kChunks) tmem_ld16(trow + 16 * (c0 + u), sb[u]);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int u = 0; u < kGroup; ++u) {
-                        const int c = c0 + u;
-                        if (c >= kChunks) break;
-                        float v[16];
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) v[e] = __uint_as_float(sb[u][e]);
-                        if (mask_chunks & (1u << c)) {
-#pragma unroll
-                            for (int e = 0; e < 16; ++e)
-                                v[e] = (16 * c + e >= c_lo && 16 * c + e <= c_hi) ? v[e] : -INFINITY;
-                        }
-#pragma unroll
-                        for (int k = 0; k < 8; ++k) mx[k] = fmax3(mx[k], v[k], v[8 + k]);
-                    }
+                    for (int e = 0; e < 16; ++e)
+                        if (16 * c + e < c_lo || 16 * c + e > c_hi) sr[c][e] = __float_as_uint(-INFINITY);
                 }
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    mx[k] = fmax3(mx[k], __uint_as_float(sr[c][k]), __uint_as_float(sr[c][8 + k]));
             }
             const float tmax = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
             const float m = fmaxf(sink2, tmax * C);  // reference maximum, log2 units
             const float neg_m = (m == -INFINITY) ? 0.f : -m;
             float l = (sink2 == -INFINITY) ? 0.f : ex2(sink2 + neg_m);  // the sink's mass
-
-            // ---- pass 2: P = exp2(S C - m) as bf16 over S, and its row sum
             {
+                // P = exp2(S C - m) as bf16 over the first KN/2 columns of S, and its row sum
+                // (masked columns hold -inf: exp2 gives exactly 0 there)
                 const float2 C2 = make_float2(C, C), M2 = make_float2(neg_m, neg_m);
                 float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-                uint32_t sb[2][16];
-                tmem_ld16(trow, sb[0]);
-                tmem_wait_ld();
 #pragma unroll
                 for (int c = 0; c < kChunks; ++c) {
-                    if (c + 1 < kChunks) tmem_ld16(trow + 16 * (c + 1), sb[(c + 1) & 1]);
                     uint32_t pk[8];
-                    const bool msk = (mask_chunks & (1u << c)) != 0;
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        const float2 x = ffma2(make_float2(__uint_as_float(sb[c & 1][2 * e]),
-                                                           __uint_as_float(sb[c & 1][2 * e + 1])),
+                        const float2 x = ffma2(make_float2(__uint_as_float(sr[c][2 * e]),
+                                                           __uint_as_float(sr[c][2 * e + 1])),
                                                C2, M2);
-                        float2 pe = make_float2(ex2(x.x), ex2(x.y));
-                        if (msk) {
-                            const int c0 = 16 * c + 2 * e;
-                            pe.x = (c0 >= c_lo && c0 <= c_hi) ? pe.x : 0.f;
-                            pe.y = (c0 + 1 >= c_lo && c0 + 1 <= c_hi) ? pe.y : 0.f;
-                        }
+                        const float2 pe = make_float2(ex2(x.x), ex2(x.y));
                         acc[e & 1] = fadd2(acc[e & 1], pe);
                         pk[e] = pack_bf16x2(pe.x, pe.y);
                     }
                     tmem_st8(trow + 8 * c, pk);
-                    tmem_wait_ld();
                 }
                 l += (acc[0].x + acc[0].y) + (acc[1].x + acc[1].y);
             }
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(p_full);
+            mbar_arrive(&p_full[wg]);
 
-            // ---- epilogue: O / l, lse
-            if (!__all_sync(0xffffffffu, mbar_wait(o_done, r & 1u, abort_flag, p.status, p.timeout_ns))) break;
+            // ---- epilogue: O / l into the item's Q buffer, one tensor store
+            if (!__all_sync(0xffffffffu, mbar_wait<false>(&o_done[wg], (r >> 1) & 1u, abort_flag, p.status, p.timeout_ns)))
+                break;
             tc_fence_after();
             uint32_t o[2][32];
             tmem_ld32(trow + kTmO, o[0]);
             tmem_ld32(trow + kTmO + 32, o[1]);
             tmem_wait_ld();
             tc_fence_before();
-            mbar_arrive(o_free);
-            if (row_valid) {
-                const float inv = l > 0.f ? 1.f / l : 0.f;
-                // the item's output rows, looked up again here rather than kept
-                // live (in registers) through both softmax passes
-                const BandItem te = band_item(p, w);
-                uint4 *dst = reinterpret_cast<uint4 *>(p.out + ((size_t)(te.orow0 + pos) * p.Hq + h) * kD);
+            mbar_arrive(&o_free[wg]);
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            uint4 ov[8];
 #pragma unroll
-                for (int c = 0; c < kD / 8; ++c) {
-                    const uint32_t *src = &o[c / 4][(c % 4) * 8];
-                    uint4 v;
-                    v.x = pack_bf16x2(__uint_as_float(src[0]) * inv, __uint_as_float(src[1]) * inv);
-                    v.y = pack_bf16x2(__uint_as_float(src[2]) * inv, __uint_as_float(src[3]) * inv);
-                    v.z = pack_bf16x2(__uint_as_float(src[4]) * inv, __uint_as_float(src[5]) * inv);
-                    v.w = pack_bf16x2(__uint_as_float(src[6]) * inv, __uint_as_float(src[7]) * inv);
-                    dst[c] = v;
+            for (int c = 0; c < 8; ++c) {
+                ov[c].x = pack_bf16x2(__uint_as_float(o[c / 4][(c % 4) * 8 + 0]) * inv,
+                                      __uint_as_float(o[c / 4][(c % 4) * 8 + 1]) * inv);
+                ov[c].y = pack_bf16x2(__uint_as_float(o[c / 4][(c % 4) * 8 + 2]) * inv,
+                                      __uint_as_float(o[c / 4][(c % 4) * 8 + 3]) * inv);
+                ov[c].z = pack_bf16x2(__uint_as_float(o[c / 4][(c % 4) * 8 + 4]) * inv,
+                                      __uint_as_float(o[c / 4][(c % 4) * 8 + 5]) * inv);
+                ov[c].w = pack_bf16x2(__uint_as_float(o[c / 4][(c % 4) * 8 + 6]) * inv,
+                                      __uint_as_float(o[c / 4][(c % 4) * 8 + 7]) * inv);
+            }
+            if (row_valid)
+                p.lse[(size_t)(t.lrow0 + (long long)h * p.lse_hs + pos)] = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
+            // A box that would run past the end of a packed sequence (into the
+            // next one) is written row by row; otherwise one tensor store, whose
+            // box the TMA clips at the end of a fixed-length sequence.  The
+            // storing thread waits (bounded) until all 128 rows are staged.
+            uint8_t *stg = Cfg::kStageInK ? smem + Cfg::kOffK + st * Cfg::kKVBytes : smem + Cfg::kOffQ + st * Cfg::kQBytes;
+            uint64_t *stg_free = Cfg::kStageInK ? &k_empty[st] : &q_empty[st];
+            const bool ragged = p.cu_q != nullptr && t.pos0 + p.P > t.Lq;
+            if (ragged) {
+                if (row_valid) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(p.out + ((size_t)(t.orow0 + pos) * p.Hq + h) * kD);
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) dst[c] = ov[c];
                 }
-                p.lse[(size_t)(te.lrow0 + (long long)h * p.lse_hs + pos)] = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
+            } else {
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    *reinterpret_cast<uint4 *>(stg + row * 128 + ((c ^ (row & 7)) << 4)) = ov[c];
+                fence_proxy_async_smem();
+            }
+            mbar_arrive(&stg_ready[wg]);
+            if (storer) {
+                if (!mbar_wait<false>(&stg_ready[wg], (r >> 1) & 1u, abort_flag, p.status, p.timeout_ns)) break;
+                if (!ragged) {
+                    tma_store_4d(&tmO, stg, 0, t.h0, t.qrow0 + t.pos0, t.tb);
+                    bulk_commit_group();
+                    bulk_wait_read_all();  // the buffer may take its next load once the store has read it
+                    stores_issued = true;
+                }
+                mbar_arrive(stg_free);
             }
         }
+        if (storer && stores_issued) bulk_wait_all();  // every tensor store completes before the CTA exits
     }
 
     tc_fence_before();
@@ -425,11 +483,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 }
 
 template <int KN>
-cudaError_t launch_kn(const void *q, const void *k, const void *v, const BandParams &p, const AttnShape &s,
-                      cudaStream_t st)
+cudaError_t launch_kn(const void *q, const void *k, const void *v, void *out, const BandParams &p,
+                      const AttnShape &s, cudaStream_t st)
 {
     using Cfg = BandCfg<KN>;
-    alignas(64) CUtensorMap mq, mk, mv;
+    alignas(64) CUtensorMap mq, mk, mv, mo;
     // fixed-length batches: [B][L][H][D]; packed sequences: [1][total][H][D]
     const uint64_t qrows = s.cu_q ? (uint64_t)s.total_q : (uint64_t)s.Lq;
     const uint64_t krows = s.cu_q ? (uint64_t)s.total_k : (uint64_t)s.Lk;
@@ -438,7 +496,8 @@ cudaError_t launch_kn(const void *q, const void *k, const void *v, const BandPar
         const uint64_t dims[4] = {(uint64_t)kD, (uint64_t)s.Hq, qrows, outer};
         const uint64_t strides[3] = {(uint64_t)kD * 2, (uint64_t)s.Hq * kD * 2, qrows * s.Hq * kD * 2};
         const uint32_t box[4] = {(uint32_t)kD, (uint32_t)p.Gp, (uint32_t)p.P, 1u};
-        if (!encode_tensor_map_4d(&mq, const_cast<void *>(q), 2, dims, strides, box, true))
+        if (!encode_tensor_map_4d(&mq, const_cast<void *>(q), 2, dims, strides, box, true) ||
+            !encode_tensor_map_4d(&mo, out, 2, dims, strides, box, true))
             return cudaErrorInvalidValue;
     }
     {
@@ -450,9 +509,20 @@ cudaError_t launch_kn(const void *q, const void *k, const void *v, const BandPar
             return cudaErrorInvalidValue;
     }
     auto kern = fwd_band_kernel<KN>;
+    // The register moves inside the kernel are sized for a launch at exactly
+    // kRegsLaunch registers per thread; a build that compiled to fewer would
+    // leave the softmax warpgroups waiting for registers that never come.
+    static int regs = -1;
+    if (regs < 0) {
+        cudaFuncAttributes a;
+        cudaError_t e = cudaFuncGetAttributes(&a, kern);
+        if (e != cudaSuccess) return e;
+        regs = a.numRegs;
+    }
+    if (regs != kRegsLaunch) return cudaErrorInvalidConfiguration;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
     if (e != cudaSuccess) return e;
-    kern<<<p.n_items, kThreads, Cfg::kSmemBytes, st>>>(mq, mk, mv, p);
+    kern<<<p.n_items, kThreads, Cfg::kSmemBytes, st>>>(mq, mk, mv, mo, p);
     return cudaGetLastError();
 }
 
@@ -514,10 +584,10 @@ cudaError_t launch_fwd_band(const void *q, const void *k, const void *v, const f
     p.status = device_status_ptr();
     p.timeout_ns = wait_timeout_ns();
     switch (band_tile_keys(s)) {
-    case 32: return launch_kn<32>(q, k, v, p, s, st);
-    case 64: return launch_kn<64>(q, k, v, p, s, st);
-    case 96: return launch_kn<96>(q, k, v, p, s, st);
-    case 144: return launch_kn<144>(q, k, v, p, s, st);
+    case 32: return launch_kn<32>(q, k, v, out, p, s, st);
+    case 64: return launch_kn<64>(q, k, v, out, p, s, st);
+    case 96: return launch_kn<96>(q, k, v, out, p, s, st);
+    case 144: return launch_kn<144>(q, k, v, out, p, s, st);
     default: return cudaErrorInvalidValue;
     }
 }

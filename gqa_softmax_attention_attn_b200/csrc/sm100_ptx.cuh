@@ -86,12 +86,8 @@ constexpr long long kShortWaitNs = 1000000;
 // role of the CTA winds down too.  (A suspend-time hint on try_wait was
 // measured slower at the default limit: the woken thread resumes late; it is
 // only used for limits below kShortWaitNs.)
-// The polling loop lives in one out-of-line function shared by every call
-// site: the kernels wait at a few dozen places, and a copy of the loop at each
-// one grew the code the SM's instruction cache has to hold (the backward
-// kernel lost 7 KB of code and 2.5% of its time with this).
-static __device__ __noinline__ bool mbar_wait_slow(uint64_t *bar, uint32_t parity, volatile int *abort, unsigned *status,
-                                            long long timeout_ns)
+__device__ __forceinline__ bool mbar_poll(uint64_t *bar, uint32_t parity, volatile int *abort, unsigned *status,
+                                          long long timeout_ns)
 {
     const uint64_t t0 = globaltimer_ns();
     const bool short_limit = timeout_ns < kShortWaitNs;
@@ -109,11 +105,41 @@ static __device__ __noinline__ bool mbar_wait_slow(uint64_t *bar, uint32_t parit
     }
 }
 
+// The polling loop lives in one out-of-line function shared by every call
+// site: the kernels wait at a few dozen places, and a copy of the loop at each
+// one grew the code the SM's instruction cache has to hold (the backward
+// kernel lost 7 KB of code and 2.5% of its time with this).
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t *bar, uint32_t parity, volatile int *abort, unsigned *status,
+                                            long long timeout_ns)
+{
+    return mbar_poll(bar, parity, abort, status, timeout_ns);
+}
+
+// kCall = false keeps the loop inline: a kernel that moves registers between
+// warpgroups (setmaxnreg) cannot make calls inside the moved regions.
+template <bool kCall = true>
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
                                           unsigned *status, long long timeout_ns)
 {
     if (mbar_try_wait(bar, parity)) return true;
-    return mbar_wait_slow(bar, parity, abort, status, timeout_ns);
+    if constexpr (kCall)
+        return mbar_wait_slow(bar, parity, abort, status, timeout_ns);
+    else
+        return mbar_poll(bar, parity, abort, status, timeout_ns);
+}
+
+// Register reallocation between warpgroups (all four warps of a warpgroup
+// execute it).  The shares after the moves must add up to at most what the
+// block was launched with (threads x registers per thread at launch).
+template <int N>
+__device__ __forceinline__ void regs_release()
+{
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_claim()
+{
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(N));
 }
 
 // ---------------------------------------------------------------- cluster launch control
@@ -159,7 +185,7 @@ constexpr int kClcDepth = ATTN_SINK_CLC_DEPTH;
 // Up to DEPTH launch-control requests in flight, answered in the order they
 // were issued; used by one thread (the producer).  bar: DEPTH mbarriers
 // initialised with count 1; resp: DEPTH 16-byte response slots.
-template <int DEPTH>
+template <int DEPTH, bool kCallWait = true>
 struct ClcQueue {
     uint64_t *bar;
     uint8_t *resp;
@@ -184,7 +210,7 @@ struct ClcQueue {
     {
         while (consumed != issued) {
             const int s = consumed % DEPTH;
-            if (!mbar_wait(&bar[s], (consumed / DEPTH) & 1u, abort, status, timeout_ns)) {
+            if (!mbar_wait<kCallWait>(&bar[s], (consumed / DEPTH) & 1u, abort, status, timeout_ns)) {
                 failed = stop = true;
                 return -1;
             }
@@ -201,7 +227,7 @@ struct ClcQueue {
         int never = 0;
         const long long tmo = timeout_ns > 1000000000LL ? timeout_ns : 1000000000LL;
         for (; consumed != issued; ++consumed)
-            mbar_wait(&bar[consumed % DEPTH], (consumed / DEPTH) & 1u, &never, status, tmo);
+            mbar_wait<kCallWait>(&bar[consumed % DEPTH], (consumed / DEPTH) & 1u, &never, status, tmo);
     }
 };
 
@@ -232,6 +258,23 @@ __device__ __forceinline__ void tma_reduce_add_4d(const CUtensorMap *map, const 
         "r"(smem_u32(smem_src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
         : "memory");
 }
+// 4-D tiled bulk tensor store shared -> global (coordinates in elements; the
+// box is clipped at the tensor's bounds), bulk-group completion.
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap *map, const void *smem_src, int c0, int c1, int c2,
+                                             int c3)
+{
+    asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(smem_u32(smem_src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+                 : "memory");
+}
+
+// Barrier among `nthreads` threads (whole warps) on hardware barrier `id` (1..15).
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // wait until every committed bulk group has finished READING its shared-memory source
 __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }

@@ -494,8 +494,9 @@ int attn_sink_bwd(const void *q, const void *k, const void *v, const float *sink
     float *terms = Drow + rows;
     float *dq_acc = reinterpret_cast<float *>(static_cast<char *>(workspace) +
                                               (bwd_simt_workspace_bytes(s) + 255) / 256 * 256);
+    // the row pre-pass also clears the dQ accumulator the main pass adds into
     cudaError_t e = launch_bwd_rows<bf>(static_cast<const bf *>(out), static_cast<const bf *>(dout), lse, sinks, Drow,
-                                        terms, s, st);
+                                        terms, dq_acc, s, st);
     if (e == cudaSuccess) e = launch_bwd_tc(q, k, v, dout, lse, Drow, dq_acc, dq, dk, dv, s, st);
     if (e == cudaSuccess) e = launch_dsink_reduce(terms, dsinks, s, st);
     return launch_status(e);

@@ -626,8 +626,8 @@ cudaError_t launch_bwd_tc(const void *q, const void *k, const void *v, const voi
         !encode_tensor_map_4d(&mv, const_cast<void *>(v), 2, kd, ks2, kbox, true) ||
         !encode_tensor_map_4d(&mdq, dq_acc, 4, qd, qs4, dqbox, true))
         return cudaErrorInvalidValue;
-    cudaError_t e = cudaMemsetAsync(dq_acc, 0, bwd_tc_dq_acc_bytes(s), st);
-    if (e != cudaSuccess) return e;
+    // dq_acc arrives zeroed (the row pre-pass clears it)
+    cudaError_t e;
     const long long n_cta = (long long)((s.Lk + kM - 1) / kM) * s.Hkv * s.B;
     if (n_cta > 0x7fffffffLL) return cudaErrorInvalidValue;
     const dim3 grid((unsigned)n_cta);

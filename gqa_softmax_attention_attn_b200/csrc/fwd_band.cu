@@ -21,9 +21,11 @@
 //    starting at a negative row where the band reaches before key 0: the TMA
 //    fills rows outside the tensor with zeros) in four stages, so items ahead
 //    of the two being computed are in flight.
-//  * Warp 1: the MMA issue loop (whole warp, one elected lane issuing):
-//    S = Q K^T of item r + 2 goes right after P.V of item r, into the TMEM
-//    half of item r's warpgroup (the tensor pipe runs them in order).
+//  * Warp 1: the MMA issue loop (whole warp, one elected lane issuing),
+//    polling the barriers of both warpgroups' items and issuing whichever
+//    product is ready: P.V of item r as soon as its P is written, S = Q K^T
+//    of item r + 2 into the same TMEM half once P.V(r) is issued (the tensor
+//    pipe runs them in order) and its Q, K have landed.
 //  * Warps 4-7 and 8-11 (registers moved to them from warpgroup 0 with
 //    setmaxnreg), one thread per row: the whole score row (KN columns)
 //    comes out of TMEM in one go into registers; masks only on the 16-column
@@ -282,14 +284,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------------------ MMA issuer
         const uint32_t id_s = idesc_bf16_f32(kM, KN, 0);
         const uint32_t id_pv = idesc_bf16_f32(kM, kD, 1);
-        auto wait_all = [&](uint64_t *bar, uint32_t parity) {
-            return __all_sync(0xffffffffu, mbar_wait<false>(bar, parity, abort_flag, p.status, p.timeout_ns));
-        };
-        // S = Q K^T of item r into its warpgroup's TMEM half; false on abort
-        auto issue_s = [&](int r) -> bool {
+        // every lane has seen the phase complete (a lane that has not yet is retried later)
+        auto ready = [&](uint64_t *bar, uint32_t parity) { return __all_sync(0xffffffffu, mbar_test(bar, parity)); };
+        // S = Q K^T of item r into its warpgroup's TMEM half
+        auto issue_s = [&](int r) {
             const int st = r % kNS;
-            const uint32_t ph = (r / kNS) & 1u;
-            if (!wait_all(&q_full[st], ph) || !wait_all(&k_full[st], ph)) return false;
             tc_fence_after();
             const uint32_t qa = smem_u32(smem + Cfg::kOffQ + st * Cfg::kQBytes);
             const uint32_t kb = smem_u32(smem + Cfg::kOffK + st * Cfg::kKVBytes);
@@ -302,15 +301,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mma_commit(Cfg::kStageInK ? &q_empty[st] : &k_empty[st]);  // the other one stages O
             }
             __syncwarp();
-            return true;
         };
-        // O = P V of item r, once its warpgroup has written P, V has landed and
-        // the warpgroup's previous epilogue has read its O out
-        auto issue_pv = [&](int r) -> bool {
+        // O = P V of item r
+        auto issue_pv = [&](int r) {
             const int st = r % kNS, wg = r & 1;
-            if (!wait_all(&p_full[wg], (r >> 1) & 1u) || !wait_all(&v_full[st], (r / kNS) & 1u) ||
-                !wait_all(&o_free[wg], ((r >> 1) & 1u) ^ 1u))
-                return false;
             tc_fence_after();
             const uint32_t vb = smem_u32(smem + Cfg::kOffV + st * Cfg::kKVBytes);
             if (elect_one()) {
@@ -322,17 +316,68 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mma_commit(&v_empty[st]);
             }
             __syncwarp();
-            return true;
         };
-        int w_cur = consumer_item(0);
-        int w_nxt = w_cur >= 0 ? consumer_item(1) : -1;
-        bool ok = (w_cur < 0 || issue_s(0)) && (w_nxt < 0 || issue_s(1));
-        for (int r = 0; ok && w_cur >= 0; ++r) {
-            if (!issue_pv(r)) break;
-            const int w2 = w_nxt >= 0 ? consumer_item(r + 2) : -1;
-            if (w2 >= 0 && !issue_s(r + 2)) break;
-            w_cur = w_nxt;
-            w_nxt = w2;
+        // Out-of-order issue between the two warpgroups' streams, so that a
+        // product whose operands are ready never waits behind one whose loads
+        // are still in flight:
+        //  * P.V of item r once S(r) is issued, P(r) written, V(r) landed and
+        //    the warpgroup's previous epilogue has read its O;
+        //  * S of item r once its warpgroup's TMEM half is free (P.V(r - 2)
+        //    issued: the tensor pipe runs one thread's MMAs in order) and Q(r),
+        //    K(r) have landed.
+        // Items come from the ring without blocking; the loop polls, and gives
+        // up (abort flag, status bit) after the wait limit without progress.
+        int n_valid = 0, next_s = 0, next_pv = 0;
+        bool end = false;
+        uint64_t t_last = globaltimer_ns();
+        while (true) {
+            bool progress = false;
+            if (!end && n_valid < next_pv + 3) {
+                const int sl = n_valid & 3;
+                if (ready(&item_full[sl], (n_valid >> 2) & 1u)) {
+                    const int w = ring[sl];
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&item_empty[sl]);
+                    if (w < 0)
+                        end = true;
+                    else
+                        ++n_valid;
+                    progress = true;
+                }
+            }
+            if (next_pv < next_s) {
+                const int r = next_pv, wg = r & 1;
+                if (ready(&p_full[wg], (r >> 1) & 1u) && ready(&v_full[r % kNS], (r / kNS) & 1u) &&
+                    ready(&o_free[wg], ((r >> 1) & 1u) ^ 1u)) {
+                    issue_pv(r);
+                    ++next_pv;
+                    progress = true;
+                }
+            }
+            if (next_s < n_valid && next_s < next_pv + 2) {
+                const int r = next_s;
+                const uint32_t ph = (r / kNS) & 1u;
+                if (ready(&q_full[r % kNS], ph) && ready(&k_full[r % kNS], ph)) {
+                    issue_s(r);
+                    ++next_s;
+                    progress = true;
+                }
+            }
+            if (end && next_pv == n_valid) break;
+            const uint64_t now = globaltimer_ns();
+            if (progress) {
+                t_last = now;
+            } else {
+                if (*abort_flag) break;
+                if ((long long)(now - t_last) > p.timeout_ns) {
+                    if (lane == 0) {
+                        *abort_flag = 1;
+                        atomicOr(p.status, STATUS_TIMEOUT);
+                    }
+                    __syncwarp();
+                    break;
+                }
+            }
         }
         if (elect_one()) mma_commit(drain);
         __syncwarp();

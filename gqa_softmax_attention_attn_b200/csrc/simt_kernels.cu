@@ -130,28 +130,95 @@ __global__ void __launch_bounds__(128) fwd_simt_kernel(const T *__restrict__ q, 
 
 // ------------------------------------------------------------------ backward
 // (1) per row: D_i = <dO_i, O_i>, dsink term -exp(sink - lse_i) * D_i.
+// HBM-bound (one read of O and dO): a row of 64 values is 128 or 256 bytes,
+// read as 16-byte chunks by kTpr neighbouring threads (8 for bf16, 16 for
+// fp32) whose partial dot products meet in a shuffle reduction; each thread
+// takes kRowsPerThread rows with all their loads issued first, so enough bytes
+// are in flight per SM to cover the memory latency.  When `zero` is given
+// (the fp32 dQ accumulator of the tensor-core backward, rows in the same
+// [B, Lq, Hq] order), the same threads clear its rows in this pass.
+template <typename T>
+struct PreRows {
+    static constexpr int kElems = 16 / sizeof(T);  // values per 16-byte chunk
+    static constexpr int kTpr = kD / kElems;       // threads per row
+    static constexpr int kRowsPerThread = 4;
+    static constexpr int kRowsPerCta = 256 / kTpr * kRowsPerThread;
+};
+
+__device__ __forceinline__ float dot16(const uint4 &a, const uint4 &b, float)
+{
+    const float *x = reinterpret_cast<const float *>(&a), *y = reinterpret_cast<const float *>(&b);
+    return x[0] * y[0] + x[1] * y[1] + x[2] * y[2] + x[3] * y[3];
+}
+__device__ __forceinline__ float dot16(const uint4 &a, const uint4 &b, __nv_bfloat16)
+{
+    const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
+    float acc = 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float2 fa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&wa[j]));
+        const float2 fb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&wb[j]));
+        acc = fmaf(fa.x, fb.x, acc);
+        acc = fmaf(fa.y, fb.y, acc);
+    }
+    return acc;
+}
+
 template <typename T>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const T *__restrict__ out, const T *__restrict__ dout,
                                                       const float *__restrict__ lse,
                                                       const float *__restrict__ sinks, float *__restrict__ Drow,
-                                                      float *__restrict__ terms, AttnShape s)
+                                                      float *__restrict__ terms, float *__restrict__ zero,
+                                                      AttnShape s)
 {
-    const int lane = threadIdx.x & 31;
-    const long row = (long)blockIdx.x * 8 + (threadIdx.x >> 5);  // row over [B, Lq, Hq]
+    using R = PreRows<T>;
+    const int sub = threadIdx.x % R::kTpr;  // chunk of the row
     const long nrows = (long)s.B * s.Lq * s.Hq;
-    if (row >= nrows) return;
-    const int h = (int)(row % s.Hq);
-    const long bi = row / s.Hq;
-    const int i = (int)(bi % s.Lq), b = (int)(bi / s.Lq);
-    const size_t base = (size_t)row * kD;
-    float d = to_f(out[base + lane]) * to_f(dout[base + lane]) + to_f(out[base + lane + 32]) * to_f(dout[base + lane + 32]);
-    d = warp_sum(d);
-    if (lane == 0) {
-        const size_t li = ((size_t)b * s.Hq + h) * s.Lq + i;
-        const float L = lse[li];
-        Drow[li] = d;
-        const float ps = (L == -INFINITY) ? 0.f : expf(sinks[h] - L);
-        terms[(size_t)h * s.B * s.Lq + (size_t)b * s.Lq + i] = -ps * d;
+    const long row0 = (long)blockIdx.x * R::kRowsPerCta + threadIdx.x / R::kTpr;
+    constexpr int kStride = 256 / R::kTpr;  // rows between a thread's successive rows
+    uint4 a[R::kRowsPerThread], b[R::kRowsPerThread];
+#pragma unroll
+    for (int u = 0; u < R::kRowsPerThread; ++u) {
+        const long row = row0 + (long)u * kStride;
+        if (row < nrows) {
+            const size_t off = (size_t)row * kD + (size_t)sub * R::kElems;
+            a[u] = *reinterpret_cast<const uint4 *>(out + off);
+            b[u] = *reinterpret_cast<const uint4 *>(dout + off);
+            if (zero) {
+                constexpr int kF = kD / R::kTpr;  // fp32 values of the row per thread
+                float4 *z = reinterpret_cast<float4 *>(zero + (size_t)row * kD + (size_t)sub * kF);
+#pragma unroll
+                for (int c = 0; c < kF / 4; ++c) z[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        } else {
+            a[u] = b[u] = make_uint4(0u, 0u, 0u, 0u);
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < R::kRowsPerThread; ++u) {
+        float d = dot16(a[u], b[u], T{});
+#pragma unroll
+        for (int w = R::kTpr / 2; w > 0; w >>= 1) d += __shfl_xor_sync(0xffffffffu, d, w);
+        const long row = row0 + (long)u * kStride;
+        if (sub == 0 && row < nrows) {  // row over [B, Lq, Hq]
+            int h, i, bb;
+            if (nrows <= 0xffffffffL) {  // 32-bit division where it suffices
+                const uint32_t r32 = (uint32_t)row, bi = r32 / (uint32_t)s.Hq;
+                h = (int)(r32 - bi * (uint32_t)s.Hq);
+                bb = (int)(bi / (uint32_t)s.Lq);
+                i = (int)(bi - (uint32_t)bb * (uint32_t)s.Lq);
+            } else {
+                h = (int)(row % s.Hq);
+                const long bi = row / s.Hq;
+                i = (int)(bi % s.Lq);
+                bb = (int)(bi / s.Lq);
+            }
+            const size_t li = ((size_t)bb * s.Hq + h) * s.Lq + i;
+            const float L = lse[li];
+            Drow[li] = d;
+            const float ps = (L == -INFINITY) ? 0.f : expf(sinks[h] - L);
+            terms[(size_t)h * s.B * s.Lq + (size_t)bb * s.Lq + i] = -ps * d;
+        }
     }
 }
 
@@ -495,7 +562,8 @@ cudaError_t launch_bwd_simt(const T *q, const T *k, const T *v, const float *sin
     const size_t rows = (size_t)s.B * s.Hq * s.Lq;
     float *Drow = static_cast<float *>(ws);
     float *terms = Drow + rows;
-    bwd_pre_kernel<T><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(out, dout, lse, sinks, Drow, terms, s);
+    bwd_pre_kernel<T><<<(unsigned)((rows + PreRows<T>::kRowsPerCta - 1) / PreRows<T>::kRowsPerCta), 256, 0, st>>>(
+        out, dout, lse, sinks, Drow, terms, nullptr, s);
     bwd_dq_kernel<T><<<dim3((s.Lq + 15) / 16, s.Hq, s.B), 128, 0, st>>>(q, k, v, dout, lse, Drow, dq, s);
     bwd_dkdv_kernel<T><<<dim3((s.Lk + 31) / 32, s.Hkv, s.B), 128, 0, st>>>(q, k, v, dout, lse, Drow, dk, dv, s);
     dsink_reduce_kernel<<<s.Hq, 256, 0, st>>>(terms, dsinks, (long)s.B * s.Lq);
@@ -504,10 +572,12 @@ cudaError_t launch_bwd_simt(const T *q, const T *k, const T *v, const float *sin
 
 template <typename T>
 cudaError_t launch_bwd_rows(const T *out, const T *dout, const float *lse, const float *sinks, float *Drow,
-                            float *terms, const AttnShape &s, cudaStream_t st)
+                            float *terms, float *zero_rows, const AttnShape &s, cudaStream_t st)
 {
     const size_t rows = (size_t)s.B * s.Hq * s.Lq;
-    bwd_pre_kernel<T><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(out, dout, lse, sinks, Drow, terms, s);
+    const size_t ctas = (rows + PreRows<T>::kRowsPerCta - 1) / PreRows<T>::kRowsPerCta;
+    if (ctas > 0x7fffffffu) return cudaErrorInvalidValue;
+    bwd_pre_kernel<T><<<(unsigned)ctas, 256, 0, st>>>(out, dout, lse, sinks, Drow, terms, zero_rows, s);
     return cudaGetLastError();
 }
 
@@ -543,7 +613,7 @@ cudaError_t launch_decode_combine(const int *seqlens, const float *sinks, T *out
                                             const T *, const float *, T *, T *, T *, float *,                 \
                                             const AttnShape &, void *, cudaStream_t);                         \
     template cudaError_t launch_bwd_rows<T>(const T *, const T *, const float *, const float *, float *, float *, \
-                                            const AttnShape &, cudaStream_t);                                 \
+                                            float *, const AttnShape &, cudaStream_t);                                 \
     template cudaError_t launch_decode_simt<T>(const T *, const T *, const T *, const int *, const float *,   \
                                                T *, float *, const DecodeShape &, float *, float *,           \
                                                cudaStream_t);                                                 \

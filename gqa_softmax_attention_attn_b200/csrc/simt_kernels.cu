@@ -141,7 +141,8 @@ template <typename T>
 struct PreRows {
     static constexpr int kElems = 16 / sizeof(T);  // values per 16-byte chunk
     static constexpr int kTpr = kD / kElems;       // threads per row
-    static constexpr int kRowsPerThread = 4;
+    static constexpr int kRowsPerThread = 2;  // with four CTAs per SM (measured best of 2/4/8 rows)
+    static constexpr int kMinCtas = 4;
     static constexpr int kRowsPerCta = 256 / kTpr * kRowsPerThread;
 };
 
@@ -165,7 +166,7 @@ __device__ __forceinline__ float dot16(const uint4 &a, const uint4 &b, __nv_bflo
 }
 
 template <typename T>
-__global__ void __launch_bounds__(256) bwd_pre_kernel(const T *__restrict__ out, const T *__restrict__ dout,
+__global__ void __launch_bounds__(256, PreRows<T>::kMinCtas) bwd_pre_kernel(const T *__restrict__ out, const T *__restrict__ dout,
                                                       const float *__restrict__ lse,
                                                       const float *__restrict__ sinks, float *__restrict__ Drow,
                                                       float *__restrict__ terms, float *__restrict__ zero,
@@ -176,7 +177,11 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const T *__restrict__ out,
     const long nrows = (long)s.B * s.Lq * s.Hq;
     const long row0 = (long)blockIdx.x * R::kRowsPerCta + threadIdx.x / R::kTpr;
     constexpr int kStride = 256 / R::kTpr;  // rows between a thread's successive rows
+    // every load of the thread's rows first (O, dO, and the row's lse and sink,
+    // which all kTpr threads of the row read), so one memory latency covers them
     uint4 a[R::kRowsPerThread], b[R::kRowsPerThread];
+    float Lr[R::kRowsPerThread], sk[R::kRowsPerThread];
+    size_t li[R::kRowsPerThread], ti[R::kRowsPerThread];
 #pragma unroll
     for (int u = 0; u < R::kRowsPerThread; ++u) {
         const long row = row0 + (long)u * kStride;
@@ -184,24 +189,7 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const T *__restrict__ out,
             const size_t off = (size_t)row * kD + (size_t)sub * R::kElems;
             a[u] = *reinterpret_cast<const uint4 *>(out + off);
             b[u] = *reinterpret_cast<const uint4 *>(dout + off);
-            if (zero) {
-                constexpr int kF = kD / R::kTpr;  // fp32 values of the row per thread
-                float4 *z = reinterpret_cast<float4 *>(zero + (size_t)row * kD + (size_t)sub * kF);
-#pragma unroll
-                for (int c = 0; c < kF / 4; ++c) z[c] = make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-        } else {
-            a[u] = b[u] = make_uint4(0u, 0u, 0u, 0u);
-        }
-    }
-#pragma unroll
-    for (int u = 0; u < R::kRowsPerThread; ++u) {
-        float d = dot16(a[u], b[u], T{});
-#pragma unroll
-        for (int w = R::kTpr / 2; w > 0; w >>= 1) d += __shfl_xor_sync(0xffffffffu, d, w);
-        const long row = row0 + (long)u * kStride;
-        if (sub == 0 && row < nrows) {  // row over [B, Lq, Hq]
-            int h, i, bb;
+            int h, i, bb;  // row over [B, Lq, Hq]
             if (nrows <= 0xffffffffL) {  // 32-bit division where it suffices
                 const uint32_t r32 = (uint32_t)row, bi = r32 / (uint32_t)s.Hq;
                 h = (int)(r32 - bi * (uint32_t)s.Hq);
@@ -213,11 +201,32 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const T *__restrict__ out,
                 i = (int)(bi % s.Lq);
                 bb = (int)(bi / s.Lq);
             }
-            const size_t li = ((size_t)bb * s.Hq + h) * s.Lq + i;
-            const float L = lse[li];
-            Drow[li] = d;
-            const float ps = (L == -INFINITY) ? 0.f : expf(sinks[h] - L);
-            terms[(size_t)h * s.B * s.Lq + (size_t)bb * s.Lq + i] = -ps * d;
+            li[u] = ((size_t)bb * s.Hq + h) * s.Lq + i;
+            ti[u] = (size_t)h * s.B * s.Lq + (size_t)bb * s.Lq + i;
+            Lr[u] = lse[li[u]];
+            sk[u] = sinks[h];
+            if (zero) {
+                constexpr int kF = kD / R::kTpr;  // fp32 values of the row per thread
+                float4 *z = reinterpret_cast<float4 *>(zero + (size_t)row * kD + (size_t)sub * kF);
+#pragma unroll
+                for (int c = 0; c < kF / 4; ++c) z[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        } else {
+            a[u] = b[u] = make_uint4(0u, 0u, 0u, 0u);
+            Lr[u] = sk[u] = 0.f;
+            li[u] = ti[u] = 0;
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < R::kRowsPerThread; ++u) {
+        float d = dot16(a[u], b[u], T{});
+#pragma unroll
+        for (int w = R::kTpr / 2; w > 0; w >>= 1) d += __shfl_xor_sync(0xffffffffu, d, w);
+        const long row = row0 + (long)u * kStride;
+        if (sub == 0 && row < nrows) {
+            Drow[li[u]] = d;
+            const float ps = (Lr[u] == -INFINITY) ? 0.f : expf(sk[u] - Lr[u]);
+            terms[ti[u]] = -ps * d;
         }
     }
 }

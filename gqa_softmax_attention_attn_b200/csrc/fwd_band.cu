@@ -72,7 +72,13 @@ struct BandCfg {
     static constexpr int kOffQ = 0;                       // [kNS]
     static constexpr int kOffK = kNS * kQBytes;           // [kNS]
     static constexpr int kOffV = kOffK + kNS * kKVBytes;  // [kNS]
-    static constexpr int kOffBar = kOffV + kNS * kKVBytes;
+    // The band's staircase mask as one more K = 16 step of the score MMA:
+    // S += E_q E_k^T with E_q[row][k] = (k == the row's position in the item)
+    // and E_k[col][k] = -2^100 where key col is outside position k's window,
+    // else 0 (bf16, K-major without swizzle: 8-row groups of 256 bytes).
+    static constexpr int kOffEq = kOffV + kNS * kKVBytes;  // 128 rows x 32 bytes
+    static constexpr int kOffEk = kOffEq + kM * 32;        // KN rows x 32 bytes
+    static constexpr int kOffBar = kOffEk + KN * 32;
     // The item's O is staged in its K buffer when that holds 16 KB (K is dead
     // once S is done and is only needed again two items of this warpgroup
     // later), else in its Q buffer.
@@ -97,6 +103,7 @@ struct BandParams {
     long long lse_hs;        // lse stride between heads: Lq, or total_q for packed sequences
     int G, Gp, P;
     int n_ptiles, n_htiles, n_items;
+    int mask_mma;  // P <= 16: the staircase mask comes from the extra MMA step
     float c_log2;  // scale * log2(e)
     const float *sinks;
     __nv_bfloat16 *out;
@@ -202,6 +209,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
     }
+    if (p.mask_mma) {
+        // E_q and E_k of the mask step, element (row, k) at byte
+        // (row / 8) 256 + (k / 8) 128 + (row % 8) 16 + (k % 8) 2
+        uint16_t *eq = reinterpret_cast<uint16_t *>(smem + Cfg::kOffEq);
+        uint16_t *ek = reinterpret_cast<uint16_t *>(smem + Cfg::kOffEk);
+        constexpr uint16_t kOne = 0x3F80u, kBig = 0xF180u;  // bf16 1 and -2^100
+        for (int i = threadIdx.x; i < (kM + KN) * 16; i += kThreads) {
+            const bool isq = i < kM * 16;
+            const int j = isq ? i : i - kM * 16;
+            const int row = j >> 4, k = j & 15;
+            const uint16_t v = isq ? ((k == row / p.Gp) ? kOne : (uint16_t)0)
+                                   : ((k < p.P && (row < k || row > k + p.window - 1)) ? kBig : (uint16_t)0);
+            (isq ? eq : ek)[((row >> 3) * 256 + (k >> 3) * 128 + (row & 7) * 16 + (k & 7) * 2) >> 1] = v;
+        }
+        fence_proxy_async_smem();  // read by the tensor core
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -284,6 +307,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------------------ MMA issuer
         const uint32_t id_s = idesc_bf16_f32(kM, KN, 0);
         const uint32_t id_pv = idesc_bf16_f32(kM, kD, 1);
+        const uint64_t eq_desc = smem_desc_noswz(smem_u32(smem + Cfg::kOffEq), 128, 256);
+        const uint64_t ek_desc = smem_desc_noswz(smem_u32(smem + Cfg::kOffEk), 128, 256);
         // every lane has seen the phase complete (a lane that has not yet is retried later)
         auto ready = [&](uint64_t *bar, uint32_t parity) { return __all_sync(0xffffffffu, mbar_test(bar, parity)); };
         // S = Q K^T of item r into its warpgroup's TMEM half
@@ -297,6 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int kk = 0; kk < kD / 16; ++kk)
                     mma_ss(tmem + 256 * (r & 1), smem_desc_sw128(qa + kk * 32, 16, 1024),
                            smem_desc_sw128(kb + kk * 32, 16, 1024), id_s, kk > 0 ? 1u : 0u);
+                if (p.mask_mma) mma_ss(tmem + 256 * (r & 1), eq_desc, ek_desc, id_s, 1u);  // + the band's mask
                 mma_commit(&s_full[r & 1]);
                 mma_commit(Cfg::kStageInK ? &q_empty[st] : &k_empty[st]);  // the other one stages O
             }
@@ -406,9 +432,32 @@ __global__ void __launch_bounds__(kThreads, 1)
             // columns c of the tile (key js + c) this row sees: c in [c_lo, c_hi]
             const int c_lo = max(dp, -t.js);
             const int c_hi = row_valid ? min(dp + p.window - 1, t.Lk - 1 - t.js) : -1;
+            // an item whose every row is valid and whose band lies inside the
+            // sequence is masked by the MMA step alone (same for the whole item)
+            const bool interior = p.mask_mma && t.js >= 0 && t.pos0 + p.P <= t.Lq && t.Lk - t.js >= p.P + p.window - 1;
             if (!__all_sync(0xffffffffu, mbar_wait<false>(&s_full[wg], (r >> 1) & 1u, abort_flag, p.status, p.timeout_ns)))
                 break;
             tc_fence_after();
+
+            // ---- masks of items at the edges of a sequence (or with more than 16
+            // positions): masked scores become -inf in tensor memory, chunk by
+            // chunk in a rolled loop, only where some row of the warp needs it;
+            // the other items are masked by the MMA step, so the unrolled path
+            // below carries no mask code
+            if (!interior) {
+#pragma unroll 1
+                for (int c = 0; c < kChunks; ++c) {
+                    if (!__any_sync(0xffffffffu, 16 * c < c_lo || 16 * c + 15 > c_hi)) continue;
+                    uint32_t v[16];
+                    tmem_ld16(trow + 16 * c, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        if (16 * c + e < c_lo || 16 * c + e > c_hi) v[e] = __float_as_uint(-INFINITY);
+                    tmem_st16(trow + 16 * c, v);
+                }
+                tmem_wait_st();
+            }
 
             // ---- the score row, all KN columns, in one TMEM read
             uint32_t sr[kChunks][16];
@@ -419,17 +468,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int k = 0; k < 8; ++k) mx[k] = -INFINITY;
 #pragma unroll
-            for (int c = 0; c < kChunks; ++c) {
-                // masks only where some row of the warp does not see the whole chunk
-                if (__any_sync(0xffffffffu, 16 * c < c_lo || 16 * c + 15 > c_hi)) {
-#pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        if (16 * c + e < c_lo || 16 * c + e > c_hi) sr[c][e] = __float_as_uint(-INFINITY);
-                }
+            for (int c = 0; c < kChunks; ++c)
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
                     mx[k] = fmax3(mx[k], __uint_as_float(sr[c][k]), __uint_as_float(sr[c][8 + k]));
-            }
             const float tmax = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
             const float m = fmaxf(sink2, tmax * C);  // reference maximum, log2 units
             const float neg_m = (m == -INFINITY) ? 0.f : -m;
@@ -622,6 +664,7 @@ cudaError_t launch_fwd_band(const void *q, const void *k, const void *v, const f
     const long long n_items = (long long)p.n_ptiles * p.n_htiles * s.B;
     if (n_items > 0x7fffffffLL) return cudaErrorInvalidValue;
     p.n_items = (int)n_items;
+    p.mask_mma = p.P <= 16;
     p.c_log2 = s.scale * kLog2e;
     p.sinks = sinks;
     p.out = static_cast<__nv_bfloat16 *>(out);

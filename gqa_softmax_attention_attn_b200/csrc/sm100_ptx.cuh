@@ -460,6 +460,19 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
 //   bits 4-5 D format (1 = f32), 7-9 A format (1 = bf16), 10-12 B format,
 //   bit 15 A major (0 = K), bit 16 B major (0 = K, 1 = MN),
 //   bits 17-22 N >> 3, bits 24-28 M >> 4.
+// Shared-memory matrix descriptor, K-major without swizzle: 8-row x 16-byte
+// core matrices, k_core_bytes between core matrices along K, group_bytes
+// between 8-row groups.
+__device__ __forceinline__ uint64_t smem_desc_noswz(uint32_t saddr, uint32_t k_core_bytes, uint32_t group_bytes)
+{
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((k_core_bytes >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((group_bytes >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1u << 46;
+    return d;
+}
+
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int b_mn_major, int a_mn_major = 0)
 {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn_major << 15) | ((uint32_t)b_mn_major << 16) |

@@ -437,12 +437,13 @@ def leg_entry(ms, flops, nbytes, bound, shape):
     return e
 
 
-def prefill_legs(dev, which=("bwd", "train", "varlen", "prologue", "long"), reps=5, warmup=2):
+def prefill_legs(dev, which=("bwd", "train", "fp8", "varlen", "prologue", "long"), reps=5, warmup=2):
     """Forward / backward legs beyond the headline step, each with its own roofline
     fraction (dense layers against the tensor peak, window-128 layers against HBM),
     L2 flushed before every timed run:
       bwd:   the backward at the prefill shape (B1 L4096 Hq64 Hkv8);
       train: forward and backward at the training shape (B8 L8192 Hq64 Hkv8);
+      fp8:   the prefill with e4m3 q, k, v (one scale per head);
       varlen: a prefill batch of 12 packed sequences of mixed lengths;
       prologue: bias + YaRN rotary embedding + split of the prefill's QKV rows;
       long:  the long-context layers (window 128 at L = 131072, dense at L = 32768)."""
@@ -483,6 +484,29 @@ def prefill_legs(dev, which=("bwd", "train", "varlen", "prologue", "long"), reps
         run_shape("", B, L, 1.0, 2002, (0, WIN), True, False)
     if "train" in which:
         run_shape("train_", 8, 8192, 1.0, 2003, (0, WIN), True, True)
+    if "fp8" in which:
+        # the gpt-oss-20b prefill with e4m3 q, k, v (one scale per head), both layers
+        from gqa_softmax_attention_attn_b200.inputs import quantize_e4m3_per_head
+
+        t = device_prefill(B, L, HQ, HKV, 1.0, 2009, dev, False)
+        q8, qs = quantize_e4m3_per_head(t["q"])
+        k8, ks = quantize_e4m3_per_head(t["k"])
+        v8, vs = quantize_e4m3_per_head(t["v"])
+        out = torch.empty(B, L, HQ, D, dtype=torch.bfloat16, device=dev)
+        lse = torch.empty(B, HQ, L, device=dev, dtype=torch.float32)
+        shape = f"B{B} L{L} Hq{HQ} Hkv{HKV} D{D}, e4m3 q/k/v"
+        nbytes = B * L * HQ * D + 2 * B * L * HKV * D + 4 * (HQ + 2 * HKV) + 2 * B * L * HQ * D + 4 * B * HQ * L
+        ws = torch.empty(attn.attn_sink_fwd_fp8_workspace_size(B, L, HKV, D), dtype=torch.uint8, device=dev)
+        for window in (0, WIN):
+            fn = lambda: attn.attn_sink_fwd_fp8(q8, k8, v8, qs, ks, vs, t["sinks"], out, lse, window, SCALE, ws,
+                                                stream)
+            ms = timed(dev, fn, reps, warmup, flush)
+            tag = "dense" if window <= 0 else "window128"
+            e = leg_entry(ms, fwd_flops(B, L, HQ, window), nbytes, "tensor" if window <= 0 else "hbm", shape)
+            # the score product runs at the 8-bit rate (twice the bf16 peak), P.V at the 16-bit one
+            e["frac_tensor_fp8_qk"] = e["TFLOP/s"] / (2 * peaks()[1])
+            legs[f"fp8_fwd_{tag}"] = e
+        assert attn.attn_sink_get_device_status(stream) == 0
     if "varlen" in which:
         # a prefill batch of mixed lengths packed back to back (seeded lengths in [256, 4096])
         import numpy as np
@@ -619,7 +643,7 @@ def main():
     ap.add_argument("--no-legs", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["decode", "bwd", "train", "varlen", "prologue", "long"], default=None,
+    ap.add_argument("--only", choices=["decode", "bwd", "train", "fp8", "varlen", "prologue", "long"], default=None,
                     help="run just one leg (reps = --steps, warm-up = --warmup); used for profiling")
     ap.add_argument("--decode-batch", type=int, default=None, help="sequences in the decode leg (default 64)")
     args = ap.parse_args()

@@ -14,6 +14,8 @@ from ._native import (  # noqa: F401
     attn_sink_bwd_workspace_size,
     attn_sink_decode,
     attn_sink_decode_fp8,
+    attn_sink_fwd_fp8,
+    attn_sink_fwd_fp8_workspace_size,
     attn_sink_decode_noalloc,
     attn_sink_decode_paged,
     attn_sink_decode_paged_workspace_size,

@@ -71,6 +71,10 @@ def load():
         lib.attn_sink_decode_workspace_size.restype = Z
         lib.attn_sink_decode_fp8.argtypes = [P] * 9 + [I] * 6 + [F, I, P, Z, P]
         lib.attn_sink_decode_fp8.restype = I
+        lib.attn_sink_fwd_fp8.argtypes = [P] * 9 + [I] * 7 + [F, P, Z, P]
+        lib.attn_sink_fwd_fp8.restype = I
+        lib.attn_sink_fwd_fp8_workspace_size.argtypes = [I] * 4
+        lib.attn_sink_fwd_fp8_workspace_size.restype = Z
         lib.attn_sink_decode_paged.argtypes = [P] * 8 + [I] * 8 + [F, I, P, Z, I, P]
         lib.attn_sink_decode_paged.restype = I
         lib.attn_sink_decode_paged_workspace_size.argtypes = [I] * 7
@@ -219,6 +223,29 @@ def attn_sink_decode_fp8(q, k_cache, v_cache, k_scale, v_scale, seqlens, sinks, 
                                      Hkv, D, int(window), float(scale), int(num_splits), ws_ptr, ws_bytes,
                                      _stream(stream))
     _check(rc, "attn_sink_decode_fp8")
+
+
+def attn_sink_fwd_fp8_workspace_size(B: int, Lk: int, Hkv: int, D: int) -> int:
+    return int(load().attn_sink_fwd_fp8_workspace_size(B, Lk, Hkv, D))
+
+
+def attn_sink_fwd_fp8(q, k, v, q_scale, k_scale, v_scale, sinks, out, lse, window: int, scale: float, workspace,
+                      stream=None):
+    """q [B,Lq,Hq,D], k/v [B,Lk,Hkv,D] e4m3 codes (uint8 or float8_e4m3fn), q_scale [Hq], k_scale/v_scale
+    [Hkv] fp32, workspace of attn_sink_fwd_fp8_workspace_size bytes -> writes out [B,Lq,Hq,D] bf16,
+    lse [B,Hq,Lq]."""
+    B, Lq, Hq, D = q.shape
+    Lk, Hkv = k.shape[1], k.shape[2]
+    for name, c in (("q", q), ("k", k), ("v", v)):
+        if c.element_size() != 1:
+            raise TypeError(f"{name} must hold one-byte e4m3 codes, got {c.dtype}")
+    rc = load().attn_sink_fwd_fp8(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(q_scale, "q_scale", torch.float32),
+                                  _dev(k_scale, "k_scale", torch.float32), _dev(v_scale, "v_scale", torch.float32),
+                                  _dev(sinks, "sinks", torch.float32), _dev(out, "out", torch.bfloat16),
+                                  _dev(lse, "lse", torch.float32), B, Lq, Lk, Hq, Hkv, D, int(window), float(scale),
+                                  _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+                                  _stream(stream))
+    _check(rc, "attn_sink_fwd_fp8")
 
 
 def attn_sink_decode_paged_workspace_size(B: int, Hq: int, D: int, max_pages_per_seq: int, page_size: int,

@@ -191,6 +191,12 @@ long long wait_timeout_ns() { return g_timeout_ns.load(); }
 bool encode_tensor_map_4d(void *map, void *gaddr, int elem_bytes, const uint64_t dims[4],
                           const uint64_t strides_bytes[3], const uint32_t box[4], bool swizzle128)
 {
+    return encode_tensor_map_4d_sw(map, gaddr, elem_bytes, dims, strides_bytes, box, swizzle128 ? 128 : 0);
+}
+
+bool encode_tensor_map_4d_sw(void *map, void *gaddr, int elem_bytes, const uint64_t dims[4],
+                             const uint64_t strides_bytes[3], const uint32_t box[4], int swizzle_bytes)
+{
     std::call_once(g_encode_once, []() {
         void *fn = nullptr;
         cudaDriverEntryPointQueryResult q;
@@ -201,6 +207,7 @@ bool encode_tensor_map_4d(void *map, void *gaddr, int elem_bytes, const uint64_t
             cudaGetLastError();
     });
     if (!g_encode || (elem_bytes != 1 && elem_bytes != 2 && elem_bytes != 4)) return false;
+    if (swizzle_bytes != 0 && swizzle_bytes != 64 && swizzle_bytes != 128) return false;
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     const CUtensorMapDataType dt = elem_bytes == 1   ? CU_TENSOR_MAP_DATA_TYPE_UINT8
                                    : elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
@@ -209,7 +216,9 @@ bool encode_tensor_map_4d(void *map, void *gaddr, int elem_bytes, const uint64_t
                                 reinterpret_cast<const cuuint64_t *>(dims),
                                 reinterpret_cast<const cuuint64_t *>(strides_bytes),
                                 reinterpret_cast<const cuuint32_t *>(box), estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                                swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                                swizzle_bytes == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                      : CU_TENSOR_MAP_SWIZZLE_NONE,
                                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -270,6 +279,34 @@ int attn_sink_fwd(const void *q, const void *k, const void *v, const float *sink
                                                     static_cast<float *>(out), lse, s, st));
     if (!fwd_tc_supported(s)) return ATTN_SINK_ERR_UNSUPPORTED;
     return launch_status(launch_fwd_tc(q, k, v, sinks, out, lse, s, st));
+}
+
+size_t attn_sink_fwd_fp8_workspace_size(int B, int Lk, int Hkv, int D)
+{
+    if (B <= 0 || Lk <= 0 || Hkv <= 0 || D <= 0) return 0;
+    AttnShape s{B, 1, Lk, Hkv, Hkv, D, 0, 1.f};
+    return fwd_fp8_workspace_bytes(s);
+}
+
+int attn_sink_fwd_fp8(const void *q, const void *k, const void *v, const float *q_scale, const float *k_scale,
+                      const float *v_scale, const float *sinks, void *out, float *lse, int B, int Lq, int Lk, int Hq,
+                      int Hkv, int D, int window, float scale, void *workspace, size_t ws_bytes, void *stream)
+{
+    if (!q || !k || !v || !q_scale || !k_scale || !v_scale || !sinks || !out || !lse) return ATTN_SINK_ERR_INVALID_ARG;
+    int rc = check_common(B, Lq, Lk, Hq, Hkv, D, ATTN_SINK_DTYPE_BF16);
+    if (rc != ATTN_SINK_OK) return rc;
+    if (!(scale > 0.f && scale < INFINITY)) return ATTN_SINK_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q_scale) || !aligned16(k_scale) ||
+        !aligned16(v_scale) || !aligned16(out) || !aligned16(lse) || !aligned16(sinks))
+        return ATTN_SINK_ERR_MISALIGNED;
+    AttnShape s{B, Lq, Lk, Hq, Hkv, D, window, scale};
+    if (!workspace || ws_bytes < fwd_fp8_workspace_bytes(s)) return ATTN_SINK_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return ATTN_SINK_ERR_MISALIGNED;
+    rc = ensure_device();
+    if (rc != ATTN_SINK_OK) return rc;
+    if (!fwd_tc_supported(s)) return ATTN_SINK_ERR_UNSUPPORTED;
+    return launch_status(launch_fwd_tc_fp8(q, k, v, q_scale, k_scale, v_scale, sinks, out, lse, workspace, s,
+                                           static_cast<cudaStream_t>(stream)));
 }
 
 int attn_sink_fwd_varlen(const void *q, const void *k, const void *v, const float *sinks, void *out, float *lse,

@@ -119,33 +119,9 @@ __device__ __forceinline__ void mma16816_f16(float (&d)[4], const uint32_t (&a)[
                  : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// two e4m3 codes (low byte first) -> their exact values as an f16 pair
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes)
-{
-    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two_codes & 0xffffu), __NV_E4M3);
-    return (uint32_t)h.x | ((uint32_t)h.y << 16);
-}
-
-__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi)
-{
-    const __half2 v = __floats2half2_rn(lo, hi);
-    return *reinterpret_cast<const uint32_t *>(&v);
-}
-
 // byte offset of (row, 16-byte chunk) in a 128-byte-swizzled tile
 __device__ __forceinline__ uint32_t swz(int row, int chunk) { return row * 128 + ((chunk ^ (row & 7)) << 4); }
 
-// 16 e4m3 codes (byte i = element i) -> their 16 exact f16 values, elements
-// 0-7 in lo and 8-15 in hi (element 2m in the low half of word m)
-__device__ __forceinline__ void e4m3x16_to_f16(const uint4 &raw, uint4 &lo, uint4 &hi)
-{
-    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-    uint32_t o[8];
-#pragma unroll
-    for (int m = 0; m < 8; ++m) o[m] = e4m3x2_to_f16x2(w[m >> 1] >> (16 * (m & 1)));
-    lo = make_uint4(o[0], o[1], o[2], o[3]);
-    hi = make_uint4(o[4], o[5], o[6], o[7]);
-}
 
 template <bool kRows16, bool kPaged, bool kFp8>
 __global__ void __launch_bounds__(kThreads)

@@ -108,18 +108,26 @@ constexpr bool FWD_SPEC = ATTN_SINK_FWD_SPEC != 0;
 constexpr int kClcDepthDense = 1;
 constexpr int pow2_at_least(int x) { return x <= 32 ? 32 : x <= 64 ? 64 : x <= 128 ? 128 : x <= 256 ? 256 : 512; }
 
-template <int BN, int NS, int CPS, int SPLIT>
+// F8: q and k as e4m3 codes (one fp32 scale per query head for q, per KV head
+// for k), S = Q K^T on the 8-bit tensor-core path (the products of e4m3
+// values are exact, accumulated in fp32); v arrives widened exactly to f16
+// (by widen_e4m3_kernel; its scale per KV head multiplies O), so P (f16) V
+// runs on the 16-bit path.
+template <int BN, int NS, int CPS, int SPLIT, bool F8 = false>
 struct FwdCfg {
     static_assert(SPLIT == 1 || SPLIT == 2, "one or two softmax warps per row");
     static_assert(BN % (16 * SPLIT) == 0, "each softmax warp takes whole 16-column chunks");
     static constexpr int kThreads = 64 + 128 * SPLIT;
     static constexpr int kCols = BN / SPLIT;  // score columns per softmax thread
-    static constexpr int kQBytes = kM * kD * 2;
-    static constexpr int kKVBytes = BN * kD * 2;
+    static constexpr int kEB = F8 ? 1 : 2;  // bytes per q, k element (v is 16-bit either way)
+    static constexpr int kQBytes = kM * kD * kEB;
+    static constexpr int kKBytes = BN * kD * kEB;
+    static constexpr int kVBytes = BN * kD * 2;
     static constexpr int kOffQ = 0;  // two Q buffers
     static constexpr int kOffK = 2 * kQBytes;
-    static constexpr int kOffV = kOffK + NS * kKVBytes;
-    static constexpr int kOffBar = kOffV + NS * kKVBytes;
+    static constexpr int kOffV = kOffK + NS * kKBytes;
+    static_assert(kQBytes % 1024 == 0 && kKBytes % 1024 == 0 && kVBytes % 1024 == 0, "tiles on 1024-byte boundaries");
+    static constexpr int kOffBar = kOffV + NS * kVBytes;
     // q_full[2], q_empty[2], k_full[NS], k_empty[NS], v_full[NS], v_empty[NS],
     // s_full[2], p_full[2], o_done, o_free, drain, xchg[4], item_full[4], item_empty[4], clc[kClcDepthDense]
     static constexpr int kNumBar = 4 + 4 * NS + 4 + 3 + 4 + 8 + kClcDepthDense;
@@ -144,6 +152,7 @@ struct FwdTcParams {
     const int *cu_q, *cu_k;  // packed ragged sequences (else nullptr)
     int total_q, total_k;
     long long lse_hs;        // lse stride between heads: Lq, or total_q for packed sequences
+    const float *q_scale, *k_scale, *v_scale;  // F8: per query head, per KV head, per KV head
     int G, Gp, P;  // group size, query heads packed per tile, positions per tile
     int n_ptiles, n_htiles, n_items;
     float c_log2;  // scale * log2(e)
@@ -205,12 +214,12 @@ __device__ __forceinline__ bool wait_noabort(uint64_t *bar, uint32_t parity, uns
     return mbar_wait(bar, parity, &never, status, tmo > 1000000000LL ? tmo : 1000000000LL);
 }
 
-template <int BN, int NS, int EMU, int CPS, int SPLIT>
-__global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT>::kThreads, CPS)
+template <int BN, int NS, int EMU, int CPS, int SPLIT, bool F8 = false>
+__global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT, F8>::kThreads, CPS)
     fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdTcParams p)
 {
-    using Cfg = FwdCfg<BN, NS, CPS, SPLIT>;
+    using Cfg = FwdCfg<BN, NS, CPS, SPLIT, F8>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kOffBar);
@@ -332,15 +341,15 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT>::kThreads, CPS)
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&k_full[st], Cfg::kKVBytes);
-                    tma_load_4d(smem + Cfg::kOffK + st * Cfg::kKVBytes, &tmK, 0, g, t.krow0 + j0, t.tb, &k_full[st]);
+                    mbar_arrive_expect_tx(&k_full[st], Cfg::kKBytes);
+                    tma_load_4d(smem + Cfg::kOffK + st * Cfg::kKBytes, &tmK, 0, g, t.krow0 + j0, t.tb, &k_full[st]);
                     ++k_issued[st];
                     if (!mbar_wait(&v_empty[st], ph ^ 1u, abort_flag, p.status, p.timeout_ns)) {
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&v_full[st], Cfg::kKVBytes);
-                    tma_load_4d(smem + Cfg::kOffV + st * Cfg::kKVBytes, &tmV, 0, g, t.krow0 + j0, t.tb, &v_full[st]);
+                    mbar_arrive_expect_tx(&v_full[st], Cfg::kVBytes);
+                    tma_load_4d(smem + Cfg::kOffV + st * Cfg::kVBytes, &tmV, 0, g, t.krow0 + j0, t.tb, &v_full[st]);
                     ++v_issued[st];
                 }
                 ++item_n;
@@ -359,8 +368,8 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT>::kThreads, CPS)
         // ------------------------------------------------------------ MMA issuer
         // The whole warp runs this loop (so every operand is warp-uniform) and
         // one elected lane issues the MMAs and their commits.
-        const uint32_t id_s = idesc_bf16_f32(kM, BN, 0);
-        const uint32_t id_pv = idesc_bf16_f32(kM, kD, 1);
+        const uint32_t id_s = F8 ? idesc_e4m3_f32(kM, BN) : idesc_bf16_f32(kM, BN, 0);
+        const uint32_t id_pv = F8 ? idesc_f16_f32(kM, kD, 1) : idesc_bf16_f32(kM, kD, 1);
         const uint32_t k_addr = smem_u32(smem + Cfg::kOffK);
         const uint32_t v_addr = smem_u32(smem + Cfg::kOffV);
         auto wait_all = [&](uint64_t *bar, uint32_t parity) {
@@ -376,7 +385,7 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT>::kThreads, CPS)
             if (!wait_all(&p_full[sb], (t >> 1) & 1u)) return false;
             if (!wait_all(&v_full[st], (t / NS) & 1u)) return false;
             tc_fence_after();
-            const uint32_t vb = v_addr + st * Cfg::kKVBytes;
+            const uint32_t vb = v_addr + st * Cfg::kVBytes;
             if (elect_one()) {
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk) {
@@ -408,13 +417,21 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT>::kThreads, CPS)
                     break;
                 }
                 tc_fence_after();
-                const uint32_t kb = k_addr + st * Cfg::kKVBytes;
+                const uint32_t kb = k_addr + st * Cfg::kKBytes;
                 if (elect_one()) {
+                    if (F8) {
+                        // e4m3 rows of 64 bytes, 64-byte swizzle: K = 32 codes (32 bytes) per step
+#pragma unroll
+                        for (int kk = 0; kk < kD / 32; ++kk)
+                            mma_ss_f8(tmem + Cfg::kTmS0 + sb * BN, smem_desc_sw64(q_addr + kk * 32, 512),
+                                      smem_desc_sw64(kb + kk * 32, 512), id_s, kk > 0 ? 1u : 0u);
+                    } else {
 #pragma unroll
                     for (int kk = 0; kk < kD / 16; ++kk) {
                         const uint64_t adesc = smem_desc_sw128(q_addr + kk * 32, 16, 1024);
                         const uint64_t bdesc = smem_desc_sw128(kb + kk * 32, 16, 1024);
                         mma_ss(tmem + Cfg::kTmS0 + sb * BN, adesc, bdesc, id_s, kk > 0 ? 1u : 0u);
+                    }
                     }
                     mma_commit(&s_full[sb]);
                     mma_commit(&k_empty[st]);
@@ -449,7 +466,7 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT>::kThreads, CPS)
         const int half = SPLIT == 2 ? (warp - 2) >> 2 : 0;
         const int r = quad * 32 + lane;
         const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
-        const float C = p.c_log2;
+        float C = p.c_log2;  // F8: times the row's q and k scales (set per item)
         uint32_t it = 0, xc = 0;
         bool ok = true;
         // publish v, get the other half's value (bounded wait; false on abort)
@@ -470,6 +487,7 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT>::kThreads, CPS)
             const bool row_valid = pos < t.Lq;
             const long pabs = pos + ((long)t.Lk - t.Lq);
             const float sink2 = p.sinks[h] * kLog2e;  // the sink logit in log2 units
+            if (F8) C = p.c_log2 * p.q_scale[h] * p.k_scale[h / p.G];
             float m = sink2;                           // reference maximum, log2 units
             // running sum, seeded with the sink's mass (in column half 0 only)
             float l = (sink2 == -INFINITY || half != 0) ? 0.f : 1.f;
@@ -529,7 +547,7 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT>::kThreads, CPS)
                             const bool emu = kEmu && (EMU == 4 ? (e & 1) != 0 : (e & 3) == EMU);
                             const float2 pe = emu ? fast_exp2x2(x) : make_float2(ex2(x.x), ex2(x.y));
                             acc[e & 1] = fadd2(acc[e & 1], pe);
-                            pk[e] = pack_bf16x2(pe.x, pe.y);
+                            pk[e] = F8 ? pack_f16x2(pe.x, pe.y) : pack_bf16x2(pe.x, pe.y);
                         }
                         if (kTrack) {
 #pragma unroll
@@ -642,7 +660,7 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT>::kThreads, CPS)
                 l += other;
             }
             if (row_valid) {
-                const float inv = l > 0.f ? 1.f / l : 0.f;
+                const float inv = l > 0.f ? (F8 ? p.v_scale[h / p.G] : 1.f) / l : 0.f;
                 uint4 *dst =
                     reinterpret_cast<uint4 *>(p.out + ((size_t)(t.orow0 + pos) * p.Hq + h) * kD + half * kOC);
 #pragma unroll
@@ -671,12 +689,16 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT>::kThreads, CPS)
     }
 }
 
-template <int BN, int NS, int EMU, int CPS, int SPLIT>
+template <int BN, int NS, int EMU, int CPS, int SPLIT, bool F8 = false>
 cudaError_t launch_cfg(const void *q, const void *k, const void *v, const float *sinks, void *out, float *lse,
-                       const AttnShape &s, cudaStream_t st)
+                       const AttnShape &s, cudaStream_t st, const float *q_scale = nullptr,
+                       const float *k_scale = nullptr, const float *v_scale = nullptr)
 {
-    using Cfg = FwdCfg<BN, NS, CPS, SPLIT>;
+    using Cfg = FwdCfg<BN, NS, CPS, SPLIT, F8>;
     FwdTcParams p;
+    p.q_scale = q_scale;
+    p.k_scale = k_scale;
+    p.v_scale = v_scale;
     p.B = s.B;
     p.Lq = s.Lq;
     p.Lk = s.Lk;
@@ -710,23 +732,28 @@ cudaError_t launch_cfg(const void *q, const void *k, const void *v, const float 
     const uint64_t qrows = s.cu_q ? (uint64_t)s.total_q : (uint64_t)s.Lq;
     const uint64_t krows = s.cu_q ? (uint64_t)s.total_k : (uint64_t)s.Lk;
     const uint64_t outer = s.cu_q ? 1u : (uint64_t)s.B;
+    // bf16: 128-byte rows, 128-byte swizzle; e4m3 q and k: 64-byte rows,
+    // 64-byte swizzle; v (bf16, or f16 widened from e4m3) as bf16
+    constexpr int eb = Cfg::kEB;
+    constexpr int swz_qk = F8 ? 64 : 128;
     {
         const uint64_t dims[4] = {(uint64_t)kD, (uint64_t)s.Hq, qrows, outer};
-        const uint64_t strides[3] = {(uint64_t)kD * 2, (uint64_t)s.Hq * kD * 2, qrows * s.Hq * kD * 2};
+        const uint64_t strides[3] = {(uint64_t)kD * eb, (uint64_t)s.Hq * kD * eb, qrows * s.Hq * kD * eb};
         const uint32_t box[4] = {(uint32_t)kD, (uint32_t)p.Gp, (uint32_t)p.P, 1u};
-        if (!encode_tensor_map_4d(&mq, const_cast<void *>(q), 2, dims, strides, box, true))
+        if (!encode_tensor_map_4d_sw(&mq, const_cast<void *>(q), eb, dims, strides, box, swz_qk))
             return cudaErrorInvalidValue;
     }
     {
         const uint64_t dims[4] = {(uint64_t)kD, (uint64_t)s.Hkv, krows, outer};
-        const uint64_t strides[3] = {(uint64_t)kD * 2, (uint64_t)s.Hkv * kD * 2, krows * s.Hkv * kD * 2};
+        const uint64_t strides[3] = {(uint64_t)kD * eb, (uint64_t)s.Hkv * kD * eb, krows * s.Hkv * kD * eb};
         const uint32_t box[4] = {(uint32_t)kD, 1u, (uint32_t)BN, 1u};
-        if (!encode_tensor_map_4d(&mk, const_cast<void *>(k), 2, dims, strides, box, true))
+        if (!encode_tensor_map_4d_sw(&mk, const_cast<void *>(k), eb, dims, strides, box, swz_qk))
             return cudaErrorInvalidValue;
-        if (!encode_tensor_map_4d(&mv, const_cast<void *>(v), 2, dims, strides, box, true))
+        const uint64_t vstrides[3] = {(uint64_t)kD * 2, (uint64_t)s.Hkv * kD * 2, krows * s.Hkv * kD * 2};
+        if (!encode_tensor_map_4d_sw(&mv, const_cast<void *>(v), 2, dims, vstrides, box, 128))
             return cudaErrorInvalidValue;
     }
-    auto kern = fwd_tc_kernel<BN, NS, EMU, CPS, SPLIT>;
+    auto kern = fwd_tc_kernel<BN, NS, EMU, CPS, SPLIT, F8>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
     if (e != cudaSuccess) return e;
     // one CTA per item: as many start as fit (kCtasPerSm per SM), the rest are
@@ -753,6 +780,43 @@ cudaError_t launch_fwd_tc(const void *q, const void *k, const void *v, const flo
                           ATTN_SINK_FWD_BAND_SPLIT>(q, k, v, sinks, out, lse, s, st);
     return launch_cfg<ATTN_SINK_FWD_DENSE_BN, ATTN_SINK_FWD_DENSE_NS, ATTN_SINK_FWD_DENSE_EMU, ATTN_SINK_FWD_DENSE_CPS,
                       ATTN_SINK_FWD_DENSE_SPLIT>(q, k, v, sinks, out, lse, s, st);
+}
+
+namespace {
+// e4m3 -> f16, exactly (16 codes per thread, 16-byte loads, 32-byte stores)
+__global__ void __launch_bounds__(256) widen_e4m3_kernel(const uint8_t *__restrict__ src, uint8_t *__restrict__ dst,
+                                                         size_t n16)
+{
+    const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n16) return;
+    uint4 lo, hi;
+    e4m3x16_to_f16(reinterpret_cast<const uint4 *>(src)[i], lo, hi);
+    reinterpret_cast<uint4 *>(dst)[2 * i] = lo;
+    reinterpret_cast<uint4 *>(dst)[2 * i + 1] = hi;
+}
+}  // namespace
+
+size_t fwd_fp8_workspace_bytes(const AttnShape &s) { return (size_t)s.B * s.Lk * s.Hkv * s.D * 2; }
+
+cudaError_t launch_fwd_tc_fp8(const void *q, const void *k, const void *v, const float *q_scale,
+                              const float *k_scale, const float *v_scale, const float *sinks, void *out, float *lse,
+                              void *v16, const AttnShape &s, cudaStream_t st)
+{
+    if (s.cu_q) return cudaErrorInvalidValue;  // fixed-length batches only
+    // v widened once into the workspace; the attention kernels read it as 16-bit tiles
+    const size_t n16 = (size_t)s.B * s.Lk * s.Hkv * s.D / 16;
+    if ((n16 + 255) / 256 > 0x7fffffffu) return cudaErrorInvalidValue;
+    if (n16 > 0) {
+        widen_e4m3_kernel<<<(unsigned)((n16 + 255) / 256), 256, 0, st>>>(static_cast<const uint8_t *>(v),
+                                                                        static_cast<uint8_t *>(v16), n16);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    if (s.window > 0 && s.window <= 1024)
+        return launch_cfg<ATTN_SINK_FWD_BAND_BN, ATTN_SINK_FWD_BAND_NS, -1, ATTN_SINK_FWD_BAND_CPS, 1, true>(
+            q, k, v16, sinks, out, lse, s, st, q_scale, k_scale, v_scale);
+    return launch_cfg<ATTN_SINK_FWD_DENSE_BN, ATTN_SINK_FWD_DENSE_NS, ATTN_SINK_FWD_DENSE_EMU, ATTN_SINK_FWD_DENSE_CPS,
+                      1, true>(q, k, v16, sinks, out, lse, s, st, q_scale, k_scale, v_scale);
 }
 
 }  // namespace attn_sink

@@ -102,6 +102,12 @@ bool fwd_band_supported(const AttnShape &s);
 // Tensor-core (tcgen05 / TMEM / TMA) bf16 prefill forward.
 cudaError_t launch_fwd_tc(const void *q, const void *k, const void *v, const float *sinks, void *out,
                           float *lse, const AttnShape &s, cudaStream_t st);
+// e4m3 q, k, v with fp32 scales per query head (q) and per KV head (k, v);
+// fixed-length batches; v16 holds fwd_fp8_workspace_bytes (v widened to f16)
+size_t fwd_fp8_workspace_bytes(const AttnShape &s);
+cudaError_t launch_fwd_tc_fp8(const void *q, const void *k, const void *v, const float *q_scale,
+                              const float *k_scale, const float *v_scale, const float *sinks, void *out, float *lse,
+                              void *v16, const AttnShape &s, cudaStream_t st);
 bool fwd_tc_supported(const AttnShape &s);
 
 // bf16 split-KV decode: TMA-staged K/V, tensor-core (mma.sync) group scores.
@@ -125,5 +131,8 @@ cudaError_t launch_qkv_prologue(const void *qkv, const float *bias, const int *p
 // Driver entry point for cuTensorMapEncodeTiled (resolved once through the runtime).
 bool encode_tensor_map_4d(void *map, void *gaddr, int elem_bytes, const uint64_t dims[4],
                           const uint64_t strides_bytes[3], const uint32_t box[4], bool swizzle128);
+// the same with the swizzle span given in bytes (0, 64 or 128)
+bool encode_tensor_map_4d_sw(void *map, void *gaddr, int elem_bytes, const uint64_t dims[4],
+                             const uint64_t strides_bytes[3], const uint32_t box[4], int swizzle_bytes);
 
 }  // namespace attn_sink

@@ -126,6 +126,40 @@ ATTN_SINK_API int attn_sink_fwd_varlen(const void *q, const void *k, const void 
                   int window, float scale, void *stream);
 
 /*
+ * Prefill forward with q, k and v in FP8 (e4m3): the operation of
+ * attn_sink_fwd with q, k and v read at one byte per element.  The pages
+ * serve gpt-oss at FP8 precision ("GPT-OSS on day 0", section "GPT-OSS a
+ * Hopper"); the format and its scale granularity are not given there: here
+ * every query head has one fp32 scale for q and every KV head one for k and
+ * one for v (the value of an element is code * its head's scale).
+ *   q        [B, Lq, Hq, D] e4m3 codes     k, v [B, Lk, Hkv, D] e4m3 codes
+ *            (OCP FP8 E4M3: bias 7, 3 mantissa bits, subnormals, 0x7f / 0xff
+ *            NaN; NaN codes in the inputs give NaN outputs)
+ *   q_scale  [Hq] fp32, k_scale, v_scale [Hkv] fp32, device; positive and
+ *            finite (the kernel takes the row maximum of the raw products)
+ *   sinks, window, scale: as attn_sink_fwd (scale positive and finite)
+ *   out      [B, Lq, Hq, D] bf16          lse [B, Hq, Lq] fp32
+ *   workspace device memory of attn_sink_fwd_fp8_workspace_size(B, Lk, Hkv, D)
+ *            bytes (v widened to f16), 16-byte aligned, owned by the caller;
+ *            its contents on return are unspecified.
+ * Q K^T runs on the 8-bit tensor-core path: the products of e4m3 values are
+ * exact and accumulate in fp32; the scales then multiply the logits.  V is
+ * widened exactly to f16 (one pass into the workspace) and P (in f16) times V
+ * runs on the 16-bit path, so the result carries the rounding of the bf16
+ * forward, not of FP8 attention probabilities.  Fixed-length batches only.
+ * Errors as attn_sink_fwd, INVALID_ARG for a null scale pointer, WORKSPACE
+ * for a missing or short workspace.  Nothing is allocated; asynchronous on
+ * stream.
+ */
+ATTN_SINK_API int attn_sink_fwd_fp8(const void *q, const void *k, const void *v, const float *q_scale,
+                  const float *k_scale, const float *v_scale, const float *sinks, void *out,
+                  float *lse, int B, int Lq, int Lk, int Hq, int Hkv, int D, int window,
+                  float scale, void *workspace, size_t ws_bytes, void *stream);
+
+/* Bytes of workspace attn_sink_fwd_fp8 needs (B * Lk * Hkv * D * 2; 0 for a non-positive size). */
+ATTN_SINK_API size_t attn_sink_fwd_fp8_workspace_size(int B, int Lk, int Hkv, int D);
+
+/*
  * QKV prologue: the step just before attention, in one pass over the QKV
  * projection's output.  The pages give gpt-oss QKV projections with biases
  * and YaRN rotary position encoding "as in DeepSeek-V3" ("GPT-OSS on day 0",
@@ -213,7 +247,7 @@ ATTN_SINK_API size_t attn_sink_decode_workspace_size(int B, int Hq, int D, int L
  *   seqlens, sinks, window, scale, num_splits, workspace: as attn_sink_decode
  *            (the workspace size is attn_sink_decode_workspace_size's).
  *   out      [B, Hq, D] bf16           lse [B, Hq] fp32
- * Each code is widened exactly (e4m3 -> bf16) and the scales are applied in
+ * Each code is widened exactly (e4m3 -> f16) and the scales are applied in
  * fp32: K's to the logits, V's to the output.  Cache rows beyond a sequence's
  * length may hold any bytes, NaN codes included.  Errors as attn_sink_decode;
  * a null scale pointer is INVALID_ARG.

@@ -195,6 +195,20 @@ def decode_fp8(q, k_codes, v_codes, k_scale, v_scale, seqlens, sinks, window: in
     return decode(q, k, v, seqlens, sinks, window, scale)
 
 
+def fwd_fp8(q_codes, k_codes, v_codes, q_scale, k_scale, v_scale, sinks, window: int, scale: float):
+    """Prefill forward over e4m3 inputs: every code is widened to its exact
+    value and multiplied by its head's scale in fp64 (q per query head, k and
+    v per KV head), then the forward definition runs unchanged.  q [B, Lq,
+    Hq, D], k/v [B, Lk, Hkv, D] codes; scales [Hq], [Hkv], [Hkv]."""
+    qs = np.asarray(_f64(q_scale))
+    ks = np.asarray(_f64(k_scale))
+    vs = np.asarray(_f64(v_scale))
+    q = e4m3_values(q_codes) * qs[None, None, :, None]
+    k = e4m3_values(k_codes) * ks[None, None, :, None]
+    v = e4m3_values(v_codes) * vs[None, None, :, None]
+    return fwd(q, k, v, sinks, window, scale)
+
+
 def fwd_varlen(q, k, v, sinks, cu_q, cu_k, window: int, scale: float):
     """Packed ragged sequences: sequence b is the independent problem
     q[cu_q[b]:cu_q[b+1]] against k, v[cu_k[b]:cu_k[b+1]], run through fwd with

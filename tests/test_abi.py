@@ -116,6 +116,34 @@ def test_decode_fp8_host_checks():
     assert call(wbytes=need - 4) == WORKSPACE
 
 
+def test_fwd_fp8_host_checks():
+    """Argument checks of the FP8 prefill, all on the host (no kernel runs)."""
+    lib = attn.load()
+    q, k, v, qs, ks, vs, s, o = _fake(8)
+    l = _fake(9)[8]
+
+    ws = _fake(10)[9]
+    need = attn.attn_sink_fwd_fp8_workspace_size(1, 128, 2, 64)
+    assert need == 1 * 128 * 2 * 64 * 2
+
+    def call(q_scale=qs, k_scale=ks, B=1, Lq=128, Lk=128, Hq=8, Hkv=2, D=64, scale=0.125, qq=q, w=ws, wbytes=need):
+        return lib.attn_sink_fwd_fp8(qq, k, v, q_scale, k_scale, vs, s, o, l, B, Lq, Lk, Hq, Hkv, D, 0, scale, w,
+                                     wbytes, None)
+
+    assert call(q_scale=None) == INVALID
+    assert call(k_scale=None) == INVALID
+    assert call(B=0) == INVALID
+    assert call(Hkv=3) == INVALID
+    assert call(D=128) == UNSUPPORTED
+    assert call(scale=0.0) == UNSUPPORTED
+    assert call(scale=-1.0) == UNSUPPORTED
+    assert call(qq=q + 4) == MISALIGNED
+    assert call(q_scale=qs + 4) == MISALIGNED
+    assert call(w=None, wbytes=0) == WORKSPACE
+    assert call(wbytes=need - 1) == WORKSPACE
+    assert call(w=ws + 4) == MISALIGNED
+
+
 def test_decode_paged_host_checks():
     lib = attn.load()
     q, kp, vp, pt, sl, s, o, l = _fake(8)

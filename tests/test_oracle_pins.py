@@ -354,6 +354,30 @@ def test_decode_fp8_is_decode_of_the_scaled_codes():
         np.testing.assert_allclose(l2, l, rtol=0, atol=1e-12)
 
 
+def test_fwd_fp8_is_fwd_of_the_scaled_codes():
+    """fwd_fp8 = fwd over code * scale (q per query head, k and v per KV
+    head): checked against the forward of inputs widened by torch's own e4m3
+    cast, with per-head scales that differ (a head mapped to the wrong scale
+    fails), and by the scale invariances (q's and k's scales only rescale the
+    logits, v's scale the output)."""
+    from gqa_softmax_attention_attn_b200.inputs import prefill_inputs, quantize_e4m3_per_head
+
+    t = prefill_inputs(2, 24, 30, 4, 2, 16, torch.float32, 0.5, 1.0, seed=83)
+    q8, qs = quantize_e4m3_per_head(t["q"] * torch.linspace(0.5, 2.0, 4)[None, None, :, None])
+    k8, ks = quantize_e4m3_per_head(t["k"] * torch.tensor([1.0, 3.0])[None, None, :, None])
+    v8, vs = quantize_e4m3_per_head(t["v"])
+    assert len(set(qs.tolist())) == 4 and len(set(ks.tolist())) == 2
+    wid = lambda c, sc: c.view(torch.float8_e4m3fn).double() * sc.double()[None, None, :, None]
+    for window in (0, 5):
+        o, l = oracle.fwd_fp8(q8, k8, v8, qs, ks, vs, t["sinks"], window, 0.25)
+        ro, rl = oracle.fwd(wid(q8, qs), wid(k8, ks), wid(v8, vs), t["sinks"], window, 0.25)
+        np.testing.assert_allclose(o, ro, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(l, rl, rtol=0, atol=1e-12)
+        o2, l2 = oracle.fwd_fp8(q8, k8, v8, qs * 2, ks * 4, vs * 8, t["sinks"], window, 0.25 / 8)
+        np.testing.assert_allclose(o2, 8 * o, rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(l2, l, rtol=0, atol=1e-12)
+
+
 # ----------------------------------------------------------------------------- packed ragged sequences
 def test_fwd_varlen_is_the_batch_when_lengths_agree_and_skips_empty_sequences():
     """fwd_varlen over B equal-length sequences packed back to back equals fwd

@@ -26,8 +26,8 @@
 //    with P read back from TMEM.  Warps 2-5: one thread per row --
 //    tcgen05.ld of S, masking, the exp2 softmax, P written over S as bf16,
 //    conditional rescale of O, epilogue.  (Compile-time option SPLIT = 2:
-//    warps 2-9, two per row on half the columns each, trading partial maxima
-//    and sums through shared memory under a per-quadrant mbarrier.)
+//    warps 2-9, two per row on half the columns each, each half with its own
+//    online softmax and O accumulator, combined once per item.)
 //  * The running maximum used for the exponentials is only moved when the
 //    true maximum exceeds it by more than 2^8, so the O rescale (which must
 //    wait for the previous PV product) is rare; the result is exact either
@@ -86,8 +86,9 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 #define ATTN_SINK_FWD_DENSE_EMU 3
 #endif
 // softmax warps per row (1 or 2) per layer type; two warps per row (half the
-// columns each, partial maxima traded every tile) measured slower on both
-// layers of the gpt-oss-20b prefill (dense 239 vs 212 us, banded 52 vs 47 us)
+// columns each, each half its own online softmax and O, combined per item)
+// measured slower on the gpt-oss-20b prefill's dense layer (234 us at 64-key
+// tiles against 207 us), as did trading partial maxima every tile (239 vs 212)
 #ifndef ATTN_SINK_FWD_DENSE_SPLIT
 #define ATTN_SINK_FWD_DENSE_SPLIT 1
 #endif
@@ -136,7 +137,7 @@ struct FwdCfg {
     static_assert(32 + 16 * kClcDepthDense <= 128, "misc area");
     // row partials exchanged by the two softmax warps of a row: [2 slots][2 halves][128 rows]
     static constexpr int kOffXchg = kOffMisc + 128;
-    static constexpr int kTmemCols = pow2_at_least(2 * BN + kD);
+    static constexpr int kTmemCols = pow2_at_least(2 * BN + kD * SPLIT);  // S double buffer + one O per column half
     static constexpr int kCtasPerSm = CPS;  // CTAs resident per SM (TMEM, registers, shared memory)
     static_assert(kTmemCols * CPS <= 512, "tensor memory over-subscribed");
     // + slack for 1024-byte alignment; a CTA that takes all 512 TMEM columns
@@ -387,16 +388,18 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT, F8>::kThreads, CPS)
             tc_fence_after();
             const uint32_t vb = v_addr + st * Cfg::kVBytes;
             if (elect_one()) {
+                // V tile [BN keys][64 d] is the MN-major B operand: 16 keys = 2048 bytes per step.
+                // Column half hh's P (its 16-key blocks, bf16 pairs at the start of its own
+                // S columns) goes into its own O accumulator.
 #pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk) {
-                    // V tile [BN keys][64 d] is the MN-major B operand: 16 keys = 2048 bytes per step
-                    const uint64_t bdesc = smem_desc_sw128(vb + kk * 2048, BN * 128, 1024);
-                    // P of keys 16kk..16kk+15: 8 packed columns; the softmax warp of
-                    // column half h writes its P at the start of its own S columns
-                    const int hcol = (16 * kk / Cfg::kCols) * (Cfg::kCols / 2);
-                    mma_ts(tmem + Cfg::kTmO, tmem + Cfg::kTmS0 + sb * BN + kk * 8 + hcol, bdesc, id_pv,
-                           (!first || kk > 0) ? 1u : 0u);
-                }
+                for (int hh = 0; hh < SPLIT; ++hh)
+#pragma unroll
+                    for (int kk = 0; kk < BN / 16 / SPLIT; ++kk) {
+                        const int kb = hh * (BN / 16 / SPLIT) + kk;  // 16-key block of the tile
+                        const uint64_t bdesc = smem_desc_sw128(vb + kb * 2048, BN * 128, 1024);
+                        mma_ts(tmem + Cfg::kTmO + kD * hh, tmem + Cfg::kTmS0 + sb * BN + hh * Cfg::kCols + kk * 8,
+                               bdesc, id_pv, (!first || kk > 0) ? 1u : 0u);
+                    }
                 mma_commit(o_done);
                 mma_commit(&v_empty[st]);
             }
@@ -456,10 +459,13 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT, F8>::kThreads, CPS)
         // ------------------------------------------------------------ softmax + epilogue
         // SPLIT warps per row: the warp of column half h (warps 2-5: h = 0,
         // warps 6-9: h = 1) takes score columns [h kCols, (h + 1) kCols) of
-        // each tile and O columns [h 64 / SPLIT, ...).  The two halves of a row
-        // trade their partial maxima every tile (and their partial sums at the
-        // end of an item) through shared memory, ordered by the quadrant's
-        // exchange barrier, so both take the same reference maximum.
+        // each tile and runs its own online softmax over them (its own
+        // reference maximum, sum and O accumulator; the sink seeds half 0).
+        // At the end of an item the two halves trade their maxima and sums
+        // through shared memory, ordered by the quadrant's exchange barrier,
+        // combine O0 and O1 and write columns [h 64 / SPLIT, ...) each --
+        // exact, since each half's numerator and denominator share its own
+        // reference.
         constexpr int kC = Cfg::kCols;
         constexpr int kOC = kD / SPLIT;  // O columns per thread
         const int quad = warp & 3;
@@ -488,7 +494,7 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT, F8>::kThreads, CPS)
             const long pabs = pos + ((long)t.Lk - t.Lq);
             const float sink2 = p.sinks[h] * kLog2e;  // the sink logit in log2 units
             if (F8) C = p.c_log2 * p.q_scale[h] * p.k_scale[h / p.G];
-            float m = sink2;                           // reference maximum, log2 units
+            float m = half == 0 ? sink2 : -INFINITY;   // reference maximum, log2 units
             // running sum, seeded with the sink's mass (in column half 0 only)
             float l = (sink2 == -INFINITY || half != 0) ? 0.f : 1.f;
             // rows beyond Lq only need finite, unused values
@@ -558,7 +564,7 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT, F8>::kThreads, CPS)
                 };
                 bool rescale = false;
                 float alpha = 1.f;
-                if (FWD_SPEC && SPLIT == 1) {
+                if (FWD_SPEC) {
                     // The exponentials first, against the current reference (it
                     // only moves when the true maximum exceeds it by 2^8, so it
                     // rarely does), with the tile maximum found in the same pass;
@@ -585,14 +591,6 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT, F8>::kThreads, CPS)
 #pragma unroll
                         for (int k = 0; k < 8; ++k) mx[k] = fmax3(mx[k], sv[c + k], sv[c + 8 + k]);
                     float tmax = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
-                    if (SPLIT == 2) {
-                        float other;
-                        if (!trade(tmax, other)) {
-                            ok = false;
-                            break;
-                        }
-                        tmax = fmaxf(tmax, other);
-                    }
                     const float m_new = fmaxf(m, tmax * C);
                     rescale = m_new > m + kRescaleThreshold;
                     alpha = rescale ? ((m == -INFINITY) ? 0.f : ex2(m - m_new)) : 1.f;
@@ -616,15 +614,16 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT, F8>::kThreads, CPS)
                     }
                     tc_fence_after();
                     if (__any_sync(0xffffffffu, rescale)) {
-                        uint32_t o[kOC / 32][32];
+                        // this half's own O accumulator (all 64 columns)
+                        uint32_t o[kD / 32][32];
 #pragma unroll
-                        for (int c = 0; c < kOC / 32; ++c) tmem_ld32(trow + Cfg::kTmO + half * kOC + 32 * c, o[c]);
+                        for (int c = 0; c < kD / 32; ++c) tmem_ld32(trow + Cfg::kTmO + kD * half + 32 * c, o[c]);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int c = 0; c < kOC; ++c)
+                        for (int c = 0; c < kD; ++c)
                             o[c / 32][c % 32] = __float_as_uint(__uint_as_float(o[c / 32][c % 32]) * alpha);
 #pragma unroll
-                        for (int c = 0; c < kOC / 32; ++c) tmem_st32(trow + Cfg::kTmO + half * kOC + 32 * c, o[c]);
+                        for (int c = 0; c < kD / 32; ++c) tmem_st32(trow + Cfg::kTmO + kD * half + 32 * c, o[c]);
                     }
                 }
                 tmem_wait_st();
@@ -635,6 +634,20 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT, F8>::kThreads, CPS)
 
             // -------------------------------------------------------- epilogue
             uint32_t o[kOC / 32][32];
+            float a_me = 1.f, a_ot = 0.f;  // SPLIT == 2: weights of this half's and the other half's O
+            if (SPLIT == 2) {
+                // the two halves' reference maxima and sums -> one reference M
+                float m_o, l_o;
+                if (!trade(m, m_o) || !trade(l, l_o)) {
+                    ok = false;
+                    break;
+                }
+                const float M = fmaxf(m, m_o);
+                a_me = (m == -INFINITY) ? 0.f : ex2(m - M);
+                a_ot = (m_o == -INFINITY) ? 0.f : ex2(m_o - M);
+                l = l * a_me + l_o * a_ot;
+                m = M;
+            }
             if (t.n_tiles > 0) {
                 if (!__all_sync(0xffffffffu,
                                 mbar_wait(o_done, (it - 1) & 1u, abort_flag, p.status, p.timeout_ns))) {
@@ -642,22 +655,28 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT, F8>::kThreads, CPS)
                     break;
                 }
                 tc_fence_after();
+                if (SPLIT == 2) {
+                    // columns [32 half, 32 half + 32) of both halves' O
+                    uint32_t o0[32], o1[32];
+                    tmem_ld32(trow + Cfg::kTmO + 32 * half, o0);
+                    tmem_ld32(trow + Cfg::kTmO + kD + 32 * half, o1);
+                    tmem_wait_ld();
+                    tc_fence_before();
+                    mbar_arrive(o_free);  // the next item's first PV may overwrite O now
+                    const float a0 = half == 0 ? a_me : a_ot, a1 = half == 0 ? a_ot : a_me;
 #pragma unroll
-                for (int c = 0; c < kOC / 32; ++c) tmem_ld32(trow + Cfg::kTmO + half * kOC + 32 * c, o[c]);
-                tmem_wait_ld();
-                tc_fence_before();
-                mbar_arrive(o_free);  // the next item's first PV may overwrite O now
+                    for (int c = 0; c < 32; ++c)
+                        o[0][c] = __float_as_uint(__uint_as_float(o0[c]) * a0 + __uint_as_float(o1[c]) * a1);
+                } else {
+#pragma unroll
+                    for (int c = 0; c < kOC / 32; ++c) tmem_ld32(trow + Cfg::kTmO + 32 * c, o[c]);
+                    tmem_wait_ld();
+                    tc_fence_before();
+                    mbar_arrive(o_free);  // the next item's first PV may overwrite O now
+                }
             } else {
 #pragma unroll
                 for (int c = 0; c < kOC; ++c) o[c / 32][c % 32] = 0u;
-            }
-            if (SPLIT == 2) {
-                float other;
-                if (!trade(l, other)) {
-                    ok = false;
-                    break;
-                }
-                l += other;
             }
             if (row_valid) {
                 const float inv = l > 0.f ? (F8 ? p.v_scale[h / p.G] : 1.f) / l : 0.f;

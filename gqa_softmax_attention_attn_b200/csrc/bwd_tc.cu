@@ -376,11 +376,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int e4 = 0; e4 < 4; ++e4) {
                     const float4 l4 = l2v[4 * (c0 + c) + e4];
                     const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-                    float pe[4];
+                    float pe[4], xa[4];
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        pe[u] = ex2(fmaf(__uint_as_float(sr[4 * e4 + u]), C, -lv[u]));
-                        if (kMasked) {
+                    for (int u = 0; u < 4; ++u) xa[u] = fmaf(__uint_as_float(sr[4 * e4 + u]), C, -lv[u]);
+                    // on tiles with no masked element, one pair in eight on the FMA
+                    // pipe (fast_exp2x2) to offload the MUFU unit (measured: 2.7 %
+                    // faster on the dense layer; a quarter or a half were slower)
+#pragma unroll
+                    for (int u = 0; u < 4; u += 2) {
+                        if (!kMasked && e4 == 3 && u == 2) {
+                            const float2 f = fast_exp2x2(make_float2(xa[u], xa[u + 1]));
+                            pe[u] = f.x;
+                            pe[u + 1] = f.y;
+                        } else {
+                            pe[u] = ex2(xa[u]);
+                            pe[u + 1] = ex2(xa[u + 1]);
+                        }
+                    }
+                    if (kMasked) {
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
                             const int pl = (16 * (c0 + c) + 4 * e4 + u) / GP;
                             pe[u] = (pl >= pl_lo && pl <= pl_hi) ? pe[u] : 0.f;
                         }

@@ -534,8 +534,7 @@ int attn_sink_bwd(const void *q, const void *k, const void *v, const float *sink
     // the row pre-pass also clears the dQ accumulator the main pass adds into
     cudaError_t e = launch_bwd_rows<bf>(static_cast<const bf *>(out), static_cast<const bf *>(dout), lse, sinks, Drow,
                                         terms, dq_acc, s, st);
-    if (e == cudaSuccess) e = launch_bwd_tc(q, k, v, dout, lse, Drow, dq_acc, dq, dk, dv, s, st);
-    if (e == cudaSuccess) e = launch_dsink_reduce(terms, dsinks, s, st);
+    if (e == cudaSuccess) e = launch_bwd_tc(q, k, v, dout, lse, Drow, terms, dsinks, dq_acc, dq, dk, dv, s, st);
     return launch_status(e);
 }
 

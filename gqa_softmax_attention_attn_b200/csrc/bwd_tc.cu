@@ -575,16 +575,38 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-__global__ void __launch_bounds__(256) dq_convert_kernel(const float *__restrict__ acc, __nv_bfloat16 *__restrict__ dq,
-                                                         size_t n)
+// The backward's last step, one launch: blocks [0, n_conv) turn the fp32 dQ
+// accumulator into bf16 (8 values per thread); block n_conv + h sums head h's
+// B * Lq dsink terms in a fixed order (deterministic).
+__global__ void __launch_bounds__(256) bwd_finish_kernel(const float *__restrict__ acc, __nv_bfloat16 *__restrict__ dq,
+                                                         size_t n8, unsigned n_conv, const float *__restrict__ terms,
+                                                         float *__restrict__ dsinks, long nterms)
 {
-    const size_t i = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) * 4;
-    if (i >= n) return;
-    const float4 v = *reinterpret_cast<const float4 *>(acc + i);
-    uint2 o;
-    o.x = pack_bf16x2(v.x, v.y);
-    o.y = pack_bf16x2(v.z, v.w);
-    *reinterpret_cast<uint2 *>(dq + i) = o;
+    if (blockIdx.x >= n_conv) {
+        __shared__ float red[256];
+        const int h = (int)(blockIdx.x - n_conv), t = threadIdx.x;
+        const float *row = terms + (size_t)h * nterms;
+        float sum = 0.f;
+        for (long e = t; e < nterms; e += 256) sum += row[e];
+        red[t] = sum;
+        __syncthreads();
+        for (int w = 128; w > 0; w >>= 1) {
+            if (t < w) red[t] += red[t + w];
+            __syncthreads();
+        }
+        if (t == 0) dsinks[h] = red[0];
+        return;
+    }
+    const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n8) return;
+    const float4 v0 = reinterpret_cast<const float4 *>(acc)[2 * i];
+    const float4 v1 = reinterpret_cast<const float4 *>(acc)[2 * i + 1];
+    uint4 o;
+    o.x = pack_bf16x2(v0.x, v0.y);
+    o.y = pack_bf16x2(v0.z, v0.w);
+    o.z = pack_bf16x2(v1.x, v1.y);
+    o.w = pack_bf16x2(v1.z, v1.w);
+    reinterpret_cast<uint4 *>(dq)[i] = o;
 }
 
 template <int GP>
@@ -602,8 +624,8 @@ cudaError_t launch_gp(const CUtensorMap &mq, const CUtensorMap &mdo, const CUten
 size_t bwd_tc_dq_acc_bytes(const AttnShape &s) { return (size_t)s.B * s.Lq * s.Hq * s.D * sizeof(float); }
 
 cudaError_t launch_bwd_tc(const void *q, const void *k, const void *v, const void *dout, const float *lse,
-                          const float *Drow, float *dq_acc, void *dq, void *dk, void *dv, const AttnShape &s,
-                          cudaStream_t st)
+                          const float *Drow, const float *terms, float *dsinks, float *dq_acc, void *dq, void *dk,
+                          void *dv, const AttnShape &s, cudaStream_t st)
 {
     BwdParams p;
     p.B = s.B;
@@ -654,8 +676,11 @@ cudaError_t launch_bwd_tc(const void *q, const void *k, const void *v, const voi
     default: e = launch_gp<16>(mq, mdo, mk, mv, mdq, p, grid, st); break;
     }
     if (e != cudaSuccess) return e;
-    const size_t n = (size_t)s.B * s.Lq * s.Hq * s.D;
-    dq_convert_kernel<<<(unsigned)((n / 4 + 255) / 256), 256, 0, st>>>(dq_acc, static_cast<__nv_bfloat16 *>(dq), n);
+    const size_t n8 = (size_t)s.B * s.Lq * s.Hq * s.D / 8;
+    const size_t n_conv = (n8 + 255) / 256;
+    if (n_conv + s.Hq > 0x7fffffffu) return cudaErrorInvalidValue;
+    bwd_finish_kernel<<<(unsigned)(n_conv + s.Hq), 256, 0, st>>>(dq_acc, static_cast<__nv_bfloat16 *>(dq), n8,
+                                                                  (unsigned)n_conv, terms, dsinks, (long)s.B * s.Lq);
     return cudaGetLastError();
 }
 

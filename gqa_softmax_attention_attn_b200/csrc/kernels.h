@@ -71,19 +71,19 @@ cudaError_t launch_bwd_simt(const T *q, const T *k, const T *v, const float *sin
                             const AttnShape &s, void *ws, cudaStream_t st);
 size_t bwd_simt_workspace_bytes(const AttnShape &s);
 // row pre-pass of the backward (D_i and the dsink terms; with zero_rows, it
-// also clears the fp32 dQ accumulator [B, Lq, Hq, 64]) and the deterministic dsink sum
+// also clears the fp32 dQ accumulator [B, Lq, Hq, 64])
 template <typename T>
 cudaError_t launch_bwd_rows(const T *out, const T *dout, const float *lse, const float *sinks, float *Drow,
                             float *terms, float *zero_rows, const AttnShape &s, cudaStream_t st);
-cudaError_t launch_dsink_reduce(const float *terms, float *dsinks, const AttnShape &s, cudaStream_t st);
 
 // Tensor-core (tcgen05) bf16 backward main pass (+ dQ fp32 accumulation and
-// conversion); dq_acc must hold zeros on entry (launch_bwd_rows clears it).
+// conversion, and the dsink sums of the row pre-pass's terms); dq_acc must
+// hold zeros on entry (launch_bwd_rows clears it).
 size_t bwd_tc_dq_acc_bytes(const AttnShape &s);
 bool bwd_tc_supported(const AttnShape &s);
 cudaError_t launch_bwd_tc(const void *q, const void *k, const void *v, const void *dout, const float *lse,
-                          const float *Drow, float *dq_acc, void *dq, void *dk, void *dv, const AttnShape &s,
-                          cudaStream_t st);
+                          const float *Drow, const float *terms, float *dsinks, float *dq_acc, void *dq, void *dk,
+                          void *dv, const AttnShape &s, cudaStream_t st);
 
 template <typename T>
 cudaError_t launch_decode_simt(const T *q, const T *kc, const T *vc, const int *seqlens, const float *sinks,

@@ -590,12 +590,6 @@ cudaError_t launch_bwd_rows(const T *out, const T *dout, const float *lse, const
     return cudaGetLastError();
 }
 
-cudaError_t launch_dsink_reduce(const float *terms, float *dsinks, const AttnShape &s, cudaStream_t st)
-{
-    dsink_reduce_kernel<<<s.Hq, 256, 0, st>>>(terms, dsinks, (long)s.B * s.Lq);
-    return cudaGetLastError();
-}
-
 template <typename T>
 cudaError_t launch_decode_simt(const T *q, const T *kc, const T *vc, const int *seqlens, const float *sinks,
                                T *out, float *lse, const DecodeShape &s, float *ws_o, float *ws_ml,

@@ -28,6 +28,12 @@
 //    P from S^T (bf16 pairs into their own TMEM columns, releasing S^T), then
 //    dS = P (dP - D) from dP^T; dS^T goes back over the half's read columns
 //    of dP^T as bf16, dS to shared memory.
+//  * With at most 16 positions per q tile the causal / window mask is one
+//    more K = 16 step of S^T: a per-key-row table of 0 / -2^100 over the q
+//    tile's positions times the one-hot of each column's position.  The load
+//    warp writes the table with the tile's lse and D (one per stage), only
+//    for q tiles that hide some key, and the MMA warp adds the step only
+//    there, so the P pass never tests visibility.
 //  * Warps 6-9 move each dQ tile from TMEM to shared memory (two 128-byte-
 //    swizzled fp32 halves) and add it into an fp32 dQ accumulator in global
 //    memory with TMA reduce-adds (L2 atomics; the summation order over key
@@ -63,7 +69,14 @@ constexpr int kOffDO = kOffQ + 2 * kTile;  // 2 stages
 constexpr int kOffDS = kOffDO + 2 * kTile;  // dS, MN-major: two 64-row atoms of 16 KB
 constexpr int kOffStg = kOffDS + 2 * kTile;  // fp32 dQ staging: two [128][32] halves, 128-byte swizzle
 constexpr int kOffLD = kOffStg + 128 * 64 * 4;  // [2 stages][lse2 | D][128] fp32
-constexpr int kOffBar = kOffLD + 2 * 2 * 128 * 4;
+// mask operands of the extra K = 16 step of S^T (no swizzle, K-major; element
+// (row, k) at (row / 8) * 256 + (k / 8) * 128 + (row % 8) * 16 + (k % 8) * 2):
+// [2 stages] per key row, 0 where the q tile's position k sees the key, else
+// -2^100; per q column c, the one-hot of its position c / GP
+constexpr int kEBytes = kM * 32;
+constexpr int kOffEK = kOffLD + 2 * 2 * 128 * 4;
+constexpr int kOffEQ = kOffEK + 2 * kEBytes;
+constexpr int kOffBar = kOffEQ + kEBytes;
 // kv_full, qdo_full[2], qdo_empty[2], s_full, s_consumed, dp_full, p_ready,
 // pt_free, ds_free, dq_full, dq_free, stg_full, stg_free, dkv_done, drain
 constexpr int kNumBar = 17;
@@ -137,6 +150,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int n_q = pos_hi >= pos_lo ? (int)(pos_hi / P - pos_lo / P + 1) : 0;
     const int qt_lo = (int)(pos_lo / P);
     const int n_iter = n_q * p.n_htiles;
+    // at most 16 positions per q tile: the mask comes from an extra MMA step
+    constexpr bool mask_mma = GP >= 8;
 
     if (threadIdx.x == 0) {
         mbar_init(kv_full, 1);
@@ -173,6 +188,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         h0 = g * p.G + ht * GP;
         pos0 = qt * P;
     };
+    // does q tile i hide some key of this tile from some of its positions?
+    // key j sees positions [max(jrel, 0), jrel + window - 1] of the tile,
+    // jrel = j - first position - (Lk - Lq); keys past Lk see none
+    auto tile_masked = [&](int i) {
+        int h0, pos0;
+        iter_head(i, h0, pos0);
+        const long jr0 = (long)k0 - pos0 - off;
+        return jr0 + kM - 1 > 0 || k0 + kM > p.Lk || (p.window > 0 && jr0 + p.window - 1 < P - 1);
+    };
 
     if (warp == 0) {
         // ------------------------------------------------------------ loads
@@ -185,10 +209,57 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_4d(smem + kOffK, &tmK, 0, g, k0, b, kv_full);
             tma_load_4d(smem + kOffV, &tmV, 0, g, k0, b, kv_full);
         }
+        if (mask_mma) {
+            // the one-hot of each column's position (covered by the first
+            // stage's proxy fence below)
+#pragma unroll
+            for (int t = 0; t < 8; ++t) {
+                const int c = lane + 32 * (t >> 1), k = 8 * (t & 1);
+                uint32_t w[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    w[u] = (k + 2 * u == c / GP ? 0x3F80u : 0u) | ((k + 2 * u + 1 == c / GP ? 0x3F80u : 0u) << 16);
+                *reinterpret_cast<uint4 *>(smem + kOffEQ + (c >> 3) * 256 + (t & 1) * 128 + (c & 7) * 16) =
+                    make_uint4(w[0], w[1], w[2], w[3]);
+            }
+        }
+        static_assert(kM == 32 * 4, "one group of 4 lse / D values per lane");
         for (int i = 0; i < n_iter && ok; ++i) {
             const int st = i & 1;
             int h0, pos0;
             iter_head(i, h0, pos0);
+            // lse and D of the tile, read before the stage is free so that the
+            // loads overlap the wait: lane l reads 4 consecutive positions of
+            // one head (16-byte loads when aligned)
+            const int hl = lane * 4 / P, pl0 = lane * 4 % P;  // head within the tile, first position
+            const size_t li0 = ((size_t)b * p.Hq + h0 + hl) * p.Lq + pos0 + pl0;
+            float L4[4], D4[4];
+            if (pos0 + pl0 + 3 < p.Lq && (li0 & 3) == 0) {
+                const float4 a = *reinterpret_cast<const float4 *>(p.lse + li0);
+                const float4 d = *reinterpret_cast<const float4 *>(p.Drow + li0);
+                L4[0] = a.x; L4[1] = a.y; L4[2] = a.z; L4[3] = a.w;
+                D4[0] = d.x; D4[1] = d.y; D4[2] = d.z; D4[3] = d.w;
+            } else {
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const bool in = pos0 + pl0 + u < p.Lq;
+                    L4[u] = in ? p.lse[li0 + u] : -INFINITY;
+                    D4[u] = in ? p.Drow[li0 + u] : 0.f;
+                }
+            }
+            // the mask rows' visibility bounds: key k0 + lane + 32 t sees
+            // positions [lo[t], hi[t]] of the tile
+            const bool masked = mask_mma && tile_masked(i);
+            int lo[4], hi[4];
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                const long j = (long)k0 + lane + 32 * t, jrel = j - pos0 - off;
+                long lo_l = max(jrel, 0L);
+                const long hi_l = p.window > 0 ? jrel + p.window - 1 : (long)P - 1;
+                if (j >= p.Lk) lo_l = P;
+                lo[t] = (int)min(lo_l, (long)P);
+                hi[t] = (int)max(-1L, min(hi_l, (long)P - 1));
+            }
             if (lane == 0) {
                 ok = mbar_wait(&qdo_empty[st], ((i >> 1) & 1u) ^ 1u, abort_flag, p.status, p.timeout_ns);
                 if (ok) {
@@ -200,34 +271,36 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
-            // log2-domain lse (+inf for rows that do not exist or see nothing) and
-            // D: lane l reads 4 consecutive positions of one head (16-byte loads
-            // when aligned) and scatters them to columns pos * GP + head
-            for (int e = lane * 4; e < kM; e += 128) {
-                const int hl = e / P, pl0 = e % P;  // head within the tile, first position
-                const int h = h0 + hl;
-                const size_t li0 = ((size_t)b * p.Hq + h) * p.Lq + pos0 + pl0;
-                float L4[4], D4[4];
-                if (pos0 + pl0 + 3 < p.Lq && (li0 & 3) == 0) {
-                    const float4 a = *reinterpret_cast<const float4 *>(p.lse + li0);
-                    const float4 d = *reinterpret_cast<const float4 *>(p.Drow + li0);
-                    L4[0] = a.x; L4[1] = a.y; L4[2] = a.z; L4[3] = a.w;
-                    D4[0] = d.x; D4[1] = d.y; D4[2] = d.z; D4[3] = d.w;
-                } else {
+            // log2-domain lse (+inf for rows that do not exist or see nothing)
+            // and D, scattered to columns pos * GP + head
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const bool in = pos0 + pl0 + u < p.Lq;
-                        L4[u] = in ? p.lse[li0 + u] : -INFINITY;
-                        D4[u] = in ? p.Drow[li0 + u] : 0.f;
+            for (int u = 0; u < 4; ++u) {
+                const int c = (pl0 + u) * GP + hl;
+                ld[(st * 2 + 0) * kM + c] = (L4[u] == -INFINITY) ? INFINITY : L4[u] * kLog2e;
+                ld[(st * 2 + 1) * kM + c] = D4[u];
+            }
+            if (masked) {
+                // the stage's mask rows (S^T two tiles back, their last reader,
+                // completed before qdo_empty): 0 where the position sees the key
+                uint8_t *ek = smem + kOffEK + st * kEBytes;
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    const int r = lane + 32 * t;
+#pragma unroll
+                    for (int kh = 0; kh < 2; ++kh) {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const int k = 8 * kh + 2 * u;
+                            w[u] = ((k >= lo[t] && k <= hi[t]) ? 0u : 0xF180u) |
+                                   ((k + 1 >= lo[t] && k + 1 <= hi[t]) ? 0u : 0xF180u) << 16;
+                        }
+                        *reinterpret_cast<uint4 *>(ek + (r >> 3) * 256 + kh * 128 + (r & 7) * 16) =
+                            make_uint4(w[0], w[1], w[2], w[3]);
                     }
                 }
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int c = (pl0 + u) * GP + hl;
-                    ld[(st * 2 + 0) * kM + c] = (L4[u] == -INFINITY) ? INFINITY : L4[u] * kLog2e;
-                    ld[(st * 2 + 1) * kM + c] = D4[u];
-                }
             }
+            if (mask_mma) fence_proxy_async_smem();  // the tables are read by the tensor core
             __syncwarp();
             if (lane == 0) mbar_arrive(&qdo_full[st]);
         }
@@ -252,6 +325,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         auto wait_all = [&](uint64_t *bar, uint32_t parity) {
             return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, p.status, p.timeout_ns));
         };
+        const uint64_t d_ek = smem_desc_noswz(smem_u32(smem + kOffEK), 128, 256);
+        const uint64_t d_eq = smem_desc_noswz(smem_u32(smem + kOffEQ), 128, 256);
         bool ok = n_iter > 0 && wait_all(kv_full, 0);
         // S^T(i) = K Q(i)^T into its own TMEM tile; issued for tile i+1 as
         // soon as the softmax-gradient threads have read S^T(i) out.
@@ -261,9 +336,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (i > 0 && !wait_all(s_consumed, (i - 1) & 1u)) return false;
             tc_fence_after();
             const uint64_t q_st = d_q + (uint64_t)((st * kTile) >> 4);
+            const bool extra = mask_mma && tile_masked(i);
             if (elect_one()) {
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk) mma_ss(tmem + kTmST, d_k + 2 * kk, q_st + 2 * kk, id_t, kk > 0);
+                if (extra)  // + 0 / -2^100 where the position does not see the key
+                    mma_ss(tmem + kTmST, d_ek + (uint64_t)((st * kEBytes) >> 4), d_eq, id_t, 1u);
                 mma_commit(s_full);
             }
             __syncwarp();
@@ -360,7 +438,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (j >= p.Lk) lo_l = P;  // keys past Lk see nothing
             const int pl_lo = (int)min(lo_l, (long)P);
             const int pl_hi = (int)max(-1L, min(hi_l, (long)P - 1));
-            const bool need_mask = __any_sync(0xffffffffu, pl_lo > 0 || pl_hi < P - 1);
+            const bool need_mask = !mask_mma && __any_sync(0xffffffffu, pl_lo > 0 || pl_hi < P - 1);
             const float4 *l2v = reinterpret_cast<const float4 *>(ld + (st * 2 + 0) * kM);
             const float4 *ddv = reinterpret_cast<const float4 *>(ld + (st * 2 + 1) * kM);
 
@@ -415,10 +493,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_wait_ld();
                 }
             };
-            if (need_mask)
-                phase1(std::true_type{});
-            else
+            if constexpr (mask_mma) {
                 phase1(std::false_type{});
+            } else {
+                if (need_mask)
+                    phase1(std::true_type{});
+                else
+                    phase1(std::false_type{});
+            }
             // P^T into its columns once dV(i-1) has read the previous P^T
             if (i > 0 &&
                 !__all_sync(0xffffffffu, mbar_wait(pt_free, (i - 1) & 1u, abort_flag, p.status, p.timeout_ns))) {
@@ -635,8 +717,13 @@ cudaError_t launch_bwd_tc(const void *q, const void *k, const void *v, const voi
     p.Hkv = s.Hkv;
     p.window = s.window;
     p.G = s.Hq / s.Hkv;
+    // query heads per q tile: the largest power of two up to 16 dividing G;
+    // with 8 or more the mask is an MMA step whose -2^100 times
+    // scale * log2(e) must stay far below any exponent, so a smaller scale
+    // takes 4 (the per-element mask)
+    const int gp_max = s.scale >= 0x1p-60f ? 16 : 4;
     int gp = 1;
-    while (gp * 2 <= 16 && p.G % (gp * 2) == 0) gp *= 2;
+    while (gp * 2 <= gp_max && p.G % (gp * 2) == 0) gp *= 2;
     p.P = kM / gp;
     p.n_htiles = p.G / gp;
     p.c_log2 = s.scale * kLog2e;

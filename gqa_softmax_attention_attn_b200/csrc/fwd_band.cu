@@ -664,7 +664,8 @@ cudaError_t launch_fwd_band(const void *q, const void *k, const void *v, const f
     const long long n_items = (long long)p.n_ptiles * p.n_htiles * s.B;
     if (n_items > 0x7fffffffLL) return cudaErrorInvalidValue;
     p.n_items = (int)n_items;
-    p.mask_mma = p.P <= 16;
+    // the mask's -2^100 times scale * log2(e) must stay far below any exponent
+    p.mask_mma = p.P <= 16 && s.scale >= 0x1p-60f;
     p.c_log2 = s.scale * kLog2e;
     p.sinks = sinks;
     p.out = static_cast<__nv_bfloat16 *>(out);

@@ -70,6 +70,25 @@ def test_bf16_bwd_small(shape, window):
     _check_bf16(t, window, 0.125, f"{shape} w={window}")
 
 
+@pytest.mark.parametrize("window", [0, 128])
+def test_bf16_tiny_scale(window):
+    """A scale below 2^-60: the -2^100 of the mask step would no longer vanish
+    after the scaling, so both kernels take their per-element masks (the
+    backward with 4 query heads per tile instead of 8) -- forward and backward
+    against the oracle on a group of 8 query heads."""
+    scale = 2.0**-70
+    t = prefill_inputs(1, 200, 200, 8, 1, 64, torch.bfloat16, 0.5, 1.0, 0.1, seed=77, with_dout=True)
+    dev = "cuda"
+    q, k, v, s = (t[x].to(dev) for x in ("q", "k", "v", "sinks"))
+    out = torch.empty_like(q)
+    lse = torch.empty(1, 8, 200, device=dev, dtype=torch.float32)
+    attn_sink_fwd(q, k, v, s, out, lse, window, scale)
+    torch.cuda.synchronize()
+    ro, rl = oracle.fwd(t["q"], t["k"], t["v"], t["sinks"], window, scale)
+    assert_close_bf16(out, ro, f"tiny scale w={window} out")
+    _check_bf16(t, window, scale, f"tiny scale w={window}")
+
+
 @pytest.mark.parametrize("window", [0, WINDOW])
 def test_bf16_bwd_one_train_group(window):
     """One (b, kv-group) slice with the training shape's group layout (all 8

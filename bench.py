@@ -315,21 +315,11 @@ def decode_legs(dev, reps=20, warmup=3, batch=None):
         ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
         kv_rows = sum(min(n, window) if window > 0 else n for n in lens)
         by = kv_rows * w.Hkv * w.D * 2 * 2 + nb * w.Hq * w.D * 2 * 2 + nb * w.Hq * 4 + 4 * nb
-        times = []
-        for it in range(reps + warmup):
-            flush.zero_()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            attn.attn_sink_decode(d["q"], d["k_cache"], d["v_cache"], d["seqlens"], d["sinks"], out, lse, window,
-                                  SCALE, 0, ws, stream)
-            e1.record(stream)
-            torch.cuda.synchronize(dev)
-            if it >= warmup:
-                times.append(e0.elapsed_time(e1))
-        ms = statistics.median(times)
+        ms = timed(dev, lambda: attn.attn_sink_decode(d["q"], d["k_cache"], d["v_cache"], d["seqlens"], d["sinks"],
+                                                      out, lse, window, SCALE, 0, ws, stream), reps, warmup, flush)
         gbs = by / (ms * 1e-3) / 1e9
         legs[name] = {"ms": ms, "GB/s": gbs, "frac_hbm": gbs / hbm, "bytes": by,
-                      "flops": 4.0 * w.D * kv_rows * (w.Hq // w.Hkv) * w.Hkv}
+                      "flops": 4.0 * w.D * kv_rows * (w.Hq // w.Hkv) * w.Hkv, "sm_mhz": LEG_CLOCK.last_leg_mhz()}
     # the same caches in FP8 (e4m3 codes, one scale per KV head): half the bytes
     from gqa_softmax_attention_attn_b200.inputs import quantize_e4m3_per_head
 
@@ -340,20 +330,11 @@ def decode_legs(dev, reps=20, warmup=3, batch=None):
         ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
         kv_rows = sum(min(n, window) if window > 0 else n for n in lens)
         by = kv_rows * w.Hkv * w.D * 2 + nb * w.Hq * w.D * 2 * 2 + nb * w.Hq * 4 + 4 * nb + 2 * 4 * w.Hkv
-        times = []
-        for it in range(reps + warmup):
-            flush.zero_()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            attn.attn_sink_decode_fp8(d["q"], k8, v8, ks, vs, d["seqlens"], d["sinks"], out, lse, window, SCALE, 0,
-                                      ws, stream)
-            e1.record(stream)
-            torch.cuda.synchronize(dev)
-            if it >= warmup:
-                times.append(e0.elapsed_time(e1))
-        ms = statistics.median(times)
+        ms = timed(dev, lambda: attn.attn_sink_decode_fp8(d["q"], k8, v8, ks, vs, d["seqlens"], d["sinks"], out, lse,
+                                                          window, SCALE, 0, ws, stream), reps, warmup, flush)
         gbs = by / (ms * 1e-3) / 1e9
-        legs[name] = {"ms": ms, "GB/s": gbs, "frac_hbm": gbs / hbm, "bytes": by, "kv_dtype": "e4m3"}
+        legs[name] = {"ms": ms, "GB/s": gbs, "frac_hbm": gbs / hbm, "bytes": by, "kv_dtype": "e4m3",
+                      "sm_mhz": LEG_CLOCK.last_leg_mhz()}
     del k8, v8
     # the same caches as a pool of 16-key pages in seeded random order, read
     # through a page table (same compulsory bytes; the table is not credited)
@@ -370,20 +351,11 @@ def decode_legs(dev, reps=20, warmup=3, batch=None):
         nbytes = attn.attn_sink_decode_paged_workspace_size(nb, w.Hq, w.D, maxp, ps, window, 0)
         ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
         by = legs[name.replace("paged16_", "")]["bytes"]
-        times = []
-        for it in range(reps + warmup):
-            flush.zero_()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            attn.attn_sink_decode_paged(d["q"], kp, vp, table, d["seqlens"], d["sinks"], out, lse, window, SCALE, 0,
-                                        ws, stream)
-            e1.record(stream)
-            torch.cuda.synchronize(dev)
-            if it >= warmup:
-                times.append(e0.elapsed_time(e1))
-        ms = statistics.median(times)
+        ms = timed(dev, lambda: attn.attn_sink_decode_paged(d["q"], kp, vp, table, d["seqlens"], d["sinks"], out,
+                                                            lse, window, SCALE, 0, ws, stream), reps, warmup, flush)
         gbs = by / (ms * 1e-3) / 1e9
-        legs[name] = {"ms": ms, "GB/s": gbs, "frac_hbm": gbs / hbm, "bytes": by, "page_size": ps}
+        legs[name] = {"ms": ms, "GB/s": gbs, "frac_hbm": gbs / hbm, "bytes": by, "page_size": ps,
+                      "sm_mhz": LEG_CLOCK.last_leg_mhz()}
     return legs
 
 
@@ -411,11 +383,61 @@ def device_prefill(B_, L_, Hq_, Hkv_, sink_std, seed, dev, with_dout):
     return t
 
 
+class LegClock:
+    """The SM clock read through NVML every ~2 ms while the legs run, so that
+    each leg reports the median clock of its own timed repetitions (a leg run
+    right after a heavy one can start below the maximum clock)."""
+
+    def __init__(self):
+        self.samples, self.window, self.nv = [], None, None
+        self.stop_ev = threading.Event()
+
+    def start(self, gpu_index: int):
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(gpu_index)
+            self.nv = pynvml
+        except Exception:
+            return
+        self.t = threading.Thread(target=self._run, daemon=True)
+        self.t.start()
+
+    def _run(self):
+        while not self.stop_ev.is_set():
+            try:
+                self.samples.append((time.time(), self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)))
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def stop(self):
+        if self.nv is not None:
+            self.stop_ev.set()
+            self.t.join(timeout=2)
+
+    def last_leg_mhz(self):
+        if self.window is None:
+            return None
+        vals = [c for t, c in self.samples if self.window[0] <= t <= self.window[1]]
+        return statistics.median(vals) if vals else None
+
+
+LEG_CLOCK = LegClock()
+LEG_PAUSE_S = 0.5  # idle time before each leg, so that the previous leg's load does not set its clock
+
+
 def timed(dev, fn, reps, warmup, flush):
     """Median device time (ms) of fn() over `reps` runs after `warmup`, L2 flushed before each."""
     stream = torch.cuda.current_stream(dev)
     times = []
+    torch.cuda.synchronize(dev)
+    time.sleep(LEG_PAUSE_S)
+    t0 = None
     for it in range(reps + warmup):
+        if it == warmup:
+            t0 = time.time()
         flush.zero_()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
@@ -424,6 +446,7 @@ def timed(dev, fn, reps, warmup, flush):
         torch.cuda.synchronize(dev)
         if it >= warmup:
             times.append(e0.elapsed_time(e1))
+    LEG_CLOCK.window = (t0, time.time())
     return statistics.median(times)
 
 
@@ -432,12 +455,12 @@ def leg_entry(ms, flops, nbytes, bound, shape):
     tf = flops / (ms * 1e-3) / 1e12
     gbs = nbytes / (ms * 1e-3) / 1e9
     e = {"ms": ms, "TFLOP/s": tf, "frac_tensor": tf / tf_burst, "GB/s": gbs, "frac_hbm": gbs / hbm,
-         "flops": flops, "bytes": nbytes, "bound": bound, "shape": shape}
+         "flops": flops, "bytes": nbytes, "bound": bound, "shape": shape, "sm_mhz": LEG_CLOCK.last_leg_mhz()}
     e["frac"] = e["frac_hbm"] if bound == "hbm" else e["frac_tensor"]
     return e
 
 
-def prefill_legs(dev, which=("bwd", "train", "fp8", "varlen", "prologue", "long"), reps=5, warmup=2):
+def prefill_legs(dev, which=("bwd", "train", "fp8", "varlen", "prologue", "long"), reps=10, warmup=3):
     """Forward / backward legs beyond the headline step, each with its own roofline
     fraction (dense layers against the tensor peak, window-128 layers against HBM),
     L2 flushed before every timed run:
@@ -665,16 +688,20 @@ def main():
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     if args.only is not None:
+        LEG_CLOCK.start(dev.index if dev.index is not None else 0)
         legs = (decode_legs(dev, args.steps, args.warmup, args.decode_batch) if args.only == "decode"
                 else prefill_legs(dev, (args.only,), args.steps, args.warmup))
+        LEG_CLOCK.stop()
         print(json.dumps({"only": args.only, "legs": legs}), flush=True)
         return
     res = run_ours(args, rank, world, dev)
     if rank == 0:
         if not args.no_legs and world == 1:
             res["legs"] = {}
+            LEG_CLOCK.start(dev.index if dev.index is not None else 0)
             res["legs"].update(decode_legs(dev))
             res["legs"].update(prefill_legs(dev))
+            LEG_CLOCK.stop()
         if not args.no_cpu_baseline and world == 1:
             v, cores, desc, _, _ = oracle_sample(12.0)
             res["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc,

@@ -34,6 +34,8 @@
 #include <cuda_fp8.h>
 #include <math.h>
 
+#include <type_traits>
+
 #include "kernels.h"
 #include "sm100_ptx.cuh"
 
@@ -51,13 +53,15 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
 // Shared-memory layout; kFp8: K/V cached as e4m3 (one byte per element).
-template <bool kFp8>
+// kStages: TMA ring depth (bf16: 4, or 3 when a split spans at most three
+// tiles, so that more CTAs fit an SM at once; e4m3: ATTN_SINK_DEC_FP8_STAGES)
+template <bool kFp8, int kStages>
 struct DecLayout {
     // keys per tile: the e4m3 tile spans twice the keys, so a tile's bytes (and
     // its fixed costs: TMA issue, barrier round trips) are those of a bf16 tile
     static constexpr int kT = kFp8 ? 128 : 64;
     static constexpr int kSlices = kT / 64;  // 16-key slices per consumer warp and tile
-    static constexpr int kNS = kFp8 ? ATTN_SINK_DEC_FP8_STAGES : 4;
+    static constexpr int kNS = kStages;
     static constexpr int kRowBytes = kFp8 ? kD : kD * 2;  // one cached K or V row
     static constexpr int kTileBytes = kT * kRowBytes;
     static constexpr int kStageBytes = 2 * kTileBytes;  // K and V
@@ -123,12 +127,12 @@ __device__ __forceinline__ void mma16816_f16(float (&d)[4], const uint32_t (&a)[
 __device__ __forceinline__ uint32_t swz(int row, int chunk) { return row * 128 + ((chunk ^ (row & 7)) << 4); }
 
 
-template <bool kRows16, bool kPaged, bool kFp8>
+template <bool kRows16, bool kPaged, bool kFp8, int kStages>
 __global__ void __launch_bounds__(kThreads)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                      const DecodeParams p)
 {
-    using L = DecLayout<kFp8>;
+    using L = DecLayout<kFp8, kStages>;
     constexpr int kT = L::kT;
     static_assert(!(kPaged && kFp8), "paged caches are bf16 only");
     extern __shared__ uint8_t smem_raw[];
@@ -511,7 +515,7 @@ cudaError_t launch_decode_bf16(const void *q, const void *kc, const void *vc, co
     p.k_scale = k_scale;
     p.v_scale = v_scale;
     p.sh = s;
-    const int kT = fp8 ? DecLayout<true>::kT : DecLayout<false>::kT;
+    const int kT = fp8 ? DecLayout<true, ATTN_SINK_DEC_FP8_STAGES>::kT : DecLayout<false, 4>::kT;
     p.box_rows = s.page_size > 0 && s.page_size < kT ? s.page_size : kT;
     p.B = s.B;
     p.Lmax = s.Lmax;
@@ -552,14 +556,28 @@ cudaError_t launch_decode_bf16(const void *q, const void *kc, const void *vc, co
         kern<<<grid, kThreads, smem_bytes, st>>>(mk, mv, p);
         return cudaGetLastError();
     };
-    constexpr int sb = DecLayout<false>::kSmemBytes, s8 = DecLayout<true>::kSmemBytes;
+    constexpr int kF8S = ATTN_SINK_DEC_FP8_STAGES;
+    constexpr int s8 = DecLayout<true, kF8S>::kSmemBytes;
     if (fp8) {
         if (paged) return cudaErrorInvalidValue;  // e4m3 caches are contiguous only
-        return p.G > 8 ? launch(decode_tc_kernel<true, false, true>, s8) : launch(decode_tc_kernel<false, false, true>, s8);
+        return p.G > 8 ? launch(decode_tc_kernel<true, false, true, kF8S>, s8)
+                       : launch(decode_tc_kernel<false, false, true, kF8S>, s8);
     }
-    if (p.G > 8)
-        return paged ? launch(decode_tc_kernel<true, true, false>, sb) : launch(decode_tc_kernel<true, false, false>, sb);
-    return paged ? launch(decode_tc_kernel<false, true, false>, sb) : launch(decode_tc_kernel<false, false, false>, sb);
+    // a split of at most 192 keys (a window of 128: 128 keys anywhere, or
+    // three whole tiles of a paged cache) needs about three 64-key tiles:
+    // three stages hold them, and the smaller ring lets four CTAs share an SM
+    // (measured on the window-128 decode of 64 sequences: 17.2 -> 15.4 us;
+    // long splits keep four stages, 336.6 vs 338.8 us dense)
+    auto pick = [&](auto stages) -> cudaError_t {
+        constexpr int kS = decltype(stages)::value;
+        constexpr int sb = DecLayout<false, kS>::kSmemBytes;
+        if (p.G > 8)
+            return paged ? launch(decode_tc_kernel<true, true, false, kS>, sb)
+                         : launch(decode_tc_kernel<true, false, false, kS>, sb);
+        return paged ? launch(decode_tc_kernel<false, true, false, kS>, sb)
+                     : launch(decode_tc_kernel<false, false, false, kS>, sb);
+    };
+    return s.chunk <= 192 ? pick(std::integral_constant<int, 3>{}) : pick(std::integral_constant<int, 4>{});
 }
 
 }  // namespace attn_sink

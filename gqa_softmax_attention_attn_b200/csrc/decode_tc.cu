@@ -128,9 +128,7 @@ __device__ __forceinline__ uint32_t swz(int row, int chunk) { return row * 128 +
 
 
 template <bool kRows16, bool kPaged, bool kFp8, int kStages>
-__global__ void __launch_bounds__(kThreads)
-    decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                     const DecodeParams p)
+__device__ __forceinline__ void decode_tc_body(const CUtensorMap &tmK, const CUtensorMap &tmV, const DecodeParams &p)
 {
     using L = DecLayout<kFp8, kStages>;
     constexpr int kT = L::kT;
@@ -497,6 +495,25 @@ __global__ void __launch_bounds__(kThreads)
     }
 }
 
+// The kernel entry points: the default register allocation, and one held to
+// four CTAs per SM (at most 102 registers per thread) for the short e4m3
+// splits, whose two-stage ring then fits four CTAs per SM.
+template <bool kRows16, bool kPaged, bool kFp8, int kStages>
+__global__ void __launch_bounds__(kThreads)
+    decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                     const DecodeParams p)
+{
+    decode_tc_body<kRows16, kPaged, kFp8, kStages>(tmK, tmV, p);
+}
+
+template <bool kRows16, bool kPaged, bool kFp8, int kStages>
+__global__ void __launch_bounds__(kThreads, 4)
+    decode_tc_kernel_4(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                       const DecodeParams p)
+{
+    decode_tc_body<kRows16, kPaged, kFp8, kStages>(tmK, tmV, p);
+}
+
 }  // namespace
 
 bool decode_bf16_supported(const DecodeShape &s)
@@ -557,11 +574,21 @@ cudaError_t launch_decode_bf16(const void *q, const void *kc, const void *vc, co
         return cudaGetLastError();
     };
     constexpr int kF8S = ATTN_SINK_DEC_FP8_STAGES;
-    constexpr int s8 = DecLayout<true, kF8S>::kSmemBytes;
     if (fp8) {
         if (paged) return cudaErrorInvalidValue;  // e4m3 caches are contiguous only
-        return p.G > 8 ? launch(decode_tc_kernel<true, false, true, kF8S>, s8)
-                       : launch(decode_tc_kernel<false, false, true, kF8S>, s8);
+        // a split of at most 256 keys (two or three 128-key tiles): two stages
+        // and at most 102 registers per thread, so four CTAs share an SM
+        auto pick8 = [&](auto stages) -> cudaError_t {
+            constexpr int kS = decltype(stages)::value;
+            constexpr int s8 = DecLayout<true, kS>::kSmemBytes;
+            if constexpr (kS == 2)
+                return p.G > 8 ? launch(decode_tc_kernel_4<true, false, true, 2>, s8)
+                               : launch(decode_tc_kernel_4<false, false, true, 2>, s8);
+            else
+                return p.G > 8 ? launch(decode_tc_kernel<true, false, true, kS>, s8)
+                               : launch(decode_tc_kernel<false, false, true, kS>, s8);
+        };
+        return s.chunk <= 256 ? pick8(std::integral_constant<int, 2>{}) : pick8(std::integral_constant<int, kF8S>{});
     }
     // a split of at most 192 keys (a window of 128: 128 keys anywhere, or
     // three whole tiles of a paged cache) needs about three 64-key tiles:

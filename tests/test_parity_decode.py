@@ -92,6 +92,19 @@ def test_decode_edges_bf16(window):
             assert_lse(lse, rl, f"edges Hq={Hq} Hkv={Hkv} w={window} s={splits}")
 
 
+@pytest.mark.parametrize("window,splits", [(160, 0), (192, 0), (192, 1), (0, 8)])
+def test_decode_short_splits(window, splits):
+    """Splits of at most 192 keys run with a three-stage ring: windows of 160
+    and 192 keys and dense splits of 188 keys span up to four 64-key tiles, so
+    the ring wraps within a split."""
+    d = decode_inputs(9, 1500, 16, 2, 64, 1, 1500, torch.bfloat16, 0.5, 1.0, seed=29 + window + splits)
+    d["seqlens"] = torch.tensor([1, 1500, 191, 192, 193, 255, 256, 257, 1023], dtype=torch.int32)
+    out, lse = run_decode(d, window, 0.125, splits)
+    ro, rl = oracle.decode(d["q"], d["k_cache"], d["v_cache"], d["seqlens"], d["sinks"], window, 0.125)
+    assert_close_bf16(out, ro, f"short splits w={window} s={splits}")
+    assert_lse(lse, rl, f"short splits w={window} s={splits}")
+
+
 @pytest.mark.parametrize("window", [0, 128])
 def test_decode_fp32_exact(window):
     d = decode_inputs(4, 600, 8, 2, 64, 1, 600, torch.float32, 1.0, 1.0, seed=23)

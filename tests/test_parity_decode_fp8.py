@@ -81,6 +81,18 @@ def _workload():
     return _cache["d"]
 
 
+@pytest.mark.parametrize("window,splits", [(200, 0), (256, 0), (0, 6)])
+def test_fp8_short_splits(window, splits):
+    """Splits of at most 256 keys run with a two-stage ring (four CTAs per
+    SM): windows of 200 and 256 keys and dense splits of 250 keys span up to
+    three 128-key tiles, so the ring wraps within a split."""
+    d = fp8_inputs(9, 1500, 16, 2, 1, 1500, seed=71 + window + splits)
+    out, lse = run_fp8(d, window, 0.125, splits)
+    ro, rl = oracle_fp8(d, window, 0.125)
+    assert_close_bf16(out, ro, f"fp8 short splits w={window} s={splits}")
+    assert_lse(lse, rl, f"fp8 short splits w={window} s={splits}")
+
+
 @pytest.mark.parametrize("window", [0, WINDOW])
 def test_fp8_decode_workload_full(window):
     """The 64-sequence decode workload (lengths U[1024, 32768], Hq64 Hkv8) with

@@ -21,6 +21,8 @@ from ._native import (  # noqa: F401
     attn_sink_decode_paged_workspace_size,
     attn_sink_decode_workspace_size,
     attn_sink_fwd,
+    attn_sink_fwd_host,
+    attn_sink_fwd_host_workspace_size,
     attn_sink_fwd_varlen,
     attn_sink_get_device_status,
     attn_sink_qkv_prologue,

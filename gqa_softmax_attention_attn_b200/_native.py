@@ -75,6 +75,10 @@ def load():
         lib.attn_sink_fwd_fp8.restype = I
         lib.attn_sink_fwd_fp8_workspace_size.argtypes = [I] * 4
         lib.attn_sink_fwd_fp8_workspace_size.restype = Z
+        lib.attn_sink_fwd_host.argtypes = [P] * 6 + [I] * 7 + [F, I, P, Z, P]
+        lib.attn_sink_fwd_host.restype = I
+        lib.attn_sink_fwd_host_workspace_size.argtypes = [I] * 6
+        lib.attn_sink_fwd_host_workspace_size.restype = Z
         lib.attn_sink_decode_paged.argtypes = [P] * 8 + [I] * 8 + [F, I, P, Z, I, P]
         lib.attn_sink_decode_paged.restype = I
         lib.attn_sink_decode_paged_workspace_size.argtypes = [I] * 7
@@ -119,6 +123,16 @@ def _dev(t: torch.Tensor, name: str, dtype=None) -> int:
     return t.data_ptr()
 
 
+def _host(t: torch.Tensor, name: str, dtype=None) -> int:
+    if not isinstance(t, torch.Tensor) or t.device.type != "cpu":
+        raise ValueError(f"{name} must be a host (CPU) tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return t.data_ptr()
+
+
 def _stream(stream) -> int:
     if stream is None:
         return torch.cuda.current_stream().cuda_stream
@@ -141,6 +155,27 @@ def attn_sink_fwd(q, k, v, sinks, out, lse, window: int, scale: float, stream=No
                               _dev(out, "out", dt), _dev(lse, "lse", torch.float32), B, Lq, Lk, Hq, Hkv, D,
                               int(window), float(scale), _dtype_code(q), _stream(stream))
     _check(rc, "attn_sink_fwd")
+
+
+def attn_sink_fwd_host_workspace_size(B: int, Lq: int, Lk: int, Hq: int, Hkv: int, D: int) -> int:
+    return int(load().attn_sink_fwd_host_workspace_size(B, Lq, Lk, Hq, Hkv, D))
+
+
+def attn_sink_fwd_host(q, k, v, sinks, out, lse, window: int, scale: float, workspace, n_chunks: int = 8,
+                       stream=None):
+    """The bf16 prefill forward on HOST tensors (pin them for the copies to overlap): q [B,Lq,Hq,D],
+    k/v [B,Lk,Hkv,D] bf16, sinks [Hq] fp32 -> writes out [B,Lq,Hq,D] bf16, lse [B,Hq,Lq] fp32 in host
+    memory; workspace: a CUDA tensor of attn_sink_fwd_host_workspace_size bytes.  Asynchronous on
+    `stream`: synchronise it before reading out or lse."""
+    B, Lq, Hq, D = q.shape
+    Lk, Hkv = k.shape[1], k.shape[2]
+    bf = torch.bfloat16
+    rc = load().attn_sink_fwd_host(_host(q, "q", bf), _host(k, "k", bf), _host(v, "v", bf),
+                                   _host(sinks, "sinks", torch.float32), _host(out, "out", bf),
+                                   _host(lse, "lse", torch.float32), B, Lq, Lk, Hq, Hkv, D, int(window), float(scale),
+                                   int(n_chunks), _dev(workspace, "workspace"),
+                                   workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "attn_sink_fwd_host")
 
 
 def attn_sink_qkv_prologue(qkv, bias, positions, q_out, k_out, v_out, rope_theta: float, rope_factor: float = 1.0,

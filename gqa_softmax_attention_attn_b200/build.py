@@ -11,7 +11,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB_DIR = os.path.join(HERE, "lib")
 LIB = os.path.join(LIB_DIR, "libattn_sink.so")
-SOURCES = ["attn_sink_api.cu", "simt_kernels.cu", "fwd_tc.cu", "fwd_band.cu", "decode_tc.cu", "bwd_tc.cu", "prologue.cu"]
+SOURCES = ["attn_sink_api.cu", "simt_kernels.cu", "fwd_tc.cu", "fwd_band.cu", "decode_tc.cu", "bwd_tc.cu", "prologue.cu",
+           "host_fwd.cu"]
 HEADERS = ["kernels.h", "sm100_ptx.cuh", "selftest.cu"]
 SELFTEST_LIB = os.path.join(LIB_DIR, "libattn_sink_selftest.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

@@ -281,6 +281,31 @@ int attn_sink_fwd(const void *q, const void *k, const void *v, const float *sink
     return launch_status(launch_fwd_tc(q, k, v, sinks, out, lse, s, st));
 }
 
+size_t attn_sink_fwd_host_workspace_size(int B, int Lq, int Lk, int Hq, int Hkv, int D)
+{
+    if (check_common(B, Lq, Lk, Hq, Hkv, D, ATTN_SINK_DTYPE_BF16) != ATTN_SINK_OK) return 0;
+    return fwd_host_workspace_bytes(AttnShape{B, Lq, Lk, Hq, Hkv, D, 0, 1.f});
+}
+
+int attn_sink_fwd_host(const void *q_host, const void *k_host, const void *v_host, const float *sinks_host,
+                       void *out_host, float *lse_host, int B, int Lq, int Lk, int Hq, int Hkv, int D, int window,
+                       float scale, int n_chunks, void *workspace, size_t ws_bytes, void *stream)
+{
+    if (!q_host || !k_host || !v_host || !sinks_host || !out_host || !lse_host) return ATTN_SINK_ERR_INVALID_ARG;
+    if (n_chunks < 1 || n_chunks > kFwdHostMaxChunks) return ATTN_SINK_ERR_INVALID_ARG;
+    int rc = check_common(B, Lq, Lk, Hq, Hkv, D, ATTN_SINK_DTYPE_BF16);
+    if (rc != ATTN_SINK_OK) return rc;
+    if (!(scale > 0.f && scale < INFINITY) || Lq > Lk) return ATTN_SINK_ERR_UNSUPPORTED;
+    const AttnShape s{B, Lq, Lk, Hq, Hkv, D, window, scale};
+    if (!fwd_tc_supported(s)) return ATTN_SINK_ERR_UNSUPPORTED;
+    if (!workspace || ws_bytes < fwd_host_workspace_bytes(s)) return ATTN_SINK_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return ATTN_SINK_ERR_MISALIGNED;
+    rc = ensure_device();
+    if (rc != ATTN_SINK_OK) return rc;
+    return launch_status(run_fwd_host(q_host, k_host, v_host, sinks_host, out_host, lse_host, s, n_chunks, workspace,
+                                      static_cast<cudaStream_t>(stream)));
+}
+
 size_t attn_sink_fwd_fp8_workspace_size(int B, int Lk, int Hkv, int D)
 {
     if (B <= 0 || Lk <= 0 || Hkv <= 0 || D <= 0) return 0;

@@ -655,7 +655,7 @@ cudaError_t launch_fwd_band(const void *q, const void *k, const void *v, const f
     p.cu_k = s.cu_k;
     p.total_q = s.total_q;
     p.total_k = s.total_k;
-    p.lse_hs = s.cu_q ? s.total_q : s.Lq;
+    p.lse_hs = s.lse_hs > 0 ? s.lse_hs : (s.cu_q ? s.total_q : s.Lq);
     p.G = s.Hq / s.Hkv;
     p.Gp = packed_heads(s);
     p.P = kM / p.Gp;

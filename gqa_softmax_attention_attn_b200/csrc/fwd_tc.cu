@@ -728,7 +728,7 @@ cudaError_t launch_cfg(const void *q, const void *k, const void *v, const float 
     p.cu_k = s.cu_k;
     p.total_q = s.total_q;
     p.total_k = s.total_k;
-    p.lse_hs = s.cu_q ? s.total_q : s.Lq;
+    p.lse_hs = s.lse_hs > 0 ? s.lse_hs : (s.cu_q ? s.total_q : s.Lq);
     p.G = s.Hq / s.Hkv;
     int gp = 1;
     while (gp * 2 <= 16 && p.G % (gp * 2) == 0) gp *= 2;

@@ -19,6 +19,9 @@ struct AttnShape {
     // sequence's query count (an upper bound).  nullptr: fixed-length batch.
     const int *cu_q = nullptr, *cu_k = nullptr;
     int total_q = 0, total_k = 0;
+    // > 0: lse's stride between heads (B = 1 only), so that a launch over some
+    // query positions writes its lse into the columns of a wider [Hq, L] array
+    int lse_hs = 0;
 };
 
 struct DecodeShape {
@@ -109,6 +112,13 @@ cudaError_t launch_fwd_tc_fp8(const void *q, const void *k, const void *v, const
                               const float *k_scale, const float *v_scale, const float *sinks, void *out, float *lse,
                               void *v16, const AttnShape &s, cudaStream_t st);
 bool fwd_tc_supported(const AttnShape &s);
+
+// The bf16 prefill forward from and to host memory, chunks of query positions
+// overlapping their transfers with the computation (host_fwd.cu); Lq <= Lk.
+constexpr int kFwdHostMaxChunks = 64;
+size_t fwd_host_workspace_bytes(const AttnShape &s);
+cudaError_t run_fwd_host(const void *q_h, const void *k_h, const void *v_h, const float *sinks_h, void *out_h,
+                         float *lse_h, const AttnShape &s, int n_chunks, void *workspace, cudaStream_t st);
 
 // bf16 split-KV decode: TMA-staged K/V, tensor-core (mma.sync) group scores.
 // With k_scale / v_scale ([Hkv] fp32, device) the caches hold e4m3 values

@@ -99,6 +99,40 @@ ATTN_SINK_API int attn_sink_fwd(const void *q, const void *k, const void *v, con
                   int window, float scale, int dtype, void *stream);
 
 /*
+ * The bf16 prefill forward of attn_sink_fwd with every tensor in HOST memory:
+ * q, k, v, sinks are read from host memory and out, lse written back to it,
+ * with the transfers overlapped with the computation.  The query positions
+ * are cut into up to `n_chunks` chunks (1..64; multiples of 128 positions): chunk c's
+ * rows need only the keys up to its last position, so while chunk c is
+ * computed, chunk c + 1's q rows and new k, v rows travel to the device and
+ * chunk c - 1's out rows and lse travel back (host-to-device and
+ * device-to-host copies run on two streams of the library's own, the kernels
+ * on `stream`; the call returns once everything is enqueued, and `stream` is
+ * ordered after the last copy, so synchronising `stream` waits for the whole
+ * call).  Each row's arithmetic is that of attn_sink_fwd on the same inputs
+ * (the chunks hold whole work items of the forward, so the same tiles), so
+ * the results are bit-for-bit identical.
+ *   q_host [B, Lq, Hq, D], k_host, v_host [B, Lk, Hkv, D] bf16; sinks_host
+ *   [Hq] fp32; out_host [B, Lq, Hq, D] bf16 and lse_host [B, Hq, Lq] fp32
+ *   (written).  Host buffers should be page-locked (cudaHostAlloc, or
+ *   torch's pin_memory) for the copies to overlap; pageable memory gives the
+ *   same results without the overlap.  The caller keeps them alive and
+ *   unchanged until `stream` has passed the call.
+ *   workspace: device memory of attn_sink_fwd_host_workspace_size() bytes,
+ *   16-byte aligned, owned by the caller (the device copies of q, k, v,
+ *   sinks, out and lse); it must not be in use by other work on other
+ *   streams during the call.
+ *   Lq <= Lk (else ATTN_SINK_ERR_UNSUPPORTED); other arguments and errors as
+ *   for attn_sink_fwd with dtype BF16; ATTN_SINK_ERR_INVALID_ARG for
+ *   n_chunks outside 1..64.
+ */
+ATTN_SINK_API size_t attn_sink_fwd_host_workspace_size(int B, int Lq, int Lk, int Hq, int Hkv, int D);
+ATTN_SINK_API int attn_sink_fwd_host(const void *q_host, const void *k_host, const void *v_host,
+                  const float *sinks_host, void *out_host, float *lse_host, int B, int Lq, int Lk,
+                  int Hq, int Hkv, int D, int window, float scale, int n_chunks,
+                  void *workspace, size_t ws_bytes, void *stream);
+
+/*
  * Prefill forward over packed ragged sequences ("varlen"): a batch of B
  * sequences of different lengths stored back to back, as a prefill server
  * that gathers requests of any length receives them (the pages separate the

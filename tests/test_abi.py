@@ -144,6 +144,32 @@ def test_fwd_fp8_host_checks():
     assert call(w=ws + 4) == MISALIGNED
 
 
+def test_fwd_host_buffers_checks():
+    """Argument checks of the host-buffer prefill, all on the host (nothing is enqueued)."""
+    lib = attn.load()
+    q, k, v, s, o, l, ws = _fake(7)
+    need = attn.attn_sink_fwd_host_workspace_size(2, 100, 120, 8, 2, 64)
+    # q and out, k and v, lse [B, Hq, Lq], sinks; 256-byte sections
+    a256 = lambda x: (x + 255) // 256 * 256
+    assert need == (2 * a256(2 * 100 * 8 * 64 * 2) + 2 * a256(2 * 120 * 2 * 64 * 2) + a256(2 * 8 * 100 * 4) + a256(8 * 4))
+    assert attn.attn_sink_fwd_host_workspace_size(2, 100, 120, 8, 3, 64) == 0
+
+    def call(B=2, Lq=100, Lk=120, Hq=8, Hkv=2, D=64, scale=0.125, chunks=4, qq=q, w=ws, wbytes=need):
+        return lib.attn_sink_fwd_host(qq, k, v, s, o, l, B, Lq, Lk, Hq, Hkv, D, 0, scale, chunks, w, wbytes, None)
+
+    assert call(qq=None) == INVALID
+    assert call(chunks=0) == INVALID
+    assert call(chunks=65) == INVALID
+    assert call(B=0) == INVALID
+    assert call(Hkv=3) == INVALID
+    assert call(D=128) == UNSUPPORTED
+    assert call(scale=0.0) == UNSUPPORTED
+    assert call(Lq=121) == UNSUPPORTED  # more queries than keys
+    assert call(w=None, wbytes=0) == WORKSPACE
+    assert call(wbytes=need - 1) == WORKSPACE
+    assert call(w=ws + 4) == MISALIGNED
+
+
 def test_decode_paged_host_checks():
     lib = attn.load()
     q, kp, vp, pt, sl, s, o, l = _fake(8)

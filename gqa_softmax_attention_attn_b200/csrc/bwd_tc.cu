@@ -638,8 +638,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive(stg_full);
             if (issuer) {
                 if (!mbar_wait(stg_full, i & 1u, abort_flag, p.status, p.timeout_ns)) break;
-                tma_reduce_add_4d(&tmDQ, stg, 0, h0, pos0, b);
-                tma_reduce_add_4d(&tmDQ, reinterpret_cast<uint8_t *>(stg) + kM * 128, kD / 2, h0, pos0, b);
+                // the accumulator's lines stay in L2 ahead of the streamed q and
+                // dO tiles, for the other key tiles' adds and the final
+                // conversion (window-128 backward 135 -> 132 us at B1 L4096)
+                const uint64_t pol = l2_policy_evict_last();
+                tma_reduce_add_4d_hint(&tmDQ, stg, 0, h0, pos0, b, pol);
+                tma_reduce_add_4d_hint(&tmDQ, reinterpret_cast<uint8_t *>(stg) + kM * 128, kD / 2, h0, pos0, b, pol);
                 bulk_commit_group();
                 bulk_wait_read_all();
                 mbar_arrive(stg_free);

@@ -264,6 +264,25 @@ __device__ __forceinline__ void tma_load_4d(void *smem_dst, const CUtensorMap *m
         : "memory");
 }
 
+// L2 cache policy for the cache-hinted copies below (all of the access
+// fraction): lines kept past others.
+__device__ __forceinline__ uint64_t l2_policy_evict_last()
+{
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+// tma_reduce_add_4d with an L2 cache policy for the lines it adds into
+__device__ __forceinline__ void tma_reduce_add_4d_hint(const CUtensorMap *map, const void *smem_src, int c0, int c1,
+                                                       int c2, int c3, uint64_t policy)
+{
+    asm volatile(
+        "cp.reduce.async.bulk.tensor.4d.global.shared::cta.add.bulk_group.L2::cache_hint [%0, {%2, %3, %4, %5}], [%1], "
+        "%6;" ::"l"(reinterpret_cast<uint64_t>(map)),
+        "r"(smem_u32(smem_src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "l"(policy)
+        : "memory");
+}
+
 // 4-D tiled bulk tensor reduce-add shared -> global (fp32 add in L2), bulk-group completion.
 __device__ __forceinline__ void tma_reduce_add_4d(const CUtensorMap *map, const void *smem_src, int c0, int c1,
                                                   int c2, int c3)

@@ -136,6 +136,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     float *ld = reinterpret_cast<float *>(smem + kOffLD);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // The launch overlaps the row pre-pass (programmatic dependent launch):
+    // the set-up, K, V, Q and dO loads and the first scores need nothing from
+    // it; the load warp waits for it before reading D, the dQ warps before
+    // their first add into the accumulator it clears.  The finish kernel may
+    // start once every CTA of this grid is running.
+    grid_dep_launch();
     // 1-D grid, key tile slowest: under a causal mask the first key tiles see
     // the most q tiles, so every head's and batch's longest CTAs start first
     const int per_kt = p.Hkv * p.B;
@@ -224,6 +230,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         static_assert(kM == 32 * 4, "one group of 4 lse / D values per lane");
+        grid_dep_wait();  // D comes from the pre-pass
         for (int i = 0; i < n_iter && ok; ++i) {
             const int st = i & 1;
             int h0, pos0;
@@ -604,6 +611,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int row = quad * 32 + lane;
         const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
         const bool issuer = (warp == 6 && lane == 0);
+        grid_dep_wait();  // the pre-pass clears the accumulator
         float *stg = reinterpret_cast<float *>(smem + kOffStg);
         for (int i = 0; i < n_iter; ++i) {
             int h0, pos0;
@@ -668,6 +676,7 @@ __global__ void __launch_bounds__(256) bwd_finish_kernel(const float *__restrict
                                                          size_t n8, unsigned n_conv, const float *__restrict__ terms,
                                                          float *__restrict__ dsinks, long nterms)
 {
+    grid_dep_wait();  // launched ahead of the main kernel's end: its dQ and the pre-pass's terms
     if (blockIdx.x >= n_conv) {
         __shared__ float red[256];
         const int h = (int)(blockIdx.x - n_conv), t = threadIdx.x;
@@ -701,8 +710,17 @@ cudaError_t launch_gp(const CUtensorMap &mq, const CUtensorMap &mdo, const CUten
 {
     cudaError_t e = cudaFuncSetAttribute(bwd_tc_kernel<GP>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
-    bwd_tc_kernel<GP><<<grid, kThreads, kSmemBytes, st>>>(mq, mdo, mk, mv, mdq, p);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, bwd_tc_kernel<GP>, mq, mdo, mk, mv, mdq, p);
 }
 
 }  // namespace
@@ -770,9 +788,17 @@ cudaError_t launch_bwd_tc(const void *q, const void *k, const void *v, const voi
     const size_t n8 = (size_t)s.B * s.Lq * s.Hq * s.D / 8;
     const size_t n_conv = (n8 + 255) / 256;
     if (n_conv + s.Hq > 0x7fffffffu) return cudaErrorInvalidValue;
-    bwd_finish_kernel<<<(unsigned)(n_conv + s.Hq), 256, 0, st>>>(dq_acc, static_cast<__nv_bfloat16 *>(dq), n8,
-                                                                  (unsigned)n_conv, terms, dsinks, (long)s.B * s.Lq);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(n_conv + s.Hq));
+    cfg.blockDim = dim3(256);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, bwd_finish_kernel, (const float *)dq_acc, static_cast<__nv_bfloat16 *>(dq), n8,
+                              (unsigned)n_conv, terms, dsinks, (long)s.B * s.Lq);
 }
 
 bool bwd_tc_supported(const AttnShape &s)

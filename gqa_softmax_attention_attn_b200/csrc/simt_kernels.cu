@@ -8,6 +8,7 @@
 #include <math.h>
 
 #include "kernels.h"
+#include "sm100_ptx.cuh"
 
 namespace attn_sink {
 namespace {
@@ -173,6 +174,9 @@ __global__ void __launch_bounds__(256, PreRows<T>::kMinCtas) bwd_pre_kernel(cons
                                                       AttnShape s)
 {
     using R = PreRows<T>;
+    // the backward's main kernel may start its set-up (it waits for this
+    // grid before it reads D or adds into the accumulator)
+    grid_dep_launch();
     const int sub = threadIdx.x % R::kTpr;  // chunk of the row
     const long nrows = (long)s.B * s.Lq * s.Hq;
     const long row0 = (long)blockIdx.x * R::kRowsPerCta + threadIdx.x / R::kTpr;

@@ -264,6 +264,14 @@ __device__ __forceinline__ void tma_load_4d(void *smem_dst, const CUtensorMap *m
         : "memory");
 }
 
+// Programmatic dependent launch: a grid launched with the programmatic
+// stream-serialisation attribute may start before the grid ahead of it on the
+// stream has finished; grid_dep_wait() blocks until that grid has completed
+// and its memory operations are visible, grid_dep_launch() lets the next such
+// grid start (both are no-ops for grids launched without the attribute).
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // L2 cache policy for the cache-hinted copies below (all of the access
 // fraction): lines kept past others.
 __device__ __forceinline__ uint64_t l2_policy_evict_last()

@@ -48,6 +48,24 @@ def test_prologue_matches_oracle(interleaved, rope, with_bias):
     assert_close_bf16(v, rv, f"v {rope} interleaved={interleaved}")
 
 
+@pytest.mark.parametrize("shape", [(9, 8, 1), (7, 300, 4), (5, 600, 8), (3, 784, 8), (130, 4, 4)])
+def test_prologue_row_widths(shape):
+    """Narrow and very wide rows (10 to 800 heads), token counts that leave
+    the last 8-token CTA ragged."""
+    T, Hq, Hkv = shape
+    qkv, bias, pos = make_qkv(T, Hq, Hkv, seed=221 + Hq, max_pos=131072)
+    dev = "cuda"
+    q = torch.empty(T, Hq, 64, dtype=torch.bfloat16, device=dev)
+    k = torch.empty(T, Hkv, 64, dtype=torch.bfloat16, device=dev)
+    v = torch.empty_like(k)
+    attn_sink_qkv_prologue(qkv.to(dev), bias.to(dev), pos.to(dev), q, k, v, **YARN)
+    torch.cuda.synchronize()
+    rq, rk, rv = oracle.qkv_prologue(qkv, bias, pos, Hq, Hkv, 64, **ORACLE_YARN)
+    assert_close_bf16(q, rq, f"q {shape}")
+    assert_close_bf16(k, rk, f"k {shape}")
+    assert_close_bf16(v, rv, f"v {shape}")
+
+
 def test_prologue_appends_to_a_decode_cache():
     """kv_rows sends token t's k and v to row b * Lmax + p of a [B, Lmax] cache;
     every other row keeps its contents, and rows outside the cache are skipped."""

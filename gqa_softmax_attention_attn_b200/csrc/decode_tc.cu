@@ -594,7 +594,10 @@ cudaError_t launch_decode_bf16(const void *q, const void *kc, const void *vc, co
     // three whole tiles of a paged cache) needs about three 64-key tiles:
     // three stages hold them, and the smaller ring lets four CTAs share an SM
     // (measured on the window-128 decode of 64 sequences: 17.2 -> 15.4 us;
-    // long splits keep four stages, 336.6 vs 338.8 us dense)
+    // long contiguous splits keep four stages, 336.6 vs 338.8 us dense).  A
+    // paged cache moves its tiles in page-sized boxes, and more CTAs per SM
+    // keep more of them in flight: three stages there too (dense decode over
+    // 16-key pages 388 -> 379 us).
     auto pick = [&](auto stages) -> cudaError_t {
         constexpr int kS = decltype(stages)::value;
         constexpr int sb = DecLayout<false, kS>::kSmemBytes;
@@ -604,7 +607,7 @@ cudaError_t launch_decode_bf16(const void *q, const void *kc, const void *vc, co
         return paged ? launch(decode_tc_kernel<false, true, false, kS>, sb)
                      : launch(decode_tc_kernel<false, false, false, kS>, sb);
     };
-    return s.chunk <= 192 ? pick(std::integral_constant<int, 3>{}) : pick(std::integral_constant<int, 4>{});
+    return (s.chunk <= 192 || paged) ? pick(std::integral_constant<int, 3>{}) : pick(std::integral_constant<int, 4>{});
 }
 
 }  // namespace attn_sink

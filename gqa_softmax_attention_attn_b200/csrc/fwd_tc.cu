@@ -102,6 +102,16 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 #define ATTN_SINK_FWD_SPEC 1
 #endif
 constexpr bool FWD_SPEC = ATTN_SINK_FWD_SPEC != 0;
+// 1: with FWD_SPEC, the pass tracks no maximum; a tile whose exponentials sum
+// past kSumLimit (so one of them may exceed it) takes the rare path, which
+// finds the maximum (measured on the gpt-oss-20b prefill's dense layer:
+// 208.9 -> 206.9 us); 0: the maximum tracked in the pass, the rare path when
+// it exceeds the reference by 2^8
+#ifndef ATTN_SINK_FWD_SUMCHECK
+#define ATTN_SINK_FWD_SUMCHECK 1
+#endif
+constexpr bool FWD_SUMCHECK = ATTN_SINK_FWD_SUMCHECK != 0;
+constexpr float kSumLimit = 1024.f;
 // launch-control requests in flight: dense items are long, so one hides the
 // round trip (measured on the gpt-oss-20b prefill's dense layer: 205.6 us at
 // one, 206.8 at two, 230.5 at four, where CTAs hold on to items others could
@@ -566,19 +576,42 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT, F8>::kThreads, CPS)
                 float alpha = 1.f;
                 if (FWD_SPEC) {
                     // The exponentials first, against the current reference (it
-                    // only moves when the true maximum exceeds it by 2^8, so it
-                    // rarely does), with the tile maximum found in the same pass;
-                    // a row whose maximum did move redoes the pass (S is still in
-                    // registers, P not yet handed to the MMA).
+                    // only moves when a tile's exponentials grow past a bound, so
+                    // it rarely does); a row whose reference does move redoes the
+                    // pass (S is still in registers, P not yet handed to the MMA).
                     const float neg_m0 = (m == -INFINITY) ? 0.f : -m;
-                    if (need_mask)
-                        exp_pass(neg_m0, std::true_type{}, std::false_type{});
-                    else
-                        exp_pass(neg_m0, std::true_type{}, std::true_type{});
-                    const float tmax =
-                        fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
-                    const float m_new = fmaxf(m, tmax * C);
-                    rescale = m_new > m + kRescaleThreshold;
+                    float m_new = m;
+                    if (FWD_SUMCHECK) {
+                        if (need_mask)
+                            exp_pass(neg_m0, std::false_type{}, std::false_type{});
+                        else
+                            exp_pass(neg_m0, std::false_type{}, std::true_type{});
+                        // every exponential is at most their sum: a sum within
+                        // kSumLimit (NaN fails the test) keeps the reference; a
+                        // row with no reference yet (sink -inf) takes the rare
+                        // path until a tile gives it one
+                        const float tsum = (acc[0].x + acc[0].y) + (acc[1].x + acc[1].y);
+                        const bool big = !(tsum <= kSumLimit) || m == -INFINITY;
+                        if (__any_sync(0xffffffffu, big)) {
+#pragma unroll
+                            for (int c = 0; c < kC; c += 16)
+#pragma unroll
+                                for (int k = 0; k < 8; ++k) mx[k] = fmax3(mx[k], sv[c + k], sv[c + 8 + k]);
+                            const float tmax =
+                                fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
+                            m_new = fmaxf(m, tmax * C);
+                            rescale = big && m_new > m;
+                        }
+                    } else {
+                        if (need_mask)
+                            exp_pass(neg_m0, std::true_type{}, std::false_type{});
+                        else
+                            exp_pass(neg_m0, std::true_type{}, std::true_type{});
+                        const float tmax =
+                            fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
+                        m_new = fmaxf(m, tmax * C);
+                        rescale = m_new > m + kRescaleThreshold;
+                    }
                     if (__any_sync(0xffffffffu, rescale)) {
                         alpha = rescale ? ((m == -INFINITY) ? 0.f : ex2(m - m_new)) : 1.f;
                         if (rescale) m = m_new;

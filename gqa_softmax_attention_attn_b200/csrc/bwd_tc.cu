@@ -36,9 +36,12 @@
 //    there, so the P pass never tests visibility.
 //  * Warps 6-9 move each dQ tile from TMEM to shared memory (two 128-byte-
 //    swizzled fp32 halves) and add it into an fp32 dQ accumulator in global
-//    memory with TMA reduce-adds (L2 atomics; the summation order over key
-//    tiles is not fixed).  dK and dV of the tile are written once, at the end
-//    (deterministic).
+//    memory with TMA reduce-adds (L2 atomics, evict_last so the accumulator
+//    stays in L2; the summation order over key tiles is not fixed).  dK and
+//    dV of the tile are written once, at the end (deterministic).  A finish
+//    kernel turns the accumulator into bf16 dQ and sums dsink in a fixed
+//    order; the main and finish kernels are chained to the row pre-pass by
+//    programmatic dependent launch.
 //  * One CTA per SM (512 TMEM columns); the 14 warps cap registers at 128 per
 //    thread.  The grid is 1-D with the key tile slowest, so the causally
 //    longest CTAs of every head and batch start first.

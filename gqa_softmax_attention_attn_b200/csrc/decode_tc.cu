@@ -10,8 +10,9 @@
 // Design (B200): the path is HBM-bound (8 flop per byte of KV at GQA group 8).
 //  * CTA = (split c, KV head g, sequence b).  Warp 0 streams the split's K and
 //    V rows of head g with 2-D-tiled TMA boxes (64 keys x 128 bytes, 128-byte
-//    swizzle) into a 4-stage shared-memory ring; every byte of KV is read
-//    from HBM once, for all G query heads of the group.
+//    swizzle) into a shared-memory ring (4 stages; 3 for short splits and for
+//    paged caches, so four CTAs share an SM); every byte of KV is read from
+//    HBM once, for all G query heads of the group.
 //  * Warps 1-4 take 16 keys of each 64-key tile: the G query heads of the
 //    group (padded to 16 rows) are scored with mma.sync m16n8k16 -- FP32 CUDA
 //    cores cannot sustain 8 flop/byte at HBM rate -- then an exp2 online

@@ -131,6 +131,7 @@ __device__ __forceinline__ uint32_t swz(int row, int chunk) { return row * 128 +
 template <bool kRows16, bool kPaged, bool kFp8, int kStages>
 __device__ __forceinline__ void decode_tc_body(const CUtensorMap &tmK, const CUtensorMap &tmV, const DecodeParams &p)
 {
+    grid_dep_launch();  // the split combine may be launched now; it waits for this grid
     using L = DecLayout<kFp8, kStages>;
     constexpr int kT = L::kT;
     static_assert(!(kPaged && kFp8), "paged caches are bf16 only");

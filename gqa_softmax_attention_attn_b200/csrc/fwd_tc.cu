@@ -327,6 +327,10 @@ __global__ void __launch_bounds__(FwdCfg<BN, NS, CPS, SPLIT, F8>::kThreads, CPS)
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
+            // e4m3 inputs: v comes widened from the kernel ahead, whose grid
+            // lets this one start early (programmatic dependent launch); the
+            // loads wait for it (no-op for a grid launched the plain way)
+            if (F8) grid_dep_wait();
             tma_prefetch_desc(&tmQ);
             tma_prefetch_desc(&tmK);
             tma_prefetch_desc(&tmV);
@@ -810,8 +814,22 @@ cudaError_t launch_cfg(const void *q, const void *k, const void *v, const float 
     if (e != cudaSuccess) return e;
     // one CTA per item: as many start as fit (kCtasPerSm per SM), the rest are
     // taken over by running CTAs before they launch
-    kern<<<p.n_items, Cfg::kThreads, Cfg::kSmemBytes, st>>>(mq, mk, mv, p);
-    return cudaGetLastError();
+    if (!F8) {
+        kern<<<p.n_items, Cfg::kThreads, Cfg::kSmemBytes, st>>>(mq, mk, mv, p);
+        return cudaGetLastError();
+    }
+    // e4m3: chained to the widening kernel (programmatic dependent launch)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)p.n_items);
+    cfg.blockDim = dim3(Cfg::kThreads);
+    cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, p);
 }
 
 }  // namespace
@@ -839,6 +857,7 @@ namespace {
 __global__ void __launch_bounds__(256) widen_e4m3_kernel(const uint8_t *__restrict__ src, uint8_t *__restrict__ dst,
                                                          size_t n16)
 {
+    grid_dep_launch();  // the attention kernel may start its set-up
     const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= n16) return;
     uint4 lo, hi;

@@ -521,6 +521,7 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const int *__restri
                                                              const float *__restrict__ ws_o,
                                                              const float *__restrict__ ws_ml, DecodeShape s)
 {
+    grid_dep_wait();  // the split partials of the decode grid ahead (programmatic dependent launch)
     const int lane = threadIdx.x & 31;
     const long bh = (long)blockIdx.x * 4 + (threadIdx.x >> 5);
     if (bh >= (long)s.B * s.Hq) return;
@@ -609,8 +610,16 @@ cudaError_t launch_decode_combine(const int *seqlens, const float *sinks, T *out
                                   const DecodeShape &s, const float *ws_o, const float *ws_ml, cudaStream_t st)
 {
     const long n = (long)s.B * s.Hq;
-    decode_combine_kernel<T><<<(unsigned)((n + 3) / 4), 128, 0, st>>>(seqlens, sinks, out, lse, ws_o, ws_ml, s);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((n + 3) / 4));
+    cfg.blockDim = dim3(128);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, decode_combine_kernel<T>, seqlens, sinks, out, lse, ws_o, ws_ml, s);
 }
 
 #define ATTN_SINK_INSTANTIATE(T)                                                                              \

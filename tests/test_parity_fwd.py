@@ -62,6 +62,17 @@ def test_bf16_small_shapes(shape, window):
     assert_lse(lse, rl, f"lse {shape} w={window}")
 
 
+@pytest.mark.parametrize("window", [0, 128])
+def test_bf16_many_heads(window):
+    """1040 query heads in groups of 8 (130 KV heads): a wide head dimension of
+    the grid for both forward kernels."""
+    t = prefill_inputs(1, 40, 40, 1040, 130, 64, torch.bfloat16, 0.5, 1.0, seed=41 + window)
+    out, lse = run_fwd(t, window, 0.125)
+    ro, rl = oracle.fwd(t["q"], t["k"], t["v"], t["sinks"], window, 0.125)
+    assert_close_bf16(out, ro, f"1040 heads w={window}")
+    assert_lse(lse, rl, f"1040 heads w={window}")
+
+
 @pytest.mark.parametrize("sink", [float("-inf"), 50.0, -30.0])
 def test_bf16_extreme_sinks(sink):
     t = prefill_inputs(1, 150, 150, 16, 2, 64, torch.bfloat16, 0.5, 1.0, seed=7, sink_fill=sink)

@@ -56,6 +56,28 @@ cudaError_t pipe_init(HostPipe &hp)
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Chunk c of the Lq positions spans [bnd[c], bnd[c + 1]); returns the number of
+// chunks (at most n).  The first chunk's copy-in and the last chunk's kernel
+// and copy-out overlap nothing, so with three or more chunks those two get
+// weight 1 and the others weight 2; every end but the last is rounded to a
+// whole 128-position block.  (Four chunks of a B1 L4096 dense layer: 1.21 ms
+// against 1.29-1.30 ms for equal chunks.)
+int chunk_bounds(int Lq, int n, int *bnd)
+{
+    const long long wsum = n <= 2 ? n : 2 * (long long)n - 2;
+    long long cum = 0;
+    int nc = 0;
+    bnd[0] = 0;
+    for (int c = 0; c < n; ++c) {
+        cum += (n <= 2 || c == 0 || c == n - 1) ? 1 : 2;
+        int e = (int)((Lq * cum + wsum / 2) / wsum);
+        e = c == n - 1 ? Lq : (e + 64) / 128 * 128;
+        if (e > Lq) e = Lq;
+        if (e > bnd[nc]) bnd[++nc] = e;
+    }
+    return nc;
+}
+
 }  // namespace
 
 size_t fwd_host_workspace_bytes(const AttnShape &s)
@@ -98,9 +120,8 @@ cudaError_t run_fwd_host(const void *q_h, const void *k_h, const void *v_h, cons
                   *vh = static_cast<const uint8_t *>(v_h);
     uint8_t *oh = static_cast<uint8_t *>(out_h);
     const int off = s.Lk - s.Lq;  // >= 0
-    int len = (s.Lq + n_chunks - 1) / n_chunks;
-    len = (len + 127) / 128 * 128;  // whole items per chunk
-    const int nc = (s.Lq + len - 1) / len;
+    int bnd[kFwdHostMaxChunks + 1];
+    const int nc = chunk_bounds(s.Lq, n_chunks, bnd);  // whole items per chunk
 
 #define ATTN_SINK_CK(x)                  \
     do {                                 \
@@ -113,7 +134,7 @@ cudaError_t run_fwd_host(const void *q_h, const void *k_h, const void *v_h, cons
     ATTN_SINK_CK(cudaMemcpyAsync(sinks_d, sinks_h, (size_t)s.Hq * 4, cudaMemcpyHostToDevice, hp.h2d));
     int kv_done = 0;  // key rows already sent (the same for every batch element)
     for (int c = 0; c < nc; ++c) {
-        const int p0 = c * len, p1 = p0 + len < s.Lq ? p0 + len : s.Lq;
+        const int p0 = bnd[c], p1 = bnd[c + 1];
         const int kneed = p1 + off;  // keys the chunk's rows can see
         const size_t nq = (size_t)(p1 - p0) * row_q;
         // in: the chunk's q rows and the keys it adds

@@ -102,10 +102,12 @@ ATTN_SINK_API int attn_sink_fwd(const void *q, const void *k, const void *v, con
  * The bf16 prefill forward of attn_sink_fwd with every tensor in HOST memory:
  * q, k, v, sinks are read from host memory and out, lse written back to it,
  * with the transfers overlapped with the computation.  The query positions
- * are cut into up to `n_chunks` chunks (1..64; multiples of 128 positions): chunk c's
+ * are cut into up to `n_chunks` chunks (1..64; multiples of 128 positions;
+ * with three or more, the first and the last hold half as many positions as
+ * the others, since nothing overlaps their copies): chunk c's
  * rows need only the keys up to its last position, so while chunk c is
  * computed, chunk c + 1's q rows and new k, v rows travel to the device and
- * chunk c - 1's out rows and lse travel back (host-to-device and
+ * chunk c - 1's out rows travel back (lse once, at the end; host-to-device and
  * device-to-host copies run on two streams of the library's own, the kernels
  * on `stream`; the call returns once everything is enqueued, and `stream` is
  * ordered after the last copy, so synchronising `stream` waits for the whole

@@ -419,6 +419,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float C = p.c_log2;
         const bool storer = (warp == 4 + 4 * wg) && lane == 0;  // issues the warpgroup's tensor stores
         bool stores_issued = false;
+        // The buffer an item's O was staged in is released once its tensor
+        // store has read it; the storer checks that only in the next item's
+        // pass, after that item's scores are in registers, instead of waiting
+        // for the read right after the store.  The next item of the warpgroup
+        // uses another stage, so its own loads never wait for that release.
+        static_assert(kNS > 2, "a warpgroup's consecutive items in different stages");
+        uint64_t *store_free = nullptr;
         for (int r = wg;; r += 2) {
             const int w = consumer_item(r);
             if (w < 0) break;
@@ -464,6 +471,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int c = 0; c < kChunks; ++c) tmem_ld16(trow + 16 * c, sr[c]);
             tmem_wait_ld();
+            if (storer && store_free != nullptr) {
+                bulk_wait_read_all();
+                mbar_arrive(store_free);
+                store_free = nullptr;
+            }
             float mx[8];
 #pragma unroll
             for (int k = 0; k < 8; ++k) mx[k] = -INFINITY;
@@ -551,11 +563,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ragged) {
                     tma_store_4d(&tmO, stg, 0, t.h0, t.qrow0 + t.pos0, t.tb);
                     bulk_commit_group();
-                    bulk_wait_read_all();  // the buffer may take its next load once the store has read it
                     stores_issued = true;
+                    store_free = stg_free;  // released once the store has read it (above)
+                } else {
+                    mbar_arrive(stg_free);
                 }
-                mbar_arrive(stg_free);
             }
+        }
+        if (storer && store_free != nullptr) {
+            bulk_wait_read_all();
+            mbar_arrive(store_free);
         }
         if (storer && stores_issued) bulk_wait_all();  // every tensor store completes before the CTA exits
     }

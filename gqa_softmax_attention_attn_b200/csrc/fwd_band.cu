@@ -34,7 +34,9 @@
 //    item's K buffer (its Q buffer for narrow bands; either is dead once S is
 //    done) in the 128-byte-swizzled layout of an output box, and stored with
 //    one TMA tensor store (a box that would run into the next packed sequence
-//    is stored row by row instead); lse row by row.
+//    is stored row by row instead); lse row by row.  The buffer goes back to
+//    the producer once the store has read it, which the storing thread checks
+//    in the warpgroup's next item rather than waiting for it right away.
 //  * Every wait is bounded; on expiry the CTA raises a status bit, waits
 //    (bounded) for its own TMA loads, stores and MMAs, frees tensor memory and
 //    exits.

@@ -73,10 +73,13 @@ def test_host_against_oracle(window):
     assert_lse(lse, rl, f"host fwd w={window}")
 
 
+@pytest.mark.parametrize("chunks", [4, 8])
 @pytest.mark.parametrize("window", [0, 128])
-def test_host_prefill_20b(window):
-    """The gpt-oss-20b prefill (B1 L4096 Hq64 Hkv8) in eight chunks, bit for bit."""
+def test_host_prefill_20b(window, chunks):
+    """The gpt-oss-20b prefill (B1 L4096 Hq64 Hkv8), bit for bit: four chunks
+    (640, 1408, 1408, 640 positions: the end chunks take half the others') and
+    eight."""
     t = prefill_inputs(1, 4096, 4096, 64, 8, 64, torch.bfloat16, 0.5, 1.0, 0.1, seed=99 + window)
-    o1, l1 = host_call(t, window, 8)
+    o1, l1 = host_call(t, window, chunks)
     o2, l2 = device_call(t, window)
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
